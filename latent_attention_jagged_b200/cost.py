@@ -1,0 +1,91 @@
+"""Algorithmic work of one forward pass, counted from the jagged lengths.
+
+The count follows the cost structure of the pyramidal schedule (LLaTTE notes,
+huaxiaozhuan.com appendix A.2: attention O(T_{l+1} T_l d), FFN O(T_{l+1} d^2),
+i.e. projections and FFN on the kept query rows only, attention over the
+visible (query, key) pairs only) with the constants of the absorbed MLA form
+(appendix A.3: per-head queries in the rank-r latent, one shared K=V latent).
+
+Per user and layer, with T history rows in, n = min(T, keep) kept, q = n + n_q:
+  kv      2 T d r
+  q       2 q d h r + 2 d_ctx h r          (context term once per user)
+  attn    4 h r P,  P = n_q T + n T - n (n - 1) / 2  visible pairs
+  o       2 q h r d
+  ffn1    2 q d (m d)      ffn2  2 q (m d) d        (m = FFN multiplier)
+  readout 2 d d_out per user (final layer)
+Masked pairs and padding are not counted.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Sequence
+
+import numpy as np
+
+
+@dataclass
+class LayerWork:
+    T: np.ndarray
+    n: np.ndarray
+    q: np.ndarray
+    pairs: np.ndarray
+    flops: Dict[str, float] = field(default_factory=dict)
+
+
+def visible_pairs(T: np.ndarray, n: np.ndarray, n_q: int) -> np.ndarray:
+    T = np.asarray(T, dtype=np.int64)
+    n = np.asarray(n, dtype=np.int64)
+    return n_q * T + n * T - n * (n - 1) // 2
+
+
+def layer_work(lengths: Sequence[int], dims) -> List[LayerWork]:
+    T = np.asarray(lengths, dtype=np.int64)
+    d, h, r, dc, m = dims.d, dims.heads, dims.rank, dims.d_ctx, dims.ffn_mult
+    out = []
+    for k in dims.keep:
+        n = np.minimum(T, k)
+        q = n + dims.n_q
+        P = visible_pairs(T, n, dims.n_q)
+        B = T.shape[0]
+        f = {
+            "kv": 2.0 * T.sum() * d * r,
+            "q": 2.0 * q.sum() * d * h * r + 2.0 * B * dc * h * r,
+            "attn": 4.0 * h * r * P.sum(),
+            "o": 2.0 * q.sum() * h * r * d,
+            "ffn1": 2.0 * q.sum() * d * m * d,
+            "ffn2": 2.0 * q.sum() * m * d * d,
+        }
+        out.append(LayerWork(T=T.copy(), n=n, q=q, pairs=P, flops=f))
+        T = n
+    return out
+
+
+def total_flops(lengths: Sequence[int], dims) -> float:
+    work = layer_work(lengths, dims)
+    tot = sum(sum(w.flops.values()) for w in work)
+    if dims.d_out:
+        tot += 2.0 * len(lengths) * dims.d * dims.d_out
+    return float(tot)
+
+
+def flops_by_step(lengths: Sequence[int], dims) -> Dict[str, float]:
+    acc: Dict[str, float] = {}
+    for w in layer_work(lengths, dims):
+        for k, v in w.flops.items():
+            acc[k] = acc.get(k, 0.0) + float(v)
+    if dims.d_out:
+        acc["readout"] = 2.0 * len(lengths) * dims.d * dims.d_out
+    return acc
+
+
+def io_bytes(lengths: Sequence[int], dims, elem: int = 2) -> float:
+    """Bytes a forward must move at least: the inputs read once, the
+    weights read once, the outputs written once (fp32)."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    B = lengths.shape[0]
+    d, hd, r, dc, f = dims.d, dims.heads * dims.d_head, dims.rank, dims.d_ctx, dims.d_ffn
+    inp = (lengths.sum() + B * dims.n_q) * d * elem + B * dc * elem + (B + 1) * 8
+    per_layer_w = (r * d + r + hd * (d + dc) + 2 * hd * r + d * hd + 2 * d + 2 * f * d) * elem
+    w = dims.n_layers * per_layer_w + dims.d_out * d * elem
+    out = B * (dims.d_out if dims.d_out else dims.n_q * d) * 4
+    return float(inp + w + out)

@@ -1,0 +1,128 @@
+"""Model dimensions and the five synthetic workloads.
+
+The shapes follow the LLaTTE pages: the online ranker looks at roughly 400
+recent events per source with candidate/context query tokens (huaxiaozhuan.com
+LLaTTE notes, sec. 1.6.4 and 1.7.1), the upstream user model encodes
+1600-token histories with user-only query tokens and a 2048-d transfer
+embedding (paper-daily.com deep reading, pipeline diagram; huaxiaozhuan.com
+sec. 1.6.1), and the horizon sweep uses T in {200, 400, 800, 1600}
+(huaxiaozhuan.com sec. 1.5.3). Depth/width values come from the d >= 256,
+L in {1,2,4,8} grid of huaxiaozhuan.com sec. 1.5.2.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Tuple
+
+
+@dataclass(frozen=True)
+class Dims:
+    """Sequence-module dimensions.
+
+    d        token width
+    heads    attention heads h
+    d_head   per-head width d_h (attention scale is 1/sqrt(d_h))
+    rank     MLA latent rank r (shared K=V latent width)
+    d_ctx    width of the non-sequence context vector c (0 = none)
+    n_q      query (candidate) tokens appended per user
+    keep     per-layer count of most recent HISTORY rows kept as queries
+             and as the next layer's sequence (non-increasing)
+    d_out    readout width (0 = output the final query-token rows)
+    ffn_mult FFN hidden width multiplier (hidden = ffn_mult * d)
+    eps      RMSNorm epsilon
+    kv_norm  1 = RMSNorm on the KV latent, 0 = plain down-projection
+    dtype    storage type of activations and weights: "bf16" or "fp32"
+    """
+
+    d: int
+    heads: int
+    d_head: int
+    rank: int
+    d_ctx: int
+    n_q: int
+    keep: Tuple[int, ...]
+    d_out: int = 0
+    ffn_mult: int = 4
+    eps: float = 1e-6
+    kv_norm: int = 1
+    dtype: str = "bf16"
+
+    @property
+    def n_layers(self) -> int:
+        return len(self.keep)
+
+    @property
+    def d_ffn(self) -> int:
+        return self.ffn_mult * self.d
+
+
+@dataclass(frozen=True)
+class Workload:
+    """A seeded synthetic batch: dims, batch size, length law and value law.
+
+    lengths: ("uniform", lo, hi) inclusive, ("fixed", T) or
+             ("lognormal", mu, sigma, lo, hi) rounded then clipped.
+    semantic: add a semantic-content term N(0,1) @ W_sem (W_sem: 128 -> d,
+              entries N(0, 1/128)) to ID embeddings N(0,1).
+    """
+
+    name: str
+    dims: Dims
+    batch: int
+    lengths: tuple
+    seed: int
+    semantic: bool = False
+    sem_dim: int = 128
+    description: str = field(default="", compare=False)
+
+
+def _sweep(L: int) -> Workload:
+    return Workload(
+        name=f"sweep{L}",
+        dims=Dims(d=256, heads=4, d_head=64, rank=128, d_ctx=64, n_q=32,
+                  keep=(L, L // 2, L // 4, L // 8)),
+        batch=128, lengths=("fixed", L), seed=3, semantic=True,
+        description=f"sequence-length sweep at L={L}: B=128, d=256, 4 heads, r=128, "
+                    "4 layers halving, 32 candidates, c in R^64")
+
+
+WORKLOADS = {
+    "tiny": Workload(
+        name="tiny",
+        dims=Dims(d=64, heads=2, d_head=32, rank=32, d_ctx=16, n_q=4, keep=(64, 32),
+                  dtype="fp32"),
+        batch=4, lengths=("uniform", 16, 64), seed=0,
+        description="tiny fp32 case: B=4, T~U[16,64], d=64, 2 heads, r=32, 2 layers"),
+    "online": Workload(
+        name="online",
+        dims=Dims(d=256, heads=4, d_head=64, rank=128, d_ctx=64, n_q=64,
+                  keep=(400, 200, 100, 50)),
+        batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
+        description="online ranker: B=256, T~U[100,400], d=256, 4 heads, r=128, "
+                    "4 layers 400->200->100->50, 64 candidates, c in R^64"),
+    "upstream": Workload(
+        name="upstream",
+        dims=Dims(d=512, heads=8, d_head=64, rank=256, d_ctx=0, n_q=0,
+                  keep=(1600, 800, 400, 200, 100, 100, 100, 100), d_out=2048),
+        batch=64, lengths=("fixed", 1600), seed=2,
+        description="upstream user model: B=64, T=1600, d=512, 8 heads, r=256, "
+                    "8 layers, mean of final rows projected to 2048"),
+    "sweep200": _sweep(200),
+    "sweep400": _sweep(400),
+    "sweep800": _sweep(800),
+    "sweep1600": _sweep(1600),
+    "skewed": Workload(
+        name="skewed",
+        dims=Dims(d=256, heads=4, d_head=64, rank=128, d_ctx=64, n_q=256,
+                  keep=tuple(512 >> l for l in range(6))),
+        batch=512, lengths=("lognormal", 5.5, 0.8, 8, 1600), seed=4, semantic=True,
+        description="skewed jagged batch: B=512, T~lognormal(5.5,0.8) clipped to "
+                    "[8,1600], d=256, 4 heads, r=128, 6 layers keep 512>>l, 256 candidates"),
+}
+
+
+def workload(name: str) -> Workload:
+    try:
+        return WORKLOADS[name]
+    except KeyError:
+        raise KeyError(f"unknown workload {name!r}; known: {sorted(WORKLOADS)}") from None
