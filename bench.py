@@ -1,0 +1,360 @@
+"""Throughput benchmark of the LLaTTE sequence-module forward (user-seqs/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload online|upstream|sweepL|skewed]
+
+One step = one whole forward pass (plan, gather, every layer's KV latent,
+absorbed queries, latent attention, output projection + norm, FFN + norm,
+readout) over one batch of the workload, inputs resident in HBM.  L2 is
+flushed (a 256 MiB write) before every timed step, outside the timed events.
+Multi-GPU: one process per GPU, each rank runs its own batch (users are
+independent, no collective on the data path): weak scaling.  Rank 0 prints
+one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on
+the host cores, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import make_inputs, workload  # noqa: E402
+
+# ncu-measured DRAM traffic per launch (bytes) of the dominant kernel, keyed by
+# (kernel, workload); filled from the committed profiles/ summaries.  None =
+# not captured for the current kernel version.
+TRAFFIC = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"llatte_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "samples": len(rows),
+                "reasons": reasons}
+
+
+def gpu_identifier(local_rank: int) -> str:
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[local_rank] if vis else str(local_rank)
+
+
+def cpu_baseline_sample(inp, budget_s: float):
+    """Time the oracle on the first users until the budget is used."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    done = 0
+    while done < inp.batch and time.perf_counter() - t0 < budget_s:
+        oracle.forward(inp, users=[done])
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "user-seqs/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"first {done} of {inp.batch} users of one batch, fp64 NumPy oracle "
+                      f"(absorbed form), {dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    """Reference arm: the fp64 oracle on host cores, bounded sample per step."""
+    inp = make_inputs(wl)
+    budget = float(os.environ.get("LLATTE_REF_STEP_S", "3.0"))
+    for _ in range(args.warmup):
+        cpu_baseline_sample(inp, min(budget, 1.0))
+    vals, samples = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cb = cpu_baseline_sample(inp, budget)
+        vals.append(cb["value"])
+        samples.append(cb)
+    wall = time.perf_counter() - t0
+    value = float(np.mean(vals))
+    cb = dict(samples[-1])
+    cb["value"] = value
+    line = {
+        "impl": "reference", "metric": "user-seqs/s", "value": value, "unit": "user-seqs/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wall * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": wl.batch, "seq_len": wl.lengths,
+                   "parallelism": "host cores"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "user-seqs/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="online")
+    ap.add_argument("--second", default="upstream",
+                    help="second workload measured in the same run ('' = none)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = workload(args.workload)
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from latent_attention_jagged_b200 import Llatte, cost
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def measure(wl, steps, warmup, sample_clocks):
+        inp = make_inputs(wl, seed=wl.seed + 1000 * rank)
+        dt = torch.bfloat16 if inp.dims.dtype == "bf16" else torch.float32
+        h = Llatte(inp.dims, inp.layers, inp.W_e, max_batch=inp.batch,
+                   max_len=int(inp.lengths.max()))
+        values = torch.from_numpy(inp.values).cuda().to(dt)
+        offsets = torch.from_numpy(inp.offsets).cuda()
+        ctx = torch.from_numpy(inp.ctx).cuda().to(dt) if inp.dims.d_ctx else None
+        cand = torch.from_numpy(inp.cand).cuda().to(dt) if inp.dims.n_q else None
+        out = torch.empty(h.out_shape(inp.batch), dtype=torch.float32, device="cuda")
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            h.forward(values, offsets, ctx, cand, out=out)
+        torch.cuda.synchronize()
+        assert h.status() == 0, "device status word set during warm-up"
+
+        # ---- device-resident timing
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        sampler = ClockSampler(gpu_identifier(local)) if sample_clocks else None
+        if sampler:
+            sampler.start()
+        barrier()
+        torch.cuda.synchronize()
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            h.forward(values, offsets, ctx, cand, out=out)
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        clocks = sampler.stop() if sampler else None
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        ms = max_over_ranks(ms)
+        users = world * inp.batch * steps
+        value = users / (ms / 1e3)
+
+        # ---- per-step timing (same loop, profiling events inside the library)
+        h.profile_reset()
+        h.set_profiling(True)
+        prof_steps = max(3, min(steps, 50))
+        for _ in range(prof_steps):
+            flush.fill_(1)
+            h.forward(values, offsets, ctx, cand, out=out)
+        torch.cuda.synchronize()
+        prof = h.profile()
+        h.set_profiling(False)
+        launches_per_fwd = sum(v["launches"] for v in prof.values()) / prof_steps
+
+        # ---- end to end: pinned host inputs -> device -> forward -> host output
+        hv = torch.from_numpy(inp.values).to(dt).pin_memory()
+        ho = torch.from_numpy(inp.offsets).pin_memory()
+        hc = torch.from_numpy(inp.ctx).to(dt).pin_memory() if inp.dims.d_ctx else None
+        hq = torch.from_numpy(inp.cand).to(dt).pin_memory() if inp.dims.n_q else None
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        e2e_steps = max(3, min(steps, 50))
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(e2e_steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for a, b in ev2:
+            flush.fill_(1)
+            a.record(stream)
+            values.copy_(hv, non_blocking=True)
+            offsets.copy_(ho, non_blocking=True)
+            if hc is not None:
+                ctx.copy_(hc, non_blocking=True)
+            if hq is not None:
+                cand.copy_(hq, non_blocking=True)
+            h.forward(values, offsets, ctx, cand, out=out)
+            hout.copy_(out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2))
+        h2d = hv.numel() * hv.element_size() + ho.numel() * 8 + \
+            (hc.numel() * hc.element_size() if hc is not None else 0) + \
+            (hq.numel() * hq.element_size() if hq is not None else 0)
+        e2e = {"value": world * inp.batch * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4)}
+        assert h.status() == 0
+
+        # ---- roofline of the dominant step (largest device time)
+        flops = cost.flops_by_step(inp.lengths, inp.dims)
+        dom = max((k for k in prof if k in flops), key=lambda k: prof[k]["ms"])
+        dom_ms = prof[dom]["ms"] / max(1, prof[dom]["calls"])       # per launch of the step
+        per_launch_flops = flops[dom] / (prof[dom]["calls"] / prof_steps)
+        achieved = per_launch_flops / (dom_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peaks['source']} sustained bf16 (cuBLAS loop)",
+                "traffic": TRAFFIC.get((dom, wl.name)),
+                "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms}
+        total_flops = cost.total_flops(inp.lengths, inp.dims)
+        step_ms = ms / steps
+        whole = {"achieved_tflops": total_flops / (step_ms / 1e3) / 1e12,
+                 "frac_of_peak": total_flops / (step_ms / 1e3) / 1e12 / peak,
+                 "flops_per_step": total_flops}
+        steps_ms = {k: round(v["ms"] / prof_steps, 4) for k, v in prof.items() if v["calls"]}
+        res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
+                   clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
+                   dtype=inp.dims.dtype)
+        h.close()
+        return res
+
+    main_res = measure(wl, args.steps, args.warmup, sample_clocks=(rank == 0))
+    second = None
+    if args.second and args.second != args.workload:
+        wl2 = workload(args.second)
+        s_steps = max(5, min(args.steps, 40))
+        r2 = measure(wl2, s_steps, args.warmup, sample_clocks=False)
+        second = {"workload": wl2.name, "value": r2["value"], "unit": "user-seqs/s",
+                  "ms_per_step": r2["ms"], "steps": s_steps, "roofline": r2["roofline"],
+                  "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(main_res["inp"], args.cpu_budget)
+
+    if rank == 0:
+        inp = main_res["inp"]
+        line = {
+            "metric": "user-seqs/s", "value": main_res["value"], "unit": "user-seqs/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": main_res["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": main_res["dtype"], "data": "synthetic",
+            "config": {"workload": wl.name, "global_batch": inp.batch * world,
+                       "seq_len": list(wl.lengths), "d": inp.dims.d, "layers": inp.dims.n_layers,
+                       "parallelism": f"users sharded, dp{world}",
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "roofline": main_res["roofline"],
+            "whole_step": main_res["whole"],
+            "cpu_baseline": cpu,
+            "e2e": main_res["e2e"],
+            "gpu_launches": int(round(main_res["launches"] * args.steps)),
+            "clocks": main_res["clocks"],
+            "steps_ms": main_res["steps_ms"],
+            "second": second,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * llatte.h - C ABI of the B200 (sm_100a) LLaTTE sequence-module forward pass.
+ *
+ * What it computes (LLaTTE notes, huaxiaozhuan.com, appendix A.2 "Sequence
+ * Module" and A.3 "Multi-head Latent Attention"; target-aware query from the
+ * daiwk.github.io notes, "core formula"):
+ *
+ *   per user u: history tokens x_1..x_T (earliest first), n_q query tokens
+ *   (candidates), a context vector c.  Fused input = [history ; query tokens].
+ *   For each layer l with keep_l:
+ *     n      = min(T, keep_l)                  kept history rows
+ *     R      = [last n history rows ; query tokens]        (query rows)
+ *     c_kv   = RMSNorm_{g_kv}(H W_dkv^T)       latent K = V, rank r, all T rows
+ *     per head j:  q~ = (W_uk,j^T W_q,j) [R_i ; c] / sqrt(d_h)
+ *                  a  = softmax over visible keys t of q~ . c_kv,t
+ *                  o~ = sum_t a_t c_kv,t
+ *     A      = sum_j (W_o,j W_uv,j) o~_j
+ *     Z      = RMSNorm_{g1}(R + A)
+ *     X      = RMSNorm_{g2}(Z + W2 SiLU(W1 Z))
+ *     history <- X[:n], query tokens <- X[n:], T <- n
+ *   Visibility: a history query at position p sees keys t <= p; a query token
+ *   sees every current history key and no query token; no key -> zero output.
+ *   Output: the final query-token rows, or, with d_out > 0, W_e times the mean
+ *   of the final layer's rows.
+ *
+ * Conventions
+ *   - All matrices are row-major [out, in] as on the pages.
+ *   - dtype LLATTE_BF16: activations/weights in bfloat16, fp32 accumulation,
+ *     fp32 softmax and RMSNorm statistics.  LLATTE_FP32: everything fp32 on
+ *     CUDA cores (no tensor-core tf32).
+ *   - Every call returns LLATTE_OK (0) or a negative LLATTE_ERR_* code; bad
+ *     arguments are rejected on the host before anything is launched.
+ *   - Faults that only the device can see (offsets not monotone, a user
+ *     longer than max_len, a batch larger than max_total, a bounded wait that
+ *     ran out) set bits in a device status word instead of trapping; the
+ *     forward then does no further work and `out` is unspecified.
+ *     llatte_get_status reads and clears that word.
+ */
+#ifndef LLATTE_H
+#define LLATTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LLATTE_MAX_LAYERS 16
+
+enum {
+  LLATTE_OK = 0,
+  LLATTE_ERR_ARG = -1,          /* null pointer, bad size or bad schedule      */
+  LLATTE_ERR_UNSUPPORTED = -2,  /* dims outside what the kernels implement     */
+  LLATTE_ERR_CUDA = -3,         /* a CUDA runtime call failed                  */
+  LLATTE_ERR_OOM = -4,          /* device allocation failed                    */
+  LLATTE_ERR_DEVICE = -5        /* device status word is non-zero              */
+};
+
+enum { LLATTE_BF16 = 0, LLATTE_FP32 = 1 };
+
+/* Bits of the device status word. */
+enum {
+  LLATTE_DEV_BAD_OFFSETS = 1,   /* offsets decrease or are negative            */
+  LLATTE_DEV_TOO_LONG = 2,      /* a history longer than max_len               */
+  LLATTE_DEV_TOO_MANY_ROWS = 4, /* sum of lengths above max_total              */
+  LLATTE_DEV_TIMEOUT = 8        /* a bounded device wait gave up               */
+};
+
+/*
+ * Model dimensions (sizes and pyramid schedule).
+ *   d, heads, d_head      token width, heads h, head width d_h (scale 1/sqrt(d_h))
+ *   rank                  MLA latent rank r
+ *   d_ctx                 context width (0 = no context)
+ *   n_q                   query tokens per user (0 allowed)
+ *   n_layers, keep[]      layers and, per layer, the number of most recent
+ *                         HISTORY rows kept (non-increasing; 0 = cross mode)
+ *   d_out                 readout width (0 = output the final query-token rows)
+ *   ffn_mult              FFN hidden = ffn_mult * d
+ *   dtype                 LLATTE_BF16 or LLATTE_FP32
+ *   kv_norm               1 = RMSNorm on the KV latent (the pages' form), 0 = none
+ *   eps                   RMSNorm epsilon
+ *   max_batch             largest B a forward may pass
+ *   max_len               longest history a user may have
+ *   max_total             largest sum of lengths in one batch (0 = max_batch*max_len)
+ */
+typedef struct {
+  int32_t d, heads, d_head, rank, d_ctx, n_q, n_layers;
+  int32_t keep[LLATTE_MAX_LAYERS];
+  int32_t d_out, ffn_mult, dtype, kv_norm;
+  float eps;
+  int32_t max_batch;
+  int64_t max_len;
+  int64_t max_total;
+} llatte_dims;
+
+/*
+ * Weights of one layer, non-absorbed, in `dtype` (row-major [out, in]):
+ *   W_dkv [r, d]        KV down-projection         g_kv [r]   latent RMSNorm gain
+ *   W_q   [h*d_h, d+d_ctx]  query projection of [x ; c]
+ *   W_uk  [h*d_h, r]    K up-projection            W_uv [h*d_h, r] V up-projection
+ *   W_o   [d, h*d_h]    output projection          g1 [d]     post-attention gain
+ *   W1    [ffn_mult*d, d]   W2 [d, ffn_mult*d]     g2 [d]     post-FFN gain
+ */
+typedef struct {
+  const void *W_dkv, *g_kv, *W_q, *W_uk, *W_uv, *W_o, *g1, *W1, *W2, *g2;
+} llatte_layer_w;
+
+typedef struct llatte_handle llatte_handle;
+
+/*
+ * Create a handle on the current CUDA device.  The weights (host memory if
+ * weights_on_device == 0, device memory otherwise) are copied; the caller may
+ * free them afterwards.  The absorbed matrices W_uk^T W_q / sqrt(d_h) and
+ * W_o W_uv are formed on the device in fp32 and stored in `dtype`.  W_e is
+ * [d_out, d] (ignored when d_out == 0).  The handle owns a workspace sized
+ * from max_batch / max_total; llatte_workspace_bytes reports its size.
+ * Synchronous.
+ */
+int llatte_create(llatte_handle** handle, const llatte_dims* dims,
+                  const llatte_layer_w* layers, const void* W_e, int weights_on_device);
+
+/*
+ * One forward pass, asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream), with no host synchronisation.
+ *   values  device [offsets[B] rows, d] in dtype: all users' histories, user u
+ *           in rows offsets[u] .. offsets[u+1]-1, earliest event first;
+ *           16-byte aligned (as are cand and context)
+ *   offsets device int64 [B+1], non-decreasing, offsets[0] >= 0
+ *   B       number of users, 0 <= B <= max_batch (B = 0 launches nothing)
+ *   context device [B, d_ctx] in dtype (may be NULL when d_ctx == 0)
+ *   cand    device [B, n_q, d] in dtype (may be NULL when n_q == 0)
+ *   out     device fp32 [B, n_q, d] (d_out == 0) or [B, d_out]
+ * Inputs are only read; `out` is the only caller memory written.  Calls on
+ * one handle must not overlap in time (they share its workspace).
+ */
+int llatte_forward(llatte_handle* handle, const void* values, const int64_t* offsets,
+                   int32_t B, const void* context, const void* cand, float* out,
+                   void* stream);
+
+/*
+ * Copy the pyramid plan of the most recent forward (for bit-exact checks):
+ * for every layer l = 0..n_layers-1 the history-row offsets then the
+ * query-row offsets, dst = device int64 [n_layers][2][B+1] with B the last
+ * forward's batch.  History rows of layer l: T_{l,u} = hist[u+1]-hist[u];
+ * query rows: n_{l,u} + n_q = query[u+1]-query[u].  Asynchronous on stream.
+ */
+int llatte_plan_export(llatte_handle* handle, int64_t* dst, void* stream);
+
+/*
+ * Synchronise the device, read the status word into *device_status (0 = no
+ * fault) and clear it.  Returns LLATTE_ERR_DEVICE when it was non-zero.
+ */
+int llatte_get_status(llatte_handle* handle, int32_t* device_status);
+
+/* Bytes of device workspace a handle with these dims allocates (0 on bad dims). */
+size_t llatte_workspace_bytes(const llatte_dims* dims);
+
+/* Human-readable name of an LLATTE_* return code. */
+const char* llatte_error_string(int code);
+
+/*
+ * Per-step device timing, a profiling aid.  With profiling enabled every
+ * forward records a CUDA event pair on its stream around each step (plan,
+ * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout); llatte_profile_step
+ * synchronises on the recorded events and returns, for step index `step`
+ * (0 .. 9), its name, the accumulated milliseconds, the number of kernels the
+ * step launched and the number of times it ran since the last reset.
+ * Returns LLATTE_ERR_ARG for a step index out of range.
+ */
+int llatte_set_profiling(llatte_handle* handle, int enable);
+int llatte_profile_reset(llatte_handle* handle);
+int llatte_profile_step(llatte_handle* handle, int step, const char** name, double* total_ms,
+                        int64_t* kernel_launches, int64_t* calls);
+
+/* Free the handle and everything it owns (synchronises its device). */
+void llatte_destroy(llatte_handle* handle);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLATTE_H */

@@ -1,0 +1,246 @@
+"""ctypes binding of libllatte.so: the same entry points as include/llatte.h,
+with argument marshalling from torch tensors (device memory and streams only;
+every step of the forward runs in the library's kernels).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libllatte.so")
+MAX_LAYERS = 16
+STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout")
+
+LLATTE_OK, LLATTE_ERR_ARG, LLATTE_ERR_UNSUPPORTED, LLATTE_ERR_CUDA, LLATTE_ERR_OOM, \
+    LLATTE_ERR_DEVICE = 0, -1, -2, -3, -4, -5
+LLATTE_BF16, LLATTE_FP32 = 0, 1
+DEV_BAD_OFFSETS, DEV_TOO_LONG, DEV_TOO_MANY_ROWS, DEV_TIMEOUT = 1, 2, 4, 8
+
+
+class LlatteError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {error_string(code)} ({code})")
+
+
+class llatte_dims(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
+                ("rank", ctypes.c_int32), ("d_ctx", ctypes.c_int32), ("n_q", ctypes.c_int32),
+                ("n_layers", ctypes.c_int32), ("keep", ctypes.c_int32 * MAX_LAYERS),
+                ("d_out", ctypes.c_int32), ("ffn_mult", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("kv_norm", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("max_batch", ctypes.c_int32), ("max_len", ctypes.c_int64),
+                ("max_total", ctypes.c_int64)]
+
+
+LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2")
+
+
+class llatte_layer_w(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in LAYER_KEYS]
+
+
+EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
+           "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
+           "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step")
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Open libllatte.so (raises if it has not been built: there is no fallback)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with "
+                           "`python -m latent_attention_jagged_b200.build`")
+    lib = ctypes.CDLL(p)
+    P, I32, I64, VP = ctypes.POINTER, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
+    lib.llatte_create.argtypes = [P(VP), P(llatte_dims), P(llatte_layer_w), VP, ctypes.c_int]
+    lib.llatte_create.restype = ctypes.c_int
+    lib.llatte_forward.argtypes = [VP, VP, VP, I32, VP, VP, VP, VP]
+    lib.llatte_forward.restype = ctypes.c_int
+    lib.llatte_plan_export.argtypes = [VP, VP, VP]
+    lib.llatte_plan_export.restype = ctypes.c_int
+    lib.llatte_get_status.argtypes = [VP, P(I32)]
+    lib.llatte_get_status.restype = ctypes.c_int
+    lib.llatte_workspace_bytes.argtypes = [P(llatte_dims)]
+    lib.llatte_workspace_bytes.restype = ctypes.c_size_t
+    lib.llatte_error_string.argtypes = [ctypes.c_int]
+    lib.llatte_error_string.restype = ctypes.c_char_p
+    lib.llatte_destroy.argtypes = [VP]
+    lib.llatte_destroy.restype = None
+    lib.llatte_set_profiling.argtypes = [VP, ctypes.c_int]
+    lib.llatte_set_profiling.restype = ctypes.c_int
+    lib.llatte_profile_reset.argtypes = [VP]
+    lib.llatte_profile_reset.restype = ctypes.c_int
+    lib.llatte_profile_step.argtypes = [VP, ctypes.c_int, P(ctypes.c_char_p),
+                                        P(ctypes.c_double), P(I64), P(I64)]
+    lib.llatte_profile_step.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def error_string(code: int) -> str:
+    try:
+        return load_library().llatte_error_string(code).decode()
+    except Exception:
+        return "unknown"
+
+
+def make_dims(dims, max_batch: int, max_len: int, max_total: int = 0) -> llatte_dims:
+    """Fill the C struct from any object with the Dims attributes."""
+    if len(dims.keep) > MAX_LAYERS:
+        raise ValueError(f"at most {MAX_LAYERS} layers")
+    c = llatte_dims()
+    c.d, c.heads, c.d_head, c.rank = dims.d, dims.heads, dims.d_head, dims.rank
+    c.d_ctx, c.n_q, c.n_layers = dims.d_ctx, dims.n_q, len(dims.keep)
+    for i, k in enumerate(dims.keep):
+        c.keep[i] = int(k)
+    c.d_out, c.ffn_mult = dims.d_out, dims.ffn_mult
+    c.dtype = {"bf16": LLATTE_BF16, "fp32": LLATTE_FP32}[dims.dtype]
+    c.kv_norm, c.eps = dims.kv_norm, float(dims.eps)
+    c.max_batch, c.max_len, c.max_total = int(max_batch), int(max_len), int(max_total)
+    return c
+
+
+def torch_dtype(dims) -> torch.dtype:
+    return {"bf16": torch.bfloat16, "fp32": torch.float32}[dims.dtype]
+
+
+def _host(a, dt: torch.dtype) -> torch.Tensor:
+    t = a if isinstance(a, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(a))
+    return t.detach().to(device="cpu", dtype=dt).contiguous()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+class Llatte:
+    """A forward handle: weights (non-absorbed, pages' layout) are copied and
+    absorbed at construction; `forward` runs the whole sequence module."""
+
+    def __init__(self, dims, layers: Sequence[dict], W_e=None, max_batch: int = 1,
+                 max_len: int = 0, max_total: int = 0, lib_path: Optional[str] = None):
+        self.lib = load_library(lib_path)
+        self.dims = dims
+        self.cdims = make_dims(dims, max_batch, max_len, max_total)
+        self.dt = torch_dtype(dims)
+        if len(layers) != len(dims.keep):
+            raise ValueError("one weight dict per layer is required")
+        keep_alive = []
+        arr = (llatte_layer_w * len(layers))()
+        for i, w in enumerate(layers):
+            for k in LAYER_KEYS:
+                t = _host(w[k], self.dt)
+                keep_alive.append(t)
+                setattr(arr[i], k, t.data_ptr())
+        we = None
+        if dims.d_out:
+            we = _host(W_e, self.dt)
+            keep_alive.append(we)
+        h = ctypes.c_void_p()
+        rc = self.lib.llatte_create(ctypes.byref(h), ctypes.byref(self.cdims), arr,
+                                    _ptr(we), 0)
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_create")
+        self.h = h
+        self.last_B = 0
+
+    def workspace_bytes(self) -> int:
+        return int(self.lib.llatte_workspace_bytes(ctypes.byref(self.cdims)))
+
+    def out_shape(self, B: int):
+        d = self.dims
+        return (B, d.d_out) if d.d_out else (B, d.n_q, d.d)
+
+    def forward(self, values: torch.Tensor, offsets: torch.Tensor, context=None, cand=None,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        d = self.dims
+        B = int(offsets.numel()) - 1
+        if B < 0:
+            raise ValueError("offsets needs B+1 entries")
+        for name, t, dt in (("values", values, self.dt), ("offsets", offsets, torch.int64),
+                            ("context", context, self.dt), ("cand", cand, self.dt)):
+            if t is None:
+                continue
+            if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+        if values.dim() != 2 or values.shape[1] != d.d:
+            raise ValueError(f"values must be [rows, {d.d}]")
+        if d.d_ctx and (context is None or tuple(context.shape) != (B, d.d_ctx)):
+            raise ValueError(f"context must be [{B}, {d.d_ctx}]")
+        if d.n_q and (cand is None or tuple(cand.shape) != (B, d.n_q, d.d)):
+            raise ValueError(f"cand must be [{B}, {d.n_q}, {d.d}]")
+        if out is None:
+            out = torch.empty(self.out_shape(B), dtype=torch.float32, device=values.device)
+        elif (tuple(out.shape) != self.out_shape(B) or out.dtype != torch.float32
+              or not out.is_contiguous()):
+            raise ValueError(f"out must be a contiguous float32 {self.out_shape(B)} tensor")
+        rc = self.lib.llatte_forward(self.h, _ptr(values), _ptr(offsets), B, _ptr(context),
+                                     _ptr(cand), _ptr(out), _stream_ptr(stream))
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_forward")
+        self.last_B = B
+        return out
+
+    def plan_export(self, stream=None) -> torch.Tensor:
+        L, B = len(self.dims.keep), self.last_B
+        dst = torch.empty((L, 2, B + 1), dtype=torch.int64, device="cuda")
+        rc = self.lib.llatte_plan_export(self.h, _ptr(dst), _stream_ptr(stream))
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_plan_export")
+        return dst
+
+    def status(self) -> int:
+        v = ctypes.c_int32(0)
+        rc = self.lib.llatte_get_status(self.h, ctypes.byref(v))
+        if rc not in (LLATTE_OK, LLATTE_ERR_DEVICE):
+            raise LlatteError(rc, "llatte_get_status")
+        return int(v.value)
+
+    def set_profiling(self, on: bool = True):
+        self.lib.llatte_set_profiling(self.h, 1 if on else 0)
+
+    def profile_reset(self):
+        self.lib.llatte_profile_reset(self.h)
+
+    def profile(self) -> dict:
+        res = {}
+        for i in range(len(STEPS)):
+            name = ctypes.c_char_p()
+            ms = ctypes.c_double()
+            nl = ctypes.c_int64()
+            nc = ctypes.c_int64()
+            rc = self.lib.llatte_profile_step(self.h, i, ctypes.byref(name), ctypes.byref(ms),
+                                              ctypes.byref(nl), ctypes.byref(nc))
+            if rc != LLATTE_OK:
+                raise LlatteError(rc, "llatte_profile_step")
+            res[name.value.decode()] = {"ms": ms.value, "launches": nl.value, "calls": nc.value}
+        return res
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.llatte_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

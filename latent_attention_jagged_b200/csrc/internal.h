@@ -1,0 +1,144 @@
+// Internal structures of the LLaTTE forward library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/llatte.h"
+
+namespace llatte {
+
+// Step kinds, for the optional per-step timing.
+enum Step { ST_PLAN = 0, ST_GATHER, ST_CTX, ST_KV, ST_Q, ST_ATTN, ST_O, ST_FFN1, ST_FFN2,
+            ST_READOUT, ST_COUNT };
+extern const char* const kStepNames[ST_COUNT];
+
+// Device-side pyramid plan.  Layer index l runs over 0..L where l = L is the
+// virtual layer holding the final rows (its keep is unbounded).
+struct PlanDev {
+  int64_t* hist_off;   // [(L+1) * (max_batch+1)]  exclusive scan of T_{l,u}
+  int64_t* query_off;  // [(L+1) * (max_batch+1)]  exclusive scan of n_{l,u} + n_q
+  int32_t* T;          // [(L+1) * max_batch]
+  int32_t* n;          // [(L+1) * max_batch]
+  int64_t* totals;     // [(L+1) * 2]: sum T_l, sum (n_l + n_q)
+  int32_t* status;     // device status word
+  int32_t* work;       // attention work items, [(L) * max_work] (tensor-core path)
+  int32_t* work_count; // [L]
+  int32_t* work_next;  // [L] dynamic scheduling counters
+  int64_t stride;      // max_batch + 1
+  int32_t max_work;
+
+  __host__ __device__ const int64_t* hoff(int l) const { return hist_off + l * stride; }
+  __host__ __device__ const int64_t* qoff(int l) const { return query_off + l * stride; }
+  __host__ __device__ const int32_t* Tl(int l) const { return T + l * (stride - 1); }
+  __host__ __device__ const int32_t* nl(int l) const { return n + l * (stride - 1); }
+  __host__ __device__ const int64_t* hist_total(int l) const { return totals + 2 * l; }
+  __host__ __device__ const int64_t* query_total(int l) const { return totals + 2 * l + 1; }
+};
+
+struct LayerDev {
+  void* W_dkv;     // [r, d]
+  void* g_kv;      // [r]
+  void* W_qk;      // [h*r, d]   absorbed W_uk^T W_q (x columns), scaled 1/sqrt(d_h)
+  float* W_qkc;    // [h*r, d_ctx] fp32 absorbed context columns (NULL if d_ctx == 0)
+  void* W_ov;      // [d, h*r]   absorbed W_o W_uv
+  void* g1;        // [d]
+  void* W1;        // [f, d]
+  void* W2;        // [d, f]
+  void* g2;        // [d]
+};
+
+struct ProfRec { int step; cudaEvent_t a, b; int launches; };
+
+}  // namespace llatte
+
+struct llatte_handle {
+  llatte_dims dims;
+  int device;
+  int elem;                       // bytes per stored element
+  int use_tc;                     // tensor-core (tcgen05) path for bf16
+  int num_sms;
+  llatte::LayerDev layers[LLATTE_MAX_LAYERS];
+  void* W_e;                      // [d_out, d]
+  std::vector<void*> allocs;
+
+  // workspace
+  llatte::PlanDev plan;
+  int64_t max_rows_h, max_rows_q;
+  void* Xh[2];
+  void* Xq[2];
+  void* C;
+  void* Qt;
+  void* Ot;
+  void* Z;
+  void* Hd;
+  float* acc32;        // fp32 pre-norm rows (CUDA-core path)
+  float* ctxbias;      // [max_batch, h*r]
+  float* final_rows;   // [max_rows_q, d] fp32 (readout only)
+  float* mean_rows;    // [max_batch, d] fp32
+  size_t ws_bytes;
+  int last_B;
+
+  // profiling
+  int profiling;
+  std::vector<llatte::ProfRec> pending;
+  std::vector<cudaEvent_t> event_pool;
+  double step_ms[llatte::ST_COUNT];
+  int64_t step_launches[llatte::ST_COUNT];
+  int64_t step_calls[llatte::ST_COUNT];
+};
+
+namespace llatte {
+
+// ---- launchers (each returns cudaGetLastError()) ----
+cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, cudaStream_t s);
+cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
+                          const void* cand, int B, cudaStream_t s);
+
+// CUDA-core path
+struct GemmArgs {
+  const void* A; int64_t lda;        // [M, K]
+  const void* W;                     // [N, K] row-major
+  void* D; int64_t ldd;              // [M, N]
+  int64_t M_host; const int64_t* M_dev;  // M from device when M_dev != NULL
+  int64_t M_max;                     // grid bound
+  int N, K;
+  int epi;                           // EPI_*
+  const float* bias; const int64_t* seg_off; int B;  // EPI_USERBIAS
+};
+enum { EPI_STORE = 0, EPI_USERBIAS, EPI_SILU, EPI_F32 };
+cudaError_t launch_gemm_simt(int elem_a, int elem_w, int elem_d, const GemmArgs& g, cudaStream_t s);
+
+struct NormArgs {
+  const float* acc; int N;           // [M, N] fp32 rows
+  const void* resid;                 // [M, N] storage type or NULL
+  const void* g; float eps;
+  const int64_t* M_dev; int64_t M_max;
+  int mode;                          // NORM_PLAIN / NORM_SCATTER
+  void* dst;                         // NORM_PLAIN: [M, N]
+  // NORM_SCATTER (FFN2 output of layer l -> inputs of layer l+1 / outputs)
+  const int64_t *qoff_l, *hoff_n, *qoff_n; const int32_t *n_l, *n_n; int B; int n_q;
+  void* Xh_n; void* Xq_n; int last; float* out; float* final_rows;
+};
+enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
+cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+  const void* Qt;                    // [sum q, h*r]
+  const void* C;                     // [sum T, r]
+  void* Ot;                          // [sum q, h*r]
+  const int64_t *qoff, *hoff; const int32_t *T, *n;
+  const int64_t* Mq_dev; int64_t Mq_max;
+  int B, heads, r;
+};
+cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
+
+cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
+                             cudaStream_t s);
+cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
+                          const void* W_o, int d, int d_ctx, int heads, int d_head, int r,
+                          void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s);
+
+}  // namespace llatte

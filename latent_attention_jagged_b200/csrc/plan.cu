@@ -1,0 +1,176 @@
+// Pyramid plan and jagged gather.
+//
+// Plan (LLaTTE notes, huaxiaozhuan.com, appendix A.2 "Transformer Layers and
+// Pyramidal Schedule"): per user u and layer l, T_{0,u} = offsets[u+1] -
+// offsets[u]; n_{l,u} = min(T_{l,u}, keep_l); T_{l+1,u} = n_{l,u}.  History
+// (key) rows of layer l are packed per user in hist_off_l = exscan(T_l); its
+// query rows (the last n_l history rows, then the n_q query tokens, i.e. the
+// pages' tail slice of the fused sequence) in query_off_l = exscan(n_l + n_q).
+// The layer after the last one is a virtual layer L whose keep is unbounded:
+// its query rows are the final rows.  One CTA computes all layers; the
+// offsets are validated first and a bad batch turns every count to zero (no
+// later kernel then does any work) and sets the device status word.
+//
+// Gather (appendix A.2 step 2, X_input = Concat(X_seq, Q)): layer 0's
+// history rows are a straight copy of `values`; its query rows are the last
+// n_0 history rows of each user followed by the user's query tokens.  One
+// warp per row, 16-byte vector loads/stores.
+#include "common.cuh"
+#include "internal.h"
+
+namespace llatte {
+
+struct KeepArr { int32_t k[LLATTE_MAX_LAYERS + 1]; };
+
+constexpr int kPlanThreads = 1024;
+
+// Block-wide exclusive scan of two int64 values (one per thread).
+__device__ void block_exscan2(int64_t a, int64_t b, int64_t* out_a, int64_t* out_b,
+                              int64_t* tot_a, int64_t* tot_b) {
+  __shared__ int64_t wa[32], wb[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int64_t ta = __shfl_up_sync(0xffffffffu, ia, o);
+    int64_t tb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) { ia += ta; ib += tb; }
+  }
+  if (lane == 31) { wa[warp] = ia; wb[warp] = ib; }
+  __syncthreads();
+  if (warp == 0) {
+    int64_t xa = wa[lane], xb = wb[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int64_t ta = __shfl_up_sync(0xffffffffu, xa, o);
+      int64_t tb = __shfl_up_sync(0xffffffffu, xb, o);
+      if (lane >= o) { xa += ta; xb += tb; }
+    }
+    wa[lane] = xa; wb[lane] = xb;
+  }
+  __syncthreads();
+  int64_t pa = warp ? wa[warp - 1] : 0, pb = warp ? wb[warp - 1] : 0;
+  *out_a = pa + ia - a;
+  *out_b = pb + ib - b;
+  *tot_a = wa[31];
+  *tot_b = wb[31];
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep, int L, int n_q,
+            int64_t max_len, int64_t max_total) {
+  __shared__ int s_err;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_err = 0;
+  __syncthreads();
+  int err = 0;
+  for (int u = tid; u < B; u += kPlanThreads) {
+    int64_t a = offsets[u], b = offsets[u + 1];
+    if (a < 0 || b < a) err |= LLATTE_DEV_BAD_OFFSETS;
+    else if (b - a > max_len) err |= LLATTE_DEV_TOO_LONG;
+  }
+  if (err) atomicOr(&s_err, err);
+  __syncthreads();
+  if (tid == 0 && s_err == 0 && offsets[B] - offsets[0] > max_total)
+    s_err |= LLATTE_DEV_TOO_MANY_ROWS;
+  __syncthreads();
+  if (s_err) {
+    if (tid == 0) atomicOr(p.status, s_err);
+    for (int i = tid; i < 2 * (L + 1); i += kPlanThreads) p.totals[i] = 0;
+    for (int i = tid; i < L; i += kPlanThreads) p.work_count[i] = 0;
+    for (int64_t i = tid; i < (int64_t)(L + 1) * p.stride; i += kPlanThreads) {
+      p.hist_off[i] = 0;
+      p.query_off[i] = 0;
+    }
+    return;
+  }
+  const int chunk = (B + kPlanThreads - 1) / kPlanThreads;
+  const int u0 = min(B, tid * chunk), u1 = min(B, u0 + chunk);
+  const int64_t bstride = p.stride - 1;
+  for (int l = 0; l <= L; ++l) {
+    int32_t* Tl = p.T + l * bstride;
+    int32_t* nl = p.n + l * bstride;
+    const int32_t* nprev = p.n + (l - 1) * bstride;
+    int64_t sT = 0, sQ = 0;
+    for (int u = u0; u < u1; ++u) {
+      int32_t t = (l == 0) ? (int32_t)(offsets[u + 1] - offsets[u]) : nprev[u];
+      int32_t nn = (l == L) ? t : min(t, keep.k[l]);
+      Tl[u] = t;
+      nl[u] = nn;
+      sT += t;
+      sQ += nn + n_q;
+    }
+    int64_t bT, bQ, totT, totQ;
+    block_exscan2(sT, sQ, &bT, &bQ, &totT, &totQ);
+    int64_t* ho = p.hist_off + l * p.stride;
+    int64_t* qo = p.query_off + l * p.stride;
+    for (int u = u0; u < u1; ++u) {
+      ho[u] = bT;
+      qo[u] = bQ;
+      bT += Tl[u];
+      bQ += nl[u] + n_q;
+    }
+    if (tid == 0) {
+      ho[B] = totT;
+      qo[B] = totQ;
+      p.totals[2 * l] = totT;
+      p.totals[2 * l + 1] = totQ;
+    }
+  }
+}
+
+cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, cudaStream_t s) {
+  KeepArr k;
+  const int L = h->dims.n_layers;
+  for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < L ? h->dims.keep[i] : 0;
+  plan_kernel<<<1, kPlanThreads, 0, s>>>(offsets, B, h->plan, k, L, h->dims.n_q, h->dims.max_len,
+                                          h->max_rows_h);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- gather
+
+__global__ void __launch_bounds__(256)
+gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offsets,
+              const uint4* __restrict__ cand, int B, PlanDev p, uint4* __restrict__ Xh,
+              uint4* __restrict__ Xq, int row_vecs, int n_q) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nh = *p.hist_total(0), nq = *p.query_total(0);
+  const int64_t base = nh ? offsets[0] : 0;
+  for (int64_t row = w0; row < nh + nq; row += warps) {
+    const uint4* src;
+    uint4* dst;
+    if (row < nh) {
+      src = values + (base + row) * row_vecs;
+      dst = Xh + row * row_vecs;
+    } else {
+      const int64_t m = row - nh;
+      const int64_t* qo = p.qoff(0);
+      const int u = segment_of(qo, B, m);
+      const int64_t j = m - qo[u];
+      const int32_t n = p.nl(0)[u];
+      if (j < n) {
+        const int64_t T = p.Tl(0)[u];
+        src = values + (offsets[u] + T - n + j) * row_vecs;
+      } else {
+        src = cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
+      }
+      dst = Xq + m * row_vecs;
+    }
+    for (int v = lane; v < row_vecs; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
+                          const void* cand, int B, cudaStream_t s) {
+  const int row_vecs = h->dims.d * h->elem / 16;
+  gather_kernel<<<h->num_sms * 4, 256, 0, s>>>(
+      (const uint4*)values, offsets, (const uint4*)cand, B, h->plan, (uint4*)h->Xh[0],
+      (uint4*)h->Xq[0], row_vecs, h->dims.n_q);
+  return cudaGetLastError();
+}
+
+}  // namespace llatte

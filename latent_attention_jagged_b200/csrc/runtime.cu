@@ -1,0 +1,466 @@
+// Host runtime of the LLaTTE forward library: argument checks, weight
+// absorption, workspace, the per-layer launch sequence and per-step timing.
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+
+#include "internal.h"
+
+using namespace llatte;
+
+namespace llatte {
+const char* const kStepNames[ST_COUNT] = {"plan", "gather", "ctx_bias", "kv", "q",
+                                          "attn", "o",      "ffn1",     "ffn2", "readout"};
+}
+
+namespace {
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  int64_t rows_h, rows_q;
+  size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
+      off_work_count, off_work_next;
+  size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
+      off_final, off_mean;
+  size_t total;
+  int32_t max_work;
+};
+
+int check_dims(const llatte_dims* d) {
+  if (!d) return LLATTE_ERR_ARG;
+  if (d->n_layers < 1 || d->n_layers > LLATTE_MAX_LAYERS) return LLATTE_ERR_ARG;
+  if (d->d <= 0 || d->heads <= 0 || d->d_head <= 0 || d->rank <= 0) return LLATTE_ERR_ARG;
+  if (d->d_ctx < 0 || d->n_q < 0 || d->d_out < 0 || d->ffn_mult <= 0) return LLATTE_ERR_ARG;
+  if (d->dtype != LLATTE_BF16 && d->dtype != LLATTE_FP32) return LLATTE_ERR_ARG;
+  if (!(d->eps > 0.f)) return LLATTE_ERR_ARG;
+  if (d->max_batch <= 0 || d->max_len < 0 || d->max_total < 0) return LLATTE_ERR_ARG;
+  if (d->kv_norm != 0 && d->kv_norm != 1) return LLATTE_ERR_ARG;
+  for (int l = 0; l < d->n_layers; ++l) {
+    if (d->keep[l] < 0) return LLATTE_ERR_ARG;
+    if (l && d->keep[l] > d->keep[l - 1]) return LLATTE_ERR_ARG;  // T_{l+1} <= T_l
+  }
+  const int elem = d->dtype == LLATTE_BF16 ? 2 : 4;
+  if ((d->d * elem) % 16 != 0) return LLATTE_ERR_UNSUPPORTED;     // 16-byte row vectors
+  if (d->rank > 256) return LLATTE_ERR_UNSUPPORTED;
+  return LLATTE_OK;
+}
+
+Layout layout_of(const llatte_dims* d) {
+  Layout L;
+  const int elem = d->dtype == LLATTE_BF16 ? 2 : 4;
+  const int64_t B = d->max_batch;
+  L.rows_h = d->max_total ? d->max_total : B * d->max_len;
+  L.rows_q = std::min<int64_t>(L.rows_h, B * (int64_t)d->keep[0]) + B * d->n_q;
+  const int64_t hr = (int64_t)d->heads * d->rank, f = (int64_t)d->ffn_mult * d->d;
+  const int nl = d->n_layers;
+  // attention work items: (user, 128-row block of (query row, head) pairs)
+  const int64_t max_work = (L.rows_q * d->heads + 127) / 128 + B;
+  L.max_work = (int32_t)std::min<int64_t>(max_work, 1 << 30);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o += align_up(bytes); return r; };
+  L.off_hist_off = take(sizeof(int64_t) * (nl + 1) * (B + 1));
+  L.off_query_off = take(sizeof(int64_t) * (nl + 1) * (B + 1));
+  L.off_T = take(sizeof(int32_t) * (nl + 1) * B);
+  L.off_n = take(sizeof(int32_t) * (nl + 1) * B);
+  L.off_totals = take(sizeof(int64_t) * 2 * (nl + 1));
+  L.off_status = take(sizeof(int32_t));
+  L.off_work = take(sizeof(int32_t) * 2 * nl * (size_t)L.max_work);
+  L.off_work_count = take(sizeof(int32_t) * nl);
+  L.off_work_next = take(sizeof(int32_t) * nl);
+  for (int i = 0; i < 2; ++i) L.off_Xh[i] = take((size_t)L.rows_h * d->d * elem);
+  for (int i = 0; i < 2; ++i) L.off_Xq[i] = take((size_t)L.rows_q * d->d * elem);
+  L.off_C = take((size_t)L.rows_h * d->rank * elem);
+  L.off_Qt = take((size_t)L.rows_q * hr * elem);
+  L.off_Ot = take((size_t)L.rows_q * hr * elem);
+  L.off_Z = take((size_t)L.rows_q * d->d * elem);
+  L.off_Hd = take((size_t)L.rows_q * f * elem);
+  L.off_acc32 = take(sizeof(float) * std::max<size_t>((size_t)L.rows_h * d->rank,
+                                                      (size_t)L.rows_q * d->d));
+  L.off_ctxbias = take(sizeof(float) * B * hr);
+  L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
+  L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
+  L.total = o;
+  return L;
+}
+
+#define CK(x)                                                   \
+  do {                                                          \
+    cudaError_t e_ = (x);                                       \
+    if (e_ != cudaSuccess) {                                    \
+      fprintf(stderr, "llatte: %s failed: %s (%s:%d)\n", #x,    \
+              cudaGetErrorString(e_), __FILE__, __LINE__);      \
+      return LLATTE_ERR_CUDA;                                   \
+    }                                                           \
+  } while (0)
+
+void* dev_alloc(llatte_handle* h, size_t bytes) {
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes ? bytes : 16) != cudaSuccess) return nullptr;
+  h->allocs.push_back(p);
+  return p;
+}
+
+// Copy one weight array to a fresh device buffer.
+void* upload(llatte_handle* h, const void* src, size_t bytes, int on_device) {
+  void* p = dev_alloc(h, bytes);
+  if (!p) return nullptr;
+  if (bytes && cudaMemcpy(p, src, bytes, on_device ? cudaMemcpyDeviceToDevice
+                                                    : cudaMemcpyHostToDevice) != cudaSuccess)
+    return nullptr;
+  return p;
+}
+
+cudaEvent_t take_event(llatte_handle* h) {
+  if (!h->event_pool.empty()) {
+    cudaEvent_t e = h->event_pool.back();
+    h->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct StepTimer {
+  llatte_handle* h;
+  cudaStream_t s;
+  int step;
+  cudaEvent_t a = nullptr;
+  StepTimer(llatte_handle* h_, cudaStream_t s_, int step_) : h(h_), s(s_), step(step_) {
+    if (h->profiling) {
+      a = take_event(h);
+      cudaEventRecord(a, s);
+    }
+  }
+  void done(int launches) {
+    if (!h->profiling) return;
+    cudaEvent_t b = take_event(h);
+    cudaEventRecord(b, s);
+    h->pending.push_back(ProfRec{step, a, b, launches});
+  }
+};
+
+int drain_profile(llatte_handle* h) {
+  for (auto& r : h->pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return LLATTE_ERR_CUDA;
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    h->step_ms[r.step] += ms;
+    h->step_launches[r.step] += r.launches;
+    h->step_calls[r.step] += 1;
+    h->event_pool.push_back(r.a);
+    h->event_pool.push_back(r.b);
+  }
+  h->pending.clear();
+  return LLATTE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t llatte_workspace_bytes(const llatte_dims* dims) {
+  if (check_dims(dims) != LLATTE_OK) return 0;
+  return layout_of(dims).total;
+}
+
+const char* llatte_error_string(int code) {
+  switch (code) {
+    case LLATTE_OK: return "ok";
+    case LLATTE_ERR_ARG: return "invalid argument";
+    case LLATTE_ERR_UNSUPPORTED: return "unsupported dimensions";
+    case LLATTE_ERR_CUDA: return "CUDA runtime error";
+    case LLATTE_ERR_OOM: return "device allocation failed";
+    case LLATTE_ERR_DEVICE: return "device-side fault reported in the status word";
+    default: return "unknown error";
+  }
+}
+
+void llatte_destroy(llatte_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  for (auto& r : h->pending) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+  for (auto e : h->event_pool) cudaEventDestroy(e);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_layer_w* layers,
+                  const void* W_e, int weights_on_device) {
+  if (!out) return LLATTE_ERR_ARG;
+  *out = nullptr;
+  int rc = check_dims(dims);
+  if (rc != LLATTE_OK) return rc;
+  if (!layers) return LLATTE_ERR_ARG;
+  const llatte_dims& D = *dims;
+  for (int l = 0; l < D.n_layers; ++l) {
+    const llatte_layer_w& w = layers[l];
+    if (!w.W_dkv || !w.g_kv || !w.W_q || !w.W_uk || !w.W_uv || !w.W_o || !w.g1 || !w.W1 ||
+        !w.W2 || !w.g2)
+      return LLATTE_ERR_ARG;
+  }
+  if (D.d_out > 0 && !W_e) return LLATTE_ERR_ARG;
+
+  llatte_handle* h = new (std::nothrow) llatte_handle();
+  if (!h) return LLATTE_ERR_OOM;
+  h->dims = D;
+  h->elem = D.dtype == LLATTE_BF16 ? 2 : 4;
+  h->use_tc = 0;
+  h->profiling = 0;
+  h->last_B = 0;
+  for (int i = 0; i < ST_COUNT; ++i) { h->step_ms[i] = 0; h->step_launches[i] = 0; h->step_calls[i] = 0; }
+  auto fail = [&](int code) { llatte_destroy(h); return code; };
+  if (cudaGetDevice(&h->device) != cudaSuccess) return fail(LLATTE_ERR_CUDA);
+  if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
+    return fail(LLATTE_ERR_CUDA);
+
+  const size_t e = h->elem;
+  const int d = D.d, r = D.rank, hd = D.heads * D.d_head, hr = D.heads * D.rank,
+            f = D.ffn_mult * D.d, dc = D.d_ctx;
+  for (int l = 0; l < D.n_layers; ++l) {
+    const llatte_layer_w& w = layers[l];
+    LayerDev& L = h->layers[l];
+    L.W_dkv = upload(h, w.W_dkv, e * r * d, weights_on_device);
+    L.g_kv = upload(h, w.g_kv, e * r, weights_on_device);
+    L.g1 = upload(h, w.g1, e * d, weights_on_device);
+    L.W1 = upload(h, w.W1, e * (size_t)f * d, weights_on_device);
+    L.W2 = upload(h, w.W2, e * (size_t)d * f, weights_on_device);
+    L.g2 = upload(h, w.g2, e * d, weights_on_device);
+    L.W_qk = dev_alloc(h, e * (size_t)hr * d);
+    L.W_qkc = dc ? (float*)dev_alloc(h, sizeof(float) * (size_t)hr * dc) : nullptr;
+    L.W_ov = dev_alloc(h, e * (size_t)d * hr);
+    if (!L.W_dkv || !L.g_kv || !L.g1 || !L.W1 || !L.W2 || !L.g2 || !L.W_qk || !L.W_ov ||
+        (dc && !L.W_qkc))
+      return fail(LLATTE_ERR_OOM);
+    // temporaries for absorption
+    void *tq = nullptr, *tuk = nullptr, *tuv = nullptr, *to = nullptr;
+    bool ok = cudaMalloc(&tq, e * (size_t)hd * (d + dc)) == cudaSuccess &&
+              cudaMalloc(&tuk, e * (size_t)hd * r) == cudaSuccess &&
+              cudaMalloc(&tuv, e * (size_t)hd * r) == cudaSuccess &&
+              cudaMalloc(&to, e * (size_t)d * hd) == cudaSuccess;
+    cudaMemcpyKind k = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    ok = ok && cudaMemcpy(tq, w.W_q, e * (size_t)hd * (d + dc), k) == cudaSuccess &&
+         cudaMemcpy(tuk, w.W_uk, e * (size_t)hd * r, k) == cudaSuccess &&
+         cudaMemcpy(tuv, w.W_uv, e * (size_t)hd * r, k) == cudaSuccess &&
+         cudaMemcpy(to, w.W_o, e * (size_t)d * hd, k) == cudaSuccess;
+    ok = ok && launch_absorb(h->elem, tq, tuk, tuv, to, d, dc, D.heads, D.d_head, r, L.W_qk,
+                             L.W_qkc, L.W_ov, 0) == cudaSuccess;
+    ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+    cudaFree(tq); cudaFree(tuk); cudaFree(tuv); cudaFree(to);
+    if (!ok) return fail(LLATTE_ERR_CUDA);
+  }
+  h->W_e = nullptr;
+  if (D.d_out > 0) {
+    h->W_e = upload(h, W_e, e * (size_t)D.d_out * d, weights_on_device);
+    if (!h->W_e) return fail(LLATTE_ERR_OOM);
+  }
+
+  Layout Lo = layout_of(&D);
+  char* ws = (char*)dev_alloc(h, Lo.total);
+  if (!ws) return fail(LLATTE_ERR_OOM);
+  if (cudaMemset(ws, 0, Lo.total) != cudaSuccess) return fail(LLATTE_ERR_CUDA);
+  h->ws_bytes = Lo.total;
+  h->max_rows_h = Lo.rows_h;
+  h->max_rows_q = Lo.rows_q;
+  PlanDev& p = h->plan;
+  p.hist_off = (int64_t*)(ws + Lo.off_hist_off);
+  p.query_off = (int64_t*)(ws + Lo.off_query_off);
+  p.T = (int32_t*)(ws + Lo.off_T);
+  p.n = (int32_t*)(ws + Lo.off_n);
+  p.totals = (int64_t*)(ws + Lo.off_totals);
+  p.status = (int32_t*)(ws + Lo.off_status);
+  p.work = (int32_t*)(ws + Lo.off_work);
+  p.work_count = (int32_t*)(ws + Lo.off_work_count);
+  p.work_next = (int32_t*)(ws + Lo.off_work_next);
+  p.stride = D.max_batch + 1;
+  p.max_work = Lo.max_work;
+  for (int i = 0; i < 2; ++i) { h->Xh[i] = ws + Lo.off_Xh[i]; h->Xq[i] = ws + Lo.off_Xq[i]; }
+  h->C = ws + Lo.off_C;
+  h->Qt = ws + Lo.off_Qt;
+  h->Ot = ws + Lo.off_Ot;
+  h->Z = ws + Lo.off_Z;
+  h->Hd = ws + Lo.off_Hd;
+  h->acc32 = (float*)(ws + Lo.off_acc32);
+  h->ctxbias = (float*)(ws + Lo.off_ctxbias);
+  h->final_rows = D.d_out ? (float*)(ws + Lo.off_final) : nullptr;
+  h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLATTE_ERR_CUDA);
+  *out = h;
+  return LLATTE_OK;
+}
+
+int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
+                   const void* context, const void* cand, float* out, void* stream) {
+  if (!h) return LLATTE_ERR_ARG;
+  const llatte_dims& D = h->dims;
+  if (B < 0 || B > D.max_batch) return LLATTE_ERR_ARG;
+  if (B == 0) { h->last_B = 0; return LLATTE_OK; }
+  if (!values || !offsets) return LLATTE_ERR_ARG;
+  if (D.d_ctx > 0 && !context) return LLATTE_ERR_ARG;
+  if (D.n_q > 0 && !cand) return LLATTE_ERR_ARG;
+  const bool has_out = D.d_out > 0 || D.n_q > 0;
+  if (has_out && !out) return LLATTE_ERR_ARG;
+  if (((uintptr_t)values | (uintptr_t)cand) & 15) return LLATTE_ERR_ARG;  // 16-byte rows
+  cudaStream_t s = (cudaStream_t)stream;
+  const int L = D.n_layers, e = h->elem;
+  const int d = D.d, r = D.rank, hr = D.heads * D.rank, f = D.ffn_mult * D.d;
+  const PlanDev& p = h->plan;
+  h->last_B = B;
+
+  { StepTimer t(h, s, ST_PLAN); CK(launch_plan(h, offsets, B, s)); t.done(1); }
+  { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, B, s)); t.done(1); }
+
+  for (int l = 0; l < L; ++l) {
+    const LayerDev& W = h->layers[l];
+    void* Xh_l = h->Xh[l & 1];
+    void* Xq_l = h->Xq[l & 1];
+    void* Xh_n = h->Xh[(l + 1) & 1];
+    void* Xq_n = h->Xq[(l + 1) & 1];
+    const bool last = l == L - 1;
+
+    if (D.d_ctx > 0) {
+      StepTimer t(h, s, ST_CTX);
+      GemmArgs g = {};
+      g.A = context; g.lda = D.d_ctx; g.W = W.W_qkc; g.D = h->ctxbias; g.ldd = hr;
+      g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = hr; g.K = D.d_ctx; g.epi = EPI_F32;
+      CK(launch_gemm_simt(e, 4, 4, g, s));
+      t.done(1);
+    }
+    {  // KV latent
+      StepTimer t(h, s, ST_KV);
+      GemmArgs g = {};
+      g.A = Xh_l; g.lda = d; g.W = W.W_dkv; g.M_dev = p.hist_total(l); g.M_max = h->max_rows_h;
+      g.N = r; g.K = d;
+      if (D.kv_norm) {
+        g.D = h->acc32; g.ldd = r; g.epi = EPI_F32;
+        CK(launch_gemm_simt(e, e, 4, g, s));
+        NormArgs a = {};
+        a.acc = h->acc32; a.N = r; a.resid = nullptr; a.g = W.g_kv; a.eps = D.eps;
+        a.M_dev = p.hist_total(l); a.M_max = h->max_rows_h; a.mode = NORM_PLAIN; a.dst = h->C;
+        CK(launch_rownorm(e, a, s));
+        t.done(2);
+      } else {
+        g.D = h->C; g.ldd = r; g.epi = EPI_STORE;
+        CK(launch_gemm_simt(e, e, e, g, s));
+        t.done(1);
+      }
+    }
+    {  // absorbed queries
+      StepTimer t(h, s, ST_Q);
+      GemmArgs g = {};
+      g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
+      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = hr; g.K = d;
+      g.epi = D.d_ctx > 0 ? EPI_USERBIAS : EPI_STORE;
+      g.bias = h->ctxbias; g.seg_off = p.qoff(l); g.B = B;
+      CK(launch_gemm_simt(e, e, e, g, s));
+      t.done(1);
+    }
+    {  // latent attention
+      StepTimer t(h, s, ST_ATTN);
+      AttnArgs a = {};
+      a.Qt = h->Qt; a.C = h->C; a.Ot = h->Ot; a.qoff = p.qoff(l); a.hoff = p.hoff(l);
+      a.T = p.Tl(l); a.n = p.nl(l); a.Mq_dev = p.query_total(l); a.Mq_max = h->max_rows_q;
+      a.B = B; a.heads = D.heads; a.r = r;
+      CK(launch_attn_simt(e, a, s));
+      t.done(1);
+    }
+    {  // output projection + residual + RMSNorm
+      StepTimer t(h, s, ST_O);
+      GemmArgs g = {};
+      g.A = h->Ot; g.lda = hr; g.W = W.W_ov; g.D = h->acc32; g.ldd = d;
+      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = hr; g.epi = EPI_F32;
+      CK(launch_gemm_simt(e, e, 4, g, s));
+      NormArgs a = {};
+      a.acc = h->acc32; a.N = d; a.resid = Xq_l; a.g = W.g1; a.eps = D.eps;
+      a.M_dev = p.query_total(l); a.M_max = h->max_rows_q; a.mode = NORM_PLAIN; a.dst = h->Z;
+      CK(launch_rownorm(e, a, s));
+      t.done(2);
+    }
+    {  // FFN up + SiLU
+      StepTimer t(h, s, ST_FFN1);
+      GemmArgs g = {};
+      g.A = h->Z; g.lda = d; g.W = W.W1; g.D = h->Hd; g.ldd = f;
+      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = f; g.K = d; g.epi = EPI_SILU;
+      CK(launch_gemm_simt(e, e, e, g, s));
+      t.done(1);
+    }
+    {  // FFN down + residual + RMSNorm, scattered into the next layer's rows
+      StepTimer t(h, s, ST_FFN2);
+      GemmArgs g = {};
+      g.A = h->Hd; g.lda = f; g.W = W.W2; g.D = h->acc32; g.ldd = d;
+      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = f; g.epi = EPI_F32;
+      CK(launch_gemm_simt(e, e, 4, g, s));
+      NormArgs a = {};
+      a.acc = h->acc32; a.N = d; a.resid = h->Z; a.g = W.g2; a.eps = D.eps;
+      a.M_dev = p.query_total(l); a.M_max = h->max_rows_q; a.mode = NORM_SCATTER;
+      a.qoff_l = p.qoff(l); a.n_l = p.nl(l); a.hoff_n = p.hoff(l + 1); a.qoff_n = p.qoff(l + 1);
+      a.n_n = p.nl(l + 1); a.B = B; a.n_q = D.n_q; a.Xh_n = Xh_n; a.Xq_n = Xq_n; a.last = last;
+      a.out = out; a.final_rows = D.d_out ? h->final_rows : nullptr;
+      CK(launch_rownorm(e, a, s));
+      t.done(2);
+    }
+  }
+  if (D.d_out > 0) {
+    StepTimer t(h, s, ST_READOUT);
+    CK(launch_mean_rows(h->final_rows, p.qoff(L - 1), B, d, h->mean_rows, s));
+    GemmArgs g = {};
+    g.A = h->mean_rows; g.lda = d; g.W = h->W_e; g.D = out; g.ldd = D.d_out;
+    g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = D.d_out; g.K = d; g.epi = EPI_F32;
+    CK(launch_gemm_simt(4, e, 4, g, s));
+    t.done(2);
+  }
+  return LLATTE_OK;
+}
+
+int llatte_plan_export(llatte_handle* h, int64_t* dst, void* stream) {
+  if (!h || !dst) return LLATTE_ERR_ARG;
+  const int B = h->last_B, L = h->dims.n_layers;
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int l = 0; l < L; ++l) {
+    CK(cudaMemcpyAsync(dst + (size_t)(2 * l) * (B + 1), h->plan.hist_off + l * h->plan.stride,
+                       sizeof(int64_t) * (B + 1), cudaMemcpyDeviceToDevice, s));
+    CK(cudaMemcpyAsync(dst + (size_t)(2 * l + 1) * (B + 1), h->plan.query_off + l * h->plan.stride,
+                       sizeof(int64_t) * (B + 1), cudaMemcpyDeviceToDevice, s));
+  }
+  return LLATTE_OK;
+}
+
+int llatte_get_status(llatte_handle* h, int32_t* device_status) {
+  if (!h || !device_status) return LLATTE_ERR_ARG;
+  CK(cudaDeviceSynchronize());
+  int32_t v = 0;
+  CK(cudaMemcpy(&v, h->plan.status, sizeof(int32_t), cudaMemcpyDeviceToHost));
+  CK(cudaMemset(h->plan.status, 0, sizeof(int32_t)));
+  *device_status = v;
+  return v ? LLATTE_ERR_DEVICE : LLATTE_OK;
+}
+
+int llatte_set_profiling(llatte_handle* h, int enable) {
+  if (!h) return LLATTE_ERR_ARG;
+  h->profiling = enable ? 1 : 0;
+  return LLATTE_OK;
+}
+
+int llatte_profile_reset(llatte_handle* h) {
+  if (!h) return LLATTE_ERR_ARG;
+  int rc = drain_profile(h);
+  for (int i = 0; i < ST_COUNT; ++i) { h->step_ms[i] = 0; h->step_launches[i] = 0; h->step_calls[i] = 0; }
+  return rc;
+}
+
+int llatte_profile_step(llatte_handle* h, int step, const char** name, double* total_ms,
+                        int64_t* kernel_launches, int64_t* calls) {
+  if (!h || step < 0 || step >= ST_COUNT) return LLATTE_ERR_ARG;
+  int rc = drain_profile(h);
+  if (rc != LLATTE_OK) return rc;
+  if (name) *name = kStepNames[step];
+  if (total_ms) *total_ms = h->step_ms[step];
+  if (kernel_launches) *kernel_launches = h->step_launches[step];
+  if (calls) *calls = h->step_calls[step];
+  return LLATTE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,302 @@
+// CUDA-core (fp32 FFMA) kernels: the whole layer for the fp32 storage type,
+// and the small steps (context bias, weight absorption, readout) for both.
+//
+// Layer equations (LLaTTE notes, huaxiaozhuan.com, appendix A.2 display and
+// A.3 absorbed MLA; target-aware query from the daiwk.github.io notes):
+//   KV    c_kv = RMSNorm_{g_kv}(X W_dkv^T)
+//   Q     q~   = X W_qk^T + (c W_qkc^T)                 (per-user context bias)
+//   ATTN  o~   = softmax(q~ . c_kv) c_kv over the visible keys
+//   O     Z    = RMSNorm_{g1}(R + o~ W_ov^T)
+//   FFN   X'   = RMSNorm_{g2}(Z + W2 SiLU(W1 Z))
+#include "common.cuh"
+#include "internal.h"
+
+namespace llatte {
+
+// ---------------------------------------------------------------- GEMM
+// D[m, n] = sum_k A[m, k] * W[n, k]   (A [M, K] row-major, W [N, K] row-major)
+// 64x64 tile, k-step 16, 256 threads, 4x4 outputs per thread.
+constexpr int SG_BM = 64, SG_BN = 64, SG_BK = 16;
+
+template <typename TA, typename TW, typename TD>
+__global__ void __launch_bounds__(256)
+gemm_simt_kernel(GemmArgs g) {
+  __shared__ float As[SG_BK][SG_BM + 4];
+  __shared__ float Ws[SG_BK][SG_BN + 4];
+  const int64_t M = g.M_dev ? *g.M_dev : g.M_host;
+  const int64_t m0 = (int64_t)blockIdx.y * SG_BM;
+  const int n0 = blockIdx.x * SG_BN;
+  if (m0 >= M) return;
+  const TA* A = (const TA*)g.A;
+  const TW* W = (const TW*)g.W;
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < g.K; k0 += SG_BK) {
+    for (int i = tid; i < SG_BM * SG_BK; i += 256) {
+      int r = i / SG_BK, c = i % SG_BK;
+      int64_t m = m0 + r;
+      int k = k0 + c;
+      As[c][r] = (m < M && k < g.K) ? to_f(A[m * g.lda + k]) : 0.f;
+      int n = n0 + r;
+      Ws[c][r] = (n < g.N && k < g.K) ? to_f(W[(int64_t)n * g.K + k]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_BK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Ws[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+    int u = 0;
+    if (g.epi == EPI_USERBIAS) u = segment_of(g.seg_off, g.B, m);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= g.N) continue;
+      float v = acc[i][j];
+      if (g.epi == EPI_USERBIAS) v += g.bias[(int64_t)u * g.N + n];
+      if (g.epi == EPI_SILU) v = silu_f(v);
+      if (g.epi == EPI_F32) ((float*)g.D)[m * g.ldd + n] = v;
+      else ((TD*)g.D)[m * g.ldd + n] = from_f<TD>(v);
+    }
+  }
+}
+
+template <typename TA, typename TW, typename TD>
+static cudaError_t gemm3(const GemmArgs& g, cudaStream_t s) {
+  dim3 grid((g.N + SG_BN - 1) / SG_BN, (unsigned)((g.M_max + SG_BM - 1) / SG_BM));
+  if (grid.y == 0) return cudaSuccess;
+  gemm_simt_kernel<TA, TW, TD><<<grid, 256, 0, s>>>(g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_simt(int ea, int ew, int ed, const GemmArgs& g, cudaStream_t s) {
+  typedef __nv_bfloat16 bf;
+  if (ea == 4 && ew == 4) return gemm3<float, float, float>(g, s);
+  if (ea == 2 && ew == 2 && ed == 2) return gemm3<bf, bf, bf>(g, s);
+  if (ea == 2 && ew == 2 && ed == 4) return gemm3<bf, bf, float>(g, s);
+  if (ea == 2 && ew == 4) return gemm3<bf, float, float>(g, s);
+  if (ea == 4 && ew == 2) return gemm3<float, bf, float>(g, s);
+  return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------- row norm
+// v = acc + resid;  y = v / sqrt(mean(v^2) + eps) * g; one warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256)
+rownorm_kernel(NormArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t M = *a.M_dev;
+  const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const int N = a.N;
+  const float* row = a.acc + m * N;
+  const T* res = (const T*)a.resid;
+  const T* g = (const T*)a.g;
+  float ss = 0.f;
+  for (int c = lane; c < N; c += 32) {
+    float v = row[c] + (res ? to_f(res[m * N + c]) : 0.f);
+    ss += v * v;
+  }
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss / N + a.eps);
+  // destinations
+  T* d1 = nullptr;
+  T* d2 = nullptr;
+  float* f1 = nullptr;
+  if (a.mode == NORM_PLAIN) {
+    d1 = (T*)a.dst + m * N;
+  } else {
+    const int u = segment_of(a.qoff_l, a.B, m);
+    const int64_t j = m - a.qoff_l[u];
+    const int32_t nl = a.n_l[u];
+    if (a.last) {
+      if (a.final_rows) f1 = a.final_rows + m * N;
+      else if (j >= nl) f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+    } else {
+      const int32_t nn = a.n_n[u];
+      if (j < nl) {
+        d1 = (T*)a.Xh_n + (a.hoff_n[u] + j) * N;
+        if (j >= nl - nn) d2 = (T*)a.Xq_n + (a.qoff_n[u] + j - (nl - nn)) * N;
+      } else {
+        d2 = (T*)a.Xq_n + (a.qoff_n[u] + nn + (j - nl)) * N;
+      }
+    }
+  }
+  for (int c = lane; c < N; c += 32) {
+    float v = row[c] + (res ? to_f(res[m * N + c]) : 0.f);
+    float y = v * inv * to_f(g[c]);
+    if (d1) d1[c] = from_f<T>(y);
+    if (d2) d2[c] = from_f<T>(y);
+    if (f1) f1[c] = y;
+  }
+}
+
+cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s) {
+  unsigned blocks = (unsigned)((a.M_max + 7) / 8);
+  if (blocks == 0) return cudaSuccess;
+  if (elem == 4) rownorm_kernel<float><<<blocks, 256, 0, s>>>(a);
+  else rownorm_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- attention
+// One warp per (query row, head).  Lane i holds latent coordinates
+// i, i+32, ...; online softmax over the visible keys of the row's user.
+template <typename T, int RV>
+__global__ void __launch_bounds__(256)
+attn_simt_kernel(AttnArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int64_t Mq = *a.Mq_dev;
+  if (w >= Mq * a.heads) return;
+  const int64_t m = w / a.heads;
+  const int j = (int)(w % a.heads);
+  const int u = segment_of(a.qoff, a.B, m);
+  const int64_t jl = m - a.qoff[u];
+  const int32_t Tu = a.T[u], n = a.n[u];
+  const int64_t vis = jl < n ? (Tu - n + jl + 1) : Tu;
+  const int r = a.r;
+  const T* q = (const T*)a.Qt + (m * a.heads + j) * r;
+  const T* C = (const T*)a.C + a.hoff[u] * r;
+  float qv[RV], o[RV];
+#pragma unroll
+  for (int i = 0; i < RV; ++i) {
+    int c = lane + 32 * i;
+    qv[i] = c < r ? to_f(q[c]) : 0.f;
+    o[i] = 0.f;
+  }
+  float mx = -INFINITY, l = 0.f;
+  for (int64_t t = 0; t < vis; ++t) {
+    const T* kr = C + t * r;
+    float kv[RV];
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < RV; ++i) {
+      int c = lane + 32 * i;
+      kv[i] = c < r ? to_f(kr[c]) : 0.f;
+      part = fmaf(qv[i], kv[i], part);
+    }
+    const float s = warp_sum(part);
+    const float mn = fmaxf(mx, s);
+    const float corr = __expf(mx - mn);
+    const float pr = __expf(s - mn);
+    l = l * corr + pr;
+#pragma unroll
+    for (int i = 0; i < RV; ++i) o[i] = fmaf(pr, kv[i], o[i] * corr);
+    mx = mn;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  T* out = (T*)a.Ot + (m * a.heads + j) * r;
+#pragma unroll
+  for (int i = 0; i < RV; ++i) {
+    int c = lane + 32 * i;
+    if (c < r) out[c] = from_f<T>(o[i] * inv);
+  }
+}
+
+template <typename T>
+static cudaError_t attn_t(const AttnArgs& a, cudaStream_t s) {
+  unsigned blocks = (unsigned)((a.Mq_max * a.heads + 7) / 8);
+  if (blocks == 0) return cudaSuccess;
+  if (a.r <= 32) attn_simt_kernel<T, 1><<<blocks, 256, 0, s>>>(a);
+  else if (a.r <= 64) attn_simt_kernel<T, 2><<<blocks, 256, 0, s>>>(a);
+  else if (a.r <= 128) attn_simt_kernel<T, 4><<<blocks, 256, 0, s>>>(a);
+  else if (a.r <= 256) attn_simt_kernel<T, 8><<<blocks, 256, 0, s>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s) {
+  return elem == 4 ? attn_t<float>(a, s) : attn_t<__nv_bfloat16>(a, s);
+}
+
+// ---------------------------------------------------------------- readout mean
+// mean[u] = (1 / rows_u) sum of the user's final rows (zero for no rows).
+__global__ void mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qoff,
+                                 int d, float* __restrict__ mean) {
+  const int u = blockIdx.x;
+  const int64_t a = qoff[u], b = qoff[u + 1];
+  const float inv = b > a ? 1.f / (float)(b - a) : 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float s = 0.f;
+    for (int64_t i = a; i < b; ++i) s += rows[i * d + c];
+    mean[(int64_t)u * d + c] = s * inv;
+  }
+}
+
+cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
+                             cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
+  mean_rows_kernel<<<B, 256, 0, s>>>(rows, qoff, d, mean);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- absorption
+// W_qk[j*r + a, k] = (1/sqrt(d_h)) sum_e W_uk[j*d_h + e, a] W_q[j*d_h + e, k]
+//   (k < d -> W_qk in the storage type, k >= d -> W_qkc in fp32)
+// W_ov[n, j*r + a] = sum_e W_o[n, j*d_h + e] W_uv[j*d_h + e, a]
+template <typename T>
+__global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int heads, int dh,
+                                int r, T* W_qk, float* W_qkc) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int K = d + dc;
+  if (idx >= (int64_t)heads * r * K) return;
+  const int k = (int)(idx % K);
+  const int row = (int)(idx / K);
+  const int j = row / r, a = row % r;
+  float s = 0.f;
+  for (int e = 0; e < dh; ++e)
+    s = fmaf(to_f(W_uk[(int64_t)(j * dh + e) * r + a]), to_f(W_q[(int64_t)(j * dh + e) * K + k]), s);
+  s *= rsqrtf((float)dh);
+  if (k < d) W_qk[(int64_t)row * d + k] = from_f<T>(s);
+  else W_qkc[(int64_t)row * dc + (k - d)] = s;
+}
+
+template <typename T>
+__global__ void absorb_o_kernel(const T* W_o, const T* W_uv, int d, int heads, int dh, int r,
+                                T* W_ov) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int HR = heads * r;
+  if (idx >= (int64_t)d * HR) return;
+  const int col = (int)(idx % HR);
+  const int nrow = (int)(idx / HR);
+  const int j = col / r, a = col % r;
+  float s = 0.f;
+  for (int e = 0; e < dh; ++e)
+    s = fmaf(to_f(W_o[(int64_t)nrow * heads * dh + j * dh + e]), to_f(W_uv[(int64_t)(j * dh + e) * r + a]), s);
+  W_ov[idx] = from_f<T>(s);
+}
+
+cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
+                          const void* W_o, int d, int dc, int heads, int dh, int r, void* W_qk,
+                          float* W_qkc, void* W_ov, cudaStream_t s) {
+  const int64_t nq = (int64_t)heads * r * (d + dc), no = (int64_t)d * heads * r;
+  const unsigned bq = (unsigned)((nq + 255) / 256), bo = (unsigned)((no + 255) / 256);
+  if (elem == 4) {
+    absorb_q_kernel<float><<<bq, 256, 0, s>>>((const float*)W_q, (const float*)W_uk, d, dc, heads,
+                                              dh, r, (float*)W_qk, W_qkc);
+    absorb_o_kernel<float><<<bo, 256, 0, s>>>((const float*)W_o, (const float*)W_uv, d, heads, dh,
+                                              r, (float*)W_ov);
+  } else {
+    typedef __nv_bfloat16 bf;
+    absorb_q_kernel<bf><<<bq, 256, 0, s>>>((const bf*)W_q, (const bf*)W_uk, d, dc, heads, dh, r,
+                                           (bf*)W_qk, W_qkc);
+    absorb_o_kernel<bf><<<bo, 256, 0, s>>>((const bf*)W_o, (const bf*)W_uv, d, heads, dh, r,
+                                           (bf*)W_ov);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace llatte

@@ -1,0 +1,94 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the public header declares, and rejects bad arguments on the host before it
+touches the device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from latent_attention_jagged_b200 import binding
+from latent_attention_jagged_b200.build import build
+from workloads import Dims, workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load_library()
+
+
+def declared_functions():
+    names = set()
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(hdr).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"\b(llatte_\w+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("llatte_create", "llatte_forward", "llatte_destroy"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(binding.EXPORTS) <= set(declared_functions())
+
+
+def test_struct_layout_matches_header(lib):
+    # int32 x 7, keep[16], 4 x int32, float, int32, (pad 4), int64, int64
+    assert ctypes.sizeof(binding.llatte_dims) == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16
+    assert ctypes.sizeof(binding.llatte_layer_w) == 10 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def _cdims(**kw):
+    base = workload("online").dims
+    fields = dict(d=base.d, heads=base.heads, d_head=base.d_head, rank=base.rank,
+                  d_ctx=base.d_ctx, n_q=base.n_q, keep=base.keep, d_out=base.d_out,
+                  ffn_mult=base.ffn_mult, eps=base.eps, kv_norm=base.kv_norm, dtype=base.dtype)
+    fields.update(kw)
+    return binding.make_dims(Dims(**fields), max_batch=256, max_len=400)
+
+
+def test_workspace_bytes_and_dim_checks(lib):
+    good = _cdims()
+    ws = lib.llatte_workspace_bytes(ctypes.byref(good))
+    assert ws > 256 * 400 * 256 * 2          # at least the history rows
+    for bad in (_cdims(keep=(100, 200)), _cdims(keep=(-1,)), _cdims(d=0), _cdims(rank=512),
+                _cdims(d=12)):
+        assert lib.llatte_workspace_bytes(ctypes.byref(bad)) == 0
+    big = _cdims()
+    big.max_total = 1000
+    assert 0 < lib.llatte_workspace_bytes(ctypes.byref(big)) < ws
+
+
+def test_create_rejects_bad_arguments_on_host(lib):
+    h = ctypes.c_void_p()
+    layers = (binding.llatte_layer_w * 4)()
+    # increasing schedule: rejected before any device call
+    bad = _cdims(keep=(10, 20, 30, 40))
+    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, 0) == \
+        binding.LLATTE_ERR_ARG
+    # null weight pointers
+    good = _cdims()
+    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(good), layers, None, 0) == \
+        binding.LLATTE_ERR_ARG
+    assert lib.llatte_create(None, ctypes.byref(good), layers, None, 0) == binding.LLATTE_ERR_ARG
+
+
+def test_forward_and_status_reject_null_handle(lib):
+    assert lib.llatte_forward(None, None, None, 1, None, None, None, None) == binding.LLATTE_ERR_ARG
+    v = ctypes.c_int32()
+    assert lib.llatte_get_status(None, ctypes.byref(v)) == binding.LLATTE_ERR_ARG
+    assert lib.llatte_plan_export(None, None, None) == binding.LLATTE_ERR_ARG
+    lib.llatte_destroy(None)
+    assert lib.llatte_error_string(binding.LLATTE_ERR_DEVICE).startswith(b"device")

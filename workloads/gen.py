@@ -31,9 +31,10 @@ LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even), kept as float32."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).reshape(a.shape)
+    u = a.view(np.uint32)
+    # finite inputs cannot overflow 32 bits here (largest finite pattern + 0x8000)
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).reshape(a.shape)
 
 
 @dataclass
@@ -67,7 +68,10 @@ def draw_lengths(spec: tuple, batch: int, rng: np.random.Generator) -> np.ndarra
 
 
 def _normal(rng, shape, std=1.0):
-    return (rng.standard_normal(size=shape) * std).astype(np.float32)
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return x
 
 
 def draw_weights(dims: Dims, rng: np.random.Generator, random_gains: bool = False):
@@ -118,8 +122,8 @@ def make_inputs(wl: Workload, batch: Optional[int] = None,
         x = _normal(rng, (n, d))
         if W_sem is not None:
             codes = _normal(rng, (n, wl.sem_dim))
-            x = x + codes @ W_sem
-        return x.astype(np.float32)
+            x += codes @ W_sem
+        return x
 
     values = tokens(total)
     cand = tokens(B * dims.n_q).reshape(B, dims.n_q, d)
