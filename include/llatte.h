@@ -125,7 +125,8 @@ int llatte_create(llatte_handle** handle, const llatte_dims* dims,
  * default stream), with no host synchronisation.
  *   values  device [offsets[B] rows, d] in dtype: all users' histories, user u
  *           in rows offsets[u] .. offsets[u+1]-1, earliest event first;
- *           16-byte aligned (as are cand and context)
+ *           16-byte aligned (as are cand and context); may be NULL when
+ *           every history is empty
  *   offsets device int64 [B+1], non-decreasing, offsets[0] >= 0
  *   B       number of users, 0 <= B <= max_batch (B = 0 launches nothing)
  *   context device [B, d_ctx] in dtype (may be NULL when d_ctx == 0)

@@ -1,0 +1,409 @@
+// Tensor-core GEMM for sm_100a: D[m, n] = sum_k A[m, k] W[n, k] (bf16 in,
+// fp32 accumulation in TMEM) with the layer's epilogues fused.
+//
+// Roles (192 threads, one CTA per SM, persistent over 128 x BN tiles):
+//   warp 0      TMA producer: A (128 x 64) and W (BN x 64) k-blocks into a
+//               STAGES-deep ring of 128-byte-swizzled shared-memory tiles
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (128 x NI x 16) and
+//               commits stage releases / accumulator-ready events
+//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), then one of
+//               STORE     bf16 store
+//               USERBIAS  + per-user context term (absorbed query projection)
+//               SILU      SiLU (FFN up-projection)
+//               NORM      + residual, RMSNorm over the full row (BN == N),
+//                         store bf16 (+ fp32 copy) or scatter into the next
+//                         layer's history / query rows (pyramid trimming)
+// The accumulator is double-buffered in TMEM when 2 * BN <= 512 columns, so
+// the epilogue of tile i overlaps the MMAs of tile i + 1.
+//
+// Equations (LLaTTE notes, huaxiaozhuan.com, appendix A.2 display and A.3):
+// KV latent RMSNorm(X W_down^KV); absorbed query X (W_uk^T W_q)^T + context
+// term; Z = RMSNorm(R + o~ (W_o W_uv)^T); FFN W2 SiLU(W1 Z) + Z, RMSNorm.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+#include "tc_gemm.h"
+
+namespace llatte {
+
+using namespace tc;
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int NI = BN > 256 ? 256 : BN;     // N of one MMA instruction
+  static constexpr int NSUB = BN / NI;
+  static constexpr int ACC_BUFS = 2 * BN <= 512 ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS =
+      ACC_BUFS * BN <= 32 ? 32 : ACC_BUFS * BN <= 64 ? 64 : ACC_BUFS * BN <= 128 ? 128
+      : ACC_BUFS * BN <= 256 ? 256 : 512;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN >= 512 ? 2 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+};
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 w = __ldg(s + j);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 f = __bfloat1622float2(h[k]);
+      v[8 * j + 2 * k] = f.x;
+      v[8 * j + 2 * k + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void add_f32x32(const float* src, float (&v)[32]) {
+  const float4* s = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float4 w = __ldg(s + j);
+    v[4 * j] += w.x; v[4 * j + 1] += w.y; v[4 * j + 2] += w.z; v[4 * j + 3] += w.w;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    d[j] = make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                      pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
+}
+
+__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) d[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+
+// Residual chunk for columns [c, c + 32) of `row`, added to v.
+__device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N, int c,
+                                          float (&v)[32]) {
+  if (!a.resid) return;
+  if (a.resid_f32) {
+    add_f32x32((const float*)a.resid + row * N + c, v);
+  } else {
+    float r[32];
+    load_bf16x32((const __nv_bfloat16*)a.resid + row * N + c, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] += r[i];
+  }
+}
+
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
+                                         bool valid, int n0) {
+  if constexpr (EPI == TC_NORM) {
+    const NormArgs& a = p.norm;
+    const int N = BN;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (valid) {
+        add_resid(a, row, N, c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      }
+    }
+    const float inv = rsqrtf(ss / (float)N + a.eps);
+    // destinations of this row
+    __nv_bfloat16* d1 = nullptr;
+    __nv_bfloat16* d2 = nullptr;
+    float* f1 = nullptr;
+    float* f2 = nullptr;
+    if (valid) {
+      if (a.mode == NORM_PLAIN) {
+        d1 = (__nv_bfloat16*)a.dst + row * N;
+        if (a.dst32) f1 = a.dst32 + row * N;
+      } else {
+        const int u = segment_of(a.qoff_l, a.B, row);
+        const int64_t j = row - a.qoff_l[u];
+        const int32_t nl = a.n_l[u];
+        if (a.last) {
+          if (a.final_rows) f1 = a.final_rows + row * N;
+          else if (j >= nl) f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+        } else {
+          const int32_t nn = a.n_n[u];
+          int64_t q = -1;
+          if (j < nl) {
+            d1 = (__nv_bfloat16*)a.Xh_n + (a.hoff_n[u] + j) * N;
+            if (j >= nl - nn) q = a.qoff_n[u] + j - (nl - nn);
+          } else {
+            q = a.qoff_n[u] + nn + (j - nl);
+          }
+          if (q >= 0) {
+            d2 = (__nv_bfloat16*)a.Xq_n + q * N;
+            if (a.Xq32_n) f2 = a.Xq32_n + q * N;
+          }
+        }
+      }
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (valid) {
+        add_resid(a, row, N, c, v);
+        float g[32];
+        load_bf16x32((const __nv_bfloat16*)a.g + c, g);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * g[i];
+        if (d1) store_bf16x32(d1 + c, v);
+        if (d2) store_bf16x32(d2 + c, v);
+        if (f1) store_f32x32(f1 + c, v);
+        if (f2) store_f32x32(f2 + c, v);
+      }
+    }
+  } else {
+    int u = 0;
+    if (EPI == TC_USERBIAS && valid) u = segment_of(p.seg_off, p.B, row);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      if (valid) {
+        const int n = n0 + c;
+        if (EPI == TC_USERBIAS) add_f32x32(p.bias + (int64_t)u * p.N + n, v);
+        if (EPI == TC_SILU) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]);
+        }
+        store_bf16x32(p.D + row * p.ldd + n, v);
+      }
+    }
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcGemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES, NI = Cfg::NI, NSUB = Cfg::NSUB, ACC_BUFS = Cfg::ACC_BUFS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint64_t* full = (uint64_t*)(sB + STAGES * Cfg::B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + ACC_BUFS;
+  uint64_t* drain = tempty + ACC_BUFS;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
+  const int n_tiles = p.N / BN;
+  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int KB = p.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kb * BK, mt * BM);
+#pragma unroll
+          for (int s2 = 0; s2 < NSUB; ++s2)
+            tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * NI * 128, kb * BK,
+                        nt * BN + s2 * NI);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, NI, false, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_base = tmem + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
+#pragma unroll
+            for (int s2 = 0; s2 < NSUB; ++s2) {
+              const uint64_t bd = sdesc_sw128(b_addr + s2 * NI * 128 + k * 32, 16, 1024);
+              umma_bf16(d_base + s2 * NI, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+      }
+      // every MMA of this CTA must be complete before TMEM is released
+      umma_commit(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, &dummy, p.status);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
+      const int64_t row = (int64_t)mt * BM + q * 32 + lane;
+      epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+template <int BN, int EPI>
+cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmParams& p,
+                       int grid, cudaStream_t s) {
+  using Cfg = GemmCfg<BN>;
+  static uint64_t attr_devices = 0;   // devices on which the smem limit was raised
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_devices >> (dev & 63) & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_devices |= 1ull << (dev & 63);
+  }
+  tc_gemm_kernel<BN, EPI><<<grid, 192, Cfg::SMEM, s>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_epi(int BN, const CUtensorMap& a, const CUtensorMap& b, const TcGemmParams& p,
+                       int grid, cudaStream_t s) {
+  switch (BN) {
+    case 64: return launch_cfg<64, EPI>(a, b, p, grid, s);
+    case 128: return launch_cfg<128, EPI>(a, b, p, grid, s);
+    case 256: return launch_cfg<256, EPI>(a, b, p, grid, s);
+    case 512:
+      if constexpr (EPI == TC_NORM) return launch_cfg<512, EPI>(a, b, p, grid, s);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+bool tc_gemm_supported(int BN, int epi, int N, int K) {
+  if (K % BK != 0 || K <= 0) return false;
+  if (BN != 64 && BN != 128 && BN != 256 && BN != 512) return false;
+  if (BN == 512 && epi != TC_NORM) return false;
+  if (epi == TC_NORM && N != BN) return false;
+  return N % BN == 0;
+}
+
+cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
+                           const TcGemmParams& p, int num_sms, cudaStream_t s) {
+  if (!tc_gemm_supported(BN, epi, p.N, p.K)) return cudaErrorInvalidValue;
+  // grid: one CTA per SM, never more CTAs than the largest possible tile count
+  const int64_t max_tiles = ((p.M_cap + BM - 1) / BM) * (p.N / BN);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, max_tiles));
+  switch (epi) {
+    case TC_STORE: return launch_epi<TC_STORE>(BN, a, b, p, grid, s);
+    case TC_USERBIAS: return launch_epi<TC_USERBIAS>(BN, a, b, p, grid, s);
+    case TC_SILU: return launch_epi<TC_SILU>(BN, a, b, p, grid, s);
+    case TC_NORM: return launch_epi<TC_NORM>(BN, a, b, p, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------- tensor maps
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+}  // namespace
+
+// 2-D bf16 tensor [rows, cols] (row-major, cols contiguous), box of
+// box_rows x 64 columns (128 bytes), 128-byte swizzle, zero fill outside.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols % 64 != 0 || ((uintptr_t)base & 15) || box_rows > 256) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace llatte

@@ -1,6 +1,7 @@
 // Internal structures of the LLaTTE forward library (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -52,6 +53,9 @@ struct LayerDev {
 
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
+// TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
+struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2; };
+
 }  // namespace llatte
 
 struct llatte_handle {
@@ -74,12 +78,20 @@ struct llatte_handle {
   void* Ot;
   void* Z;
   void* Hd;
+  float* Z32;          // fp32 residual copy of Z (bf16 storage only, else aliases Z)
+  float* Xq32[2];      // fp32 residual copy of the query rows (bf16 storage only)
   float* acc32;        // fp32 pre-norm rows (CUDA-core path)
   float* ctxbias;      // [max_batch, h*r]
   float* final_rows;   // [max_rows_q, d] fp32 (readout only)
   float* mean_rows;    // [max_batch, d] fp32
   size_t ws_bytes;
   int last_B;
+
+  // tensor-core path: TMA descriptors of the A operands and the weights,
+  // and the tile width (BN) of each GEMM
+  CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd;
+  llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
+  int bn_kv, bn_q, bn_o, bn_f1, bn_f2;
 
   // profiling
   int profiling;
@@ -113,14 +125,15 @@ cudaError_t launch_gemm_simt(int elem_a, int elem_w, int elem_d, const GemmArgs&
 
 struct NormArgs {
   const float* acc; int N;           // [M, N] fp32 rows
-  const void* resid;                 // [M, N] storage type or NULL
+  const void* resid;                 // [M, N] residual or NULL
+  int resid_f32;                     // 1: resid is fp32, 0: storage type
   const void* g; float eps;
   const int64_t* M_dev; int64_t M_max;
   int mode;                          // NORM_PLAIN / NORM_SCATTER
-  void* dst;                         // NORM_PLAIN: [M, N]
+  void* dst; float* dst32;           // NORM_PLAIN: [M, N] storage type (+ optional fp32 copy)
   // NORM_SCATTER (FFN2 output of layer l -> inputs of layer l+1 / outputs)
   const int64_t *qoff_l, *hoff_n, *qoff_n; const int32_t *n_l, *n_n; int B; int n_q;
-  void* Xh_n; void* Xq_n; int last; float* out; float* final_rows;
+  void* Xh_n; void* Xq_n; float* Xq32_n; int last; float* out; float* final_rows;
 };
 enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
 cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s);

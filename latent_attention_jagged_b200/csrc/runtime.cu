@@ -7,6 +7,7 @@
 #include <new>
 
 #include "internal.h"
+#include "tc_gemm.h"
 
 using namespace llatte;
 
@@ -24,7 +25,7 @@ struct Layout {
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
       off_work_count, off_work_next;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
-      off_final, off_mean;
+      off_final, off_mean, off_Z32, off_Xq32[2];
   size_t total;
   int32_t max_work;
 };
@@ -77,6 +78,11 @@ Layout layout_of(const llatte_dims* d) {
   L.off_Ot = take((size_t)L.rows_q * hr * elem);
   L.off_Z = take((size_t)L.rows_q * d->d * elem);
   L.off_Hd = take((size_t)L.rows_q * f * elem);
+  // fp32 copies of the residual stream (bf16 storage keeps bf16 GEMM operands
+  // plus these; fp32 storage needs none)
+  const size_t res32 = elem == 2 ? sizeof(float) * (size_t)L.rows_q * d->d : 0;
+  L.off_Z32 = take(res32);
+  for (int i = 0; i < 2; ++i) L.off_Xq32[i] = take(res32);
   L.off_acc32 = take(sizeof(float) * std::max<size_t>((size_t)L.rows_h * d->rank,
                                                       (size_t)L.rows_q * d->d));
   L.off_ctxbias = take(sizeof(float) * B * hr);
@@ -156,6 +162,47 @@ int drain_profile(llatte_handle* h) {
   }
   h->pending.clear();
   return LLATTE_OK;
+}
+
+
+// Dimensions the tensor-core kernels implement (bf16 storage).
+bool tc_dims_ok(const llatte_dims& D) {
+  const int hr = D.heads * D.rank, f = D.ffn_mult * D.d;
+  const bool d_ok = D.d == 64 || D.d == 128 || D.d == 256 || D.d == 512;
+  const bool r_ok = D.rank == 64 || D.rank == 128 || D.rank == 256;
+  return d_ok && r_ok && hr % 64 == 0 && f % 64 == 0;
+}
+
+int pick_bn(int N) { return N % 256 == 0 ? 256 : N % 128 == 0 ? 128 : 64; }
+
+bool build_tc_maps(llatte_handle* h) {
+  const llatte_dims& D = h->dims;
+  const int d = D.d, r = D.rank, hr = D.heads * D.rank, f = D.ffn_mult * D.d;
+  h->bn_kv = r;
+  h->bn_q = pick_bn(hr);
+  h->bn_o = d;
+  h->bn_f1 = pick_bn(f);
+  h->bn_f2 = d;
+  const uint64_t rh = std::max<int64_t>(h->max_rows_h, 1), rq = std::max<int64_t>(h->max_rows_q, 1);
+  bool ok = true;
+  for (int i = 0; i < 2; ++i) {
+    ok = ok && make_tmap_bf16(&h->tm_Xh[i], h->Xh[i], rh, d, 128);
+    ok = ok && make_tmap_bf16(&h->tm_Xq[i], h->Xq[i], rq, d, 128);
+  }
+  ok = ok && make_tmap_bf16(&h->tm_Ot, h->Ot, rq, hr, 128);
+  ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
+  ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
+  auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
+  for (int l = 0; l < D.n_layers && ok; ++l) {
+    const LayerDev& W = h->layers[l];
+    LayerMaps& M = h->lmaps[l];
+    ok = ok && make_tmap_bf16(&M.dkv, W.W_dkv, r, d, box(h->bn_kv));
+    ok = ok && make_tmap_bf16(&M.qk, W.W_qk, hr, d, box(h->bn_q));
+    ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
+    ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
+    ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
+  }
+  return ok;
 }
 
 }  // namespace
@@ -283,10 +330,17 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->Ot = ws + Lo.off_Ot;
   h->Z = ws + Lo.off_Z;
   h->Hd = ws + Lo.off_Hd;
+  h->Z32 = h->elem == 2 ? (float*)(ws + Lo.off_Z32) : (float*)h->Z;
+  for (int i = 0; i < 2; ++i)
+    h->Xq32[i] = h->elem == 2 ? (float*)(ws + Lo.off_Xq32[i]) : (float*)h->Xq[i];
   h->acc32 = (float*)(ws + Lo.off_acc32);
   h->ctxbias = (float*)(ws + Lo.off_ctxbias);
   h->final_rows = D.d_out ? (float*)(ws + Lo.off_final) : nullptr;
   h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
+  if (h->elem == 2 && tc_dims_ok(D)) {
+    if (!build_tc_maps(h)) return fail(LLATTE_ERR_CUDA);
+    h->use_tc = 1;
+  }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLATTE_ERR_CUDA);
   *out = h;
   return LLATTE_OK;
@@ -298,7 +352,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
   const llatte_dims& D = h->dims;
   if (B < 0 || B > D.max_batch) return LLATTE_ERR_ARG;
   if (B == 0) { h->last_B = 0; return LLATTE_OK; }
-  if (!values || !offsets) return LLATTE_ERR_ARG;
+  if (!offsets) return LLATTE_ERR_ARG;  // values may be NULL when every history is empty
   if (D.d_ctx > 0 && !context) return LLATTE_ERR_ARG;
   if (D.n_q > 0 && !cand) return LLATTE_ERR_ARG;
   const bool has_out = D.d_out > 0 || D.n_q > 0;
@@ -329,33 +383,76 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       CK(launch_gemm_simt(e, 4, 4, g, s));
       t.done(1);
     }
+    const bool tc = h->use_tc != 0;
+    // epilogue arguments shared by both paths
+    NormArgs kv_norm = {};
+    kv_norm.N = r; kv_norm.g = W.g_kv; kv_norm.eps = D.eps; kv_norm.M_dev = p.hist_total(l);
+    kv_norm.M_max = h->max_rows_h; kv_norm.mode = NORM_PLAIN; kv_norm.dst = h->C;
+    NormArgs o_norm = {};
+    o_norm.N = d; o_norm.g = W.g1; o_norm.eps = D.eps;
+    // residual: the layer input rows; in fp32 from layer 1 on (layer 0 reads
+    // the gathered inputs, exact in the storage type)
+    o_norm.resid = (l == 0) ? Xq_l : (const void*)h->Xq32[l & 1];
+    o_norm.resid_f32 = (l == 0) ? (e == 4) : 1;
+    o_norm.M_dev = p.query_total(l); o_norm.M_max = h->max_rows_q; o_norm.mode = NORM_PLAIN;
+    o_norm.dst = h->Z; o_norm.dst32 = e == 2 ? h->Z32 : nullptr;
+    NormArgs f_norm = {};
+    f_norm.N = d; f_norm.resid = h->Z32; f_norm.resid_f32 = 1; f_norm.g = W.g2; f_norm.eps = D.eps;
+    f_norm.M_dev = p.query_total(l); f_norm.M_max = h->max_rows_q; f_norm.mode = NORM_SCATTER;
+    f_norm.qoff_l = p.qoff(l); f_norm.n_l = p.nl(l); f_norm.hoff_n = p.hoff(l + 1);
+    f_norm.qoff_n = p.qoff(l + 1); f_norm.n_n = p.nl(l + 1); f_norm.B = B; f_norm.n_q = D.n_q;
+    f_norm.Xh_n = Xh_n; f_norm.Xq_n = Xq_n; f_norm.last = last;
+    f_norm.Xq32_n = (e == 2 && !last) ? h->Xq32[(l + 1) & 1] : nullptr;
+    f_norm.out = out; f_norm.final_rows = D.d_out ? h->final_rows : nullptr;
+    const LayerMaps& LM = h->lmaps[l];
+    auto tcp = [&](const int64_t* Mdev, int64_t cap, int N, int K) {
+      TcGemmParams q = {};
+      q.M_dev = Mdev; q.M_cap = cap; q.N = N; q.K = K; q.status = p.status;
+      return q;
+    };
+
     {  // KV latent
       StepTimer t(h, s, ST_KV);
-      GemmArgs g = {};
-      g.A = Xh_l; g.lda = d; g.W = W.W_dkv; g.M_dev = p.hist_total(l); g.M_max = h->max_rows_h;
-      g.N = r; g.K = d;
-      if (D.kv_norm) {
-        g.D = h->acc32; g.ldd = r; g.epi = EPI_F32;
-        CK(launch_gemm_simt(e, e, 4, g, s));
-        NormArgs a = {};
-        a.acc = h->acc32; a.N = r; a.resid = nullptr; a.g = W.g_kv; a.eps = D.eps;
-        a.M_dev = p.hist_total(l); a.M_max = h->max_rows_h; a.mode = NORM_PLAIN; a.dst = h->C;
-        CK(launch_rownorm(e, a, s));
-        t.done(2);
-      } else {
-        g.D = h->C; g.ldd = r; g.epi = EPI_STORE;
-        CK(launch_gemm_simt(e, e, e, g, s));
+      if (tc) {
+        TcGemmParams q = tcp(p.hist_total(l), h->max_rows_h, r, d);
+        q.norm = kv_norm;
+        q.D = (__nv_bfloat16*)h->C; q.ldd = r;
+        CK(launch_tc_gemm(h->bn_kv, D.kv_norm ? TC_NORM : TC_STORE, h->tm_Xh[l & 1], LM.dkv, q,
+                          h->num_sms, s));
         t.done(1);
+      } else {
+        GemmArgs g = {};
+        g.A = Xh_l; g.lda = d; g.W = W.W_dkv; g.M_dev = p.hist_total(l); g.M_max = h->max_rows_h;
+        g.N = r; g.K = d;
+        if (D.kv_norm) {
+          g.D = h->acc32; g.ldd = r; g.epi = EPI_F32;
+          CK(launch_gemm_simt(e, e, 4, g, s));
+          kv_norm.acc = h->acc32;
+          CK(launch_rownorm(e, kv_norm, s));
+          t.done(2);
+        } else {
+          g.D = h->C; g.ldd = r; g.epi = EPI_STORE;
+          CK(launch_gemm_simt(e, e, e, g, s));
+          t.done(1);
+        }
       }
     }
-    {  // absorbed queries
+    {  // absorbed queries (+ per-user context term)
       StepTimer t(h, s, ST_Q);
-      GemmArgs g = {};
-      g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
-      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = hr; g.K = d;
-      g.epi = D.d_ctx > 0 ? EPI_USERBIAS : EPI_STORE;
-      g.bias = h->ctxbias; g.seg_off = p.qoff(l); g.B = B;
-      CK(launch_gemm_simt(e, e, e, g, s));
+      if (tc) {
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);
+        q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
+        q.bias = h->ctxbias; q.seg_off = p.qoff(l); q.B = B;
+        CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1], LM.qk,
+                          q, h->num_sms, s));
+      } else {
+        GemmArgs g = {};
+        g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
+        g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = hr; g.K = d;
+        g.epi = D.d_ctx > 0 ? EPI_USERBIAS : EPI_STORE;
+        g.bias = h->ctxbias; g.seg_off = p.qoff(l); g.B = B;
+        CK(launch_gemm_simt(e, e, e, g, s));
+      }
       t.done(1);
     }
     {  // latent attention
@@ -369,38 +466,51 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     }
     {  // output projection + residual + RMSNorm
       StepTimer t(h, s, ST_O);
-      GemmArgs g = {};
-      g.A = h->Ot; g.lda = hr; g.W = W.W_ov; g.D = h->acc32; g.ldd = d;
-      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = hr; g.epi = EPI_F32;
-      CK(launch_gemm_simt(e, e, 4, g, s));
-      NormArgs a = {};
-      a.acc = h->acc32; a.N = d; a.resid = Xq_l; a.g = W.g1; a.eps = D.eps;
-      a.M_dev = p.query_total(l); a.M_max = h->max_rows_q; a.mode = NORM_PLAIN; a.dst = h->Z;
-      CK(launch_rownorm(e, a, s));
-      t.done(2);
+      if (tc) {
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, hr);
+        q.norm = o_norm;
+        CK(launch_tc_gemm(h->bn_o, TC_NORM, h->tm_Ot, LM.ov, q, h->num_sms, s));
+        t.done(1);
+      } else {
+        GemmArgs g = {};
+        g.A = h->Ot; g.lda = hr; g.W = W.W_ov; g.D = h->acc32; g.ldd = d;
+        g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = hr; g.epi = EPI_F32;
+        CK(launch_gemm_simt(e, e, 4, g, s));
+        o_norm.acc = h->acc32;
+        CK(launch_rownorm(e, o_norm, s));
+        t.done(2);
+      }
     }
     {  // FFN up + SiLU
       StepTimer t(h, s, ST_FFN1);
-      GemmArgs g = {};
-      g.A = h->Z; g.lda = d; g.W = W.W1; g.D = h->Hd; g.ldd = f;
-      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = f; g.K = d; g.epi = EPI_SILU;
-      CK(launch_gemm_simt(e, e, e, g, s));
+      if (tc) {
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, f, d);
+        q.D = (__nv_bfloat16*)h->Hd; q.ldd = f;
+        CK(launch_tc_gemm(h->bn_f1, TC_SILU, h->tm_Z, LM.w1, q, h->num_sms, s));
+      } else {
+        GemmArgs g = {};
+        g.A = h->Z; g.lda = d; g.W = W.W1; g.D = h->Hd; g.ldd = f;
+        g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = f; g.K = d; g.epi = EPI_SILU;
+        CK(launch_gemm_simt(e, e, e, g, s));
+      }
       t.done(1);
     }
     {  // FFN down + residual + RMSNorm, scattered into the next layer's rows
       StepTimer t(h, s, ST_FFN2);
-      GemmArgs g = {};
-      g.A = h->Hd; g.lda = f; g.W = W.W2; g.D = h->acc32; g.ldd = d;
-      g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = f; g.epi = EPI_F32;
-      CK(launch_gemm_simt(e, e, 4, g, s));
-      NormArgs a = {};
-      a.acc = h->acc32; a.N = d; a.resid = h->Z; a.g = W.g2; a.eps = D.eps;
-      a.M_dev = p.query_total(l); a.M_max = h->max_rows_q; a.mode = NORM_SCATTER;
-      a.qoff_l = p.qoff(l); a.n_l = p.nl(l); a.hoff_n = p.hoff(l + 1); a.qoff_n = p.qoff(l + 1);
-      a.n_n = p.nl(l + 1); a.B = B; a.n_q = D.n_q; a.Xh_n = Xh_n; a.Xq_n = Xq_n; a.last = last;
-      a.out = out; a.final_rows = D.d_out ? h->final_rows : nullptr;
-      CK(launch_rownorm(e, a, s));
-      t.done(2);
+      if (tc) {
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, f);
+        q.norm = f_norm;
+        CK(launch_tc_gemm(h->bn_f2, TC_NORM, h->tm_Hd, LM.w2, q, h->num_sms, s));
+        t.done(1);
+      } else {
+        GemmArgs g = {};
+        g.A = h->Hd; g.lda = f; g.W = W.W2; g.D = h->acc32; g.ldd = d;
+        g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = d; g.K = f; g.epi = EPI_F32;
+        CK(launch_gemm_simt(e, e, 4, g, s));
+        f_norm.acc = h->acc32;
+        CK(launch_rownorm(e, f_norm, s));
+        t.done(2);
+      }
     }
   }
   if (D.d_out > 0) {

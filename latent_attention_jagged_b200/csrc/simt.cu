@@ -102,11 +102,18 @@ rownorm_kernel(NormArgs a) {
   if (m >= M) return;
   const int N = a.N;
   const float* row = a.acc + m * N;
-  const T* res = (const T*)a.resid;
+  const T* res = a.resid_f32 ? nullptr : (const T*)a.resid;
+  const float* res32 = a.resid_f32 ? (const float*)a.resid : nullptr;
   const T* g = (const T*)a.g;
+  auto val = [&](int c) {
+    float v = row[c];
+    if (res) v += to_f(res[m * N + c]);
+    if (res32) v += res32[m * N + c];
+    return v;
+  };
   float ss = 0.f;
   for (int c = lane; c < N; c += 32) {
-    float v = row[c] + (res ? to_f(res[m * N + c]) : 0.f);
+    float v = val(c);
     ss += v * v;
   }
   ss = warp_sum(ss);
@@ -115,8 +122,10 @@ rownorm_kernel(NormArgs a) {
   T* d1 = nullptr;
   T* d2 = nullptr;
   float* f1 = nullptr;
+  float* f2 = nullptr;
   if (a.mode == NORM_PLAIN) {
     d1 = (T*)a.dst + m * N;
+    if (a.dst32) f1 = a.dst32 + m * N;
   } else {
     const int u = segment_of(a.qoff_l, a.B, m);
     const int64_t j = m - a.qoff_l[u];
@@ -126,20 +135,25 @@ rownorm_kernel(NormArgs a) {
       else if (j >= nl) f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
     } else {
       const int32_t nn = a.n_n[u];
+      int64_t q = -1;
       if (j < nl) {
         d1 = (T*)a.Xh_n + (a.hoff_n[u] + j) * N;
-        if (j >= nl - nn) d2 = (T*)a.Xq_n + (a.qoff_n[u] + j - (nl - nn)) * N;
+        if (j >= nl - nn) q = a.qoff_n[u] + j - (nl - nn);
       } else {
-        d2 = (T*)a.Xq_n + (a.qoff_n[u] + nn + (j - nl)) * N;
+        q = a.qoff_n[u] + nn + (j - nl);
+      }
+      if (q >= 0) {
+        d2 = (T*)a.Xq_n + q * N;
+        if (a.Xq32_n) f2 = a.Xq32_n + q * N;
       }
     }
   }
   for (int c = lane; c < N; c += 32) {
-    float v = row[c] + (res ? to_f(res[m * N + c]) : 0.f);
-    float y = v * inv * to_f(g[c]);
+    float y = val(c) * inv * to_f(g[c]);
     if (d1) d1[c] = from_f<T>(y);
     if (d2) d2[c] = from_f<T>(y);
     if (f1) f1[c] = y;
+    if (f2) f2[c] = y;
   }
 }
 

@@ -1,0 +1,31 @@
+// Interface of the tensor-core (tcgen05) kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace llatte {
+
+enum { TC_STORE = 0, TC_USERBIAS = 1, TC_SILU = 2, TC_NORM = 3 };
+
+struct TcGemmParams {
+  int64_t M_host;               // rows, unless M_dev != NULL
+  const int64_t* M_dev;
+  int64_t M_cap;                // largest M (sizes the grid)
+  int N, K;
+  __nv_bfloat16* D; int64_t ldd;                      // STORE / USERBIAS / SILU
+  const float* bias; const int64_t* seg_off; int B;   // USERBIAS: bias[user(row), n]
+  NormArgs norm;                                       // NORM (acc unused)
+  int32_t* status;
+};
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+bool tc_gemm_supported(int BN, int epi, int N, int K);
+cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
+                           const TcGemmParams& p, int num_sms, cudaStream_t s);
+
+}  // namespace llatte
