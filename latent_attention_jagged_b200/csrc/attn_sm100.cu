@@ -1,0 +1,408 @@
+// Fused latent attention for sm_100a (MLA as multi-query attention in the
+// rank-r latent space, LLaTTE notes, huaxiaozhuan.com, appendix A.3; target-
+// aware causal / candidate masking of appendix A.2 and the daiwk.github.io
+// "core formula").
+//
+// One work item = one user u and a block of 128 (query row, head) pairs of
+// that user (q~ rows of [sum q * h, r], heads interleaved, so all heads of a
+// query row share its mask).  Keys and values are the same latent rows c_kv
+// of the user's current history: S = Q~ C^T and O~ = softmax(S) C both read
+// one shared-memory copy of each C tile (K-major for S, MN-major for P V).
+//
+// Roles (192 threads, one CTA per SM, persistent over the sorted work list):
+//   warp 0      TMA: the Q~ block once per item, C tiles into a KV_STAGES ring
+//   warp 1      TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
+//               O += P(kt) C_kt, so the tensor pipe works while the softmax
+//               warps turn S(kt) into P(kt)
+//   warps 2..5  softmax, one TMEM lane (= one pair) per thread: masking
+//               (history row at position p sees keys t <= p; a query token
+//               sees every key t < T), online max / sum in fp32, P written to
+//               shared memory as bf16, lazy rescaling of O in TMEM (only when
+//               the running max grows by more than 2^8), final O / l to HBM.
+// TMEM: O in columns [0, r), S double-buffered after it.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_attn.h"
+#include "tc_common.cuh"
+
+namespace llatte {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kThreads = 192;
+
+template <int R>
+struct AttnCfg {
+  static constexpr int KEYS = R >= 256 ? 64 : 128;     // keys per tile
+  static constexpr int RSUB = R / 64;                  // 64-wide latent sub-tiles
+  static constexpr int KV_STAGES = 4;
+  static constexpr uint32_t Q_BYTES = 128 * R * 2;
+  static constexpr uint32_t KV_BYTES = KEYS * R * 2;
+  static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
+  static constexpr uint32_t P_BYTES = 128 * KEYS * 2;
+  static constexpr uint32_t S_COL = R;                  // S buffers after O
+  static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(R + 2 * KEYS <= 512, "TMEM budget");
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+struct Item {
+  int u, b;
+  int64_t T, n, q, hoff, qoff;
+  int nk;         // key tiles
+};
+
+__device__ __forceinline__ Item load_item(const AttnTcParams& p, int idx, int keys) {
+  Item it;
+  it.u = p.work[2 * idx];
+  it.b = p.work[2 * idx + 1];
+  it.T = p.T[it.u];
+  it.n = p.n[it.u];
+  it.q = it.n + p.n_q;
+  it.hoff = p.hoff[it.u];
+  it.qoff = p.qoff[it.u];
+  const int64_t last = min((int64_t)it.b * 128 + 127, it.q * p.heads - 1);
+  const int64_t jl = last / p.heads;
+  const int64_t kmax = jl < it.n ? it.T - it.n + jl + 1 : it.T;
+  it.nk = (int)((kmax + keys - 1) / keys);
+  return it;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
+               const AttnTcParams p) {
+  using Cfg = AttnCfg<R>;
+  constexpr int KEYS = Cfg::KEYS, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + Cfg::Q_BYTES;
+  uint8_t* sP = sKV + KS * Cfg::KV_BYTES;
+  uint64_t* bars = (uint64_t*)(sP + 2 * Cfg::P_BYTES);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;            // [KS]
+  uint64_t* kv_empty = kv_full + KS;       // [KS]
+  uint64_t* s_full = kv_empty + KS;        // [2]
+  uint64_t* s_empty = s_full + 2;          // [2]
+  uint64_t* p_full = s_empty + 2;          // [2]
+  uint64_t* p_empty = p_full + 2;          // [2]
+  uint64_t* o_free = p_empty + 2;
+  uint64_t* drain = o_free + 1;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = *p.work_count;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 4);
+      mbar_init(&p_full[s], 4);
+      mbar_init(&p_empty[s], 1);
+    }
+    mbar_init(o_free, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t itm = 0, g = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const Item it = load_item(p, idx, KEYS);
+        if (it.nk == 0) continue;
+        if (!mbar_wait(q_empty, (itm & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(q_full, Cfg::Q_BYTES);
+        const int32_t qrow = (int32_t)(it.qoff * p.heads + (int64_t)it.b * 128);
+#pragma unroll
+        for (int s = 0; s < RSUB; ++s) tma_load_2d(&tmQ, q_full, sQ + s * 16384, s * 64, qrow);
+        for (int kt = 0; kt < it.nk; ++kt, ++g) {
+          const int st = g % KS;
+          if (!mbar_wait(&kv_empty[st], ((g / KS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[st], Cfg::KV_BYTES);
+          const int32_t krow = (int32_t)(it.hoff + (int64_t)kt * KEYS);
+          uint8_t* dst = sKV + st * Cfg::KV_BYTES;
+#pragma unroll
+          for (int s = 0; s < RSUB; ++s)
+            tma_load_2d(&tmC, &kv_full[st], dst + s * Cfg::KV_SUB_BYTES, s * 64, krow);
+        }
+        ++itm;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(128, KEYS, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16(128, R, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      uint32_t itm = 0, g = 0;
+      bool ok = true;
+      auto issue_s = [&](uint32_t gg) -> bool {
+        const int st = gg % KS;
+        if (!mbar_wait(&kv_full[st], (gg / KS) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(&s_empty[gg & 1], ((gg >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);
+        const uint32_t d = tmem + Cfg::S_COL + (gg & 1) * KEYS;
+#pragma unroll
+        for (int k = 0; k < R / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(q_addr + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              sdesc_sw128(kv_addr + (k >> 2) * Cfg::KV_SUB_BYTES + (k & 3) * 32, 16, 1024);
+          umma_bf16(d, ad, bd, IDESC_S, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[gg & 1]);
+        return true;
+      };
+      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+        if (!mbar_wait(&p_full[gg & 1], (gg >> 1) & 1, abort_flag, p.status)) return false;
+        if (first && !mbar_wait(o_free, (itm & 1) ^ 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const int st = gg % KS;
+        const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);
+        const uint32_t p_addr = smem_u32(sP + (gg & 1) * Cfg::P_BYTES);
+#pragma unroll
+        for (int k = 0; k < KEYS / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(p_addr + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          // V = the same C tile read MN-major: 64-wide latent blocks are the
+          // sub-tiles (LBO apart), 16 keys per MMA step = 2048 bytes
+          const uint64_t bd = sdesc_sw128(kv_addr + k * 2048, Cfg::KV_SUB_BYTES, 1024);
+          umma_bf16(tmem, ad, bd, IDESC_O, (!first || k > 0) ? 1u : 0u);
+        }
+        // one commit per barrier: the C tile and the P buffer are free, and
+        // (through p_empty) the softmax warps learn that PV(gg) is in O
+        umma_commit(&kv_empty[st]);
+        umma_commit(&p_empty[gg & 1]);
+        return true;
+      };
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+        const Item it = load_item(p, idx, KEYS);
+        if (it.nk == 0) continue;
+        if (!mbar_wait(q_full, itm & 1, abort_flag, p.status)) break;
+        const uint32_t g0 = g;
+        for (int kt = 0; kt < it.nk; ++kt) {
+          if (!issue_s(g0 + kt)) { ok = false; break; }
+          if (kt == it.nk - 1) umma_commit(q_empty);
+          if (kt > 0 && !issue_pv(g0 + kt - 1, kt - 1 == 0)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!issue_pv(g0 + it.nk - 1, it.nk == 1)) break;
+        g += it.nk;
+        ++itm;
+      }
+      umma_commit(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, &dummy, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;              // pair within the block = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const float kLog2e = 1.4426950408889634f;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
+      const Item it = load_item(p, idx, KEYS);
+      const int64_t pair = (int64_t)it.b * 128 + row;
+      const bool valid = pair < it.q * p.heads;
+      const int64_t jl = pair / p.heads;
+      const int64_t vis = !valid ? 0 : (jl < it.n ? it.T - it.n + jl + 1 : it.T);
+      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R;
+      if (it.nk == 0) {
+        if (valid) {
+          uint4 z = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < R; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+        }
+        continue;
+      }
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
+      for (int kt = 0; kt < it.nk; ++kt, ++g) {
+        // ---- S tile -> registers
+        bool w = mbar_wait(&s_full[g & 1], (g >> 1) & 1, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        float s[KEYS];
+#pragma unroll
+        for (int c = 0; c < KEYS; c += 32) {
+          float v[32];
+          tmem_ld32(lane_base + Cfg::S_COL + (g & 1) * KEYS + c, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c + i] = v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[g & 1]);
+        // ---- mask and tile max (log2 domain)
+        const int64_t t0 = (int64_t)kt * KEYS;
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < KEYS; ++c) {
+          s[c] = (t0 + c < vis) ? s[c] * kLog2e : -INFINITY;
+          mt = fmaxf(mt, s[c]);
+        }
+        // ---- lazy rescale of O and l (only when the max grows by > 8 in log2)
+        float scale = 1.f;
+        bool resc = false;
+        if (kt == 0) {
+          m_run = mt;
+        } else if (mt > m_run + 8.f) {
+          scale = ex2(m_run - mt);
+          m_run = mt;
+          resc = true;
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // PV(g-1) must have landed in O before O is touched.  Its completion
+          // is the next phase of p_empty[(g-1)&1]: that barrier cannot run a
+          // phase further ahead because PV(g+1) needs P(g+1), not written yet.
+          bool w2 = mbar_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, p.status);
+          if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < R; c += 32) {
+            float v[32];
+            tmem_ld32(lane_base + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= scale;
+            tmem_st32(lane_base + c, v);
+          }
+          l_run *= scale;
+        }
+        // ---- probabilities
+        const bool live = m_run > -INFINITY;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < KEYS; ++c) {
+          const float e = (live && s[c] > -INFINITY) ? ex2(s[c] - m_run) : 0.f;
+          s[c] = e;
+          lsum += e;
+        }
+        l_run += lsum;
+        // ---- P tile -> shared memory (bf16, 128-byte swizzled, K-major)
+        bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
+        const uint32_t pbase = smem_u32(sP + (g & 1) * Cfg::P_BYTES);
+#pragma unroll
+        for (int ch = 0; ch < KEYS / 8; ++ch) {
+          const int sub = ch >> 3, cc = ch & 7;
+          const uint32_t addr = pbase + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+          uint4 v = make_uint4(pack_bf16(s[8 * ch], s[8 * ch + 1]), pack_bf16(s[8 * ch + 2], s[8 * ch + 3]),
+                               pack_bf16(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
+          st_shared_v4(addr, v);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[g & 1]);
+      }
+      if (!ok) break;
+      // ---- final: O / l -> HBM, once the last PV(g-1) has completed
+      bool w4 = mbar_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w4)) break;
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < R; c += 32) {
+        float v[32];
+        tmem_ld32(lane_base + c, v);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(pack_bf16(v[8 * j] * inv, v[8 * j + 1] * inv),
+                                pack_bf16(v[8 * j + 2] * inv, v[8 * j + 3] * inv),
+                                pack_bf16(v[8 * j + 4] * inv, v[8 * j + 5] * inv),
+                                pack_bf16(v[8 * j + 6] * inv, v[8 * j + 7] * inv));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+template <int R>
+cudaError_t launch_r(const CUtensorMap& q, const CUtensorMap& c, const AttnTcParams& p, int grid,
+                     cudaStream_t s) {
+  using Cfg = AttnCfg<R>;
+  static uint64_t attr_devices = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_devices >> (dev & 63) & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_devices |= 1ull << (dev & 63);
+  }
+  attn_tc_kernel<R><<<grid, kThreads, Cfg::SMEM, s>>>(q, c, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_tc_keys(int r) { return r >= 256 ? 64 : 128; }
+
+bool attn_tc_supported(int r) { return r == 64 || r == 128 || r == 256; }
+
+cudaError_t launch_attn_tc(int r, const CUtensorMap& q, const CUtensorMap& c,
+                           const AttnTcParams& p, int num_sms, cudaStream_t s) {
+  const int grid = std::max(1, std::min(num_sms, p.max_items));
+  switch (r) {
+    case 64: return launch_r<64>(q, c, p, grid, s);
+    case 128: return launch_r<128>(q, c, p, grid, s);
+    case 256: return launch_r<256>(q, c, p, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace llatte

@@ -92,6 +92,8 @@ struct llatte_handle {
   CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd;
   llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
   int bn_kv, bn_q, bn_o, bn_f1, bn_f2;
+  int attn_keys;                  // keys per attention tile (tensor-core path)
+  CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
 
   // profiling
   int profiling;

@@ -59,7 +59,7 @@ __device__ void block_exscan2(int64_t a, int64_t b, int64_t* out_a, int64_t* out
 
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep, int L, int n_q,
-            int64_t max_len, int64_t max_total) {
+            int64_t max_len, int64_t max_total, int heads, int attn_keys) {
   __shared__ int s_err;
   const int tid = threadIdx.x;
   if (tid == 0) s_err = 0;
@@ -118,6 +118,54 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
       p.totals[2 * l + 1] = totQ;
     }
   }
+  if (attn_keys <= 0) return;
+
+  // Attention work lists: one item per (user, block of 128 (query row, head)
+  // pairs), ordered by the number of key tiles the block visits, largest
+  // first (a counting sort over at most kBuckets cost classes), so that the
+  // persistent attention CTAs take the longest items first.
+  constexpr int kBuckets = 64;
+  __shared__ int32_t hist[kBuckets], cursor[kBuckets];
+  __shared__ int32_t total_items;
+  for (int l = 0; l < L; ++l) {
+    const int32_t* Tl = p.T + l * bstride;
+    const int32_t* nl = p.n + l * bstride;
+    if (tid < kBuckets) hist[tid] = 0;
+    __syncthreads();
+    auto cost_of = [&](int u, int b) {
+      const int64_t q = (int64_t)nl[u] + n_q;
+      const int64_t last = min((int64_t)b * 128 + 127, q * heads - 1);
+      const int64_t jl = last / heads;
+      const int64_t kmax = jl < nl[u] ? (int64_t)Tl[u] - nl[u] + jl + 1 : (int64_t)Tl[u];
+      const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
+      return (int)min<int64_t>(tiles, kBuckets - 1);
+    };
+    for (int u = u0; u < u1; ++u) {
+      const int64_t items = (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+      for (int b = 0; b < items; ++b) atomicAdd(&hist[cost_of(u, b)], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int32_t acc = 0;
+      for (int k = kBuckets - 1; k >= 0; --k) { cursor[k] = acc; acc += hist[k]; }
+      total_items = acc;
+    }
+    __syncthreads();
+    int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
+    for (int u = u0; u < u1; ++u) {
+      const int64_t items = (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+      for (int b = 0; b < items; ++b) {
+        const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
+        W[2 * pos] = u;
+        W[2 * pos + 1] = b;
+      }
+    }
+    if (tid == 0) {
+      p.work_count[l] = total_items;
+      p.work_next[l] = 0;
+    }
+    __syncthreads();
+  }
 }
 
 cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, cudaStream_t s) {
@@ -125,7 +173,7 @@ cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, c
   const int L = h->dims.n_layers;
   for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < L ? h->dims.keep[i] : 0;
   plan_kernel<<<1, kPlanThreads, 0, s>>>(offsets, B, h->plan, k, L, h->dims.n_q, h->dims.max_len,
-                                          h->max_rows_h);
+                                          h->max_rows_h, h->dims.heads, h->use_tc ? h->attn_keys : 0);
   return cudaGetLastError();
 }
 

@@ -7,6 +7,7 @@
 #include <new>
 
 #include "internal.h"
+#include "tc_attn.h"
 #include "tc_gemm.h"
 
 using namespace llatte;
@@ -169,7 +170,7 @@ int drain_profile(llatte_handle* h) {
 bool tc_dims_ok(const llatte_dims& D) {
   const int hr = D.heads * D.rank, f = D.ffn_mult * D.d;
   const bool d_ok = D.d == 64 || D.d == 128 || D.d == 256 || D.d == 512;
-  const bool r_ok = D.rank == 64 || D.rank == 128 || D.rank == 256;
+  const bool r_ok = attn_tc_supported(D.rank);
   return d_ok && r_ok && hr % 64 == 0 && f % 64 == 0;
 }
 
@@ -192,6 +193,9 @@ bool build_tc_maps(llatte_handle* h) {
   ok = ok && make_tmap_bf16(&h->tm_Ot, h->Ot, rq, hr, 128);
   ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
+  h->attn_keys = attn_tc_keys(r);
+  ok = ok && make_tmap_bf16(&h->tm_Qt, h->Qt, rq * D.heads, r, 128);
+  ok = ok && make_tmap_bf16(&h->tm_C, h->C, rh, r, (uint32_t)h->attn_keys);
   auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
   for (int l = 0; l < D.n_layers && ok; ++l) {
     const LayerDev& W = h->layers[l];
@@ -455,7 +459,16 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       }
       t.done(1);
     }
-    {  // latent attention
+    if (tc) {  // latent attention, tensor cores
+      StepTimer t(h, s, ST_ATTN);
+      AttnTcParams a = {};
+      a.work = p.work + (int64_t)l * 2 * p.max_work; a.work_count = p.work_count + l;
+      a.max_items = p.max_work; a.T = p.Tl(l); a.n = p.nl(l); a.hoff = p.hoff(l);
+      a.qoff = p.qoff(l); a.n_q = D.n_q; a.heads = D.heads; a.Ot = (__nv_bfloat16*)h->Ot;
+      a.status = p.status;
+      CK(launch_attn_tc(r, h->tm_Qt, h->tm_C, a, h->num_sms, s));
+      t.done(1);
+    } else {  // latent attention, CUDA cores
       StepTimer t(h, s, ST_ATTN);
       AttnArgs a = {};
       a.Qt = h->Qt; a.C = h->C; a.Ot = h->Ot; a.qoff = p.qoff(l); a.hoff = p.hoff(l);
