@@ -138,7 +138,7 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
       const int64_t jl = last / heads;
       const int64_t kmax = jl < nl[u] ? (int64_t)Tl[u] - nl[u] + jl + 1 : (int64_t)Tl[u];
       const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
-      return (int)min<int64_t>(tiles, kBuckets - 1);
+      return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
     };
     for (int u = u0; u < u1; ++u) {
       const int64_t items = (((int64_t)nl[u] + n_q) * heads + 127) / 128;
