@@ -52,12 +52,6 @@ struct AttnCfg {
   static_assert(R + 2 * KEYS <= 512, "TMEM budget");
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -290,7 +284,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (kt == 0) {
           m_run = mt;
         } else if (mt > m_run + 8.f) {
-          scale = ex2(m_run - mt);
+          scale = ex2_approx(m_run - mt);
           m_run = mt;
           resc = true;
         }
@@ -316,7 +310,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         float lsum = 0.f;
 #pragma unroll
         for (int c = 0; c < KEYS; ++c) {
-          const float e = (live && s[c] > -INFINITY) ? ex2(s[c] - m_run) : 0.f;
+          const float e = (live && s[c] > -INFINITY) ? ex2_approx(s[c] - m_run) : 0.f;
           s[c] = e;
           lsum += e;
         }

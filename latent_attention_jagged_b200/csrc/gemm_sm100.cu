@@ -181,7 +181,7 @@ __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, 
         if (EPI == TC_USERBIAS) add_f32x32(p.bias + (int64_t)u * p.N + n, v);
         if (EPI == TC_SILU) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]);
+          for (int i = 0; i < 32; ++i) v[i] = silu_approx(v[i]);
         }
         store_bf16x32(p.D + row * p.ldd + n, v);
       }
