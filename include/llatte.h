@@ -174,6 +174,35 @@ int llatte_profile_reset(llatte_handle* handle);
 int llatte_profile_step(llatte_handle* handle, int step, const char** name, double* total_ms,
                         int64_t* kernel_launches, int64_t* calls);
 
+/*
+ * The pyramid plan of one batch computed without allocating any device
+ * memory, for callers that cannot call cudaMalloc where they need it (code
+ * running under another framework's memory pool or allocator hook, or with
+ * all device memory reserved up front).  It needs no handle.  The paper has
+ * no counterpart of this call: it only serves such callers.
+ *
+ *   dims       host; uses n_layers, keep[], n_q, max_batch, max_len, max_total
+ *   offsets    device int64 [B+1], as for llatte_forward
+ *   B          0 <= B <= min(dims->max_batch, LLATTE_PLAN_STATIC_MAX_BATCH)
+ *   plan_out   device int64 [n_layers][2][B+1]: the same values and layout as
+ *              llatte_plan_export after llatte_forward on this batch
+ *   status_out device int32: 0, or the LLATTE_DEV_* bits of a rejected batch
+ *              (then plan_out holds zeros)
+ *
+ * Its scratch is one fixed device array of about 1.7 MB inside the library,
+ * held on every GPU that loads the library until the process exits.  A batch
+ * larger than LLATTE_PLAN_STATIC_MAX_BATCH users returns
+ * LLATTE_ERR_UNSUPPORTED without launching anything.  The first call on a
+ * device looks up that array's device address (with the device current);
+ * make the first call before any stream capture.  Every call on a device
+ * shares the array: calls that can run at the same time on the GPU race, so
+ * order them (one stream, or synchronise in between).  Asynchronous on
+ * `stream`; it calls no cudaMalloc or cudaFree.
+ */
+#define LLATTE_PLAN_STATIC_MAX_BATCH 4096
+int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t B,
+                       int64_t* plan_out, int32_t* status_out, void* stream);
+
 /* Free the handle and everything it owns (synchronises its device). */
 void llatte_destroy(llatte_handle* handle);
 

@@ -47,7 +47,9 @@ class llatte_layer_w(ctypes.Structure):
 
 EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
-           "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step")
+           "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
+           "llatte_plan_static")
+PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
 
@@ -84,6 +86,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_profile_step.argtypes = [VP, ctypes.c_int, P(ctypes.c_char_p),
                                         P(ctypes.c_double), P(I64), P(I64)]
     lib.llatte_profile_step.restype = ctypes.c_int
+    lib.llatte_plan_static.argtypes = [P(llatte_dims), VP, I32, VP, VP, VP]
+    lib.llatte_plan_static.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -244,3 +248,28 @@ class Llatte:
             self.close()
         except Exception:
             pass
+
+
+def plan_static(dims, offsets: torch.Tensor, max_batch: int, max_len: int, max_total: int = 0,
+                stream=None, out: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None):
+    """Pyramid plan of one batch through llatte_plan_static, the entry point
+    that allocates no device memory (its scratch is a fixed array inside the
+    library).  Pass `out` / `status` to reuse caller-owned buffers.  Returns
+    (plan [n_layers, 2, B+1] int64, status int32 tensor)."""
+    lib = load_library()
+    cd = make_dims(dims, max_batch, max_len, max_total)
+    B = int(offsets.numel()) - 1
+    if not offsets.is_cuda or offsets.dtype != torch.int64 or not offsets.is_contiguous():
+        raise ValueError("offsets must be a contiguous CUDA int64 tensor")
+    if out is None:
+        out = torch.empty((len(dims.keep), 2, B + 1), dtype=torch.int64, device=offsets.device)
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=offsets.device)
+    if tuple(out.shape) != (len(dims.keep), 2, B + 1) or out.dtype != torch.int64:
+        raise ValueError("out must be int64 [n_layers, 2, B+1]")
+    rc = lib.llatte_plan_static(ctypes.byref(cd), _ptr(offsets), B, _ptr(out), _ptr(status),
+                                _stream_ptr(stream))
+    if rc != LLATTE_OK:
+        raise LlatteError(rc, "llatte_plan_static")
+    return out, status

@@ -108,6 +108,9 @@ namespace llatte {
 
 // ---- launchers (each returns cudaGetLastError()) ----
 cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, cudaStream_t s);
+// The plan kernel on caller-described storage (no work lists).
+cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_total,
+                           const int64_t* offsets, int B, cudaStream_t s);
 cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
                           const void* cand, int B, cudaStream_t s);
 

@@ -177,6 +177,15 @@ cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_total,
+                           const int64_t* offsets, int B, cudaStream_t s) {
+  KeepArr k;
+  for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < d.n_layers ? d.keep[i] : 0;
+  plan_kernel<<<1, kPlanThreads, 0, s>>>(offsets, B, p, k, d.n_layers, d.n_q, d.max_len,
+                                          max_total, d.heads, 0);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- gather
 
 __global__ void __launch_bounds__(256)
