@@ -7,9 +7,9 @@ One step = one whole forward pass (plan, gather, every layer's KV latent,
 absorbed queries, latent attention, output projection + norm, FFN + norm,
 readout) over one batch of the workload, inputs resident in HBM.  L2 is
 flushed (a 256 MiB write) before every timed step, outside the timed events.
-Multi-GPU: one process per GPU, each rank runs its own batch (users are
-independent, no collective on the data path): weak scaling.  Rank 0 prints
-one JSON line.
+Multi-GPU: one process per GPU; a global batch of N x B users is split by
+user (longest-processing-time first on per-user FLOPs), weights replicated,
+no collective on the data path: weak scaling.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only reference there is) on
 the host cores, each step a bounded sample of the same workload.
@@ -29,7 +29,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import make_inputs, workload  # noqa: E402
+from workloads import draw_lengths, make_inputs, workload  # noqa: E402
+from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 
 # ncu-measured DRAM traffic per launch (bytes) of the dominant kernel, keyed by
 # (kernel, workload); filled from the committed profiles/ summaries.  None =
@@ -171,6 +172,8 @@ def main():
                     help="second workload measured in the same run ('' = none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch every kernel eagerly instead of replaying one CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -210,8 +213,24 @@ def main():
     peaks = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
+    def rank_inputs(wl):
+        """N = 1: the workload's batch.  N > 1: one global batch of N x B users
+        (lengths from the workload's law), split by LPT on per-user FLOPs; each
+        rank draws the tokens of its own users, all ranks share the weights."""
+        if world == 1:
+            return make_inputs(wl)
+        rng = np.random.Generator(np.random.PCG64(wl.seed))
+        lengths = draw_lengths(wl.lengths, wl.batch * world, rng)
+        offsets = np.zeros(lengths.shape[0] + 1, dtype=np.int64)
+        np.cumsum(lengths, out=offsets[1:])
+        shard = shard_batch(offsets, wl.dims, world)[rank]
+        inp = make_inputs(wl, lengths=lengths[shard.users], seed=wl.seed + 1000 + rank)
+        shared = make_inputs(wl, lengths=np.zeros(1, dtype=np.int64), seed=wl.seed)
+        inp.layers, inp.W_e = shared.layers, shared.W_e
+        return inp
+
     def measure(wl, steps, warmup, sample_clocks):
-        inp = make_inputs(wl, seed=wl.seed + 1000 * rank)
+        inp = rank_inputs(wl)
         dt = torch.bfloat16 if inp.dims.dtype == "bf16" else torch.float32
         h = Llatte(inp.dims, inp.layers, inp.W_e, max_batch=inp.batch,
                    max_len=int(inp.lengths.max()))
@@ -225,6 +244,20 @@ def main():
             h.forward(values, offsets, ctx, cand, out=out)
         torch.cuda.synchronize()
         assert h.status() == 0, "device status word set during warm-up"
+        # the whole forward as one CUDA graph (no host work between kernels)
+        graph = None
+        if args.graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                h.forward(values, offsets, ctx, cand, out=out)
+            graph.replay()
+            torch.cuda.synchronize()
+
+        def step():
+            if graph is not None:
+                graph.replay()
+            else:
+                h.forward(values, offsets, ctx, cand, out=out)
 
         # ---- device-resident timing
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -237,15 +270,19 @@ def main():
         for a, b in ev:
             flush.fill_(1)
             a.record(stream)
-            h.forward(values, offsets, ctx, cand, out=out)
+            step()
             b.record(stream)
         torch.cuda.synchronize()
         barrier()
         clocks = sampler.stop() if sampler else None
         ms = sum(a.elapsed_time(b) for a, b in ev)
         ms = max_over_ranks(ms)
-        users = world * inp.batch * steps
-        value = users / (ms / 1e3)
+        users_all = inp.batch
+        if world > 1:
+            t = torch.tensor([inp.batch], dtype=torch.int64, device="cuda")
+            dist.all_reduce(t)
+            users_all = int(t.item())
+        value = users_all * steps / (ms / 1e3)
 
         # ---- per-step timing (same loop, profiling events inside the library)
         h.profile_reset()
@@ -279,7 +316,7 @@ def main():
                 ctx.copy_(hc, non_blocking=True)
             if hq is not None:
                 cand.copy_(hq, non_blocking=True)
-            h.forward(values, offsets, ctx, cand, out=out)
+            step()
             hout.copy_(out, non_blocking=True)
             b.record(stream)
         torch.cuda.synchronize()
@@ -288,7 +325,7 @@ def main():
         h2d = hv.numel() * hv.element_size() + ho.numel() * 8 + \
             (hc.numel() * hc.element_size() if hc is not None else 0) + \
             (hq.numel() * hq.element_size() if hq is not None else 0)
-        e2e = {"value": world * inp.batch * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
+        e2e = {"value": users_all * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4)}
         assert h.status() == 0
 
@@ -312,7 +349,8 @@ def main():
         steps_ms = {k: round(v["ms"] / prof_steps, 4) for k, v in prof.items() if v["calls"]}
         res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
                    clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
-                   dtype=inp.dims.dtype)
+                   dtype=inp.dims.dtype, users_all=users_all)
+        del graph
         h.close()
         return res
 
@@ -337,10 +375,11 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": main_res["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": main_res["dtype"], "data": "synthetic",
-            "config": {"workload": wl.name, "global_batch": inp.batch * world,
+            "config": {"workload": wl.name, "global_batch": main_res["users_all"],
                        "seq_len": list(wl.lengths), "d": inp.dims.d, "layers": inp.dims.n_layers,
-                       "parallelism": f"users sharded, dp{world}",
-                       "l2": "flushed (256 MiB write) before every timed step"},
+                       "parallelism": f"users sharded by LPT on FLOPs, dp{world}",
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "launch": "one CUDA graph replay per step" if args.graph else "eager"},
             "roofline": main_res["roofline"],
             "whole_step": main_res["whole"],
             "cpu_baseline": cpu,

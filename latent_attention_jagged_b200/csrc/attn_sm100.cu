@@ -236,7 +236,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int quad = warp & 3;
     const int row = quad * 32 + lane;              // pair within the block = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const float kLog2e = 1.4426950408889634f;
     uint32_t g = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
@@ -270,14 +269,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[g & 1]);
-        // ---- mask and tile max (log2 domain)
+        // ---- mask (only on tiles this row does not see entirely) and tile
+        // max; scores are already in log2 units (log2 e folded into q~)
         const int64_t t0 = (int64_t)kt * KEYS;
-        float mt = -INFINITY;
+        if (t0 + KEYS > vis) {
+          const int64_t lim = vis - t0;
 #pragma unroll
-        for (int c = 0; c < KEYS; ++c) {
-          s[c] = (t0 + c < vis) ? s[c] * kLog2e : -INFINITY;
-          mt = fmaxf(mt, s[c]);
+          for (int c = 0; c < KEYS; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
         }
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < KEYS; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
+        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         // ---- lazy rescale of O and l (only when the max grows by > 8 in log2)
         float scale = 1.f;
         bool resc = false;
@@ -305,16 +313,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           l_run *= scale;
         }
-        // ---- probabilities
-        const bool live = m_run > -INFINITY;
-        float lsum = 0.f;
+        // ---- probabilities: 2^(s - m); masked scores are -inf and give 0.  A
+        // row that sees no key at all keeps m = -inf: subtract 0 instead so
+        // that -inf - (-inf) never happens.
+        const float m_use = m_run > -INFINITY ? m_run : 0.f;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < KEYS; ++c) {
-          const float e = (live && s[c] > -INFINITY) ? ex2_approx(s[c] - m_run) : 0.f;
-          s[c] = e;
-          lsum += e;
-        }
-        l_run += lsum;
+        for (int c = 0; c < KEYS; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s[c + i] = ex2_approx(s[c + i] - m_use);
+            l8[i] += s[c + i];
+          }
+        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         // ---- P tile -> shared memory (bf16, 128-byte swizzled, K-major)
         bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }

@@ -1,18 +1,21 @@
 // Tensor-core GEMM for sm_100a: D[m, n] = sum_k A[m, k] W[n, k] (bf16 in,
 // fp32 accumulation in TMEM) with the layer's epilogues fused.
 //
-// Roles (192 threads, one CTA per SM, persistent over 128 x BN tiles):
+// Roles (320 threads, one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: A (128 x 64) and W (BN x 64) k-blocks into a
 //               STAGES-deep ring of 128-byte-swizzled shared-memory tiles
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (128 x NI x 16) and
 //               commits stage releases / accumulator-ready events
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), then one of
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant, each taking half
+//               of the tile's columns: TMEM -> registers (tcgen05.ld), then one of
 //               STORE     bf16 store
 //               USERBIAS  + per-user context term (absorbed query projection)
 //               SILU      SiLU (FFN up-projection)
-//               NORM      + residual, RMSNorm over the full row (BN == N),
-//                         store bf16 (+ fp32 copy) or scatter into the next
-//                         layer's history / query rows (pyramid trimming)
+//               NORM      + residual (read once: the sum is staged back in
+//                         TMEM), RMSNorm over the full row (BN == N; the two
+//                         halves' sums of squares meet in shared memory),
+//                         store bf16 (+ fp16 residual copy) or scatter into the
+//                         next layer's history / query rows (pyramid trimming)
 // The accumulator is double-buffered in TMEM when 2 * BN <= 512 columns, so
 // the epilogue of tile i overlaps the MMAs of tile i + 1.
 //
@@ -20,6 +23,7 @@
 // KV latent RMSNorm(X W_down^KV); absorbed query X (W_uk^T W_q)^T + context
 // term; Z = RMSNorm(R + o~ (W_o W_uv)^T); FFN W2 SiLU(W1 Z) + Z, RMSNorm.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 
@@ -35,6 +39,8 @@ using namespace tc;
 namespace {
 
 constexpr int BM = 128, BK = 64;
+constexpr int kEpiWarps = 8;                        // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 template <int BN>
 struct GemmCfg {
@@ -48,7 +54,7 @@ struct GemmCfg {
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 512 ? 2 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4;
 };
 
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
@@ -89,47 +95,82 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
   for (int j = 0; j < 8; ++j) d[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
-// Residual chunk for columns [c, c + 32) of `row`, added to v.
-__device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N, int c,
-                                          float (&v)[32]) {
-  if (!a.resid) return;
-  if (a.resid_f32) {
-    add_f32x32((const float*)a.resid + row * N + c, v);
-  } else {
-    float r[32];
-    load_bf16x32((const __nv_bfloat16*)a.resid + row * N + c, r);
+__device__ __forceinline__ void load_f16x32(const __half* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] += r[i];
+  for (int j = 0; j < 4; ++j) {
+    uint4 w = __ldg(s + j);
+    const __half2* h = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float2 f = __half22float2(h[k]);
+      v[8 * j + 2 * k] = f.x;
+      v[8 * j + 2 * k + 1] = f.y;
+    }
   }
 }
 
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void store_f16x32(__half* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    d[j] = make_uint4(pack_f16(v[8 * j], v[8 * j + 1]), pack_f16(v[8 * j + 2], v[8 * j + 3]),
+                      pack_f16(v[8 * j + 4], v[8 * j + 5]), pack_f16(v[8 * j + 6], v[8 * j + 7]));
+}
+
+// Residual chunk for columns [c, c + 32) of `row`, added to v (bf16 or fp16).
+__device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N, int c,
+                                          float (&v)[32]) {
+  if (!a.resid) return;
+  float r[32];
+  if (a.resid_kind == RES_F16) load_f16x32((const __half*)a.resid + row * N + c, r);
+  else load_bf16x32((const __nv_bfloat16*)a.resid + row * N + c, r);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] += r[i];
+}
+
+// Named barrier over the 8 epilogue warps (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// Epilogue of one 128 x BN tile.  Two warps share each TMEM lane quadrant;
+// `half` selects which half of the columns this thread handles.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0) {
+                                         bool valid, int n0, int half, float* red, int rrow) {
+  constexpr int HB = BN / 2;                 // columns per thread
+  const int c0 = half * HB;
   if constexpr (EPI == TC_NORM) {
     const NormArgs& a = p.norm;
     const int N = BN;
+    // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM
     float ss = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c0 + HB; c += 32) {
       float v[32];
       tmem_ld32(taddr + c, v);
-      if (valid) {
-        add_resid(a, row, N, c, v);
+      if (valid) add_resid(a, row, N, c, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-      }
+      for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+      if (a.resid) tmem_st32(taddr + c, v);
     }
+    red[half * 128 + rrow] = ss;
+    epi_bar();
+    ss += red[(half ^ 1) * 128 + rrow];
     const float inv = rsqrtf(ss / (float)N + a.eps);
     // destinations of this row
     __nv_bfloat16* d1 = nullptr;
     __nv_bfloat16* d2 = nullptr;
     float* f1 = nullptr;
-    float* f2 = nullptr;
+    __half* r1 = nullptr;
     if (valid) {
       if (a.mode == NORM_PLAIN) {
         d1 = (__nv_bfloat16*)a.dst + row * N;
-        if (a.dst32) f1 = a.dst32 + row * N;
+        if (a.dst_res) r1 = (__half*)a.dst_res + row * N;
       } else {
         const int u = segment_of(a.qoff_l, a.B, row);
         const int64_t j = row - a.qoff_l[u];
@@ -148,17 +189,17 @@ __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, 
           }
           if (q >= 0) {
             d2 = (__nv_bfloat16*)a.Xq_n + q * N;
-            if (a.Xq32_n) f2 = a.Xq32_n + q * N;
+            if (a.Xq_res_n) r1 = (__half*)a.Xq_res_n + q * N;
           }
         }
       }
     }
+    // pass 2: normalise, scale by the gain, store
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c0 + HB; c += 32) {
       float v[32];
       tmem_ld32(taddr + c, v);
       if (valid) {
-        add_resid(a, row, N, c, v);
         float g[32];
         load_bf16x32((const __nv_bfloat16*)a.g + c, g);
 #pragma unroll
@@ -166,14 +207,14 @@ __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, 
         if (d1) store_bf16x32(d1 + c, v);
         if (d2) store_bf16x32(d2 + c, v);
         if (f1) store_f32x32(f1 + c, v);
-        if (f2) store_f32x32(f2 + c, v);
+        if (r1) store_f16x32(r1 + c, v);
       }
     }
   } else {
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = segment_of(p.seg_off, p.B, row);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c0 + HB; c += 32) {
       float v[32];
       tmem_ld32(taddr + c, v);
       if (valid) {
@@ -190,7 +231,7 @@ __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, 
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcGemmParams p) {
   using Cfg = GemmCfg<BN>;
@@ -206,6 +247,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* drain = tempty + ACC_BUFS;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][2 halves][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
@@ -215,7 +257,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 4); }
+    for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -289,17 +331,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int q = warp & 3;                // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;      // which half of the tile's columns
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    int acc = 0;
+    int acc = 0, it = 0;
     uint32_t acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
-      const int64_t row = (int64_t)mt * BM + q * 32 + lane;
-      epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN);
+      const int rr = q * 32 + lane;
+      const int64_t row = (int64_t)mt * BM + rr;
+      epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
+                        red + (it & 1) * 256, rr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -327,7 +372,7 @@ cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmP
     if (e != cudaSuccess) return e;
     attr_devices |= 1ull << (dev & 63);
   }
-  tc_gemm_kernel<BN, EPI><<<grid, 192, Cfg::SMEM, s>>>(a, b, p);
+  tc_gemm_kernel<BN, EPI><<<grid, kThreads, Cfg::SMEM, s>>>(a, b, p);
   return cudaGetLastError();
 }
 

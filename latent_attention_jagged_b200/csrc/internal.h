@@ -78,8 +78,8 @@ struct llatte_handle {
   void* Ot;
   void* Z;
   void* Hd;
-  float* Z32;          // fp32 residual copy of Z (bf16 storage only, else aliases Z)
-  float* Xq32[2];      // fp32 residual copy of the query rows (bf16 storage only)
+  void* Zres;          // fp16 residual copy of Z (bf16 storage only; NULL for fp32)
+  void* Xqres[2];      // fp16 residual copy of the query rows (bf16 storage only)
   float* acc32;        // fp32 pre-norm rows (CUDA-core path)
   float* ctxbias;      // [max_batch, h*r]
   float* final_rows;   // [max_rows_q, d] fp32 (readout only)
@@ -128,17 +128,21 @@ struct GemmArgs {
 enum { EPI_STORE = 0, EPI_USERBIAS, EPI_SILU, EPI_F32 };
 cudaError_t launch_gemm_simt(int elem_a, int elem_w, int elem_d, const GemmArgs& g, cudaStream_t s);
 
+// Element type of a residual-stream buffer.
+enum { RES_STORAGE = 0, RES_F32 = 1, RES_F16 = 2 };
+
 struct NormArgs {
   const float* acc; int N;           // [M, N] fp32 rows
   const void* resid;                 // [M, N] residual or NULL
-  int resid_f32;                     // 1: resid is fp32, 0: storage type
+  int resid_kind;                    // RES_STORAGE / RES_F32 / RES_F16
   const void* g; float eps;
   const int64_t* M_dev; int64_t M_max;
   int mode;                          // NORM_PLAIN / NORM_SCATTER
-  void* dst; float* dst32;           // NORM_PLAIN: [M, N] storage type (+ optional fp32 copy)
+  int res_kind;                      // type of the residual copies written below
+  void* dst; void* dst_res;          // NORM_PLAIN: [M, N] storage type (+ optional residual copy)
   // NORM_SCATTER (FFN2 output of layer l -> inputs of layer l+1 / outputs)
   const int64_t *qoff_l, *hoff_n, *qoff_n; const int32_t *n_l, *n_n; int B; int n_q;
-  void* Xh_n; void* Xq_n; float* Xq32_n; int last; float* out; float* final_rows;
+  void* Xh_n; void* Xq_n; void* Xq_res_n; int last; float* out; float* final_rows;
 };
 enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
 cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s);
@@ -157,6 +161,6 @@ cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int 
                              cudaStream_t s);
 cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
                           const void* W_o, int d, int d_ctx, int heads, int d_head, int r,
-                          void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s);
+                          float qscale, void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s);
 
 }  // namespace llatte

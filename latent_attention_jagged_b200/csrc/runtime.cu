@@ -26,7 +26,7 @@ struct Layout {
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
       off_work_count, off_work_next;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
-      off_final, off_mean, off_Z32, off_Xq32[2];
+      off_final, off_mean, off_Zres, off_Xqres[2];
   size_t total;
   int32_t max_work;
 };
@@ -79,11 +79,11 @@ Layout layout_of(const llatte_dims* d) {
   L.off_Ot = take((size_t)L.rows_q * hr * elem);
   L.off_Z = take((size_t)L.rows_q * d->d * elem);
   L.off_Hd = take((size_t)L.rows_q * f * elem);
-  // fp32 copies of the residual stream (bf16 storage keeps bf16 GEMM operands
+  // fp16 copies of the residual stream (bf16 storage keeps bf16 GEMM operands
   // plus these; fp32 storage needs none)
-  const size_t res32 = elem == 2 ? sizeof(float) * (size_t)L.rows_q * d->d : 0;
-  L.off_Z32 = take(res32);
-  for (int i = 0; i < 2; ++i) L.off_Xq32[i] = take(res32);
+  const size_t res16 = elem == 2 ? 2 * (size_t)L.rows_q * d->d : 0;
+  L.off_Zres = take(res16);
+  for (int i = 0; i < 2; ++i) L.off_Xqres[i] = take(res16);
   L.off_acc32 = take(sizeof(float) * std::max<size_t>((size_t)L.rows_h * d->rank,
                                                       (size_t)L.rows_q * d->d));
   L.off_ctxbias = take(sizeof(float) * B * hr);
@@ -271,6 +271,10 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   const size_t e = h->elem;
   const int d = D.d, r = D.rank, hd = D.heads * D.d_head, hr = D.heads * D.rank,
             f = D.ffn_mult * D.d, dc = D.d_ctx;
+  // The tensor-core attention takes its scores in log2 units (exp2 in the
+  // softmax): fold log2(e) into the absorbed query projection for that path.
+  const bool want_tc = h->elem == 2 && tc_dims_ok(D);
+  const float qscale = want_tc ? 1.4426950408889634f : 1.0f;
   for (int l = 0; l < D.n_layers; ++l) {
     const llatte_layer_w& w = layers[l];
     LayerDev& L = h->layers[l];
@@ -297,8 +301,8 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
          cudaMemcpy(tuk, w.W_uk, e * (size_t)hd * r, k) == cudaSuccess &&
          cudaMemcpy(tuv, w.W_uv, e * (size_t)hd * r, k) == cudaSuccess &&
          cudaMemcpy(to, w.W_o, e * (size_t)d * hd, k) == cudaSuccess;
-    ok = ok && launch_absorb(h->elem, tq, tuk, tuv, to, d, dc, D.heads, D.d_head, r, L.W_qk,
-                             L.W_qkc, L.W_ov, 0) == cudaSuccess;
+    ok = ok && launch_absorb(h->elem, tq, tuk, tuv, to, d, dc, D.heads, D.d_head, r, qscale,
+                             L.W_qk, L.W_qkc, L.W_ov, 0) == cudaSuccess;
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     cudaFree(tq); cudaFree(tuk); cudaFree(tuv); cudaFree(to);
     if (!ok) return fail(LLATTE_ERR_CUDA);
@@ -334,14 +338,13 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->Ot = ws + Lo.off_Ot;
   h->Z = ws + Lo.off_Z;
   h->Hd = ws + Lo.off_Hd;
-  h->Z32 = h->elem == 2 ? (float*)(ws + Lo.off_Z32) : (float*)h->Z;
-  for (int i = 0; i < 2; ++i)
-    h->Xq32[i] = h->elem == 2 ? (float*)(ws + Lo.off_Xq32[i]) : (float*)h->Xq[i];
+  h->Zres = h->elem == 2 ? (void*)(ws + Lo.off_Zres) : nullptr;
+  for (int i = 0; i < 2; ++i) h->Xqres[i] = h->elem == 2 ? (void*)(ws + Lo.off_Xqres[i]) : nullptr;
   h->acc32 = (float*)(ws + Lo.off_acc32);
   h->ctxbias = (float*)(ws + Lo.off_ctxbias);
   h->final_rows = D.d_out ? (float*)(ws + Lo.off_final) : nullptr;
   h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
-  if (h->elem == 2 && tc_dims_ok(D)) {
+  if (want_tc) {
     if (!build_tc_maps(h)) return fail(LLATTE_ERR_CUDA);
     h->use_tc = 1;
   }
@@ -392,21 +395,27 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     NormArgs kv_norm = {};
     kv_norm.N = r; kv_norm.g = W.g_kv; kv_norm.eps = D.eps; kv_norm.M_dev = p.hist_total(l);
     kv_norm.M_max = h->max_rows_h; kv_norm.mode = NORM_PLAIN; kv_norm.dst = h->C;
+    // Residual stream: bf16 storage keeps an fp16 copy of Z and of every
+    // layer's query rows for the residual adds (the bf16 copies feed the
+    // tensor cores); fp32 storage adds to the stored rows directly.
+    const bool res16 = e == 2;
     NormArgs o_norm = {};
-    o_norm.N = d; o_norm.g = W.g1; o_norm.eps = D.eps;
-    // residual: the layer input rows; in fp32 from layer 1 on (layer 0 reads
-    // the gathered inputs, exact in the storage type)
-    o_norm.resid = (l == 0) ? Xq_l : (const void*)h->Xq32[l & 1];
-    o_norm.resid_f32 = (l == 0) ? (e == 4) : 1;
+    o_norm.N = d; o_norm.g = W.g1; o_norm.eps = D.eps; o_norm.res_kind = RES_F16;
+    // residual: the layer input rows (layer 0: the gathered inputs, exact in
+    // the storage type)
+    o_norm.resid = (l == 0 || !res16) ? Xq_l : h->Xqres[l & 1];
+    o_norm.resid_kind = (l == 0 || !res16) ? RES_STORAGE : RES_F16;
     o_norm.M_dev = p.query_total(l); o_norm.M_max = h->max_rows_q; o_norm.mode = NORM_PLAIN;
-    o_norm.dst = h->Z; o_norm.dst32 = e == 2 ? h->Z32 : nullptr;
+    o_norm.dst = h->Z; o_norm.dst_res = res16 ? h->Zres : nullptr;
     NormArgs f_norm = {};
-    f_norm.N = d; f_norm.resid = h->Z32; f_norm.resid_f32 = 1; f_norm.g = W.g2; f_norm.eps = D.eps;
+    f_norm.N = d; f_norm.resid = res16 ? h->Zres : h->Z;
+    f_norm.resid_kind = res16 ? RES_F16 : RES_STORAGE; f_norm.res_kind = RES_F16;
+    f_norm.g = W.g2; f_norm.eps = D.eps;
     f_norm.M_dev = p.query_total(l); f_norm.M_max = h->max_rows_q; f_norm.mode = NORM_SCATTER;
     f_norm.qoff_l = p.qoff(l); f_norm.n_l = p.nl(l); f_norm.hoff_n = p.hoff(l + 1);
     f_norm.qoff_n = p.qoff(l + 1); f_norm.n_n = p.nl(l + 1); f_norm.B = B; f_norm.n_q = D.n_q;
     f_norm.Xh_n = Xh_n; f_norm.Xq_n = Xq_n; f_norm.last = last;
-    f_norm.Xq32_n = (e == 2 && !last) ? h->Xq32[(l + 1) & 1] : nullptr;
+    f_norm.Xq_res_n = (res16 && !last) ? h->Xqres[(l + 1) & 1] : nullptr;
     f_norm.out = out; f_norm.final_rows = D.d_out ? h->final_rows : nullptr;
     const LayerMaps& LM = h->lmaps[l];
     auto tcp = [&](const int64_t* Mdev, int64_t cap, int N, int K) {

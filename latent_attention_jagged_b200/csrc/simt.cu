@@ -8,6 +8,8 @@
 //   ATTN  o~   = softmax(q~ . c_kv) c_kv over the visible keys
 //   O     Z    = RMSNorm_{g1}(R + o~ W_ov^T)
 //   FFN   X'   = RMSNorm_{g2}(Z + W2 SiLU(W1 Z))
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -102,13 +104,15 @@ rownorm_kernel(NormArgs a) {
   if (m >= M) return;
   const int N = a.N;
   const float* row = a.acc + m * N;
-  const T* res = a.resid_f32 ? nullptr : (const T*)a.resid;
-  const float* res32 = a.resid_f32 ? (const float*)a.resid : nullptr;
   const T* g = (const T*)a.g;
   auto val = [&](int c) {
     float v = row[c];
-    if (res) v += to_f(res[m * N + c]);
-    if (res32) v += res32[m * N + c];
+    if (a.resid) {
+      const int64_t i = m * N + c;
+      if (a.resid_kind == RES_F32) v += ((const float*)a.resid)[i];
+      else if (a.resid_kind == RES_F16) v += __half2float(((const __half*)a.resid)[i]);
+      else v += to_f(((const T*)a.resid)[i]);
+    }
     return v;
   };
   float ss = 0.f;
@@ -121,11 +125,11 @@ rownorm_kernel(NormArgs a) {
   // destinations
   T* d1 = nullptr;
   T* d2 = nullptr;
-  float* f1 = nullptr;
-  float* f2 = nullptr;
+  float* f1 = nullptr;     // fp32 output row (final layer)
+  void* r1 = nullptr;      // residual copy of this row
   if (a.mode == NORM_PLAIN) {
     d1 = (T*)a.dst + m * N;
-    if (a.dst32) f1 = a.dst32 + m * N;
+    if (a.dst_res) r1 = a.dst_res;
   } else {
     const int u = segment_of(a.qoff_l, a.B, m);
     const int64_t j = m - a.qoff_l[u];
@@ -144,16 +148,21 @@ rownorm_kernel(NormArgs a) {
       }
       if (q >= 0) {
         d2 = (T*)a.Xq_n + q * N;
-        if (a.Xq32_n) f2 = a.Xq32_n + q * N;
+        if (a.Xq_res_n) r1 = a.Xq_res_n;
       }
     }
   }
+  int64_t rrow = m;
+  if (a.mode != NORM_PLAIN && d2) rrow = (d2 - (T*)a.Xq_n) / N;
   for (int c = lane; c < N; c += 32) {
     float y = val(c) * inv * to_f(g[c]);
     if (d1) d1[c] = from_f<T>(y);
     if (d2) d2[c] = from_f<T>(y);
     if (f1) f1[c] = y;
-    if (f2) f2[c] = y;
+    if (r1) {
+      if (a.res_kind == RES_F16) ((__half*)r1)[rrow * N + c] = __float2half_rn(y);
+      else ((float*)r1)[rrow * N + c] = y;
+    }
   }
 }
 
@@ -258,12 +267,13 @@ cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int 
 }
 
 // ---------------------------------------------------------------- absorption
-// W_qk[j*r + a, k] = (1/sqrt(d_h)) sum_e W_uk[j*d_h + e, a] W_q[j*d_h + e, k]
+// W_qk[j*r + a, k] = (qscale/sqrt(d_h)) sum_e W_uk[j*d_h + e, a] W_q[j*d_h + e, k]
+//   (qscale = log2(e) when the attention kernel takes scores in log2 units)
 //   (k < d -> W_qk in the storage type, k >= d -> W_qkc in fp32)
 // W_ov[n, j*r + a] = sum_e W_o[n, j*d_h + e] W_uv[j*d_h + e, a]
 template <typename T>
 __global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int heads, int dh,
-                                int r, T* W_qk, float* W_qkc) {
+                                int r, float qscale, T* W_qk, float* W_qkc) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int K = d + dc;
   if (idx >= (int64_t)heads * r * K) return;
@@ -273,7 +283,7 @@ __global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int 
   float s = 0.f;
   for (int e = 0; e < dh; ++e)
     s = fmaf(to_f(W_uk[(int64_t)(j * dh + e) * r + a]), to_f(W_q[(int64_t)(j * dh + e) * K + k]), s);
-  s *= rsqrtf((float)dh);
+  s *= rsqrtf((float)dh) * qscale;
   if (k < d) W_qk[(int64_t)row * d + k] = from_f<T>(s);
   else W_qkc[(int64_t)row * dc + (k - d)] = s;
 }
@@ -294,19 +304,19 @@ __global__ void absorb_o_kernel(const T* W_o, const T* W_uv, int d, int heads, i
 }
 
 cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
-                          const void* W_o, int d, int dc, int heads, int dh, int r, void* W_qk,
-                          float* W_qkc, void* W_ov, cudaStream_t s) {
+                          const void* W_o, int d, int dc, int heads, int dh, int r, float qscale,
+                          void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s) {
   const int64_t nq = (int64_t)heads * r * (d + dc), no = (int64_t)d * heads * r;
   const unsigned bq = (unsigned)((nq + 255) / 256), bo = (unsigned)((no + 255) / 256);
   if (elem == 4) {
     absorb_q_kernel<float><<<bq, 256, 0, s>>>((const float*)W_q, (const float*)W_uk, d, dc, heads,
-                                              dh, r, (float*)W_qk, W_qkc);
+                                              dh, r, qscale, (float*)W_qk, W_qkc);
     absorb_o_kernel<float><<<bo, 256, 0, s>>>((const float*)W_o, (const float*)W_uv, d, heads, dh,
                                               r, (float*)W_ov);
   } else {
     typedef __nv_bfloat16 bf;
     absorb_q_kernel<bf><<<bq, 256, 0, s>>>((const bf*)W_q, (const bf*)W_uk, d, dc, heads, dh, r,
-                                           (bf*)W_qk, W_qkc);
+                                           qscale, (bf*)W_qk, W_qkc);
     absorb_o_kernel<bf><<<bo, 256, 0, s>>>((const bf*)W_o, (const bf*)W_uv, d, heads, dh, r,
                                            (bf*)W_ov);
   }

@@ -120,3 +120,23 @@ def test_device_status_reports_bad_offsets_without_fault():
     _, again = run(inp, handle=h)
     assert h.status() == 0
     assert np.array_equal(good, again)
+
+
+def test_cuda_graph_replay_matches_eager():
+    """A whole forward captured once in a CUDA graph and replayed gives the
+    same bits as launching it eagerly (no host work inside the forward)."""
+    inp = make_inputs(workload("online"), batch=48)
+    h, eager = run(inp)
+    values, offsets, ctx, cand = to_device(inp)
+    out = torch.empty(h.out_shape(inp.batch), dtype=torch.float32, device="cuda")
+    h.forward(values, offsets, ctx, cand, out=out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        h.forward(values, offsets, ctx, cand, out=out)
+    out.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert h.status() == 0
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), eager)
