@@ -163,9 +163,10 @@ const char* llatte_error_string(int code);
 /*
  * Per-step device timing, a profiling aid.  With profiling enabled every
  * forward records a CUDA event pair on its stream around each step (plan,
- * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout); llatte_profile_step
- * synchronises on the recorded events and returns, for step index `step`
- * (0 .. 9), its name, the accumulated milliseconds, the number of kernels the
+ * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout, and ffn when the FFN
+ * runs as one fused kernel); llatte_profile_step synchronises on the recorded
+ * events and returns, for step index `step` (0 .. 10), its name, the
+ * accumulated milliseconds, the number of kernels the
  * step launched and the number of times it ran since the last reset.
  * Returns LLATTE_ERR_ARG for a step index out of range.
  */

@@ -14,7 +14,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libllatte.so")
 MAX_LAYERS = 16
-STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout")
+STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout", "ffn")
 
 LLATTE_OK, LLATTE_ERR_ARG, LLATTE_ERR_UNSUPPORTED, LLATTE_ERR_CUDA, LLATTE_ERR_OOM, \
     LLATTE_ERR_DEVICE = 0, -1, -2, -3, -4, -5

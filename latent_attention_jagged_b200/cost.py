@@ -75,6 +75,7 @@ def flops_by_step(lengths: Sequence[int], dims) -> Dict[str, float]:
             acc[k] = acc.get(k, 0.0) + float(v)
     if dims.d_out:
         acc["readout"] = 2.0 * len(lengths) * dims.d * dims.d_out
+    acc["ffn"] = acc["ffn1"] + acc["ffn2"]      # the FFN as one fused step
     return acc
 
 

@@ -13,7 +13,7 @@ namespace llatte {
 
 // Step kinds, for the optional per-step timing.
 enum Step { ST_PLAN = 0, ST_GATHER, ST_CTX, ST_KV, ST_Q, ST_ATTN, ST_O, ST_FFN1, ST_FFN2,
-            ST_READOUT, ST_COUNT };
+            ST_READOUT, ST_FFN, ST_COUNT };
 extern const char* const kStepNames[ST_COUNT];
 
 // Device-side pyramid plan.  Layer index l runs over 0..L where l = L is the
@@ -54,7 +54,7 @@ struct LayerDev {
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
-struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2; };
+struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_ffn; };
 
 }  // namespace llatte
 
@@ -93,6 +93,7 @@ struct llatte_handle {
   llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
   int bn_kv, bn_q, bn_o, bn_f1, bn_f2;
   int attn_keys;                  // keys per attention tile (tensor-core path)
+  int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
 
   // profiling

@@ -8,13 +8,14 @@
 
 #include "internal.h"
 #include "tc_attn.h"
+#include "tc_ffn.h"
 #include "tc_gemm.h"
 
 using namespace llatte;
 
 namespace llatte {
-const char* const kStepNames[ST_COUNT] = {"plan", "gather", "ctx_bias", "kv", "q",
-                                          "attn", "o",      "ffn1",     "ffn2", "readout"};
+const char* const kStepNames[ST_COUNT] = {"plan", "gather", "ctx_bias", "kv",      "q",  "attn",
+                                          "o",    "ffn1",   "ffn2",     "readout", "ffn"};
 }
 
 namespace {
@@ -194,6 +195,7 @@ bool build_tc_maps(llatte_handle* h) {
   ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
   h->attn_keys = attn_tc_keys(r);
+  h->ffn_fused = ffn_tc_supported(d, f) ? 1 : 0;
   ok = ok && make_tmap_bf16(&h->tm_Qt, h->Qt, rq * D.heads, r, 128);
   ok = ok && make_tmap_bf16(&h->tm_C, h->C, rh, r, (uint32_t)h->attn_keys);
   auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
@@ -205,6 +207,7 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
+    if (h->ffn_fused) ok = ok && make_tmap_bf16(&M.w1_ffn, W.W1, f, d, 128);
   }
   return ok;
 }
@@ -502,6 +505,15 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
         CK(launch_rownorm(e, o_norm, s));
         t.done(2);
       }
+    }
+    if (tc && h->ffn_fused) {  // FFN up + SiLU + down + residual + RMSNorm, one kernel
+      StepTimer t(h, s, ST_FFN);
+      FfnTcParams q = {};
+      q.M_dev = p.query_total(l); q.M_cap = h->max_rows_q; q.F = f; q.norm = f_norm;
+      q.status = p.status;
+      CK(launch_ffn_tc(h->tm_Z, LM.w1_ffn, LM.w2, q, h->num_sms, s));
+      t.done(1);
+      continue;
     }
     {  // FFN up + SiLU
       StepTimer t(h, s, ST_FFN1);
