@@ -9,12 +9,13 @@
 // of the user's current history: S = Q~ C^T and O~ = softmax(S) C both read
 // one shared-memory copy of each C tile (K-major for S, MN-major for P V).
 //
-// Roles (192 threads, one CTA per SM, persistent over the sorted work list):
+// Roles (320 threads, one CTA per SM, persistent over the sorted work list):
 //   warp 0      TMA: the Q~ block once per item, C tiles into a KV_STAGES ring
 //   warp 1      TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
 //               O += P(kt) C_kt, so the tensor pipe works while the softmax
 //               warps turn S(kt) into P(kt)
-//   warps 2..5  softmax, one TMEM lane (= one pair) per thread: masking
+//   warps 2..9  softmax, two warps per TMEM lane (= one pair), each taking
+//               half of the columns: masking
 //               (history row at position p sees keys t <= p; a query token
 //               sees every key t < T), online max / sum in fp32, P written to
 //               shared memory as bf16, lazy rescaling of O in TMEM (only when
@@ -35,19 +36,22 @@ using namespace tc;
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;                 // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
 
 template <int R>
 struct AttnCfg {
   static constexpr int KEYS = R >= 256 ? 64 : 128;     // keys per tile
   static constexpr int RSUB = R / 64;                  // 64-wide latent sub-tiles
-  static constexpr int KV_STAGES = 4;
+  static constexpr int KV_STAGES = 3;
   static constexpr uint32_t Q_BYTES = 128 * R * 2;
   static constexpr uint32_t KV_BYTES = KEYS * R * 2;
   static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
   static constexpr uint32_t P_BYTES = 128 * KEYS * 2;
   static constexpr uint32_t S_COL = R;                  // S buffers after O
-  static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256;
+  static constexpr uint32_t RED_BYTES = 3 * 256 * 4;     // max exchange [2][2][128], sums [2][128]
+  static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256 +
+                                RED_BYTES;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(R + 2 * KEYS <= 512, "TMEM budget");
 };
@@ -106,8 +110,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* p_empty = p_full + 2;          // [2]
   uint64_t* o_free = p_empty + 2;
   uint64_t* drain = o_free + 1;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* xbar = drain + 1;              // softmax group barrier (max / sum exchange)
+  uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* red = (float*)((uint8_t*)bars + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = *p.work_count;
@@ -118,12 +124,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&s_empty[s], kSoftmaxWarps);
+      mbar_init(&p_full[s], kSoftmaxWarps);
       mbar_init(&p_empty[s], 1);
     }
-    mbar_init(o_free, 4);
+    mbar_init(o_free, kSoftmaxWarps);
     mbar_init(drain, 1);
+    mbar_init(xbar, kSoftmaxWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -233,10 +240,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
+    // Two warps per TMEM lane quadrant: `half` takes columns
+    // [half * KEYS/2, ...) of every S tile and [half * R/2, ...) of O.  The
+    // row max of a tile is the max of both halves (exchanged in shared memory
+    // behind the softmax named barrier), so both halves make the same lazy
+    // rescaling decision; the row sums are combined once per item.
+    constexpr int HK = KEYS / 2, HR = R / 2;
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;              // pair within the block = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t g = 0;
+    uint32_t g = 0, xphase = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
       const Item it = load_item(p, idx, KEYS);
@@ -244,48 +258,52 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const bool valid = pair < it.q * p.heads;
       const int64_t jl = pair / p.heads;
       const int64_t vis = !valid ? 0 : (jl < it.n ? it.T - it.n + jl + 1 : it.T);
-      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R;
+      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R + half * HR;
       if (it.nk == 0) {
         if (valid) {
           uint4 z = make_uint4(0, 0, 0, 0);
-          for (int c = 0; c < R; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+          for (int c = 0; c < HR; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
         }
         continue;
       }
-      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and this half's sum
       for (int kt = 0; kt < it.nk; ++kt, ++g) {
-        // ---- S tile -> registers
+        // ---- this half of the S tile -> registers
         bool w = mbar_wait(&s_full[g & 1], (g >> 1) & 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
-        float s[KEYS];
+        float s[HK];
 #pragma unroll
-        for (int c = 0; c < KEYS; c += 32) {
+        for (int c = 0; c < HK; c += 32) {
           float v[32];
-          tmem_ld32(lane_base + Cfg::S_COL + (g & 1) * KEYS + c, v);
+          tmem_ld32(lane_base + Cfg::S_COL + (g & 1) * KEYS + half * HK + c, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c + i] = v[i];
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[g & 1]);
-        // ---- mask (only on tiles this row does not see entirely) and tile
-        // max; scores are already in log2 units (log2 e folded into q~)
-        const int64_t t0 = (int64_t)kt * KEYS;
-        if (t0 + KEYS > vis) {
+        // ---- mask (only where this row does not see the whole tile) and the
+        // partial max; scores are already in log2 units (log2 e folded into q~)
+        const int64_t t0 = (int64_t)kt * KEYS + half * HK;
+        if (t0 + HK > vis) {
           const int64_t lim = vis - t0;
 #pragma unroll
-          for (int c = 0; c < KEYS; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+          for (int c = 0; c < HK; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
         }
         float m8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = s[i];
 #pragma unroll
-        for (int c = 8; c < KEYS; c += 8)
+        for (int c = 8; c < HK; c += 8)
 #pragma unroll
           for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        float* xm = red + (g & 1) * 256;
+        xm[half * 128 + row] = mt;
+        if (!group_sync(xbar, xphase, abort_flag, p.status)) { ok = false; break; }
+        mt = fmaxf(mt, xm[(half ^ 1) * 128 + row]);
         // ---- lazy rescale of O and l (only when the max grows by > 8 in log2)
         float scale = 1.f;
         bool resc = false;
@@ -304,12 +322,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < R; c += 32) {
+          for (int c = 0; c < HR; c += 32) {
             float v[32];
-            tmem_ld32(lane_base + c, v);
+            tmem_ld32(lane_base + half * HR + c, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= scale;
-            tmem_st32(lane_base + c, v);
+            tmem_st32(lane_base + half * HR + c, v);
           }
           l_run *= scale;
         }
@@ -319,23 +337,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
         float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < KEYS; c += 8)
+        for (int c = 0; c < HK; c += 8)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             s[c + i] = ex2_approx(s[c + i] - m_use);
             l8[i] += s[c + i];
           }
         l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        // ---- P tile -> shared memory (bf16, 128-byte swizzled, K-major)
+        // ---- this half of the P tile -> shared memory (bf16, 128-byte
+        // swizzled, K-major: 64-key sub-tiles, 16-byte chunks XOR row % 8)
         bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
         const uint32_t pbase = smem_u32(sP + (g & 1) * Cfg::P_BYTES);
 #pragma unroll
-        for (int ch = 0; ch < KEYS / 8; ++ch) {
+        for (int c8 = 0; c8 < HK / 8; ++c8) {
+          const int ch = half * (HK / 8) + c8;          // 8-key chunk within the tile
           const int sub = ch >> 3, cc = ch & 7;
           const uint32_t addr = pbase + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-          uint4 v = make_uint4(pack_bf16(s[8 * ch], s[8 * ch + 1]), pack_bf16(s[8 * ch + 2], s[8 * ch + 3]),
-                               pack_bf16(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
+          const float* x = &s[8 * c8];
+          uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                               pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
           st_shared_v4(addr, v);
         }
         fence_proxy_async_smem();
@@ -345,14 +366,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       if (!ok) break;
       // ---- final: O / l -> HBM, once the last PV(g-1) has completed
+      float* xl = red + 512;
+      xl[half * 128 + row] = l_run;
+      if (!group_sync(xbar, xphase, abort_flag, p.status)) break;
+      const float l_tot = l_run + xl[(half ^ 1) * 128 + row];
+      // both halves have read the sums before the next item writes them
+      if (!group_sync(xbar, xphase, abort_flag, p.status)) break;
       bool w4 = mbar_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w4)) break;
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < R; c += 32) {
+      for (int c = 0; c < HR; c += 32) {
         float v[32];
-        tmem_ld32(lane_base + c, v);
+        tmem_ld32(lane_base + half * HR + c, v);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll

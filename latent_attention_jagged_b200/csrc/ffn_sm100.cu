@@ -72,7 +72,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
   uint64_t* out_full = hs_empty + 2;
   uint64_t* out_empty = out_full + 1;
   uint64_t* drain = out_empty + 1;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* xbar = drain + 1;                          // epilogue group barrier
+  uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   // the residual-norm exchange lives in the first SiLU buffer: while OUT is
   // normalised no MMA reads that buffer and no SiLU chunk is being written
@@ -95,6 +96,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
     mbar_init(out_full, 1);
     mbar_init(out_empty, kEpiWarps);
     mbar_init(drain, 1);
+    mbar_init(xbar, kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmZ);
@@ -223,7 +225,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
     const int half = (warp - 2) >> 2;
     const int rr = q * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    uint32_t ti = 0, gc = 0;
+    uint32_t ti = 0, gc = 0, xphase = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++ti) {
       for (int j = 0; j < NC; ++j, ++gc) {
@@ -256,8 +258,11 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
       if (!__all_sync(0xffffffffu, w3)) break;
       tc_fence_after();
       const int64_t row = t * 128 + rr;
-      norm_epilogue<D>(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr);
-      epi_bar();   // every partner has read `red` before a SiLU chunk reuses it
+      if (!norm_epilogue<D>(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr, xbar,
+                            xphase, abort_flag, p.status))
+        break;
+      // every partner has read `red` before a SiLU chunk reuses that memory
+      if (!group_sync(xbar, xphase, abort_flag, p.status)) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(out_empty);

@@ -61,12 +61,15 @@ struct GemmCfg {
 // Epilogue of one 128 x BN tile.  Two warps share each TMEM lane quadrant;
 // `half` selects which half of the columns this thread handles.
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0, int half, float* red, int rrow) {
+__device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
+                                         bool valid, int n0, int half, float* red, int rrow,
+                                         uint64_t* xbar, uint32_t& xphase,
+                                         volatile int* abort_flag) {
   constexpr int HB = BN / 2;                 // columns per thread
   const int c0 = half * HB;
   if constexpr (EPI == TC_NORM) {
-    norm_epilogue<BN>(p.norm, taddr, row, valid, half, red, rrow);
+    return norm_epilogue<BN>(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
+                             abort_flag, p.status);
   } else {
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = segment_of(p.seg_off, p.B, row);
@@ -84,6 +87,7 @@ __device__ __forceinline__ void epilogue(const TcGemmParams& p, uint32_t taddr, 
         store_bf16x32(p.D + row * p.ldd + n, v);
       }
     }
+    return true;
   }
 }
 
@@ -102,7 +106,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + ACC_BUFS;
   uint64_t* drain = tempty + ACC_BUFS;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  uint64_t* xbar = drain + 1;                 // epilogue group barrier (norm exchange)
+  uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][2 halves][128]
 
@@ -116,6 +121,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiWarps); }
     mbar_init(drain, 1);
+    mbar_init(xbar, kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -192,7 +198,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int half = (warp - 2) >> 2;      // which half of the tile's columns
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     int acc = 0, it = 0;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, xphase = 0;
     for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -200,8 +206,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
-      epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
-                        red + (it & 1) * 256, rr);
+      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
+                             red + (it & 1) * 256, rr, xbar, xphase, abort_flag))
+        break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

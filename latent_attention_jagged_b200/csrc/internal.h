@@ -28,6 +28,7 @@ struct PlanDev {
   int32_t* work;       // attention work items, [(L) * max_work] (tensor-core path)
   int32_t* work_count; // [L]
   int32_t* work_next;  // [L] dynamic scheduling counters
+  int32_t* item_off;   // [max_batch+1] scratch: first work item of each user
   int64_t stride;      // max_batch + 1
   int32_t max_work;
 
@@ -81,7 +82,7 @@ struct llatte_handle {
   void* Zres;          // fp16 residual copy of Z (bf16 storage only; NULL for fp32)
   void* Xqres[2];      // fp16 residual copy of the query rows (bf16 storage only)
   float* acc32;        // fp32 pre-norm rows (CUDA-core path)
-  float* ctxbias;      // [max_batch, h*r]
+  float* ctxbias;      // [n_layers][B][h*r] (this forward's B)
   float* final_rows;   // [max_rows_q, d] fp32 (readout only)
   float* mean_rows;    // [max_batch, d] fp32
   size_t ws_bytes;
@@ -157,6 +158,11 @@ struct AttnArgs {
   int B, heads, r;
 };
 cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
+
+// Per-user context term of every layer's absorbed query projection.
+struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [h*r, d_ctx] per layer
+cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
+                            int dc, float* out, cudaStream_t s);
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
                              cudaStream_t s);

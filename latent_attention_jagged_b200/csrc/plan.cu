@@ -12,9 +12,11 @@
 // later kernel then does any work) and sets the device status word.
 //
 // Gather (appendix A.2 step 2, X_input = Concat(X_seq, Q)): layer 0's
-// history rows are a straight copy of `values`; its query rows are the last
-// n_0 history rows of each user followed by the user's query tokens.  One
-// warp per row, 16-byte vector loads/stores.
+// history rows are a copy of `values`; its query rows are the last n_0
+// history rows of each user followed by the user's query tokens.  Blocks per
+// (user, slice), one warp per row, 16-byte vector loads/stores.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -131,6 +133,16 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     const int32_t* Tl = p.T + l * bstride;
     const int32_t* nl = p.n + l * bstride;
     if (tid < kBuckets) hist[tid] = 0;
+    // items per user and their exclusive scan (item_off[u] = first item of u)
+    int64_t cnt = 0;
+    for (int u = u0; u < u1; ++u) cnt += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+    int64_t base, dummy, total, dummy2;
+    block_exscan2(cnt, 0, &base, &dummy, &total, &dummy2);
+    for (int u = u0; u < u1; ++u) {
+      p.item_off[u] = (int32_t)base;
+      base += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+    }
+    if (tid == 0) p.item_off[B] = (int32_t)total;
     __syncthreads();
     auto cost_of = [&](int u, int b) {
       const int64_t q = (int64_t)nl[u] + n_q;
@@ -140,9 +152,17 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
       const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
       return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
     };
-    for (int u = u0; u < u1; ++u) {
-      const int64_t items = (((int64_t)nl[u] + n_q) * heads + 127) / 128;
-      for (int b = 0; b < items; ++b) atomicAdd(&hist[cost_of(u, b)], 1);
+    auto user_of = [&](int i) {      // largest u with item_off[u] <= i
+      int lo = 0, hi = B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.item_off[mid] <= i) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    };
+    for (int i = tid; i < (int)total; i += kPlanThreads) {
+      const int u = user_of(i);
+      atomicAdd(&hist[cost_of(u, i - p.item_off[u])], 1);
     }
     __syncthreads();
     if (tid == 0) {
@@ -152,13 +172,12 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     }
     __syncthreads();
     int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
-    for (int u = u0; u < u1; ++u) {
-      const int64_t items = (((int64_t)nl[u] + n_q) * heads + 127) / 128;
-      for (int b = 0; b < items; ++b) {
-        const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
-        W[2 * pos] = u;
-        W[2 * pos + 1] = b;
-      }
+    for (int i = tid; i < (int)total; i += kPlanThreads) {
+      const int u = user_of(i);
+      const int b = i - p.item_off[u];
+      const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
+      W[2 * pos] = u;
+      W[2 * pos + 1] = b;
     }
     if (tid == 0) {
       p.work_count[l] = total_items;
@@ -188,34 +207,33 @@ cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_t
 
 // ---------------------------------------------------------------- gather
 
+// Block (u, s): slice s of user u's rows.  Rows 0..T-1 are the user's
+// history (copied to the history buffer), rows T..T+q-1 its query rows (the
+// last n history rows, then the query tokens).  One warp per row.
 __global__ void __launch_bounds__(256)
 gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offsets,
-              const uint4* __restrict__ cand, int B, PlanDev p, uint4* __restrict__ Xh,
+              const uint4* __restrict__ cand, PlanDev p, uint4* __restrict__ Xh,
               uint4* __restrict__ Xq, int row_vecs, int n_q) {
+  // a batch the plan rejected has zero rows everywhere: copy nothing
+  if (*p.hist_total(0) == 0 && *p.query_total(0) == 0) return;
+  const int u = blockIdx.x;
   const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int64_t w0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nh = *p.hist_total(0), nq = *p.query_total(0);
-  const int64_t base = nh ? offsets[0] : 0;
-  for (int64_t row = w0; row < nh + nq; row += warps) {
+  const int warps = (blockDim.x >> 5) * gridDim.y;
+  const int w0 = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t T = p.Tl(0)[u], n = p.nl(0)[u];
+  const int64_t hoff = p.hoff(0)[u], qoff = p.qoff(0)[u], src0 = offsets[u];
+  const int64_t rows = T + n + n_q;
+  for (int64_t r = w0; r < rows; r += warps) {
     const uint4* src;
     uint4* dst;
-    if (row < nh) {
-      src = values + (base + row) * row_vecs;
-      dst = Xh + row * row_vecs;
+    if (r < T) {
+      src = values + (src0 + r) * row_vecs;
+      dst = Xh + (hoff + r) * row_vecs;
     } else {
-      const int64_t m = row - nh;
-      const int64_t* qo = p.qoff(0);
-      const int u = segment_of(qo, B, m);
-      const int64_t j = m - qo[u];
-      const int32_t n = p.nl(0)[u];
-      if (j < n) {
-        const int64_t T = p.Tl(0)[u];
-        src = values + (offsets[u] + T - n + j) * row_vecs;
-      } else {
-        src = cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
-      }
-      dst = Xq + m * row_vecs;
+      const int64_t j = r - T;
+      src = j < n ? values + (src0 + T - n + j) * row_vecs
+                  : cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
+      dst = Xq + (qoff + j) * row_vecs;
     }
     for (int v = lane; v < row_vecs; v += 32) dst[v] = __ldg(src + v);
   }
@@ -223,10 +241,13 @@ gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offs
 
 cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
                           const void* cand, int B, cudaStream_t s) {
+  if (B == 0) return cudaSuccess;
   const int row_vecs = h->dims.d * h->elem / 16;
-  gather_kernel<<<h->num_sms * 4, 256, 0, s>>>(
-      (const uint4*)values, offsets, (const uint4*)cand, B, h->plan, (uint4*)h->Xh[0],
-      (uint4*)h->Xq[0], row_vecs, h->dims.n_q);
+  // enough blocks to cover every SM several times even for small batches
+  const int slices = std::max(1, std::min(64, (h->num_sms * 8 + B - 1) / B));
+  gather_kernel<<<dim3(B, slices), 256, 0, s>>>((const uint4*)values, offsets, (const uint4*)cand,
+                                                h->plan, (uint4*)h->Xh[0], (uint4*)h->Xq[0],
+                                                row_vecs, h->dims.n_q);
   return cudaGetLastError();
 }
 

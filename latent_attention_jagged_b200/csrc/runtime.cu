@@ -25,7 +25,7 @@ size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 struct Layout {
   int64_t rows_h, rows_q;
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
-      off_work_count, off_work_next;
+      off_work_count, off_work_next, off_item_off;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
       off_final, off_mean, off_Zres, off_Xqres[2];
   size_t total;
@@ -73,6 +73,7 @@ Layout layout_of(const llatte_dims* d) {
   L.off_work = take(sizeof(int32_t) * 2 * nl * (size_t)L.max_work);
   L.off_work_count = take(sizeof(int32_t) * nl);
   L.off_work_next = take(sizeof(int32_t) * nl);
+  L.off_item_off = take(sizeof(int32_t) * (B + 1));
   for (int i = 0; i < 2; ++i) L.off_Xh[i] = take((size_t)L.rows_h * d->d * elem);
   for (int i = 0; i < 2; ++i) L.off_Xq[i] = take((size_t)L.rows_q * d->d * elem);
   L.off_C = take((size_t)L.rows_h * d->rank * elem);
@@ -87,7 +88,7 @@ Layout layout_of(const llatte_dims* d) {
   for (int i = 0; i < 2; ++i) L.off_Xqres[i] = take(res16);
   L.off_acc32 = take(sizeof(float) * std::max<size_t>((size_t)L.rows_h * d->rank,
                                                       (size_t)L.rows_q * d->d));
-  L.off_ctxbias = take(sizeof(float) * B * hr);
+  L.off_ctxbias = take(sizeof(float) * nl * B * hr);
   L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
   L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
   L.total = o;
@@ -333,6 +334,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   p.work = (int32_t*)(ws + Lo.off_work);
   p.work_count = (int32_t*)(ws + Lo.off_work_count);
   p.work_next = (int32_t*)(ws + Lo.off_work_next);
+  p.item_off = (int32_t*)(ws + Lo.off_item_off);
   p.stride = D.max_batch + 1;
   p.max_work = Lo.max_work;
   for (int i = 0; i < 2; ++i) { h->Xh[i] = ws + Lo.off_Xh[i]; h->Xq[i] = ws + Lo.off_Xq[i]; }
@@ -376,6 +378,13 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
 
   { StepTimer t(h, s, ST_PLAN); CK(launch_plan(h, offsets, B, s)); t.done(1); }
   { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, B, s)); t.done(1); }
+  if (D.d_ctx > 0) {  // context term of every layer's query projection, one launch
+    StepTimer t(h, s, ST_CTX);
+    CtxWeights cw = {};
+    for (int l = 0; l < L; ++l) cw.W[l] = h->layers[l].W_qkc;
+    CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, s));
+    t.done(1);
+  }
 
   for (int l = 0; l < L; ++l) {
     const LayerDev& W = h->layers[l];
@@ -385,14 +394,6 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     void* Xq_n = h->Xq[(l + 1) & 1];
     const bool last = l == L - 1;
 
-    if (D.d_ctx > 0) {
-      StepTimer t(h, s, ST_CTX);
-      GemmArgs g = {};
-      g.A = context; g.lda = D.d_ctx; g.W = W.W_qkc; g.D = h->ctxbias; g.ldd = hr;
-      g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = hr; g.K = D.d_ctx; g.epi = EPI_F32;
-      CK(launch_gemm_simt(e, 4, 4, g, s));
-      t.done(1);
-    }
     const bool tc = h->use_tc != 0;
     // epilogue arguments shared by both paths
     NormArgs kv_norm = {};
@@ -458,7 +459,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
-        q.bias = h->ctxbias; q.seg_off = p.qoff(l); q.B = B;
+        q.bias = h->ctxbias + (int64_t)l * B * hr; q.seg_off = p.qoff(l); q.B = B;
         CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1], LM.qk,
                           q, h->num_sms, s));
       } else {
@@ -466,7 +467,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
         g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
         g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = hr; g.K = d;
         g.epi = D.d_ctx > 0 ? EPI_USERBIAS : EPI_STORE;
-        g.bias = h->ctxbias; g.seg_off = p.qoff(l); g.B = B;
+        g.bias = h->ctxbias + (int64_t)l * B * hr; g.seg_off = p.qoff(l); g.B = B;
         CK(launch_gemm_simt(e, e, e, g, s));
       }
       t.done(1);

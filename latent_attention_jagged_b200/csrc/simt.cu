@@ -245,6 +245,49 @@ cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s) {
   return elem == 4 ? attn_t<float>(a, s) : attn_t<__nv_bfloat16>(a, s);
 }
 
+// ---------------------------------------------------------------- context term
+// bias[l][u][n] = sum_k c_u[k] W_qkc,l[n][k] for every layer at once: the
+// per-user part of the absorbed target-aware query W_qk [x ; c] (daiwk.github.io
+// notes, "core formula").  Block = (16 users, one layer); the context rows sit
+// in shared memory and each thread walks output columns n with 16 sums.
+constexpr int CTX_USERS = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
+                float* __restrict__ out) {
+  extern __shared__ float cs[];                       // [CTX_USERS][dc]
+  const int l = blockIdx.y;
+  const int u0 = blockIdx.x * CTX_USERS;
+  const int nu = min(CTX_USERS, B - u0);
+  for (int i = threadIdx.x; i < CTX_USERS * dc; i += blockDim.x) {
+    const int uu = i / dc, k = i % dc;
+    cs[i] = uu < nu ? to_f(ctx[(int64_t)(u0 + uu) * dc + k]) : 0.f;
+  }
+  __syncthreads();
+  const float* W = w.W[l];
+  for (int n = threadIdx.x; n < hr; n += blockDim.x) {
+    float acc[CTX_USERS] = {};
+    const float* wr = W + (int64_t)n * dc;
+    for (int k = 0; k < dc; ++k) {
+      const float wk = __ldg(wr + k);
+#pragma unroll
+      for (int uu = 0; uu < CTX_USERS; ++uu) acc[uu] = fmaf(cs[uu * dc + k], wk, acc[uu]);
+    }
+    for (int uu = 0; uu < nu; ++uu) out[((int64_t)l * B + u0 + uu) * hr + n] = acc[uu];
+  }
+}
+
+cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
+                            int dc, float* out, cudaStream_t s) {
+  if (B == 0 || dc == 0) return cudaSuccess;
+  dim3 grid((B + CTX_USERS - 1) / CTX_USERS, L);
+  const size_t sm = sizeof(float) * CTX_USERS * dc;
+  if (elem == 4) ctx_bias_kernel<float><<<grid, 256, sm, s>>>((const float*)ctx, w, B, hr, dc, out);
+  else ctx_bias_kernel<__nv_bfloat16><<<grid, 256, sm, s>>>((const __nv_bfloat16*)ctx, w, B, hr, dc, out);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- readout mean
 // mean[u] = (1 / rows_u) sum of the user's final rows (zero for no rows).
 __global__ void mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qoff,

@@ -79,6 +79,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Synchronise a group of warps that exchange values through shared memory
+// (init `bar` with the group's warp count).  Each warp arrives once (lane 0,
+// after __syncwarp, release) and waits for the phase to complete (acquire)
+// with the bounded wait above, so a group whose other members gave up cannot
+// hang here.  `phase` counts this group's uses.  Returns false on abort.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abort_flag,
+                                           int32_t* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase & 1u, abort_flag, status);
+  ++phase;
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -217,9 +231,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// SiLU(x) = x / (1 + e^-x) = x * 1 / (1 + 2^(-x log2 e)).
+// SiLU(x) = x / (1 + e^-x) = x * sigmoid(x) = (x / 2) * (1 + tanh(x / 2)):
+// one hardware tanh approximation (a single MUFU operation) per element.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float silu_approx(float x) {
-  return x * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * x));
+  const float h = 0.5f * x;
+  return fmaf(h, tanh_approx(h), h);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {

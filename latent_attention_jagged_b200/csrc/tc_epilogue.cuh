@@ -93,18 +93,18 @@ __device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N,
   for (int i = 0; i < 32; ++i) v[i] += r[i];
 }
 
-// Named barrier over the 8 epilogue warps (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 // Residual + RMSNorm epilogue of one 128-row tile whose accumulator holds the
 // full row (BN == N columns, starting at taddr).  Two warps share each TMEM
 // lane quadrant and take half of the columns each; their partial sums of
-// squares meet in `red` ([2][128] floats) behind the epilogue named barrier.
-// Pass 1 reads the accumulator, adds the residual (read once) and stages the
-// sum back in TMEM; pass 2 normalises, applies the gain and stores.
+// squares meet in `red` ([2][128] floats) behind the group barrier `xbar`
+// (bounded wait; returns false if the CTA is aborting).  Pass 1 reads the
+// accumulator, adds the residual (read once) and stages the sum back in TMEM;
+// pass 2 normalises, applies the gain and stores.
 template <int BN>
-__device__ __forceinline__ void norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
-                                              bool valid, int half, float* red, int rrow) {
+__device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
+                                              bool valid, int half, float* red, int rrow,
+                                              uint64_t* xbar, uint32_t& xphase,
+                                              volatile int* abort_flag, int32_t* status) {
   constexpr int HB = BN / 2;
   const int c0 = half * HB;
   const int N = BN;
@@ -120,7 +120,7 @@ __device__ __forceinline__ void norm_epilogue(const NormArgs& a, uint32_t taddr,
     if (a.resid) tmem_st32(taddr + c, v);
   }
   red[half * 128 + rrow] = ss;
-  epi_bar();
+  if (!group_sync(xbar, xphase, abort_flag, status)) return false;
   ss += red[(half ^ 1) * 128 + rrow];
   const float inv = rsqrtf(ss / (float)N + a.eps);
   // destinations of this row
@@ -171,6 +171,7 @@ __device__ __forceinline__ void norm_epilogue(const NormArgs& a, uint32_t taddr,
       if (r1) store_f16x32(r1 + c, v);
     }
   }
+  return true;
 }
 
 }  // namespace tc
