@@ -72,19 +72,49 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
                              abort_flag, p.status);
   } else {
     int u = 0;
-    if (EPI == TC_USERBIAS && valid) u = segment_of(p.seg_off, p.B, row);
+    if (EPI == TC_USERBIAS && valid) u = p.row_user[row];
+    if constexpr (HB >= 64) {
+      // 64 columns per step; the bias loads are issued before the TMEM read
 #pragma unroll 1
-    for (int c = c0; c < c0 + HB; c += 32) {
-      float v[32];
-      tmem_ld32(taddr + c, v);
-      if (valid) {
+      for (int c = c0; c < c0 + HB; c += 64) {
         const int n = n0 + c;
-        if (EPI == TC_USERBIAS) add_f32x32(p.bias + (int64_t)u * p.N + n, v);
-        if (EPI == TC_SILU) {
+        float4 b[16];
+        if (EPI == TC_USERBIAS && valid) {
+          const float4* bp = reinterpret_cast<const float4*>(p.bias + (int64_t)u * p.N + n);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = silu_approx(v[i]);
+          for (int j = 0; j < 16; ++j) b[j] = __ldg(bp + j);
         }
-        store_bf16x32(p.D + row * p.ldd + n, v);
+        float v[64];
+        tmem_ld64(taddr + c, v);
+        if (valid) {
+          if (EPI == TC_USERBIAS) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              v[4 * j] += b[j].x; v[4 * j + 1] += b[j].y; v[4 * j + 2] += b[j].z; v[4 * j + 3] += b[j].w;
+            }
+          }
+          if (EPI == TC_SILU) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = silu_approx(v[i]);
+          }
+          store_bf16x32(p.D + row * p.ldd + n, *reinterpret_cast<float(*)[32]>(&v[0]));
+          store_bf16x32(p.D + row * p.ldd + n + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c = c0; c < c0 + HB; c += 32) {
+        float v[32];
+        tmem_ld32(taddr + c, v);
+        if (valid) {
+          const int n = n0 + c;
+          if (EPI == TC_USERBIAS) add_f32x32(p.bias + (int64_t)u * p.N + n, v);
+          if (EPI == TC_SILU) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = silu_approx(v[i]);
+          }
+          store_bf16x32(p.D + row * p.ldd + n, v);
+        }
       }
     }
     return true;

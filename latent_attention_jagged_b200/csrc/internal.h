@@ -29,6 +29,9 @@ struct PlanDev {
   int32_t* work_count; // [L]
   int32_t* work_next;  // [L] dynamic scheduling counters
   int32_t* item_off;   // [max_batch+1] scratch: first work item of each user
+  int32_t* row_user;   // [L][max rows_q]: user of every query row of every layer
+  int64_t row_user_stride;
+  __host__ __device__ const int32_t* ruser(int l) const { return row_user + l * row_user_stride; }
   int64_t stride;      // max_batch + 1
   int32_t max_work;
 
@@ -145,6 +148,7 @@ struct NormArgs {
   // NORM_SCATTER (FFN2 output of layer l -> inputs of layer l+1 / outputs)
   const int64_t *qoff_l, *hoff_n, *qoff_n; const int32_t *n_l, *n_n; int B; int n_q;
   void* Xh_n; void* Xq_n; void* Xq_res_n; int last; float* out; float* final_rows;
+  const int32_t* row_user;           // user of each query row of layer l (tensor-core path)
 };
 enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
 cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s);

@@ -213,7 +213,7 @@ cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_t
 __global__ void __launch_bounds__(256)
 gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offsets,
               const uint4* __restrict__ cand, PlanDev p, uint4* __restrict__ Xh,
-              uint4* __restrict__ Xq, int row_vecs, int n_q) {
+              uint4* __restrict__ Xq, int row_vecs, int n_q, int n_layers) {
   // a batch the plan rejected has zero rows everywhere: copy nothing
   if (*p.hist_total(0) == 0 && *p.query_total(0) == 0) return;
   const int u = blockIdx.x;
@@ -223,6 +223,14 @@ gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offs
   const int64_t T = p.Tl(0)[u], n = p.nl(0)[u];
   const int64_t hoff = p.hoff(0)[u], qoff = p.qoff(0)[u], src0 = offsets[u];
   const int64_t rows = T + n + n_q;
+  // user of every query row of every layer (the epilogues' row -> user map)
+  for (int l = 0; l < n_layers; ++l) {
+    const int64_t q = (int64_t)p.nl(l)[u] + n_q;
+    int32_t* dst = p.row_user + l * p.row_user_stride + p.qoff(l)[u];
+    for (int64_t j = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; j < q;
+         j += (int64_t)gridDim.y * blockDim.x)
+      dst[j] = u;
+  }
   for (int64_t r = w0; r < rows; r += warps) {
     const uint4* src;
     uint4* dst;
@@ -247,7 +255,7 @@ cudaError_t launch_gather(const llatte_handle* h, const void* values, const int6
   const int slices = std::max(1, std::min(64, (h->num_sms * 8 + B - 1) / B));
   gather_kernel<<<dim3(B, slices), 256, 0, s>>>((const uint4*)values, offsets, (const uint4*)cand,
                                                 h->plan, (uint4*)h->Xh[0], (uint4*)h->Xq[0],
-                                                row_vecs, h->dims.n_q);
+                                                row_vecs, h->dims.n_q, h->dims.n_layers);
   return cudaGetLastError();
 }
 

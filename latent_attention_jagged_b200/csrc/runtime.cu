@@ -25,7 +25,7 @@ size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 struct Layout {
   int64_t rows_h, rows_q;
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
-      off_work_count, off_work_next, off_item_off;
+      off_work_count, off_work_next, off_item_off, off_row_user;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
       off_final, off_mean, off_Zres, off_Xqres[2];
   size_t total;
@@ -74,6 +74,7 @@ Layout layout_of(const llatte_dims* d) {
   L.off_work_count = take(sizeof(int32_t) * nl);
   L.off_work_next = take(sizeof(int32_t) * nl);
   L.off_item_off = take(sizeof(int32_t) * (B + 1));
+  L.off_row_user = take(sizeof(int32_t) * nl * (size_t)L.rows_q);
   for (int i = 0; i < 2; ++i) L.off_Xh[i] = take((size_t)L.rows_h * d->d * elem);
   for (int i = 0; i < 2; ++i) L.off_Xq[i] = take((size_t)L.rows_q * d->d * elem);
   L.off_C = take((size_t)L.rows_h * d->rank * elem);
@@ -335,6 +336,8 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   p.work_count = (int32_t*)(ws + Lo.off_work_count);
   p.work_next = (int32_t*)(ws + Lo.off_work_next);
   p.item_off = (int32_t*)(ws + Lo.off_item_off);
+  p.row_user = (int32_t*)(ws + Lo.off_row_user);
+  p.row_user_stride = Lo.rows_q;
   p.stride = D.max_batch + 1;
   p.max_work = Lo.max_work;
   for (int i = 0; i < 2; ++i) { h->Xh[i] = ws + Lo.off_Xh[i]; h->Xq[i] = ws + Lo.off_Xq[i]; }
@@ -421,6 +424,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     f_norm.Xh_n = Xh_n; f_norm.Xq_n = Xq_n; f_norm.last = last;
     f_norm.Xq_res_n = (res16 && !last) ? h->Xqres[(l + 1) & 1] : nullptr;
     f_norm.out = out; f_norm.final_rows = D.d_out ? h->final_rows : nullptr;
+    f_norm.row_user = p.ruser(l);
     const LayerMaps& LM = h->lmaps[l];
     auto tcp = [&](const int64_t* Mdev, int64_t cap, int N, int K) {
       TcGemmParams q = {};
@@ -460,6 +464,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
         q.bias = h->ctxbias + (int64_t)l * B * hr; q.seg_off = p.qoff(l); q.B = B;
+        q.row_user = p.ruser(l);
         CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1], LM.qk,
                           q, h->num_sms, s));
       } else {

@@ -108,13 +108,43 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   constexpr int HB = BN / 2;
   const int c0 = half * HB;
   const int N = BN;
-  // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM
+  // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
+  // The residual chunk is loaded (raw) before the TMEM read so that the two
+  // latencies overlap.
   float ss = 0.f;
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
+    uint4 rr[4];
+    const bool have = valid && a.resid;
+    if (have) {
+      const uint4* rp = reinterpret_cast<const uint4*>(
+          (a.resid_kind == RES_F16 ? (const void*)((const __half*)a.resid + row * N + c)
+                                   : (const void*)((const __nv_bfloat16*)a.resid + row * N + c)));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rr[j] = __ldg(rp + j);
+    }
     float v[32];
     tmem_ld32(taddr + c, v);
-    if (valid) add_resid(a, row, N, c, v);
+    if (have) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float2 f[4];
+        if (a.resid_kind == RES_F16) {
+          const __half2* h2 = reinterpret_cast<const __half2*>(&rr[j]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) f[k] = __half22float2(h2[k]);
+        } else {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&rr[j]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) f[k] = __bfloat1622float2(h2[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          v[8 * j + 2 * k] += f[k].x;
+          v[8 * j + 2 * k + 1] += f[k].y;
+        }
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     if (a.resid) tmem_st32(taddr + c, v);
@@ -133,7 +163,7 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
       d1 = (__nv_bfloat16*)a.dst + row * N;
       if (a.dst_res) r1 = (__half*)a.dst_res + row * N;
     } else {
-      const int u = segment_of(a.qoff_l, a.B, row);
+      const int u = a.row_user[row];
       const int64_t j = row - a.qoff_l[u];
       const int32_t nl = a.n_l[u];
       if (a.last) {
@@ -158,11 +188,11 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   // pass 2: normalise, scale by the gain, store
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
+    float g[32];
+    load_bf16x32((const __nv_bfloat16*)a.g + c, g);
     float v[32];
     tmem_ld32(taddr + c, v);
     if (valid) {
-      float g[32];
-      load_bf16x32((const __nv_bfloat16*)a.g + c, g);
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * g[i];
       if (d1) store_bf16x32(d1 + c, v);

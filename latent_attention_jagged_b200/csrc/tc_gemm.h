@@ -18,6 +18,7 @@ struct TcGemmParams {
   int N, K;
   __nv_bfloat16* D; int64_t ldd;                      // STORE / USERBIAS / SILU
   const float* bias; const int64_t* seg_off; int B;   // USERBIAS: bias[user(row), n]
+  const int32_t* row_user;                             // user of each row
   NormArgs norm;                                       // NORM (acc unused)
   int32_t* status;
 };
