@@ -10,17 +10,19 @@
 // one shared-memory copy of each C tile (K-major for S, MN-major for P V).
 //
 // Roles (320 threads, one CTA per SM, persistent over the sorted work list):
-//   warp 0      TMA: the Q~ block once per item, C tiles into a KV_STAGES ring
+//   warp 0      TMA: the Q~ block once per item, C tiles into a 3-stage ring
 //   warp 1      TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
 //               O += P(kt) C_kt, so the tensor pipe works while the softmax
 //               warps turn S(kt) into P(kt)
-//   warps 2..9  softmax, two warps per TMEM lane (= one pair), each taking
-//               half of the columns: masking
+//   warps 2..5  softmax, one TMEM lane (= one pair) per thread: masking
 //               (history row at position p sees keys t <= p; a query token
 //               sees every key t < T), online max / sum in fp32, P written to
 //               shared memory as bf16, lazy rescaling of O in TMEM (only when
-//               the running max grows by more than 2^8), final O / l to HBM.
-// TMEM: O in columns [0, r), S double-buffered after it.
+//               the running max grows by more than 2^8)
+//   warps 6..9  epilogue: O / l from TMEM to HBM, so the softmax warps move on
+//               to the next item at once
+// TMEM: O (double-buffered across items when 2 r + 2 KEYS <= 512 columns),
+// then S double-buffered across key tiles.
 #include <cuda.h>
 
 #include <algorithm>
@@ -36,24 +38,26 @@ using namespace tc;
 
 namespace {
 
-constexpr int kSoftmaxWarps = 8;                 // two per TMEM lane quadrant
-constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
+constexpr int kThreads = 320;
 
 template <int R>
 struct AttnCfg {
   static constexpr int KEYS = R >= 256 ? 64 : 128;     // keys per tile
   static constexpr int RSUB = R / 64;                  // 64-wide latent sub-tiles
+  static constexpr int OBUF = (2 * R + 2 * KEYS <= 512) ? 2 : 1;
+  static constexpr int QBUF = R <= 128 ? 2 : 1;          // query blocks in flight
   static constexpr int KV_STAGES = 3;
   static constexpr uint32_t Q_BYTES = 128 * R * 2;
   static constexpr uint32_t KV_BYTES = KEYS * R * 2;
   static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
   static constexpr uint32_t P_BYTES = 128 * KEYS * 2;
-  static constexpr uint32_t S_COL = R;                  // S buffers after O
-  static constexpr uint32_t RED_BYTES = 3 * 256 * 4;     // max exchange [2][2][128], sums [2][128]
-  static constexpr size_t SMEM = 1024 + Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256 +
-                                RED_BYTES;
+  static constexpr uint32_t S_COL = OBUF * R;           // S buffers after O
+  static constexpr uint32_t L_BYTES = 2 * 128 * 4;      // row sums handed to the epilogue
+  static constexpr size_t SMEM =
+      1024 + QBUF * Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256 + L_BYTES;
+  static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(R + 2 * KEYS <= 512, "TMEM budget");
+  static_assert(OBUF * R + 2 * KEYS <= 512, "TMEM budget");
 };
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -69,11 +73,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 struct Item {
   int u, b;
   int64_t T, n, q, hoff, qoff;
-  int nk;         // key tiles
+  int nk;         // key tiles (0: no key at all)
 };
 
-__device__ __forceinline__ Item load_item(const AttnTcParams& p, int idx, int keys) {
+__device__ __forceinline__ Item load_item(const AttnTcParams& p, int idx, int n_items, int keys) {
   Item it;
+  if (idx >= n_items) {
+    it.u = -1; it.b = 0; it.T = it.n = it.q = it.hoff = it.qoff = 0; it.nk = 0;
+    return it;
+  }
   it.u = p.work[2 * idx];
   it.b = p.work[2 * idx + 1];
   it.T = p.T[it.u];
@@ -93,44 +101,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                const AttnTcParams p) {
   using Cfg = AttnCfg<R>;
-  constexpr int KEYS = Cfg::KEYS, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES;
+  constexpr int KEYS = Cfg::KEYS, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES, OBUF = Cfg::OBUF,
+                QBUF = Cfg::QBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + Cfg::Q_BYTES;
+  uint8_t* sKV = sQ + QBUF * Cfg::Q_BYTES;
   uint8_t* sP = sKV + KS * Cfg::KV_BYTES;
   uint64_t* bars = (uint64_t*)(sP + 2 * Cfg::P_BYTES);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;            // [KS]
+  uint64_t* q_full = bars + 0;             // [2]
+  uint64_t* q_empty = bars + 2;            // [2]
+  uint64_t* kv_full = bars + 4;            // [KS]
   uint64_t* kv_empty = kv_full + KS;       // [KS]
   uint64_t* s_full = kv_empty + KS;        // [2]
   uint64_t* s_empty = s_full + 2;          // [2]
   uint64_t* p_full = s_empty + 2;          // [2]
   uint64_t* p_empty = p_full + 2;          // [2]
-  uint64_t* o_free = p_empty + 2;
-  uint64_t* drain = o_free + 1;
-  uint64_t* xbar = drain + 1;              // softmax group barrier (max / sum exchange)
-  uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
+  uint64_t* o_full = p_empty + 2;          // [OBUF] last PV done + row sums written
+  uint64_t* o_free = o_full + 2;           // [OBUF] epilogue has read O
+  uint64_t* drain = o_free + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* red = (float*)((uint8_t*)bars + 256);
+  float* lbuf = (float*)((uint8_t*)bars + 256);   // [2][128] row sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = *p.work_count;
+  const int step = gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], kSoftmaxWarps);
-      mbar_init(&p_full[s], kSoftmaxWarps);
+      mbar_init(&s_empty[s], 4);
+      mbar_init(&p_full[s], 4);
       mbar_init(&p_empty[s], 1);
+      mbar_init(&o_full[s], 1 + 4);        // the MMA commit + the four softmax warps
+      mbar_init(&o_free[s], 4);
     }
-    mbar_init(o_free, kSoftmaxWarps);
     mbar_init(drain, 1);
-    mbar_init(xbar, kSoftmaxWarps);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -150,14 +159,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       uint32_t itm = 0, g = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-        const Item it = load_item(p, idx, KEYS);
+      Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+        const Item it = nxt;
+        nxt = load_item(p, idx + step, n_items, KEYS);   // prefetch the next item's metadata
         if (it.nk == 0) continue;
-        if (!mbar_wait(q_empty, (itm & 1) ^ 1, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(q_full, Cfg::Q_BYTES);
+        const int qb = itm % QBUF;
+        if (!mbar_wait(&q_empty[qb], ((itm / QBUF) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&q_full[qb], Cfg::Q_BYTES);
         const int32_t qrow = (int32_t)(it.qoff * p.heads + (int64_t)it.b * 128);
+        uint8_t* qdst = sQ + qb * Cfg::Q_BYTES;
 #pragma unroll
-        for (int s = 0; s < RSUB; ++s) tma_load_2d(&tmQ, q_full, sQ + s * 16384, s * 64, qrow);
+        for (int s = 0; s < RSUB; ++s) tma_load_2d(&tmQ, &q_full[qb], qdst + s * 16384, s * 64, qrow);
         for (int kt = 0; kt < it.nk; ++kt, ++g) {
           const int st = g % KS;
           if (!mbar_wait(&kv_empty[st], ((g / KS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
@@ -177,10 +190,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16(128, KEYS, false, false);
       constexpr uint32_t IDESC_O = idesc_bf16(128, R, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
       uint32_t itm = 0, g = 0;
       bool ok = true;
-      auto issue_s = [&](uint32_t gg) -> bool {
+      auto issue_s = [&](uint32_t gg, uint32_t q_addr) -> bool {
         const int st = gg % KS;
         if (!mbar_wait(&kv_full[st], (gg / KS) & 1, abort_flag, p.status)) return false;
         if (!mbar_wait(&s_empty[gg & 1], ((gg >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
@@ -197,9 +209,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         umma_commit(&s_full[gg & 1]);
         return true;
       };
-      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+      // PV of tile gg (item number `item`, O buffer ob); `first` zeroes O
+      auto issue_pv = [&](uint32_t gg, bool first, int ob, uint32_t item) -> bool {
         if (!mbar_wait(&p_full[gg & 1], (gg >> 1) & 1, abort_flag, p.status)) return false;
-        if (first && !mbar_wait(o_free, (itm & 1) ^ 1, abort_flag, p.status)) return false;
+        // the O buffer of this item is free once the epilogue has read the
+        // item that used it OBUF items ago
+        if (first && !mbar_wait(&o_free[ob], ((item / OBUF) & 1) ^ 1, abort_flag, p.status))
+          return false;
         tc_fence_after();
         const int st = gg % KS;
         const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);
@@ -210,100 +226,97 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           // V = the same C tile read MN-major: 64-wide latent blocks are the
           // sub-tiles (LBO apart), 16 keys per MMA step = 2048 bytes
           const uint64_t bd = sdesc_sw128(kv_addr + k * 2048, Cfg::KV_SUB_BYTES, 1024);
-          umma_bf16(tmem, ad, bd, IDESC_O, (!first || k > 0) ? 1u : 0u);
+          umma_bf16(tmem + ob * R, ad, bd, IDESC_O, (!first || k > 0) ? 1u : 0u);
         }
-        // one commit per barrier: the C tile and the P buffer are free, and
-        // (through p_empty) the softmax warps learn that PV(gg) is in O
+        // the C tile and the P buffer are free, and (through p_empty) the
+        // softmax warps learn that PV(gg) is in O
         umma_commit(&kv_empty[st]);
         umma_commit(&p_empty[gg & 1]);
         return true;
       };
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-        const Item it = load_item(p, idx, KEYS);
+      // The PV of a tile is issued after the S of the next tile, also across
+      // item boundaries, so the softmax of tile g overlaps S(g + 1) even for
+      // one-tile items.  `pend` is the tile whose PV is still to be issued.
+      struct Pending { uint32_t g, item; int ob; bool first, last, valid; };
+      Pending pend = {0, 0, 0, false, false, false};
+      auto flush = [&]() -> bool {
+        if (!pend.valid) return true;
+        if (!issue_pv(pend.g, pend.first, pend.ob, pend.item)) return false;
+        if (pend.last) umma_commit(&o_full[pend.ob]);   // every PV of that item is in O
+        pend.valid = false;
+        return true;
+      };
+      Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+        const Item it = nxt;
+        nxt = load_item(p, idx + step, n_items, KEYS);
         if (it.nk == 0) continue;
-        if (!mbar_wait(q_full, itm & 1, abort_flag, p.status)) break;
-        const uint32_t g0 = g;
-        for (int kt = 0; kt < it.nk; ++kt) {
-          if (!issue_s(g0 + kt)) { ok = false; break; }
-          if (kt == it.nk - 1) umma_commit(q_empty);
-          if (kt > 0 && !issue_pv(g0 + kt - 1, kt - 1 == 0)) { ok = false; break; }
+        const int ob = itm % OBUF, qb = itm % QBUF;
+        // with one query buffer the next block only arrives after the last S
+        // of this one: finish the pending PV before waiting for it
+        if (QBUF == 1 && !flush()) break;
+        if (!mbar_wait(&q_full[qb], (itm / QBUF) & 1, abort_flag, p.status)) break;
+        const uint32_t q_addr = smem_u32(sQ + qb * Cfg::Q_BYTES);
+        for (int kt = 0; kt < it.nk; ++kt, ++g) {
+          if (!issue_s(g, q_addr)) { ok = false; break; }
+          if (kt == it.nk - 1) umma_commit(&q_empty[qb]);
+          if (!flush()) { ok = false; break; }
+          pend = {g, itm, ob, kt == 0, kt == it.nk - 1, true};
         }
-        if (!ok) break;
-        if (!issue_pv(g0 + it.nk - 1, it.nk == 1)) break;
-        g += it.nk;
         ++itm;
       }
+      if (ok) flush();
       umma_commit(drain);
       int dummy = 0;
       mbar_wait(drain, 0, &dummy, p.status);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax
-    // Two warps per TMEM lane quadrant: `half` takes columns
-    // [half * KEYS/2, ...) of every S tile and [half * R/2, ...) of O.  The
-    // row max of a tile is the max of both halves (exchanged in shared memory
-    // behind the softmax named barrier), so both halves make the same lazy
-    // rescaling decision; the row sums are combined once per item.
-    constexpr int HK = KEYS / 2, HR = R / 2;
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;              // pair within the block = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t g = 0, xphase = 0;
+    uint32_t g = 0, itm = 0;
     bool ok = true;
-    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-      const Item it = load_item(p, idx, KEYS);
+    Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+      const Item it = nxt;
+      nxt = load_item(p, idx + step, n_items, KEYS);
+      if (it.nk == 0) continue;
+      const int ob = itm % OBUF;
+      const uint32_t o_col = ob * R;
       const int64_t pair = (int64_t)it.b * 128 + row;
       const bool valid = pair < it.q * p.heads;
       const int64_t jl = pair / p.heads;
       const int64_t vis = !valid ? 0 : (jl < it.n ? it.T - it.n + jl + 1 : it.T);
-      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R + half * HR;
-      if (it.nk == 0) {
-        if (valid) {
-          uint4 z = make_uint4(0, 0, 0, 0);
-          for (int c = 0; c < HR; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
-        }
-        continue;
-      }
-      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and this half's sum
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
       for (int kt = 0; kt < it.nk; ++kt, ++g) {
-        // ---- this half of the S tile -> registers
+        // ---- pass 1 over the S tile in TMEM: masked row max.  Scores are
+        // already in log2 units (log2 e folded into q~); a row is masked only
+        // on the tiles it does not see entirely.
         bool w = mbar_wait(&s_full[g & 1], (g >> 1) & 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
-        float s[HK];
-#pragma unroll
-        for (int c = 0; c < HK; c += 32) {
-          float v[32];
-          tmem_ld32(lane_base + Cfg::S_COL + (g & 1) * KEYS + half * HK + c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c + i] = v[i];
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[g & 1]);
-        // ---- mask (only where this row does not see the whole tile) and the
-        // partial max; scores are already in log2 units (log2 e folded into q~)
-        const int64_t t0 = (int64_t)kt * KEYS + half * HK;
-        if (t0 + HK > vis) {
-          const int64_t lim = vis - t0;
-#pragma unroll
-          for (int c = 0; c < HK; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
-        }
+        const uint32_t s_addr = lane_base + Cfg::S_COL + (g & 1) * KEYS;
+        const int64_t t0 = (int64_t)kt * KEYS;
+        const bool partial = t0 + KEYS > vis;
+        const int64_t lim = vis - t0;
         float m8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
-        for (int c = 8; c < HK; c += 8)
+        for (int c = 0; c < KEYS; c += 64) {
+          float v[64];
+          tmem_ld64(s_addr + c, v);
+          if (partial) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-        float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        float* xm = red + (g & 1) * 256;
-        xm[half * 128 + row] = mt;
-        if (!group_sync(xbar, xphase, abort_flag, p.status)) { ok = false; break; }
-        mt = fmaxf(mt, xm[(half ^ 1) * 128 + row]);
+            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], v[i]);
+        }
+        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         // ---- lazy rescale of O and l (only when the max grows by > 8 in log2)
         float scale = 1.f;
         bool resc = false;
@@ -322,68 +335,102 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < HR; c += 32) {
+          for (int c = 0; c < R; c += 32) {
             float v[32];
-            tmem_ld32(lane_base + half * HR + c, v);
+            tmem_ld32(lane_base + o_col + c, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= scale;
-            tmem_st32(lane_base + half * HR + c, v);
+            tmem_st32(lane_base + o_col + c, v);
           }
           l_run *= scale;
         }
-        // ---- probabilities: 2^(s - m); masked scores are -inf and give 0.  A
-        // row that sees no key at all keeps m = -inf: subtract 0 instead so
-        // that -inf - (-inf) never happens.
+        // ---- pass 2: probabilities 2^(s - m) -> bf16 P tile in shared memory
+        // (128-byte swizzled, K-major).  Masked scores are -inf and give 0; a
+        // row that sees no key at all keeps m = -inf and subtracts 0 instead,
+        // so that -inf - (-inf) never happens.
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < HK; c += 8)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            s[c + i] = ex2_approx(s[c + i] - m_use);
-            l8[i] += s[c + i];
-          }
-        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        // ---- this half of the P tile -> shared memory (bf16, 128-byte
-        // swizzled, K-major: 64-key sub-tiles, 16-byte chunks XOR row % 8)
         bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
         const uint32_t pbase = smem_u32(sP + (g & 1) * Cfg::P_BYTES);
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c8 = 0; c8 < HK / 8; ++c8) {
-          const int ch = half * (HK / 8) + c8;          // 8-key chunk within the tile
-          const int sub = ch >> 3, cc = ch & 7;
-          const uint32_t addr = pbase + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-          const float* x = &s[8 * c8];
-          uint4 v = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                               pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          st_shared_v4(addr, v);
+        for (int c = 0; c < KEYS; c += 64) {
+          float v[64];
+          tmem_ld64(s_addr + c, v);
+          if (partial) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            v[i] = ex2_approx(v[i] - m_use);
+            l8[i & 7] += v[i];
+          }
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const int ch = (c >> 3) + q4;                 // 8-key chunk within the tile
+            const int sub = ch >> 3, cc = ch & 7;
+            const uint32_t addr = pbase + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+            const float* x = &v[8 * q4];
+            uint4 pk = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                  pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+            st_shared_v4(addr, pk);
+          }
         }
+        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        // S buffer consumed (both passes done), P tile written
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[g & 1]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[g & 1]);
       }
       if (!ok) break;
-      // ---- final: O / l -> HBM, once the last PV(g-1) has completed
-      float* xl = red + 512;
-      xl[half * 128 + row] = l_run;
-      if (!group_sync(xbar, xphase, abort_flag, p.status)) break;
-      const float l_tot = l_run + xl[(half ^ 1) * 128 + row];
-      // both halves have read the sums before the next item writes them
-      if (!group_sync(xbar, xphase, abort_flag, p.status)) break;
-      bool w4 = mbar_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, p.status);
+      // ---- hand the row sum to the epilogue warps (the sum slot of this O
+      // buffer is free once the epilogue has finished the item OBUF ago)
+      bool w4 = mbar_wait(&o_free[ob], ((itm / OBUF) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w4)) break;
+      lbuf[ob * 128 + row] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_full[ob]);
+      ++itm;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t itm = 0;
+    Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+    for (int idx = blockIdx.x; idx < n_items; idx += step) {
+      const Item it = nxt;
+      nxt = load_item(p, idx + step, n_items, KEYS);
+      const int64_t pair = (int64_t)it.b * 128 + row;
+      const bool valid = pair < it.q * p.heads;
+      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R;
+      if (it.nk == 0) {                 // no key: the attention output is zero
+        if (valid) {
+          uint4 z = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < R; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
+        }
+        continue;
+      }
+      const int ob = itm % OBUF;
+      bool w = mbar_wait(&o_full[ob], (itm / OBUF) & 1, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
-      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float l = lbuf[ob * 128 + row];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < HR; c += 32) {
-        float v[32];
-        tmem_ld32(lane_base + half * HR + c, v);
+      for (int c = 0; c < R; c += 64) {
+        float v[64];
+        tmem_ld64(lane_base + ob * R + c, v);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 8; ++j)
             dst[j] = make_uint4(pack_bf16(v[8 * j] * inv, v[8 * j + 1] * inv),
                                 pack_bf16(v[8 * j + 2] * inv, v[8 * j + 3] * inv),
                                 pack_bf16(v[8 * j + 4] * inv, v[8 * j + 5] * inv),
@@ -392,7 +439,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0) mbar_arrive(&o_free[ob]);
+      ++itm;
     }
   }
   __syncthreads();
