@@ -9,6 +9,7 @@
 //   MMA1(j)  H[j % 2]  = Z W1[j]^T        (TMEM, two 128-column buffers)
 //   SiLU(j)  8 epilogue warps: H -> SiLU -> bf16 -> shared memory (A operand)
 //   MMA2(j)  OUT      += SiLU(H_j) W2[:, j]^T   (TMEM, 256 columns)
+// (each CTA starts at a different chunk and wraps around)
 // MMA1(j + 2) is issued right after MMA2(j), so the tensor pipe works on the
 // next chunks while the epilogue warps apply SiLU.  After the last chunk the
 // same warps run the residual + RMSNorm epilogue on OUT and scatter each row
@@ -83,6 +84,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
   const int64_t M = *p.M_dev;
   const int64_t num_tiles = (M + 127) / 128;
   const int NC = p.F / HC;
+  // Every CTA walks the hidden chunks in a rotated order, so that the SMs do
+  // not all read the same weight lines from L2 at the same moment.
+  const int c0 = blockIdx.x % NC;
+  auto chunk = [&](int j) { return (c0 + j) % NC; };
 
   if (threadIdx.x == 0) {
     mbar_init(z_full, 1);
@@ -148,9 +153,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
         if (!mbar_wait(z_empty, (ti & 1) ^ 1, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(z_full, Z_BYTES);
         for (int s = 0; s < D / 64; ++s) tma_load_2d(&tmZ, z_full, sZ + s * 16384, 64 * s, (int)(t * 128));
-        ok = load_w1(0) && (NC < 2 || load_w1(1));
+        ok = load_w1(chunk(0)) && (NC < 2 || load_w1(chunk(1)));
         for (int j = 0; j < NC && ok; ++j) {
-          ok = load_w2(j) && (j + 2 >= NC || load_w1(j + 2));
+          ok = load_w2(chunk(j)) && (j + 2 >= NC || load_w1(chunk(j + 2)));
         }
       }
     }
@@ -163,7 +168,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
       const uint32_t z_addr = smem_u32(sZ);
       uint32_t w = 0, ti = 0, gc = 0;
       bool ok = true;
-      auto mma1 = [&](int j, uint32_t gcj) -> bool {   // H[gcj&1] = Z W1[j]^T
+      auto mma1 = [&](int j, uint32_t gcj) -> bool {   // H[gcj&1] = Z W1[chunk(j)]^T
         const uint32_t d = tmem + H_COL + (gcj & 1) * HC;
         for (int s2 = 0; s2 < 2; ++s2) {
           const int st = w % W_STAGES;
@@ -183,7 +188,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
         if (j == NC - 1) umma_commit(z_empty);
         return true;
       };
-      auto mma2 = [&](int j, uint32_t gcj) -> bool {   // OUT += SiLU(H_j) W2[:, j]^T
+      auto mma2 = [&](int j, uint32_t gcj) -> bool {   // OUT += SiLU(H_j) W2[:, chunk(j)]^T
         if (!mbar_wait(&hs_full[gcj & 1], (gcj >> 1) & 1, abort_flag, p.status)) return false;
         if (j == 0 && !mbar_wait(out_empty, (ti & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();

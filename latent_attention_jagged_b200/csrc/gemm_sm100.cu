@@ -146,6 +146,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n_tiles = p.N / BN;
   const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles;
   const int KB = p.K / BK;
+  const int kb0 = blockIdx.x % KB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -176,10 +177,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kb * BK, mt * BM);
+          // k-blocks in a per-CTA rotated order: the SMs do not all read the
+          // same weight lines from L2 at the same moment
+          const int kx = ((kb + kb0) % KB) * BK;
+          tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kx, mt * BM);
 #pragma unroll
           for (int s2 = 0; s2 < NSUB; ++s2)
-            tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * NI * 128, kb * BK,
+            tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * NI * 128, kx,
                         nt * BN + s2 * NI);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
