@@ -204,6 +204,22 @@ int llatte_profile_step(llatte_handle* handle, int step, const char** name, doub
 int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t B,
                        int64_t* plan_out, int32_t* status_out, void* stream);
 
+/*
+ * Self-check of an arithmetic building block; the paper has no counterpart.
+ * The attention softmax computes one probability pair in four with an
+ * exponential built from fused multiply-adds (range reduction x = j + f,
+ * |f| <= 1/2, a fitted cubic for 2^f, j added to the exponent field) instead
+ * of the special-function unit.  This evaluates exactly that device function:
+ *
+ *   x     device float [n], inputs (<= 64; below -125 they act as -125)
+ *   y     device float [n], y[i] ~ 2^x[i], relative error below 1e-4
+ *   y_hw  device float [n] or NULL: 2^x[i] from the hardware ex2.approx
+ *
+ * Returns LLATTE_ERR_ARG for n < 0 or a NULL x / y with n > 0.  Asynchronous
+ * on `stream`; allocates nothing.
+ */
+int llatte_exp2_eval(const float* x, float* y, float* y_hw, int64_t n, void* stream);
+
 /* Free the handle and everything it owns (synchronises its device). */
 void llatte_destroy(llatte_handle* handle);
 

@@ -48,7 +48,7 @@ class llatte_layer_w(ctypes.Structure):
 EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
            "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
-           "llatte_plan_static")
+           "llatte_plan_static", "llatte_exp2_eval")
 PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
@@ -88,6 +88,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_profile_step.restype = ctypes.c_int
     lib.llatte_plan_static.argtypes = [P(llatte_dims), VP, I32, VP, VP, VP]
     lib.llatte_plan_static.restype = ctypes.c_int
+    lib.llatte_exp2_eval.argtypes = [VP, VP, VP, I64, VP]
+    lib.llatte_exp2_eval.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
@@ -273,3 +275,17 @@ def plan_static(dims, offsets: torch.Tensor, max_batch: int, max_len: int, max_t
     if rc != LLATTE_OK:
         raise LlatteError(rc, "llatte_plan_static")
     return out, status
+
+
+def exp2_eval(x: torch.Tensor, with_hw: bool = True, stream=None):
+    """2^x through the softmax's FMA-pipe exponential (and, with `with_hw`,
+    through the hardware ex2.approx) for a contiguous CUDA float32 tensor."""
+    lib = load_library()
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    y_hw = torch.empty_like(x) if with_hw else None
+    rc = lib.llatte_exp2_eval(_ptr(x), _ptr(y), _ptr(y_hw), x.numel(), _stream_ptr(stream))
+    if rc != LLATTE_OK:
+        raise LlatteError(rc, "llatte_exp2_eval")
+    return (y, y_hw) if with_hw else y

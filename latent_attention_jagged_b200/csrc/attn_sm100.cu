@@ -298,9 +298,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_addr = lane_base + Cfg::S_COL + (g & 1) * KEYS;
-        const int64_t t0 = (int64_t)kt * KEYS;
-        const bool partial = t0 + KEYS > vis;
-        const int64_t lim = vis - t0;
+        // keys [0, lim) of this tile are visible to the row; a 64-key chunk
+        // is masked only when some row of the warp stops inside it
+        const int64_t lim64 = vis - (int64_t)kt * KEYS;
+        const int lim = lim64 <= 0 ? 0 : (lim64 >= KEYS ? KEYS : (int)lim64);
         float m8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
@@ -308,12 +309,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < KEYS; c += 64) {
           float v[64];
           tmem_ld64(s_addr + c, v);
-          if (partial) {
+          if (__any_sync(0xffffffffu, lim < c + 64)) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : -INFINITY;
           }
 #pragma unroll
-          for (int i = 0; i < 64; ++i) m8[i & 7] = fmaxf(m8[i & 7], v[i]);
+          for (int i = 0; i < 64; i += 16) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
+          }
         }
         const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
@@ -345,27 +349,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           l_run *= scale;
         }
         // ---- pass 2: probabilities 2^(s - m) -> bf16 P tile in shared memory
-        // (128-byte swizzled, K-major).  Masked scores are -inf and give 0; a
-        // row that sees no key at all keeps m = -inf and subtracts 0 instead,
-        // so that -inf - (-inf) never happens.
+        // (128-byte swizzled, K-major).  One pair in four takes the FMA-pipe
+        // exponential, the rest the special-function unit, so that both pipes
+        // share the work.  Masked keys are set to 0 after the exponential; a
+        // row that sees no key at all keeps m = -inf and subtracts 0 instead.
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
+        const float2 nm2 = make_float2(-m_use, -m_use);
         bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
         const uint32_t pbase = smem_u32(sP + (g & 1) * Cfg::P_BYTES);
-        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float2 l4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) l4[i] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < KEYS; c += 64) {
           float v[64];
           tmem_ld64(s_addr + c, v);
-          if (partial) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : -INFINITY;
+          for (int j = 0; j < 32; ++j) {
+            float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
+            if ((j & 3) == 3) {
+              x = exp2_fma2(x);
+            } else {
+              x.x = ex2_approx(x.x);
+              x.y = ex2_approx(x.y);
+            }
+            v[2 * j] = x.x;
+            v[2 * j + 1] = x.y;
+          }
+          if (__any_sync(0xffffffffu, lim < c + 64)) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : 0.f;
           }
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            v[i] = ex2_approx(v[i] - m_use);
-            l8[i & 7] += v[i];
-          }
+          for (int j = 0; j < 32; ++j)
+            l4[j & 3] = add_f2(l4[j & 3], make_float2(v[2 * j], v[2 * j + 1]));
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             const int ch = (c >> 3) + q4;                 // 8-key chunk within the tile
@@ -377,7 +395,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             st_shared_v4(addr, pk);
           }
         }
-        l_run += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        l_run += ((l4[0].x + l4[0].y) + (l4[1].x + l4[1].y)) +
+                 ((l4[2].x + l4[2].y) + (l4[3].x + l4[3].y));
         // S buffer consumed (both passes done), P tile written
         tc_fence_before();
         __syncwarp();

@@ -274,5 +274,57 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ---------------------------------------------------------------- packed fp32
+// Two fp32 lanes per instruction (the f32x2 forms of sm_100), round to nearest.
+__device__ __forceinline__ float2 add_f2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "add.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 fma_f2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%6, %7};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for two values on the FMA pipe, so that the softmax need not send every
+// exponential through the special-function unit.  Classic range reduction:
+// x = j + f with j = rint(x) and f in [-1/2, 1/2]; 2^f from a cubic whose
+// coefficients were fitted here for least maximum relative error on that
+// interval (7.5e-5, far below the bf16 rounding of the probabilities); 2^j
+// enters by adding j to the exponent field.  rint comes from adding and
+// subtracting 1.5 * 2^23, which leaves j in the low mantissa bits of the sum.
+// Valid for x <= 64; inputs below -125 are clamped (result ~2^-125, which
+// the callers mask to zero where it matters).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = add_f2(x, make_float2(kRound, kRound));
+  const float2 j = add_f2(t, make_float2(-kRound, -kRound));
+  const float2 f = fma_f2(j, make_float2(-1.f, -1.f), x);
+  float2 p = fma_f2(make_float2(0x1.c3f76p-5f, 0x1.c3f76p-5f), f,
+                    make_float2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+  p = fma_f2(p, f, make_float2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+  p = fma_f2(p, f, make_float2(0x1.fff692p-1f, 0x1.fff692p-1f));
+  float2 r;
+  r.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
+  r.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+  return r;
+}
+
 }  // namespace tc
 }  // namespace llatte
