@@ -60,16 +60,6 @@ struct AttnCfg {
   static_assert(OBUF * R + 2 * KEYS <= 512, "TMEM budget");
 };
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
 struct Item {
   int u, b;
   int64_t T, n, q, hoff, qoff;

@@ -44,16 +44,6 @@ constexpr uint32_t W_STAGE_BYTES = 32768;            // W1: 2 boxes 128 x 64; W2
 constexpr uint32_t OUT_COL = 0, H_COL = D;           // TMEM columns
 constexpr size_t SMEM = 1024 + Z_BYTES + 2 * HS_BYTES + W_STAGES * W_STAGE_BYTES + 256;
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmW1,
               const __grid_constant__ CUtensorMap tmW2, const FfnTcParams p) {
@@ -263,8 +253,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
       if (!__all_sync(0xffffffffu, w3)) break;
       tc_fence_after();
       const int64_t row = t * 128 + rr;
+      // staging buffers: in the first hidden tile, after `red` (both hidden
+      // tiles are idle while the output epilogue runs; the group barrier
+      // below keeps the next SiLU chunk out until every warp is done)
       if (!norm_epilogue<D>(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr, xbar,
-                            xphase, abort_flag, p.status))
+                            xphase, abort_flag, p.status,
+                            smem_u32(sHs) + 1024 + (warp - 2) * kStageBytes))
         break;
       // every partner has read `red` before a SiLU chunk reuses that memory
       if (!group_sync(xbar, xphase, abort_flag, p.status)) break;

@@ -55,66 +55,57 @@ struct GemmCfg {
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 512 ? 2 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4;
+  static constexpr size_t SMEM =
+      1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4 + kEpiWarps * kStageBytes;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 // Epilogue of one 128 x BN tile.  Two warps share each TMEM lane quadrant;
-// `half` selects which half of the columns this thread handles.
+// `half` selects which half of the columns this thread handles.  Stores pass
+// through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
 __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
                                          bool valid, int n0, int half, float* red, int rrow,
                                          uint64_t* xbar, uint32_t& xphase,
-                                         volatile int* abort_flag) {
+                                         volatile int* abort_flag, uint32_t stg) {
   constexpr int HB = BN / 2;                 // columns per thread
   const int c0 = half * HB;
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue<BN>(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
-                             abort_flag, p.status);
+                             abort_flag, p.status, stg);
   } else {
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = p.row_user[row];
-    if constexpr (HB >= 64) {
-      // 64 columns per step; the bias loads are issued before the TMEM read
+    __nv_bfloat16* drow = valid ? p.D + row * p.ldd + n0 : nullptr;
+    constexpr int STEP = HB >= 64 ? 64 : 32;
+    // STEP columns per step; the bias loads are issued before the TMEM read
 #pragma unroll 1
-      for (int c = c0; c < c0 + HB; c += 64) {
-        const int n = n0 + c;
-        float4 b[16];
-        if (EPI == TC_USERBIAS && valid) {
-          const float4* bp = reinterpret_cast<const float4*>(p.bias + (int64_t)u * p.N + n);
+    for (int c = c0; c < c0 + HB; c += STEP) {
+      const int n = n0 + c;
+      float4 b[STEP / 4];
+      if (EPI == TC_USERBIAS && valid) {
+        const float4* bp = reinterpret_cast<const float4*>(p.bias + (int64_t)u * p.N + n);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) b[j] = __ldg(bp + j);
-        }
-        float v[64];
-        tmem_ld64(taddr + c, v);
-        if (valid) {
-          if (EPI == TC_USERBIAS) {
+        for (int j = 0; j < STEP / 4; ++j) b[j] = __ldg(bp + j);
+      }
+      float v[STEP];
+      if constexpr (STEP == 64) tmem_ld64(taddr + c, v);
+      else tmem_ld32(taddr + c, v);
+      if (EPI == TC_USERBIAS && valid) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              v[4 * j] += b[j].x; v[4 * j + 1] += b[j].y; v[4 * j + 2] += b[j].z; v[4 * j + 3] += b[j].w;
-            }
-          }
-          if (EPI == TC_SILU) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = silu_approx(v[i]);
-          }
-          store_bf16x32(p.D + row * p.ldd + n, *reinterpret_cast<float(*)[32]>(&v[0]));
-          store_bf16x32(p.D + row * p.ldd + n + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        for (int j = 0; j < STEP / 4; ++j) {
+          v[4 * j] += b[j].x; v[4 * j + 1] += b[j].y; v[4 * j + 2] += b[j].z; v[4 * j + 3] += b[j].w;
         }
       }
-    } else {
-#pragma unroll 1
-      for (int c = c0; c < c0 + HB; c += 32) {
-        float v[32];
-        tmem_ld32(taddr + c, v);
-        if (valid) {
-          const int n = n0 + c;
-          if (EPI == TC_USERBIAS) add_f32x32(p.bias + (int64_t)u * p.N + n, v);
-          if (EPI == TC_SILU) {
+      if (EPI == TC_SILU) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = silu_approx(v[i]);
-          }
-          store_bf16x32(p.D + row * p.ldd + n, v);
-        }
+        for (int i = 0; i < STEP; ++i) v[i] = silu_approx(v[i]);
+      }
+#pragma unroll
+      for (int h = 0; h < STEP / 32; ++h) {
+        uint4 x[4];
+        pack_bf16x32(&v[32 * h], x);
+        stage_store(stg, x, drow ? drow + c + 32 * h : nullptr);
       }
     }
     return true;
@@ -140,6 +131,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][2 halves][128]
+  uint8_t* sStage = (uint8_t*)(red + 2 * 2 * 128);                  // [epilogue warp][kStageBytes]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
@@ -241,7 +233,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
       if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
-                             red + (it & 1) * 256, rr, xbar, xphase, abort_flag))
+                             red + (it & 1) * 256, rr, xbar, xphase, abort_flag,
+                             smem_u32(sStage + (warp - 2) * kStageBytes)))
         break;
       tc_fence_before();
       __syncwarp();

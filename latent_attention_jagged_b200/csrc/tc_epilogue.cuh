@@ -1,5 +1,5 @@
-// Epilogue building blocks shared by the tensor-core kernels: vectorised
-// loads / stores of 32-column row chunks and the fused residual + RMSNorm
+// Epilogue building blocks shared by the tensor-core kernels: row staging
+// through shared memory for row-contiguous global accesses, and the fused residual + RMSNorm
 // epilogue (LLaTTE notes, huaxiaozhuan.com, appendix A.2 display: post-norm
 // Z = RMSNorm(R + MLA(R)), X = RMSNorm(Z + FFN(Z)); the FFN-down variant
 // scatters each output row into the next layer's history / query rows).
@@ -31,66 +31,69 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v
   }
 }
 
-__device__ __forceinline__ void add_f32x32(const float* src, float (&v)[32]) {
-  const float4* s = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float4 w = __ldg(s + j);
-    v[4 * j] += w.x; v[4 * j + 1] += w.y; v[4 * j + 2] += w.z; v[4 * j + 3] += w.w;
-  }
-}
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    d[j] = make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
-                      pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
-}
-
-__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
-  float4* d = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) d[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-}
-
-__device__ __forceinline__ void load_f16x32(const __half* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint4 w = __ldg(s + j);
-    const __half2* h = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float2 f = __half22float2(h[k]);
-      v[8 * j + 2 * k] = f.x;
-      v[8 * j + 2 * k + 1] = f.y;
-    }
-  }
-}
-
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void store_f16x32(__half* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    d[j] = make_uint4(pack_f16(v[8 * j], v[8 * j + 1]), pack_f16(v[8 * j + 2], v[8 * j + 3]),
-                      pack_f16(v[8 * j + 4], v[8 * j + 5]), pack_f16(v[8 * j + 6], v[8 * j + 7]));
+// ---------------------------------------------------------------- row staging
+// A TMEM load leaves one accumulator row in each lane, but global memory is
+// fastest when one instruction covers whole 32-byte sectors of few rows.  So
+// rows pass through a per-warp shared-memory buffer of 32 rows x 64 bytes
+// (kStageBytes): the 16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3),
+// which keeps both directions free of bank conflicts, and every global access
+// then moves 8 rows x 64 bytes.  All 32 lanes must take part; a lane whose
+// row has no source / destination passes a null pointer.
+constexpr uint32_t kStageBytes = 32 * 64;
+
+__device__ __forceinline__ uint32_t stage_slot(uint32_t stg, int r, int k) {
+  return stg + (uint32_t)r * 64u + ((uint32_t)(k ^ ((r >> 1) & 3)) << 4);
 }
 
-// Residual chunk for columns [c, c + 32) of `row`, added to v (bf16 or fp16).
-__device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N, int c,
-                                          float (&v)[32]) {
-  if (!a.resid) return;
-  float r[32];
-  if (a.resid_kind == RES_F16) load_f16x32((const __half*)a.resid + row * N + c, r);
-  else load_bf16x32((const __nv_bfloat16*)a.resid + row * N + c, r);
+// Lane l holds the 64 bytes x of row l; the row goes to lane l's `dst`.
+__device__ __forceinline__ void stage_store(uint32_t stg, const uint4 (&x)[4], void* dst) {
+  const int lane = threadIdx.x & 31, k = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] += r[i];
+  for (int j = 0; j < 4; ++j) st_shared_v4(stage_slot(stg, lane, j), x[j]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2);
+    char* d = reinterpret_cast<char*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), r));
+    const uint4 v = ld_shared_v4(stage_slot(stg, r, k));
+    if (d) *reinterpret_cast<uint4*>(d + 16 * k) = v;
+  }
+  __syncwarp();
+}
+
+// Global loads of the 64 bytes at lane r's `src` (zeros for a null pointer),
+// 8 rows per instruction; stage_deliver then hands each lane its own row.
+__device__ __forceinline__ void stage_fetch(const void* src, uint4 (&t)[4]) {
+  const int lane = threadIdx.x & 31, k = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2);
+    const char* s = reinterpret_cast<const char*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), r));
+    t[i] = s ? __ldg(reinterpret_cast<const uint4*>(s + 16 * k)) : make_uint4(0, 0, 0, 0);
+  }
+}
+__device__ __forceinline__ void stage_deliver(uint32_t stg, const uint4 (&t)[4], uint4 (&x)[4]) {
+  const int lane = threadIdx.x & 31, k = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) st_shared_v4(stage_slot(stg, i * 8 + (lane >> 2), k), t[i]);
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) x[j] = ld_shared_v4(stage_slot(stg, lane, j));
+  __syncwarp();
+}
+
+__device__ __forceinline__ void pack_bf16x32(const float* v, uint4 (&x)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    x[j] = make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                      pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
 // Residual + RMSNorm epilogue of one 128-row tile whose accumulator holds the
@@ -99,33 +102,32 @@ __device__ __forceinline__ void add_resid(const NormArgs& a, int64_t row, int N,
 // squares meet in `red` ([2][128] floats) behind the group barrier `xbar`
 // (bounded wait; returns false if the CTA is aborting).  Pass 1 reads the
 // accumulator, adds the residual (read once) and stages the sum back in TMEM;
-// pass 2 normalises, applies the gain and stores.
+// pass 2 normalises, applies the gain and stores.  Global reads and writes go
+// through the warp's staging buffer `stg` (kStageBytes of shared memory).
 template <int BN>
 __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
                                               bool valid, int half, float* red, int rrow,
                                               uint64_t* xbar, uint32_t& xphase,
-                                              volatile int* abort_flag, int32_t* status) {
+                                              volatile int* abort_flag, int32_t* status,
+                                              uint32_t stg) {
   constexpr int HB = BN / 2;
   const int c0 = half * HB;
   const int N = BN;
+  const bool have = a.resid != nullptr;
+  const char* rsrc = (valid && have) ? (const char*)a.resid + (row * N) * 2 : nullptr;
   // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
-  // The residual chunk is loaded (raw) before the TMEM read so that the two
+  // The residual rows are fetched before the TMEM read so that the two
   // latencies overlap.
   float ss = 0.f;
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
-    uint4 rr[4];
-    const bool have = valid && a.resid;
-    if (have) {
-      const uint4* rp = reinterpret_cast<const uint4*>(
-          (a.resid_kind == RES_F16 ? (const void*)((const __half*)a.resid + row * N + c)
-                                   : (const void*)((const __nv_bfloat16*)a.resid + row * N + c)));
-#pragma unroll
-      for (int j = 0; j < 4; ++j) rr[j] = __ldg(rp + j);
-    }
+    uint4 t[4];
+    if (have) stage_fetch(rsrc ? rsrc + 2 * c : nullptr, t);
     float v[32];
     tmem_ld32(taddr + c, v);
     if (have) {
+      uint4 rr[4];
+      stage_deliver(stg, t, rr);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float2 f[4];
@@ -147,13 +149,13 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
     }
 #pragma unroll
     for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-    if (a.resid) tmem_st32(taddr + c, v);
+    if (have) tmem_st32(taddr + c, v);
   }
   red[half * 128 + rrow] = ss;
   if (!group_sync(xbar, xphase, abort_flag, status)) return false;
   ss += red[(half ^ 1) * 128 + rrow];
   const float inv = rsqrtf(ss / (float)N + a.eps);
-  // destinations of this row
+  // destinations of this row (null: none)
   __nv_bfloat16* d1 = nullptr;
   __nv_bfloat16* d2 = nullptr;
   float* f1 = nullptr;
@@ -185,6 +187,9 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
       }
     }
   }
+  const unsigned full = 0xffffffffu;
+  const bool any_d1 = __any_sync(full, d1 != nullptr), any_d2 = __any_sync(full, d2 != nullptr);
+  const bool any_f1 = __any_sync(full, f1 != nullptr), any_r1 = __any_sync(full, r1 != nullptr);
   // pass 2: normalise, scale by the gain, store
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
@@ -192,13 +197,31 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
     load_bf16x32((const __nv_bfloat16*)a.g + c, g);
     float v[32];
     tmem_ld32(taddr + c, v);
-    if (valid) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * g[i];
-      if (d1) store_bf16x32(d1 + c, v);
-      if (d2) store_bf16x32(d2 + c, v);
-      if (f1) store_f32x32(f1 + c, v);
-      if (r1) store_f16x32(r1 + c, v);
+    for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * g[i];
+    uint4 x[4];
+    if (any_d1 || any_d2) {
+      pack_bf16x32(v, x);
+      if (any_d1) stage_store(stg, x, d1 ? d1 + c : nullptr);
+      if (any_d2) stage_store(stg, x, d2 ? d2 + c : nullptr);
+    }
+    if (any_r1) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        x[j] = make_uint4(pack_f16(v[8 * j], v[8 * j + 1]), pack_f16(v[8 * j + 2], v[8 * j + 3]),
+                          pack_f16(v[8 * j + 4], v[8 * j + 5]), pack_f16(v[8 * j + 6], v[8 * j + 7]));
+      stage_store(stg, x, r1 ? r1 + c : nullptr);
+    }
+    if (any_f1) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x[j] = make_uint4(__float_as_uint(v[16 * h + 4 * j]), __float_as_uint(v[16 * h + 4 * j + 1]),
+                            __float_as_uint(v[16 * h + 4 * j + 2]),
+                            __float_as_uint(v[16 * h + 4 * j + 3]));
+        stage_store(stg, x, f1 ? f1 + c + 16 * h : nullptr);
+      }
     }
   }
   return true;
