@@ -42,7 +42,8 @@ constexpr uint32_t Z_BYTES = 128 * D * 2;            // 64 KB: 4 sub-tiles of 12
 constexpr uint32_t HS_BYTES = 128 * HC * 2;          // 32 KB: 2 sub-tiles of 128 x 64
 constexpr uint32_t W_STAGE_BYTES = 32768;            // W1: 2 boxes 128 x 64; W2: 1 box 256 x 64
 constexpr uint32_t OUT_COL = 0, H_COL = D;           // TMEM columns
-constexpr size_t SMEM = 1024 + Z_BYTES + 2 * HS_BYTES + W_STAGES * W_STAGE_BYTES + 256;
+constexpr size_t SMEM = 1024 + Z_BYTES + 2 * HS_BYTES + W_STAGES * W_STAGE_BYTES + 256 + D * 2;
+static_assert(SMEM <= 232448, "shared memory budget");
 
 __global__ void __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmW1,
@@ -69,6 +70,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
   // the residual-norm exchange lives in the first SiLU buffer: while OUT is
   // normalised no MMA reads that buffer and no SiLU chunk is being written
   float* red = (float*)sHs;
+  __nv_bfloat16* sG = (__nv_bfloat16*)((uint8_t*)sW + W_STAGES * W_STAGE_BYTES + 256);  // gain [D]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t M = *p.M_dev;
@@ -102,6 +104,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  load_gain(p.norm, D, sG);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -249,16 +252,18 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
         if (lane == 0) mbar_arrive(&hs_full[gc & 1]);
       }
       if (!ok) break;
+      const int64_t row = t * 128 + rr;
+      uint4 pre[4];
+      norm_prefetch<D>(p.norm, row, row < M, half, pre);
       bool w3 = mbar_wait(out_full, ti & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w3)) break;
       tc_fence_after();
-      const int64_t row = t * 128 + rr;
       // staging buffers: in the first hidden tile, after `red` (both hidden
       // tiles are idle while the output epilogue runs; the group barrier
       // below keeps the next SiLU chunk out until every warp is done)
       if (!norm_epilogue<D>(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr, xbar,
                             xphase, abort_flag, p.status,
-                            smem_u32(sHs) + 1024 + (warp - 2) * kStageBytes))
+                            smem_u32(sHs) + 1024 + (warp - 2) * kStageBytes, pre, sG))
         break;
       // every partner has read `red` before a SiLU chunk reuses that memory
       if (!group_sync(xbar, xphase, abort_flag, p.status)) break;

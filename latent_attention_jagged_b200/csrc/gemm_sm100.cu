@@ -56,7 +56,8 @@ struct GemmCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 512 ? 2 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
   static constexpr size_t SMEM =
-      1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4 + kEpiWarps * kStageBytes;
+      1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4 + kEpiWarps * kStageBytes +
+      BN * 2;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -67,12 +68,13 @@ template <int BN, int EPI>
 __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
                                          bool valid, int n0, int half, float* red, int rrow,
                                          uint64_t* xbar, uint32_t& xphase,
-                                         volatile int* abort_flag, uint32_t stg) {
+                                         volatile int* abort_flag, uint32_t stg,
+                                         const uint4 (&pre)[4], const __nv_bfloat16* sg) {
   constexpr int HB = BN / 2;                 // columns per thread
   const int c0 = half * HB;
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue<BN>(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
-                             abort_flag, p.status, stg);
+                             abort_flag, p.status, stg, pre, sg);
   } else {
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = p.row_user[row];
@@ -132,6 +134,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][2 halves][128]
   uint8_t* sStage = (uint8_t*)(red + 2 * 2 * 128);                  // [epilogue warp][kStageBytes]
+  __nv_bfloat16* sG = (__nv_bfloat16*)(sStage + kEpiWarps * kStageBytes);   // RMSNorm gain [BN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
@@ -154,6 +157,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  if constexpr (EPI == TC_NORM) load_gain(p.norm, BN, sG);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -226,15 +230,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0, it = 0;
     uint32_t acc_phase = 0, xphase = 0;
     for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
+      uint4 pre[4];
+      if constexpr (EPI == TC_NORM) norm_prefetch<BN>(p.norm, row, row < M, half, pre);
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
       if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
                              red + (it & 1) * 256, rr, xbar, xphase, abort_flag,
-                             smem_u32(sStage + (warp - 2) * kStageBytes)))
+                             smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
         break;
       tc_fence_before();
       __syncwarp();

@@ -16,21 +16,6 @@
 namespace llatte {
 namespace tc {
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint4 w = __ldg(s + j);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float2 f = __bfloat1622float2(h[k]);
-      v[8 * j + 2 * k] = f.x;
-      v[8 * j + 2 * k + 1] = f.y;
-    }
-  }
-}
-
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -96,33 +81,50 @@ __device__ __forceinline__ void pack_bf16x32(const float* v, uint4 (&x)[4]) {
                       pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
+// First residual chunk of this thread's half row, fetched before the
+// accumulator is ready so that its latency overlaps the wait.
+template <int BN>
+__device__ __forceinline__ void norm_prefetch(const NormArgs& a, int64_t row, bool valid,
+                                              int half, uint4 (&t)[4]) {
+  if (a.resid)
+    stage_fetch(valid ? (const char*)a.resid + (row * BN + half * (BN / 2)) * 2 : nullptr, t);
+}
+
+// Copy the RMSNorm gain (N bf16) into shared memory; every thread of the CTA
+// calls this before the CTA's first barrier.
+__device__ __forceinline__ void load_gain(const NormArgs& a, int N, __nv_bfloat16* sg) {
+  for (int i = threadIdx.x; i < N / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(sg)[i] = __ldg(reinterpret_cast<const uint4*>(a.g) + i);
+}
+
 // Residual + RMSNorm epilogue of one 128-row tile whose accumulator holds the
 // full row (BN == N columns, starting at taddr).  Two warps share each TMEM
 // lane quadrant and take half of the columns each; their partial sums of
 // squares meet in `red` ([2][128] floats) behind the group barrier `xbar`
 // (bounded wait; returns false if the CTA is aborting).  Pass 1 reads the
-// accumulator, adds the residual (read once) and stages the sum back in TMEM;
-// pass 2 normalises, applies the gain and stores.  Global reads and writes go
-// through the warp's staging buffer `stg` (kStageBytes of shared memory).
+// accumulator, adds the residual (read once, one chunk ahead; `pre` holds the
+// first chunk from norm_prefetch) and stages the sum back in TMEM; pass 2
+// normalises, applies the gain (`sg`, in shared memory) and stores.  Global
+// reads and writes go through the warp's staging buffer `stg`.
 template <int BN>
 __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
                                               bool valid, int half, float* red, int rrow,
                                               uint64_t* xbar, uint32_t& xphase,
                                               volatile int* abort_flag, int32_t* status,
-                                              uint32_t stg) {
+                                              uint32_t stg, const uint4 (&pre)[4],
+                                              const __nv_bfloat16* sg) {
   constexpr int HB = BN / 2;
   const int c0 = half * HB;
   const int N = BN;
   const bool have = a.resid != nullptr;
   const char* rsrc = (valid && have) ? (const char*)a.resid + (row * N) * 2 : nullptr;
   // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
-  // The residual rows are fetched before the TMEM read so that the two
-  // latencies overlap.
   float ss = 0.f;
+  uint4 t[4] = {pre[0], pre[1], pre[2], pre[3]};
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
-    uint4 t[4];
-    if (have) stage_fetch(rsrc ? rsrc + 2 * c : nullptr, t);
+    uint4 tn[4];
+    if (have && c + 32 < c0 + HB) stage_fetch(rsrc ? rsrc + 2 * (c + 32) : nullptr, tn);
     float v[32];
     tmem_ld32(taddr + c, v);
     if (have) {
@@ -150,6 +152,8 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
 #pragma unroll
     for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     if (have) tmem_st32(taddr + c, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) t[j] = tn[j];
   }
   red[half * 128 + rrow] = ss;
   if (!group_sync(xbar, xphase, abort_flag, status)) return false;
@@ -194,7 +198,20 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
     float g[32];
-    load_bf16x32((const __nv_bfloat16*)a.g + c, g);
+    {
+      const uint32_t ga = smem_u32(sg + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = ld_shared_v4(ga + 16 * j);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h2[k]);
+          g[8 * j + 2 * k] = f.x;
+          g[8 * j + 2 * k + 1] = f.y;
+        }
+      }
+    }
     float v[32];
     tmem_ld32(taddr + c, v);
 #pragma unroll
