@@ -9,20 +9,25 @@
 // of the user's current history: S = Q~ C^T and O~ = softmax(S) C both read
 // one shared-memory copy of each C tile (K-major for S, MN-major for P V).
 //
-// Roles (320 threads, one CTA per SM, persistent over the sorted work list):
-//   warp 0      TMA: the Q~ block once per item, C tiles into a 3-stage ring
-//   warp 1      TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
-//               O += P(kt) C_kt, so the tensor pipe works while the softmax
-//               warps turn S(kt) into P(kt)
-//   warps 2..5  softmax, one TMEM lane (= one pair) per thread: masking
-//               (history row at position p sees keys t <= p; a query token
-//               sees every key t < T), online max / sum in fp32, P written to
-//               shared memory as bf16, lazy rescaling of O in TMEM (only when
-//               the running max grows by more than 2^8)
-//   warps 6..9  epilogue: O / l from TMEM to HBM, so the softmax warps move on
-//               to the next item at once
+// Roles (448 threads, one CTA per SM, persistent over the sorted work list):
+//   warp 0       TMA: the Q~ block once per item, C tiles into a 4-stage ring
+//   warp 1       TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
+//                O += P(kt) C_kt, so the tensor pipe works while the softmax
+//                warps turn S(kt) into P(kt)
+//   warps 2..9   softmax, two warps per TMEM lane quadrant, each taking half
+//                of the tile's keys for the quadrant's 32 pairs (one pair per
+//                thread): masking (history row at position p sees keys
+//                t <= p; a query token sees every key t < T), row max (the two
+//                halves meet in shared memory behind a bounded pair barrier),
+//                2^(s - m) in fp32, P written back over S in TMEM as bf16,
+//                lazy rescaling of O in TMEM (only when the running max grows
+//                by more than 2^8)
+//   warps 10..13 epilogue: O / l from TMEM to HBM, so the softmax warps move
+//                on to the next item at once
 // TMEM: O (double-buffered across items when 2 r + 2 KEYS <= 512 columns),
-// then S double-buffered across key tiles.
+// then S double-buffered across key tiles; P(kt) overwrites S(kt) and the
+// P V product reads it from TMEM.  The MMAs of one thread run in issue order,
+// so S(kt + 2) (issued after P(kt) V) cannot overwrite P(kt) early.
 #include <cuda.h>
 
 #include <algorithm>
@@ -31,6 +36,7 @@
 #include "internal.h"
 #include "tc_attn.h"
 #include "tc_common.cuh"
+#include "tc_epilogue.cuh"
 
 namespace llatte {
 
@@ -38,27 +44,43 @@ using namespace tc;
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kSplit = 2;                          // softmax warps per lane quadrant
+constexpr int kSoftWarps = 4 * kSplit;
+constexpr int kEpiWarps = 4;
+constexpr int kEpiWarp0 = 2 + kSoftWarps;
+constexpr int kThreads = 32 * (2 + kSoftWarps + kEpiWarps);
 
 template <int R>
 struct AttnCfg {
   static constexpr int KEYS = R >= 256 ? 64 : 128;     // keys per tile
+  static constexpr int KP = KEYS / kSplit;             // keys per softmax warp
   static constexpr int RSUB = R / 64;                  // 64-wide latent sub-tiles
   static constexpr int OBUF = (2 * R + 2 * KEYS <= 512) ? 2 : 1;
   static constexpr int QBUF = R <= 128 ? 2 : 1;          // query blocks in flight
-  static constexpr int KV_STAGES = 3;
+  static constexpr int KV_STAGES = 4;
   static constexpr uint32_t Q_BYTES = 128 * R * 2;
   static constexpr uint32_t KV_BYTES = KEYS * R * 2;
   static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
-  static constexpr uint32_t P_BYTES = 128 * KEYS * 2;
   static constexpr uint32_t S_COL = OBUF * R;           // S buffers after O
+  static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t L_BYTES = 2 * 128 * 4;      // row sums handed to the epilogue
-  static constexpr size_t SMEM =
-      1024 + QBUF * Q_BYTES + (size_t)KV_STAGES * KV_BYTES + 2 * P_BYTES + 256 + L_BYTES;
+  static constexpr uint32_t MX_BYTES = 2 * kSplit * 128 * 4;   // partial row maxima
+  static constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)KV_STAGES * KV_BYTES +
+                                 BAR_BYTES + L_BYTES + MX_BYTES + kEpiWarps * kStageBytes;
   static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(OBUF * R + 2 * KEYS <= 512, "TMEM budget");
+  static_assert(KP == 32 || KP == 64, "softmax chunk");
 };
+
+// TMEM column (relative to the S buffer) of the packed bf16 P for keys
+// [16 kk, 16 kk + 16): each softmax warp packs its KP keys into the first
+// KP / 2 columns of its own half of the buffer.
+template <int KP>
+__device__ __forceinline__ uint32_t p_col(int kk) {
+  const int key = 16 * kk;
+  return (uint32_t)((key / KP) * KP + (key % KP) / 2);
+}
 
 struct Item {
   int u, b;
@@ -86,33 +108,55 @@ __device__ __forceinline__ Item load_item(const AttnTcParams& p, int idx, int n_
   return it;
 }
 
+// KP fp32 columns of this lane's TMEM row.
+template <int KP>
+__device__ __forceinline__ void tmem_ld_kp(uint32_t taddr, float (&v)[KP]) {
+  if constexpr (KP == 64) tmem_ld64(taddr, v);
+  else tmem_ld32(taddr, v);
+}
+
+// KP / 2 packed bf16 pairs into this lane's TMEM row.
+template <int KP>
+__device__ __forceinline__ void tmem_st_packed(uint32_t taddr, const uint32_t (&w)[KP / 2]) {
+  if constexpr (KP == 64) {
+    float f[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(w[i]);
+    tmem_st32(taddr, f);          // waits for the store
+  } else {
+    tmem_st16u(taddr, w);
+    tmem_wait_st();
+  }
+}
+
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                const AttnTcParams p) {
   using Cfg = AttnCfg<R>;
-  constexpr int KEYS = Cfg::KEYS, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES, OBUF = Cfg::OBUF,
-                QBUF = Cfg::QBUF;
+  constexpr int KEYS = Cfg::KEYS, KP = Cfg::KP, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES,
+                OBUF = Cfg::OBUF, QBUF = Cfg::QBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + QBUF * Cfg::Q_BYTES;
-  uint8_t* sP = sKV + KS * Cfg::KV_BYTES;
-  uint64_t* bars = (uint64_t*)(sP + 2 * Cfg::P_BYTES);
+  uint64_t* bars = (uint64_t*)(sKV + KS * Cfg::KV_BYTES);
   uint64_t* q_full = bars + 0;             // [2]
   uint64_t* q_empty = bars + 2;            // [2]
   uint64_t* kv_full = bars + 4;            // [KS]
   uint64_t* kv_empty = kv_full + KS;       // [KS]
   uint64_t* s_full = kv_empty + KS;        // [2]
-  uint64_t* s_empty = s_full + 2;          // [2]
-  uint64_t* p_full = s_empty + 2;          // [2]
-  uint64_t* p_empty = p_full + 2;          // [2]
-  uint64_t* o_full = p_empty + 2;          // [OBUF] last PV done + row sums written
+  uint64_t* p_full = s_full + 2;           // [2] both halves of P(kt) written
+  uint64_t* p_empty = p_full + 2;          // [2] P(kt) V done (O holds it)
+  uint64_t* o_full = p_empty + 2;          // [OBUF] last PV done + row sums added
   uint64_t* o_free = o_full + 2;           // [OBUF] epilogue has read O
-  uint64_t* drain = o_free + 2;
+  uint64_t* pair_bar = o_free + 2;         // [4] the two softmax warps of a quadrant
+  uint64_t* drain = pair_bar + 4;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* lbuf = (float*)((uint8_t*)bars + 256);   // [2][128] row sums
+  float* lbuf = (float*)((uint8_t*)bars + Cfg::BAR_BYTES);   // [2][128] row sums
+  float* mx = lbuf + 2 * 128;                                  // [2][kSplit][128]
+  uint8_t* sStage = (uint8_t*)(mx + 2 * kSplit * 128);         // [kEpiWarps][kStageBytes]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = *p.work_count;
@@ -123,18 +167,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int s = 0; s < KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[s], kSoftWarps);
       mbar_init(&p_empty[s], 1);
-      mbar_init(&o_full[s], 1 + 4);        // the MMA commit + the four softmax warps
-      mbar_init(&o_free[s], 4);
+      mbar_init(&o_full[s], 1 + kSoftWarps);   // the MMA commit + every softmax warp
+      mbar_init(&o_free[s], kEpiWarps);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&pair_bar[q], kSplit);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmC);
   }
+  for (int i = threadIdx.x; i < 2 * 128; i += blockDim.x) lbuf[i] = 0.f;
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
@@ -182,10 +227,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t IDESC_O = idesc_bf16(128, R, false, true);
       uint32_t itm = 0, g = 0;
       bool ok = true;
+      // S(gg) into S buffer gg & 1.  That buffer last held P(gg - 2), whose
+      // P V product was issued before this call, so the in-order tensor pipe
+      // reads it first.
       auto issue_s = [&](uint32_t gg, uint32_t q_addr) -> bool {
         const int st = gg % KS;
         if (!mbar_wait(&kv_full[st], (gg / KS) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(&s_empty[gg & 1], ((gg >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
         tc_fence_after();
         const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);
         const uint32_t d = tmem + Cfg::S_COL + (gg & 1) * KEYS;
@@ -199,7 +246,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         umma_commit(&s_full[gg & 1]);
         return true;
       };
-      // PV of tile gg (item number `item`, O buffer ob); `first` zeroes O
+      // PV of tile gg (item number `item`, O buffer ob); `first` zeroes O.
+      // A = P(gg) from TMEM, B = the C tile read MN-major.
       auto issue_pv = [&](uint32_t gg, bool first, int ob, uint32_t item) -> bool {
         if (!mbar_wait(&p_full[gg & 1], (gg >> 1) & 1, abort_flag, p.status)) return false;
         // the O buffer of this item is free once the epilogue has read the
@@ -209,17 +257,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
         const int st = gg % KS;
         const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);
-        const uint32_t p_addr = smem_u32(sP + (gg & 1) * Cfg::P_BYTES);
+        const uint32_t p_tmem = tmem + Cfg::S_COL + (gg & 1) * KEYS;
 #pragma unroll
         for (int k = 0; k < KEYS / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(p_addr + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-          // V = the same C tile read MN-major: 64-wide latent blocks are the
-          // sub-tiles (LBO apart), 16 keys per MMA step = 2048 bytes
+          // 64-wide latent blocks are the sub-tiles (LBO apart), 16 keys per
+          // MMA step = 2048 bytes
           const uint64_t bd = sdesc_sw128(kv_addr + k * 2048, Cfg::KV_SUB_BYTES, 1024);
-          umma_bf16(tmem + ob * R, ad, bd, IDESC_O, (!first || k > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + ob * R, p_tmem + p_col<KP>(k), bd, IDESC_O,
+                       (!first || k > 0) ? 1u : 0u);
         }
-        // the C tile and the P buffer are free, and (through p_empty) the
-        // softmax warps learn that PV(gg) is in O
+        // the C tile is free, and (through p_empty) the softmax warps learn
+        // that PV(gg) is in O
         umma_commit(&kv_empty[st]);
         umma_commit(&p_empty[gg & 1]);
         return true;
@@ -261,12 +309,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_wait(drain, 0, &dummy, p.status);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ softmax
     const int quad = warp & 3;
+    const int part = (warp - 2) / 4;               // which half of the tile's keys
     const int row = quad * 32 + lane;              // pair within the block = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t g = 0, itm = 0;
+    uint32_t g = 0, itm = 0, pphase = 0;
     bool ok = true;
     Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
     for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
@@ -274,44 +323,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       nxt = load_item(p, idx + step, n_items, KEYS);
       if (it.nk == 0) continue;
       const int ob = itm % OBUF;
-      const uint32_t o_col = ob * R;
+      const uint32_t o_col = ob * R + part * (R / 2);   // this warp's half of O
       const int64_t pair = (int64_t)it.b * 128 + row;
       const bool valid = pair < it.q * p.heads;
       const int64_t jl = pair / p.heads;
       const int64_t vis = !valid ? 0 : (jl < it.n ? it.T - it.n + jl + 1 : it.T);
-      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and partial sum
       for (int kt = 0; kt < it.nk; ++kt, ++g) {
-        // ---- pass 1 over the S tile in TMEM: masked row max.  Scores are
-        // already in log2 units (log2 e folded into q~); a row is masked only
-        // on the tiles it does not see entirely.
+        // ---- masked row max over this warp's keys.  Scores are already in
+        // log2 units (log2 e folded into q~).
         bool w = mbar_wait(&s_full[g & 1], (g >> 1) & 1, abort_flag, p.status);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s_addr = lane_base + Cfg::S_COL + (g & 1) * KEYS;
-        // keys [0, lim) of this tile are visible to the row; a 64-key chunk
-        // is masked only when some row of the warp stops inside it
-        const int64_t lim64 = vis - (int64_t)kt * KEYS;
-        const int lim = lim64 <= 0 ? 0 : (lim64 >= KEYS ? KEYS : (int)lim64);
+        const uint32_t s_addr = lane_base + Cfg::S_COL + (g & 1) * KEYS + part * KP;
+        // keys [0, lim) of this warp's KP are visible to the row; masking is
+        // applied only when some row of the warp stops inside them
+        const int64_t lim64 = vis - (int64_t)kt * KEYS - part * KP;
+        const int lim = lim64 <= 0 ? 0 : (lim64 >= KP ? KP : (int)lim64);
+        const bool masked = __any_sync(0xffffffffu, lim < KP);
+        float v[KP];
+        tmem_ld_kp<KP>(s_addr, v);
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < KP; ++i) v[i] = (i < lim) ? v[i] : -INFINITY;
+        }
         float m8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < KEYS; c += 64) {
-          float v[64];
-          tmem_ld64(s_addr + c, v);
-          if (__any_sync(0xffffffffu, lim < c + 64)) {
+        for (int i = 0; i < KP; i += 16) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : -INFINITY;
-          }
-#pragma unroll
-          for (int i = 0; i < 64; i += 16) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
-          }
+          for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
         }
-        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        // ---- lazy rescale of O and l (only when the max grows by > 8 in log2)
+        float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        // the two halves of the row meet: both warps end with the same max
+        float* mxs = mx + (g & 1) * kSplit * 128;
+        mxs[part * 128 + row] = mt;
+        if (!group_sync(&pair_bar[quad], pphase, abort_flag, p.status)) { ok = false; break; }
+        mt = fmaxf(mt, mxs[(part ^ 1) * 128 + row]);
+        // ---- lazy rescale of O and l (only when the max grows by > 8 in log2);
+        // both warps of the quadrant take the same decisions
         float scale = 1.f;
         bool resc = false;
         if (kt == 0) {
@@ -329,79 +381,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < R; c += 32) {
-            float v[32];
-            tmem_ld32(lane_base + o_col + c, v);
+          for (int c = 0; c < R / 2; c += 32) {
+            float o[32];
+            tmem_ld32(lane_base + o_col + c, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= scale;
-            tmem_st32(lane_base + o_col + c, v);
+            for (int i = 0; i < 32; ++i) o[i] *= scale;
+            tmem_st32(lane_base + o_col + c, o);
           }
           l_run *= scale;
         }
-        // ---- pass 2: probabilities 2^(s - m) -> bf16 P tile in shared memory
-        // (128-byte swizzled, K-major).  One pair in four takes the FMA-pipe
-        // exponential, the rest the special-function unit, so that both pipes
-        // share the work.  Masked keys are set to 0 after the exponential; a
+        // ---- probabilities 2^(s - m) -> bf16, written over S in TMEM.  One
+        // pair in four takes the FMA-pipe exponential, the rest the special-
+        // function unit.  Masked keys are set to 0 after the exponential; a
         // row that sees no key at all keeps m = -inf and subtracts 0 instead.
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
         const float2 nm2 = make_float2(-m_use, -m_use);
-        bool w3 = mbar_wait(&p_empty[g & 1], ((g >> 1) & 1) ^ 1, abort_flag, p.status);
-        if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
-        const uint32_t pbase = smem_u32(sP + (g & 1) * Cfg::P_BYTES);
+#pragma unroll
+        for (int j = 0; j < KP / 2; ++j) {
+          float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
+          if ((j & 3) == 3) {
+            x = exp2_fma2(x);
+          } else {
+            x.x = ex2_approx(x.x);
+            x.y = ex2_approx(x.y);
+          }
+          v[2 * j] = x.x;
+          v[2 * j + 1] = x.y;
+        }
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < KP; ++i) v[i] = (i < lim) ? v[i] : 0.f;
+        }
         float2 l4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) l4[i] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < KEYS; c += 64) {
-          float v[64];
-          tmem_ld64(s_addr + c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
-            if ((j & 3) == 3) {
-              x = exp2_fma2(x);
-            } else {
-              x.x = ex2_approx(x.x);
-              x.y = ex2_approx(x.y);
-            }
-            v[2 * j] = x.x;
-            v[2 * j + 1] = x.y;
-          }
-          if (__any_sync(0xffffffffu, lim < c + 64)) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = (c + i < lim) ? v[i] : 0.f;
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            l4[j & 3] = add_f2(l4[j & 3], make_float2(v[2 * j], v[2 * j + 1]));
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const int ch = (c >> 3) + q4;                 // 8-key chunk within the tile
-            const int sub = ch >> 3, cc = ch & 7;
-            const uint32_t addr = pbase + sub * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-            const float* x = &v[8 * q4];
-            uint4 pk = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                  pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-            st_shared_v4(addr, pk);
-          }
-        }
+        for (int j = 0; j < KP / 2; ++j)
+          l4[j & 3] = add_f2(l4[j & 3], make_float2(v[2 * j], v[2 * j + 1]));
         l_run += ((l4[0].x + l4[0].y) + (l4[1].x + l4[1].y)) +
                  ((l4[2].x + l4[2].y) + (l4[3].x + l4[3].y));
-        // S buffer consumed (both passes done), P tile written
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[g & 1]);
-        fence_proxy_async_smem();
+        uint32_t pk[KP / 2];
+#pragma unroll
+        for (int j = 0; j < KP / 2; ++j) pk[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
+        tmem_st_packed<KP>(s_addr, pk);
+        // P(g) half written: the MMA may read it once both halves are in
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[g & 1]);
       }
       if (!ok) break;
-      // ---- hand the row sum to the epilogue warps (the sum slot of this O
-      // buffer is free once the epilogue has finished the item OBUF ago)
+      // ---- add this half's row sum for the epilogue warps (the sum slot of
+      // this O buffer is free, and zero, once the epilogue has finished the
+      // item OBUF ago)
       bool w4 = mbar_wait(&o_free[ob], ((itm / OBUF) & 1) ^ 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w4)) break;
-      lbuf[ob * 128 + row] = l_run;
+      atomicAdd(&lbuf[ob * 128 + row], l_run);
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_full[ob]);
       ++itm;
@@ -411,6 +445,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t stg = smem_u32(sStage + (warp - kEpiWarp0) * kStageBytes);
     uint32_t itm = 0;
     Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
     for (int idx = blockIdx.x; idx < n_items; idx += step) {
@@ -418,12 +453,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       nxt = load_item(p, idx + step, n_items, KEYS);
       const int64_t pair = (int64_t)it.b * 128 + row;
       const bool valid = pair < it.q * p.heads;
-      __nv_bfloat16* orow = p.Ot + (it.qoff * p.heads + pair) * R;
+      __nv_bfloat16* orow = valid ? p.Ot + (it.qoff * p.heads + pair) * R : nullptr;
       if (it.nk == 0) {                 // no key: the attention output is zero
-        if (valid) {
-          uint4 z = make_uint4(0, 0, 0, 0);
-          for (int c = 0; c < R; c += 8) *reinterpret_cast<uint4*>(orow + c) = z;
-        }
+        const uint4 z[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                            make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        for (int c = 0; c < R; c += 32) stage_store(stg, z, orow ? orow + c : nullptr);
         continue;
       }
       const int ob = itm % OBUF;
@@ -431,19 +465,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!__all_sync(0xffffffffu, w)) break;
       tc_fence_after();
       const float l = lbuf[ob * 128 + row];
+      lbuf[ob * 128 + row] = 0.f;        // ready for the item that reuses this buffer
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
       for (int c = 0; c < R; c += 64) {
         float v[64];
         tmem_ld64(lane_base + ob * R + c, v);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_uint4(pack_bf16(v[8 * j] * inv, v[8 * j + 1] * inv),
-                                pack_bf16(v[8 * j + 2] * inv, v[8 * j + 3] * inv),
-                                pack_bf16(v[8 * j + 4] * inv, v[8 * j + 5] * inv),
-                                pack_bf16(v[8 * j + 6] * inv, v[8 * j + 7] * inv));
+        for (int i = 0; i < 64; ++i) v[i] *= inv;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4 x[4];
+          pack_bf16x32(&v[32 * h], x);
+          stage_store(stg, x, orow ? orow + c + 32 * h : nullptr);
         }
       }
       tc_fence_before();

@@ -253,15 +253,15 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ C
       }
       if (!ok) break;
       const int64_t row = t * 128 + rr;
-      uint4 pre[4];
-      norm_prefetch<D>(p.norm, row, row < M, half, pre);
+      NormPre<D, 2> pre;   // two chunks ahead: the register budget is tight here
+      norm_prefetch(p.norm, row, row < M, half, pre);
       bool w3 = mbar_wait(out_full, ti & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w3)) break;
       tc_fence_after();
       // staging buffers: in the first hidden tile, after `red` (both hidden
       // tiles are idle while the output epilogue runs; the group barrier
       // below keeps the next SiLU chunk out until every warp is done)
-      if (!norm_epilogue<D>(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr, xbar,
+      if (!norm_epilogue(p.norm, lane_base + OUT_COL, row, row < M, half, red, rr, xbar,
                             xphase, abort_flag, p.status,
                             smem_u32(sHs) + 1024 + (warp - 2) * kStageBytes, pre, sG))
         break;

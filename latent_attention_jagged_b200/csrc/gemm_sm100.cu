@@ -69,11 +69,11 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
                                          bool valid, int n0, int half, float* red, int rrow,
                                          uint64_t* xbar, uint32_t& xphase,
                                          volatile int* abort_flag, uint32_t stg,
-                                         const uint4 (&pre)[4], const __nv_bfloat16* sg) {
+                                         NormPre<BN, 4>& pre, const __nv_bfloat16* sg) {
   constexpr int HB = BN / 2;                 // columns per thread
   const int c0 = half * HB;
   if constexpr (EPI == TC_NORM) {
-    return norm_epilogue<BN>(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
+    return norm_epilogue(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
                              abort_flag, p.status, stg, pre, sg);
   } else {
     int u = 0;
@@ -233,8 +233,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
-      uint4 pre[4];
-      if constexpr (EPI == TC_NORM) norm_prefetch<BN>(p.norm, row, row < M, half, pre);
+      NormPre<BN, 4> pre;
+      if constexpr (EPI == TC_NORM) norm_prefetch(p.norm, row, row < M, half, pre);
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();

@@ -81,13 +81,23 @@ __device__ __forceinline__ void pack_bf16x32(const float* v, uint4 (&x)[4]) {
                       pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-// First residual chunk of this thread's half row, fetched before the
-// accumulator is ready so that its latency overlaps the wait.
-template <int BN>
+// Residual chunks of this thread's half row held in registers: the first
+// PD 32-column chunks are fetched before the accumulator is ready (their
+// latency overlaps the wait); pass 1 refills each slot PD chunks ahead.
+template <int BN, int PDMAX = 4>
+struct NormPre {
+  static constexpr int CH = BN / 64;            // 32-column chunks per half row
+  static constexpr int PD = CH < PDMAX ? CH : PDMAX;   // chunks in flight
+  uint4 t[PD][4];
+};
+
+template <int BN, int PDMAX>
 __device__ __forceinline__ void norm_prefetch(const NormArgs& a, int64_t row, bool valid,
-                                              int half, uint4 (&t)[4]) {
-  if (a.resid)
-    stage_fetch(valid ? (const char*)a.resid + (row * BN + half * (BN / 2)) * 2 : nullptr, t);
+                                              int half, NormPre<BN, PDMAX>& pre) {
+  if (!a.resid) return;
+  const char* src = valid ? (const char*)a.resid + (row * BN + half * (BN / 2)) * 2 : nullptr;
+#pragma unroll
+  for (int i = 0; i < NormPre<BN, PDMAX>::PD; ++i) stage_fetch(src ? src + 64 * i : nullptr, pre.t[i]);
 }
 
 // Copy the RMSNorm gain (N bf16) into shared memory; every thread of the CTA
@@ -102,16 +112,16 @@ __device__ __forceinline__ void load_gain(const NormArgs& a, int N, __nv_bfloat1
 // lane quadrant and take half of the columns each; their partial sums of
 // squares meet in `red` ([2][128] floats) behind the group barrier `xbar`
 // (bounded wait; returns false if the CTA is aborting).  Pass 1 reads the
-// accumulator, adds the residual (read once, one chunk ahead; `pre` holds the
-// first chunk from norm_prefetch) and stages the sum back in TMEM; pass 2
+// accumulator, adds the residual (read once, from the chunks `pre` holds and
+// refills) and stages the sum back in TMEM; pass 2
 // normalises, applies the gain (`sg`, in shared memory) and stores.  Global
 // reads and writes go through the warp's staging buffer `stg`.
-template <int BN>
+template <int BN, int PDMAX>
 __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
                                               bool valid, int half, float* red, int rrow,
                                               uint64_t* xbar, uint32_t& xphase,
                                               volatile int* abort_flag, int32_t* status,
-                                              uint32_t stg, const uint4 (&pre)[4],
+                                              uint32_t stg, NormPre<BN, PDMAX>& pre,
                                               const __nv_bfloat16* sg) {
   constexpr int HB = BN / 2;
   const int c0 = half * HB;
@@ -120,16 +130,17 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   const char* rsrc = (valid && have) ? (const char*)a.resid + (row * N) * 2 : nullptr;
   // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
   float ss = 0.f;
-  uint4 t[4] = {pre[0], pre[1], pre[2], pre[3]};
-#pragma unroll 1
-  for (int c = c0; c < c0 + HB; c += 32) {
-    uint4 tn[4];
-    if (have && c + 32 < c0 + HB) stage_fetch(rsrc ? rsrc + 2 * (c + 32) : nullptr, tn);
+  constexpr int PD = NormPre<BN, PDMAX>::PD;
+#pragma unroll
+  for (int ci = 0; ci < NormPre<BN, PDMAX>::CH; ++ci) {
+    const int c = c0 + 32 * ci;
     float v[32];
     tmem_ld32(taddr + c, v);
     if (have) {
       uint4 rr[4];
-      stage_deliver(stg, t, rr);
+      stage_deliver(stg, pre.t[ci % PD], rr);
+      if (ci + PD < NormPre<BN, PDMAX>::CH)
+        stage_fetch(rsrc ? rsrc + 2 * (c + 32 * PD) : nullptr, pre.t[ci % PD]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float2 f[4];
@@ -152,8 +163,6 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
 #pragma unroll
     for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     if (have) tmem_st32(taddr + c, v);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) t[j] = tn[j];
   }
   red[half * 128 + rrow] = ss;
   if (!group_sync(xbar, xphase, abort_flag, status)) return false;
