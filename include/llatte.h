@@ -211,7 +211,7 @@ int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t 
  * |f| <= 1/2, a fitted cubic for 2^f, j added to the exponent field) instead
  * of the special-function unit.  This evaluates exactly that device function:
  *
- *   x     device float [n], inputs (<= 64; below -125 they act as -125)
+ *   x     device float [n], inputs (<= 64; x <= -125, -inf and NaN give 0)
  *   y     device float [n], y[i] ~ 2^x[i], relative error below 1e-4
  *   y_hw  device float [n] or NULL: 2^x[i] from the hardware ex2.approx
  *

@@ -84,29 +84,58 @@ __device__ __forceinline__ uint32_t p_col(int kk) {
 
 struct Item {
   int u, b;
-  int64_t T, n, q, hoff, qoff;
+  int32_t T, n, q;
   int nk;         // key tiles (0: no key at all)
+  int64_t hoff, qoff;
 };
 
-__device__ __forceinline__ Item load_item(const AttnTcParams& p, int idx, int n_items, int keys) {
-  Item it;
-  if (idx >= n_items) {
-    it.u = -1; it.b = 0; it.T = it.n = it.q = it.hoff = it.qoff = 0; it.nk = 0;
+// The items of one CTA (idx = blockIdx.x, + gridDim.x, ...) arrive through a
+// two-stage prefetch: the work entry (user, block) of the item after next and
+// the per-user metadata of the next item are loaded one item ahead, so no
+// role waits on a dependent pair of global loads at an item boundary.
+struct ItemStream {
+  int idx;
+  int2 ub;                          // work entry of item idx + step
+  int u, b;                         // item idx: work entry ...
+  int32_t T, n;                     // ... and metadata (loads in flight)
+  int64_t hoff, qoff;
+
+  __device__ __forceinline__ static int2 entry(const AttnTcParams& p, int i, int n_items) {
+    return i < n_items ? reinterpret_cast<const int2*>(p.work)[i] : make_int2(-1, 0);
+  }
+  __device__ __forceinline__ void fetch(const AttnTcParams& p, int2 e) {
+    u = e.x;
+    b = e.y;
+    if (u >= 0) {
+      T = p.T[u]; n = p.n[u]; hoff = p.hoff[u]; qoff = p.qoff[u];
+    } else {
+      T = n = 0; hoff = qoff = 0;
+    }
+  }
+  __device__ __forceinline__ void start(const AttnTcParams& p, int first, int n_items, int step) {
+    idx = first;
+    fetch(p, entry(p, first, n_items));
+    ub = entry(p, first + step, n_items);
+  }
+  // The current item, fully derived; then the prefetch moves one item on.
+  __device__ __forceinline__ Item next(const AttnTcParams& p, int n_items, int step, int keys) {
+    Item it;
+    it.u = u; it.b = b; it.T = T; it.n = n; it.hoff = hoff; it.qoff = qoff;
+    it.q = n + p.n_q;
+    if (u < 0) {
+      it.nk = 0;
+    } else {
+      const int64_t last = min((int64_t)b * 128 + 127, (int64_t)it.q * p.heads - 1);
+      const int64_t jl = last / p.heads;
+      const int64_t kmax = jl < n ? (int64_t)T - n + jl + 1 : T;
+      it.nk = (int)((kmax + keys - 1) / keys);
+    }
+    fetch(p, ub);
+    idx += step;
+    ub = entry(p, idx + step, n_items);
     return it;
   }
-  it.u = p.work[2 * idx];
-  it.b = p.work[2 * idx + 1];
-  it.T = p.T[it.u];
-  it.n = p.n[it.u];
-  it.q = it.n + p.n_q;
-  it.hoff = p.hoff[it.u];
-  it.qoff = p.qoff[it.u];
-  const int64_t last = min((int64_t)it.b * 128 + 127, it.q * p.heads - 1);
-  const int64_t jl = last / p.heads;
-  const int64_t kmax = jl < it.n ? it.T - it.n + jl + 1 : it.T;
-  it.nk = (int)((kmax + keys - 1) / keys);
-  return it;
-}
+};
 
 // KP fp32 columns of this lane's TMEM row.
 template <int KP>
@@ -194,10 +223,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       uint32_t itm = 0, g = 0;
       bool ok = true;
-      Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+      ItemStream items;
+      items.start(p, blockIdx.x, n_items, step);
       for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-        const Item it = nxt;
-        nxt = load_item(p, idx + step, n_items, KEYS);   // prefetch the next item's metadata
+        const Item it = items.next(p, n_items, step, KEYS);
         if (it.nk == 0) continue;
         const int qb = itm % QBUF;
         if (!mbar_wait(&q_empty[qb], ((itm / QBUF) & 1) ^ 1, abort_flag, p.status)) break;
@@ -284,10 +313,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         pend.valid = false;
         return true;
       };
-      Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+      ItemStream items;
+      items.start(p, blockIdx.x, n_items, step);
       for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-        const Item it = nxt;
-        nxt = load_item(p, idx + step, n_items, KEYS);
+        const Item it = items.next(p, n_items, step, KEYS);
         if (it.nk == 0) continue;
         const int ob = itm % OBUF, qb = itm % QBUF;
         // with one query buffer the next block only arrives after the last S
@@ -317,17 +346,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t g = 0, itm = 0, pphase = 0;
     bool ok = true;
-    Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+    ItemStream items;
+    items.start(p, blockIdx.x, n_items, step);
     for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-      const Item it = nxt;
-      nxt = load_item(p, idx + step, n_items, KEYS);
+      const Item it = items.next(p, n_items, step, KEYS);
       if (it.nk == 0) continue;
       const int ob = itm % OBUF;
       const uint32_t o_col = ob * R + part * (R / 2);   // this warp's half of O
       const int64_t pair = (int64_t)it.b * 128 + row;
-      const bool valid = pair < it.q * p.heads;
+      const bool valid = pair < (int64_t)it.q * p.heads;
       const int64_t jl = pair / p.heads;
-      const int64_t vis = !valid ? 0 : (jl < it.n ? it.T - it.n + jl + 1 : it.T);
+      const int64_t vis = !valid ? 0 : (jl < it.n ? (int64_t)it.T - it.n + jl + 1 : it.T);
       float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and partial sum
       for (int kt = 0; kt < it.nk; ++kt, ++g) {
         // ---- masked row max over this warp's keys.  Scores are already in
@@ -392,7 +421,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         // ---- probabilities 2^(s - m) -> bf16, written over S in TMEM.  One
         // pair in four takes the FMA-pipe exponential, the rest the special-
-        // function unit.  Masked keys are set to 0 after the exponential; a
+        // function unit; both give exactly 0 for a masked score (-inf).  A
         // row that sees no key at all keeps m = -inf and subtracts 0 instead.
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
         const float2 nm2 = make_float2(-m_use, -m_use);
@@ -407,10 +436,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           v[2 * j] = x.x;
           v[2 * j + 1] = x.y;
-        }
-        if (masked) {
-#pragma unroll
-          for (int i = 0; i < KP; ++i) v[i] = (i < lim) ? v[i] : 0.f;
         }
         float2 l4[4];
 #pragma unroll
@@ -447,12 +472,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t stg = smem_u32(sStage + (warp - kEpiWarp0) * kStageBytes);
     uint32_t itm = 0;
-    Item nxt = load_item(p, blockIdx.x, n_items, KEYS);
+    ItemStream items;
+    items.start(p, blockIdx.x, n_items, step);
     for (int idx = blockIdx.x; idx < n_items; idx += step) {
-      const Item it = nxt;
-      nxt = load_item(p, idx + step, n_items, KEYS);
+      const Item it = items.next(p, n_items, step, KEYS);
       const int64_t pair = (int64_t)it.b * 128 + row;
-      const bool valid = pair < it.q * p.heads;
+      const bool valid = pair < (int64_t)it.q * p.heads;
       __nv_bfloat16* orow = valid ? p.Ot + (it.qoff * p.heads + pair) * R : nullptr;
       if (it.nk == 0) {                 // no key: the attention output is zero
         const uint4 z[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),

@@ -353,12 +353,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // interval (7.5e-5, far below the bf16 rounding of the probabilities); 2^j
 // enters by adding j to the exponent field.  rint comes from adding and
 // subtracting 1.5 * 2^23, which leaves j in the low mantissa bits of the sum.
-// Valid for x <= 64; inputs below -125 are clamped (result ~2^-125, which
-// the callers mask to zero where it matters).
+// Valid for x <= 64; x <= -125 (also -inf) and NaN give exactly 0, as the
+// hardware exponential does for a masked score of -inf.
 __device__ __forceinline__ float2 exp2_fma2(float2 x) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
   const float2 t = add_f2(x, make_float2(kRound, kRound));
   const float2 j = add_f2(t, make_float2(-kRound, -kRound));
   const float2 f = fma_f2(j, make_float2(-1.f, -1.f), x);
@@ -369,6 +367,8 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
   float2 r;
   r.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
   r.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+  r.x = x.x > -125.f ? r.x : 0.f;
+  r.y = x.y > -125.f ? r.y : 0.f;
   return r;
 }
 

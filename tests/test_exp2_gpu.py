@@ -19,7 +19,7 @@ def _eval(x_np):
 
 def test_relative_error_over_the_softmax_range():
     # the softmax feeds s - m <= 8 (lazy rescale threshold); cover far beyond
-    x = np.concatenate([np.linspace(-125.0, 64.0, 1_000_001),
+    x = np.concatenate([np.linspace(-124.5, 64.0, 1_000_001),
                         np.random.default_rng(0).uniform(-30.0, 8.0, 200_001)]).astype(np.float32)
     y, y_hw = _eval(x)
     exact = np.exp2(x.astype(np.float64))
@@ -31,15 +31,19 @@ def test_relative_error_over_the_softmax_range():
 
 
 def test_integers_halves_and_odd_length():
-    x = np.concatenate([np.arange(-125, 65), np.arange(-125, 64) + 0.5]).astype(np.float32)
+    x = np.concatenate([np.arange(-124, 65), np.arange(-124, 64) + 0.5]).astype(np.float32)
     assert x.size % 2 == 1
     y, _ = _eval(x)
     exact = np.exp2(x.astype(np.float64))
     assert np.abs(y / exact - 1.0).max() < 1e-4
 
 
-def test_very_negative_and_non_finite_inputs_stay_tiny():
-    x = np.array([-126.0, -200.0, -1e30, -np.inf, np.nan, -125.0], dtype=np.float32)
-    y, _ = _eval(x)
-    assert np.all(np.isfinite(y)) and np.all(y >= 0.0)
-    assert np.all(y <= 2.0 ** -124)
+def test_very_negative_and_non_finite_inputs_give_zero():
+    # a masked score reaches the exponential as -inf and must give exactly 0
+    x = np.array([-125.0, -126.0, -200.0, -1e30, -np.inf, np.nan], dtype=np.float32)
+    y, y_hw = _eval(x)
+    assert np.all(y == 0.0)
+    assert y_hw[4] == 0.0
+    # just above the cut the value is the ordinary one
+    y2, _ = _eval(np.array([-124.75, -124.0], dtype=np.float32))
+    assert np.abs(y2 / np.exp2([-124.75, -124.0]) - 1.0).max() < 1e-4
