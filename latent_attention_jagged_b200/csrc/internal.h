@@ -28,7 +28,7 @@ struct PlanDev {
   int32_t* work;       // attention work items, [(L) * max_work] (tensor-core path)
   int32_t* work_count; // [L]
   int32_t* work_next;  // [L] dynamic scheduling counters
-  int32_t* item_off;   // [max_batch+1] scratch: first work item of each user
+  int32_t* item_off;   // [L][max_batch+1] scratch: first work item of each user
   int32_t* row_user;   // [L][max rows_q]: user of every query row of every layer
   int64_t row_user_stride;
   __host__ __device__ const int32_t* ruser(int l) const { return row_user + l * row_user_stride; }
@@ -47,7 +47,7 @@ struct LayerDev {
   void* W_dkv;     // [r, d]
   void* g_kv;      // [r]
   void* W_qk;      // [h*r, d]   absorbed W_uk^T W_q (x columns), scaled 1/sqrt(d_h)
-  float* W_qkc;    // [h*r, d_ctx] fp32 absorbed context columns (NULL if d_ctx == 0)
+  float* W_qkc;    // [d_ctx, h*r] fp32 absorbed context columns, transposed (NULL if d_ctx == 0)
   void* W_ov;      // [d, h*r]   absorbed W_o W_uv
   void* g1;        // [d]
   void* W1;        // [f, d]
@@ -99,6 +99,11 @@ struct llatte_handle {
   int attn_keys;                  // keys per attention tile (tensor-core path)
   int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
+
+  // the per-user context term runs on a side stream, beside the plan and
+  // the gather (forked from and joined back into the caller's stream)
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
 
   // profiling
   int profiling;
@@ -164,7 +169,7 @@ struct AttnArgs {
 cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
 
 // Per-user context term of every layer's absorbed query projection.
-struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [h*r, d_ctx] per layer
+struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [d_ctx, h*r] per layer
 cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
                             int dc, float* out, cudaStream_t s);
 

@@ -7,9 +7,9 @@
 // query rows (the last n_l history rows, then the n_q query tokens, i.e. the
 // pages' tail slice of the fused sequence) in query_off_l = exscan(n_l + n_q).
 // The layer after the last one is a virtual layer L whose keep is unbounded:
-// its query rows are the final rows.  One CTA computes all layers; the
-// offsets are validated first and a bad batch turns every count to zero (no
-// later kernel then does any work) and sets the device status word.
+// its query rows are the final rows.  One CTA per layer; the offsets are
+// validated first and a bad batch turns every count to zero (no later kernel
+// then does any work) and sets the device status word.
 //
 // Gather (appendix A.2 step 2, X_input = Concat(X_seq, Q)): layer 0's
 // history rows are a copy of `values`; its query rows are the last n_0
@@ -59,11 +59,15 @@ __device__ void block_exscan2(int64_t a, int64_t b, int64_t* out_a, int64_t* out
   __syncthreads();
 }
 
+// Block l handles layer l (block L the virtual final layer): every layer's
+// counts have a closed form in the input length, T_{l,u} = min(T_{0,u},
+// keep_0, ..., keep_{l-1}), so the layers need not wait for one another.
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep, int L, int n_q,
             int64_t max_len, int64_t max_total, int heads, int attn_keys) {
   __shared__ int s_err;
   const int tid = threadIdx.x;
+  const int l = blockIdx.x;
   if (tid == 0) s_err = 0;
   __syncthreads();
   int err = 0;
@@ -78,26 +82,33 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     s_err |= LLATTE_DEV_TOO_MANY_ROWS;
   __syncthreads();
   if (s_err) {
-    if (tid == 0) atomicOr(p.status, s_err);
-    for (int i = tid; i < 2 * (L + 1); i += kPlanThreads) p.totals[i] = 0;
-    for (int i = tid; i < L; i += kPlanThreads) p.work_count[i] = 0;
-    for (int64_t i = tid; i < (int64_t)(L + 1) * p.stride; i += kPlanThreads) {
-      p.hist_off[i] = 0;
-      p.query_off[i] = 0;
+    // every block clears its own layer; block 0 reports
+    if (tid == 0) {
+      if (l == 0) atomicOr(p.status, s_err);
+      p.totals[2 * l] = 0;
+      p.totals[2 * l + 1] = 0;
+      if (l < L) p.work_count[l] = 0;
+    }
+    for (int64_t i = tid; i < p.stride; i += kPlanThreads) {
+      p.hist_off[l * p.stride + i] = 0;
+      p.query_off[l * p.stride + i] = 0;
     }
     return;
   }
+  int32_t cap = 0x7fffffff;                  // min of the keeps of the layers before l
+  for (int k = 0; k < l; ++k) cap = min(cap, keep.k[k]);
+  const int32_t kl = l < L ? keep.k[l] : 0x7fffffff;
   const int chunk = (B + kPlanThreads - 1) / kPlanThreads;
   const int u0 = min(B, tid * chunk), u1 = min(B, u0 + chunk);
   const int64_t bstride = p.stride - 1;
-  for (int l = 0; l <= L; ++l) {
+  {
     int32_t* Tl = p.T + l * bstride;
     int32_t* nl = p.n + l * bstride;
-    const int32_t* nprev = p.n + (l - 1) * bstride;
     int64_t sT = 0, sQ = 0;
     for (int u = u0; u < u1; ++u) {
-      int32_t t = (l == 0) ? (int32_t)(offsets[u + 1] - offsets[u]) : nprev[u];
-      int32_t nn = (l == L) ? t : min(t, keep.k[l]);
+      const int64_t len = offsets[u + 1] - offsets[u];
+      const int32_t t = (int32_t)(len < cap ? len : cap);
+      const int32_t nn = min(t, kl);
       Tl[u] = t;
       nl[u] = nn;
       sT += t;
@@ -120,70 +131,69 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
       p.totals[2 * l + 1] = totQ;
     }
   }
-  if (attn_keys <= 0) return;
+  __syncthreads();
+  if (attn_keys <= 0 || l == L) return;
 
-  // Attention work lists: one item per (user, block of 128 (query row, head)
-  // pairs), ordered by the number of key tiles the block visits, largest
-  // first (a counting sort over at most kBuckets cost classes), so that the
-  // persistent attention CTAs take the longest items first.
+  // Attention work list of layer l: one item per (user, block of 128 (query
+  // row, head) pairs), ordered by the number of key tiles the block visits,
+  // largest first (a counting sort over at most kBuckets cost classes), so
+  // that the persistent attention CTAs take the longest items first.
   constexpr int kBuckets = 64;
   __shared__ int32_t hist[kBuckets], cursor[kBuckets];
   __shared__ int32_t total_items;
-  for (int l = 0; l < L; ++l) {
-    const int32_t* Tl = p.T + l * bstride;
-    const int32_t* nl = p.n + l * bstride;
-    if (tid < kBuckets) hist[tid] = 0;
-    // items per user and their exclusive scan (item_off[u] = first item of u)
-    int64_t cnt = 0;
-    for (int u = u0; u < u1; ++u) cnt += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
-    int64_t base, dummy, total, dummy2;
-    block_exscan2(cnt, 0, &base, &dummy, &total, &dummy2);
-    for (int u = u0; u < u1; ++u) {
-      p.item_off[u] = (int32_t)base;
-      base += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+  const int32_t* Tl = p.T + l * bstride;
+  const int32_t* nl = p.n + l * bstride;
+  int32_t* item_off = p.item_off + l * p.stride;
+  if (tid < kBuckets) hist[tid] = 0;
+  // items per user and their exclusive scan (item_off[u] = first item of u)
+  int64_t cnt = 0;
+  for (int u = u0; u < u1; ++u) cnt += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+  int64_t base, dummy, total, dummy2;
+  block_exscan2(cnt, 0, &base, &dummy, &total, &dummy2);
+  for (int u = u0; u < u1; ++u) {
+    item_off[u] = (int32_t)base;
+    base += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+  }
+  if (tid == 0) item_off[B] = (int32_t)total;
+  __syncthreads();
+  auto cost_of = [&](int u, int b) {
+    const int64_t q = (int64_t)nl[u] + n_q;
+    const int64_t last = min((int64_t)b * 128 + 127, q * heads - 1);
+    const int64_t jl = last / heads;
+    const int64_t kmax = jl < nl[u] ? (int64_t)Tl[u] - nl[u] + jl + 1 : (int64_t)Tl[u];
+    const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
+    return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
+  };
+  auto user_of = [&](int i) {      // largest u with item_off[u] <= i
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (item_off[mid] <= i) lo = mid; else hi = mid - 1;
     }
-    if (tid == 0) p.item_off[B] = (int32_t)total;
-    __syncthreads();
-    auto cost_of = [&](int u, int b) {
-      const int64_t q = (int64_t)nl[u] + n_q;
-      const int64_t last = min((int64_t)b * 128 + 127, q * heads - 1);
-      const int64_t jl = last / heads;
-      const int64_t kmax = jl < nl[u] ? (int64_t)Tl[u] - nl[u] + jl + 1 : (int64_t)Tl[u];
-      const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
-      return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
-    };
-    auto user_of = [&](int i) {      // largest u with item_off[u] <= i
-      int lo = 0, hi = B - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.item_off[mid] <= i) lo = mid; else hi = mid - 1;
-      }
-      return lo;
-    };
-    for (int i = tid; i < (int)total; i += kPlanThreads) {
-      const int u = user_of(i);
-      atomicAdd(&hist[cost_of(u, i - p.item_off[u])], 1);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int32_t acc = 0;
-      for (int k = kBuckets - 1; k >= 0; --k) { cursor[k] = acc; acc += hist[k]; }
-      total_items = acc;
-    }
-    __syncthreads();
-    int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
-    for (int i = tid; i < (int)total; i += kPlanThreads) {
-      const int u = user_of(i);
-      const int b = i - p.item_off[u];
-      const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
-      W[2 * pos] = u;
-      W[2 * pos + 1] = b;
-    }
-    if (tid == 0) {
-      p.work_count[l] = total_items;
-      p.work_next[l] = 0;
-    }
-    __syncthreads();
+    return lo;
+  };
+  for (int i = tid; i < (int)total; i += kPlanThreads) {
+    const int u = user_of(i);
+    atomicAdd(&hist[cost_of(u, i - item_off[u])], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int k = kBuckets - 1; k >= 0; --k) { cursor[k] = acc; acc += hist[k]; }
+    total_items = acc;
+  }
+  __syncthreads();
+  int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
+  for (int i = tid; i < (int)total; i += kPlanThreads) {
+    const int u = user_of(i);
+    const int b = i - item_off[u];
+    const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
+    W[2 * pos] = u;
+    W[2 * pos + 1] = b;
+  }
+  if (tid == 0) {
+    p.work_count[l] = total_items;
+    p.work_next[l] = 0;
   }
 }
 
@@ -191,7 +201,7 @@ cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, c
   KeepArr k;
   const int L = h->dims.n_layers;
   for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < L ? h->dims.keep[i] : 0;
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(offsets, B, h->plan, k, L, h->dims.n_q, h->dims.max_len,
+  plan_kernel<<<L + 1, kPlanThreads, 0, s>>>(offsets, B, h->plan, k, L, h->dims.n_q, h->dims.max_len,
                                           h->max_rows_h, h->dims.heads, h->use_tc ? h->attn_keys : 0);
   return cudaGetLastError();
 }
@@ -200,7 +210,7 @@ cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_t
                            const int64_t* offsets, int B, cudaStream_t s) {
   KeepArr k;
   for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < d.n_layers ? d.keep[i] : 0;
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(offsets, B, p, k, d.n_layers, d.n_q, d.max_len,
+  plan_kernel<<<d.n_layers + 1, kPlanThreads, 0, s>>>(offsets, B, p, k, d.n_layers, d.n_q, d.max_len,
                                           max_total, d.heads, 0);
   return cudaGetLastError();
 }
@@ -231,19 +241,36 @@ gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offs
          j += (int64_t)gridDim.y * blockDim.x)
       dst[j] = u;
   }
-  for (int64_t r = w0; r < rows; r += warps) {
-    const uint4* src;
-    uint4* dst;
-    if (r < T) {
-      src = values + (src0 + r) * row_vecs;
-      dst = Xh + (hoff + r) * row_vecs;
-    } else {
-      const int64_t j = r - T;
-      src = j < n ? values + (src0 + T - n + j) * row_vecs
-                  : cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
-      dst = Xq + (qoff + j) * row_vecs;
+  // four rows in flight per warp: all loads of a group before its stores
+  constexpr int RG = 4;
+  for (int64_t r0 = w0; r0 < rows; r0 += (int64_t)warps * RG) {
+    const uint4* src[RG];
+    uint4* dst[RG];
+#pragma unroll
+    for (int k = 0; k < RG; ++k) {
+      const int64_t r = r0 + (int64_t)k * warps;
+      src[k] = nullptr;
+      dst[k] = nullptr;
+      if (r >= rows) continue;
+      if (r < T) {
+        src[k] = values + (src0 + r) * row_vecs;
+        dst[k] = Xh + (hoff + r) * row_vecs;
+      } else {
+        const int64_t j = r - T;
+        src[k] = j < n ? values + (src0 + T - n + j) * row_vecs
+                       : cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
+        dst[k] = Xq + (qoff + j) * row_vecs;
+      }
     }
-    for (int v = lane; v < row_vecs; v += 32) dst[v] = __ldg(src + v);
+    for (int v = lane; v < row_vecs; v += 32) {
+      uint4 x[RG];
+#pragma unroll
+      for (int k = 0; k < RG; ++k)
+        if (src[k]) x[k] = __ldg(src[k] + v);
+#pragma unroll
+      for (int k = 0; k < RG; ++k)
+        if (dst[k]) dst[k][v] = x[k];
+    }
   }
 }
 

@@ -73,7 +73,7 @@ Layout layout_of(const llatte_dims* d) {
   L.off_work = take(sizeof(int32_t) * 2 * nl * (size_t)L.max_work);
   L.off_work_count = take(sizeof(int32_t) * nl);
   L.off_work_next = take(sizeof(int32_t) * nl);
-  L.off_item_off = take(sizeof(int32_t) * (B + 1));
+  L.off_item_off = take(sizeof(int32_t) * (B + 1) * nl);     // per layer
   L.off_row_user = take(sizeof(int32_t) * nl * (size_t)L.rows_q);
   for (int i = 0; i < 2; ++i) L.off_Xh[i] = take((size_t)L.rows_h * d->d * elem);
   for (int i = 0; i < 2; ++i) L.off_Xq[i] = take((size_t)L.rows_q * d->d * elem);
@@ -238,6 +238,9 @@ const char* llatte_error_string(int code) {
 void llatte_destroy(llatte_handle* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   for (auto& r : h->pending) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
   for (auto e : h->event_pool) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
@@ -271,6 +274,10 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   auto fail = [&](int code) { llatte_destroy(h); return code; };
   if (cudaGetDevice(&h->device) != cudaSuccess) return fail(LLATTE_ERR_CUDA);
   if (cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess)
+    return fail(LLATTE_ERR_CUDA);
+  if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess)
     return fail(LLATTE_ERR_CUDA);
 
   const size_t e = h->elem;
@@ -379,15 +386,27 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
   const PlanDev& p = h->plan;
   h->last_B = B;
 
-  { StepTimer t(h, s, ST_PLAN); CK(launch_plan(h, offsets, B, s)); t.done(1); }
-  { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, B, s)); t.done(1); }
-  if (D.d_ctx > 0) {  // context term of every layer's query projection, one launch
-    StepTimer t(h, s, ST_CTX);
+  // Context term of every layer's query projection, one launch.  It depends
+  // on nothing above, so outside profiling it runs on the side stream while
+  // the plan and the gather run here; the first query projection waits for it.
+  bool ctx_join = false;
+  if (D.d_ctx > 0) {
     CtxWeights cw = {};
     for (int l = 0; l < L; ++l) cw.W[l] = h->layers[l].W_qkc;
-    CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, s));
-    t.done(1);
+    if (h->profiling) {
+      StepTimer t(h, s, ST_CTX);
+      CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, s));
+      t.done(1);
+    } else {
+      CK(cudaEventRecord(h->ev_fork, s));
+      CK(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+      CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, h->side));
+      CK(cudaEventRecord(h->ev_join, h->side));
+      ctx_join = true;
+    }
   }
+  { StepTimer t(h, s, ST_PLAN); CK(launch_plan(h, offsets, B, s)); t.done(1); }
+  { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, B, s)); t.done(1); }
 
   for (int l = 0; l < L; ++l) {
     const LayerDev& W = h->layers[l];
@@ -459,6 +478,10 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       }
     }
     {  // absorbed queries (+ per-user context term)
+      if (ctx_join) {
+        CK(cudaStreamWaitEvent(s, h->ev_join, 0));
+        ctx_join = false;
+      }
       StepTimer t(h, s, ST_Q);
       if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);

@@ -246,45 +246,50 @@ cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------- context term
-// bias[l][u][n] = sum_k c_u[k] W_qkc,l[n][k] for every layer at once: the
+// bias[l][u][n] = sum_k c_u[k] W_qkc,l[k][n] for every layer at once: the
 // per-user part of the absorbed target-aware query W_qk [x ; c] (daiwk.github.io
-// notes, "core formula").  Block = (16 users, one layer); the context rows sit
-// in shared memory and each thread walks output columns n with 16 sums.
-constexpr int CTX_USERS = 16;
+// notes, "core formula").  Block = (128 output columns, one layer, CTX_USERS
+// users): the context rows sit in shared memory, each thread owns one column
+// n and reads the weight rows W_qkc[k][n] coalesced.
+constexpr int CTX_USERS = 8;
+constexpr int CTX_COLS = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(CTX_COLS)
 ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
                 float* __restrict__ out) {
   extern __shared__ float cs[];                       // [CTX_USERS][dc]
   const int l = blockIdx.y;
-  const int u0 = blockIdx.x * CTX_USERS;
+  const int u0 = blockIdx.z * CTX_USERS;
   const int nu = min(CTX_USERS, B - u0);
   for (int i = threadIdx.x; i < CTX_USERS * dc; i += blockDim.x) {
     const int uu = i / dc, k = i % dc;
     cs[i] = uu < nu ? to_f(ctx[(int64_t)(u0 + uu) * dc + k]) : 0.f;
   }
   __syncthreads();
-  const float* W = w.W[l];
-  for (int n = threadIdx.x; n < hr; n += blockDim.x) {
-    float acc[CTX_USERS] = {};
-    const float* wr = W + (int64_t)n * dc;
-    for (int k = 0; k < dc; ++k) {
-      const float wk = __ldg(wr + k);
+  const int n = blockIdx.x * CTX_COLS + threadIdx.x;
+  if (n >= hr) return;
+  const float* W = w.W[l] + n;
+  float acc[CTX_USERS] = {};
+#pragma unroll 4
+  for (int k = 0; k < dc; ++k) {
+    const float wk = __ldg(W + (int64_t)k * hr);
 #pragma unroll
-      for (int uu = 0; uu < CTX_USERS; ++uu) acc[uu] = fmaf(cs[uu * dc + k], wk, acc[uu]);
-    }
-    for (int uu = 0; uu < nu; ++uu) out[((int64_t)l * B + u0 + uu) * hr + n] = acc[uu];
+    for (int uu = 0; uu < CTX_USERS; ++uu) acc[uu] = fmaf(cs[uu * dc + k], wk, acc[uu]);
   }
+  for (int uu = 0; uu < nu; ++uu) out[((int64_t)l * B + u0 + uu) * hr + n] = acc[uu];
 }
 
 cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
                             int dc, float* out, cudaStream_t s) {
   if (B == 0 || dc == 0) return cudaSuccess;
-  dim3 grid((B + CTX_USERS - 1) / CTX_USERS, L);
+  dim3 grid((hr + CTX_COLS - 1) / CTX_COLS, L, (B + CTX_USERS - 1) / CTX_USERS);
   const size_t sm = sizeof(float) * CTX_USERS * dc;
-  if (elem == 4) ctx_bias_kernel<float><<<grid, 256, sm, s>>>((const float*)ctx, w, B, hr, dc, out);
-  else ctx_bias_kernel<__nv_bfloat16><<<grid, 256, sm, s>>>((const __nv_bfloat16*)ctx, w, B, hr, dc, out);
+  if (elem == 4)
+    ctx_bias_kernel<float><<<grid, CTX_COLS, sm, s>>>((const float*)ctx, w, B, hr, dc, out);
+  else
+    ctx_bias_kernel<__nv_bfloat16><<<grid, CTX_COLS, sm, s>>>((const __nv_bfloat16*)ctx, w, B, hr,
+                                                             dc, out);
   return cudaGetLastError();
 }
 
@@ -312,7 +317,8 @@ cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int 
 // ---------------------------------------------------------------- absorption
 // W_qk[j*r + a, k] = (qscale/sqrt(d_h)) sum_e W_uk[j*d_h + e, a] W_q[j*d_h + e, k]
 //   (qscale = log2(e) when the attention kernel takes scores in log2 units)
-//   (k < d -> W_qk in the storage type, k >= d -> W_qkc in fp32)
+//   (k < d -> W_qk in the storage type, k >= d -> W_qkc in fp32, stored
+//    transposed as [d_ctx][h*r] so that the context kernel reads it coalesced)
 // W_ov[n, j*r + a] = sum_e W_o[n, j*d_h + e] W_uv[j*d_h + e, a]
 template <typename T>
 __global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int heads, int dh,
@@ -328,7 +334,7 @@ __global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int 
     s = fmaf(to_f(W_uk[(int64_t)(j * dh + e) * r + a]), to_f(W_q[(int64_t)(j * dh + e) * K + k]), s);
   s *= rsqrtf((float)dh) * qscale;
   if (k < d) W_qk[(int64_t)row * d + k] = from_f<T>(s);
-  else W_qkc[(int64_t)row * dc + (k - d)] = s;
+  else W_qkc[(int64_t)(k - d) * heads * r + row] = s;
 }
 
 template <typename T>
