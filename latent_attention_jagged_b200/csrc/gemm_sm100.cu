@@ -99,13 +99,13 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
           v[4 * j] += b[j].x; v[4 * j + 1] += b[j].y; v[4 * j + 2] += b[j].z; v[4 * j + 3] += b[j].w;
         }
       }
-      if (EPI == TC_SILU) {
-#pragma unroll
-        for (int i = 0; i < STEP; ++i) v[i] = silu_approx(v[i]);
-      }
 #pragma unroll
       for (int h = 0; h < STEP / 32; ++h) {
         uint4 x[4];
+        if (EPI == TC_SILU) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[32 * h + i] = silu_approx(v[32 * h + i]);
+        }
         pack_bf16x32(&v[32 * h], x);
         stage_store(stg, x, drow ? drow + c + 32 * h : nullptr);
       }

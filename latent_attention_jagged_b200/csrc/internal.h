@@ -58,7 +58,7 @@ struct LayerDev {
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
-struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_ffn; };
+struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair; };
 
 }  // namespace llatte
 

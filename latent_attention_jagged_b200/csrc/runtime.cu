@@ -209,7 +209,11 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
-    if (h->ffn_fused) ok = ok && make_tmap_bf16(&M.w1_ffn, W.W1, f, d, 128);
+    if (h->ffn_fused) {
+      // the SM-pair FFN: each CTA loads half of a weight chunk
+      ok = ok && make_tmap_bf16(&M.w1_pair, W.W1, f, d, 64);
+      ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
+    }
   }
   return ok;
 }
@@ -540,7 +544,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       FfnTcParams q = {};
       q.M_dev = p.query_total(l); q.M_cap = h->max_rows_q; q.F = f; q.norm = f_norm;
       q.status = p.status;
-      CK(launch_ffn_tc(h->tm_Z, LM.w1_ffn, LM.w2, q, h->num_sms, s));
+      CK(launch_ffn_pair(h->tm_Z, LM.w1_pair, LM.w2_pair, q, h->num_sms, s));
       t.done(1);
       continue;
     }

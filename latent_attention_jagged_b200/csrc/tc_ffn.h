@@ -1,4 +1,4 @@
-// Interface of the fused tensor-core FFN kernel (d = 256).
+// Interface of the fused tensor-core FFN kernel (d = 256, pairs of SMs).
 #pragma once
 
 #include <cuda.h>
@@ -17,7 +17,10 @@ struct FfnTcParams {
 };
 
 bool ffn_tc_supported(int d, int f);
-cudaError_t launch_ffn_tc(const CUtensorMap& z, const CUtensorMap& w1, const CUtensorMap& w2,
-                          const FfnTcParams& p, int num_sms, cudaStream_t s);
+// X = RMSNorm(Z + W2 SiLU(W1 Z)) on pairs of SMs (cta_group::2, 256-row
+// tiles).  w1h: W1 with 64-row boxes; w2h: W2 with 128-row boxes (each CTA
+// loads half a chunk).  norm.mode must be NORM_SCATTER.
+cudaError_t launch_ffn_pair(const CUtensorMap& z, const CUtensorMap& w1h, const CUtensorMap& w2h,
+                            const FfnTcParams& p, int num_sms, cudaStream_t s);
 
 }  // namespace llatte
