@@ -32,10 +32,11 @@ sys.path.insert(0, ROOT)
 from workloads import draw_lengths, make_inputs, workload  # noqa: E402
 from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 
-# ncu-measured DRAM traffic per launch (bytes) of the dominant kernel, keyed by
-# (kernel, workload); filled from the committed profiles/ summaries.  None =
-# not captured for the current kernel version.
-TRAFFIC = {}
+# ncu-measured DRAM traffic per launch (bytes, mean over one forward's layers)
+# of the dominant kernel, keyed by (step, workload); taken from the committed
+# profiles/dram_traffic_dominant_kernels.md.  Absent = not captured for the
+# current kernel version.
+TRAFFIC = {("ffn", "online"): 7.2008e7, ("attn", "upstream"): 2.5609e8}
 
 
 def load_peaks():
