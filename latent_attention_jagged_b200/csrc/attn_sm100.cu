@@ -187,8 +187,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   float* mx = lbuf + 2 * 128;                                  // [2][kSplit][128]
   uint8_t* sStage = (uint8_t*)(mx + 2 * kSplit * 128);         // [kEpiWarps][kStageBytes]
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = *p.work_count;
   const int step = gridDim.x;
 
   if (threadIdx.x == 0) {
@@ -217,6 +217,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  const int n_items = *p.work_count;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -532,8 +535,7 @@ cudaError_t launch_r(const CUtensorMap& q, const CUtensorMap& c, const AttnTcPar
     if (e != cudaSuccess) return e;
     attr_devices |= 1ull << (dev & 63);
   }
-  attn_tc_kernel<R><<<grid, kThreads, Cfg::SMEM, s>>>(q, c, p);
-  return cudaGetLastError();
+  return launch_dependent(attn_tc_kernel<R>, dim3(grid), dim3(kThreads), Cfg::SMEM, s, 1, q, c, p);
 }
 
 }  // namespace

@@ -87,11 +87,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   __nv_bfloat16* sG = (__nv_bfloat16*)((uint8_t*)bars + 256);   // gain [D]
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-  const int64_t M = *p.M_dev;
-  const int64_t num_tiles = (M + 255) / 256;
   const int NC = p.F / HC;
   // Every pair walks the hidden chunks in a rotated order, so that the SMs
   // do not all read the same weight lines from L2 at the same moment.
@@ -130,6 +129,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
   cluster_sync();          // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  const int64_t M = *p.M_dev;
+  const int64_t num_tiles = (M + 255) / 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -484,19 +487,7 @@ cudaError_t launch_ffn_pair(const CUtensorMap& z, const CUtensorMap& w1h, const 
   }
   const int64_t max_tiles = (p.M_cap + 255) / 256;
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs(num_sms), max_tiles));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ffn_pair_kernel, z, w1h, w2h, p);
+  return launch_dependent(ffn_pair_kernel, dim3(2 * pairs), dim3(kThreads), SMEM, s, 2, z, w1h, w2h, p);
 }
 
 }  // namespace llatte

@@ -136,10 +136,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint8_t* sStage = (uint8_t*)(red + 2 * 2 * 128);                  // [epilogue warp][kStageBytes]
   __nv_bfloat16* sG = (__nv_bfloat16*)(sStage + kEpiWarps * kStageBytes);   // RMSNorm gain [BN]
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
   const int n_tiles = p.N / BN;
-  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles;
   const int KB = p.K / BK;
   const int kb0 = blockIdx.x % KB;
 
@@ -162,6 +161,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
+  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -269,8 +272,8 @@ cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmP
     if (e != cudaSuccess) return e;
     attr_devices |= 1ull << (dev & 63);
   }
-  tc_gemm_kernel<BN, EPI><<<grid, kThreads, Cfg::SMEM, s>>>(a, b, p);
-  return cudaGetLastError();
+  return launch_dependent(tc_gemm_kernel<BN, EPI>, dim3(grid), dim3(kThreads), Cfg::SMEM, s, 1,
+                          a, b, p);
 }
 
 template <int EPI>

@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/llatte.h"
 
 namespace llatte {
@@ -320,6 +322,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch.  A persistent kernel (every CTA resident from
+// the start) calls pdl_trigger() first, so the next kernel in the stream may
+// be scheduled as soon as SMs free up; that kernel sets up (barriers, TMEM,
+// descriptor prefetch) and calls pdl_wait() before it reads anything an
+// earlier kernel wrote.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- CTA pairs
 // A cluster of two CTAs on two SMs whose tensor cores work as one
 // (cta_group::2): rank 0 issues the MMAs of M = 256 rows, each CTA holds its
@@ -480,6 +493,35 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
   r.x = x.x > -125.f ? r.x : 0.f;
   r.y = x.y > -125.f ? r.y : 0.f;
   return r;
+}
+
+// Launch with programmatic stream serialisation (the kernel may start while
+// the previous kernel of the stream finishes; it must call pdl_wait() before
+// touching that kernel's results) and, for cluster_x > 1, clusters of
+// cluster_x CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace tc
