@@ -423,7 +423,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           l_run *= scale;
         }
         // ---- probabilities 2^(s - m) -> bf16, written over S in TMEM.  One
-        // pair in four takes the FMA-pipe exponential, the rest the special-
+        // pair in eight takes the FMA-pipe exponential, the rest the special-
         // function unit; both give exactly 0 for a masked score (-inf).  A
         // row that sees no key at all keeps m = -inf and subtracts 0 instead.
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
@@ -431,7 +431,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int j = 0; j < KP / 2; ++j) {
           float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
-          if ((j & 3) == 3) {
+          if ((j & 7) == 7) {
             x = exp2_fma2(x);
           } else {
             x.x = ex2_approx(x.x);
