@@ -10,7 +10,8 @@
 // one shared-memory copy of each C tile (K-major for S, MN-major for P V).
 //
 // Roles (448 threads, one CTA per SM, persistent over the sorted work list):
-//   warp 0       TMA: the Q~ block once per item, C tiles into a 4-stage ring
+//   warp 0       TMA: the Q~ block once per item, 128-key C tiles into a ring
+//                (4 stages, 2 for r = 256)
 //   warp 1       TMEM owner; lane 0 issues S(kt+1) = Q~ C_{kt+1}^T before
 //                O += P(kt) C_kt, so the tensor pipe works while the softmax
 //                warps turn S(kt) into P(kt)
@@ -52,12 +53,14 @@ constexpr int kThreads = 32 * (2 + kSoftWarps + kEpiWarps);
 
 template <int R>
 struct AttnCfg {
-  static constexpr int KEYS = R >= 256 ? 64 : 128;     // keys per tile
+  // 128 keys per tile for every rank: the S MMA then has N = 128 (an N = 64
+  // MMA takes about 54 cycles instead of 32 on this part)
+  static constexpr int KEYS = 128;
   static constexpr int KP = KEYS / kSplit;             // keys per softmax warp
   static constexpr int RSUB = R / 64;                  // 64-wide latent sub-tiles
   static constexpr int OBUF = (2 * R + 2 * KEYS <= 512) ? 2 : 1;
   static constexpr int QBUF = R <= 128 ? 2 : 1;          // query blocks in flight
-  static constexpr int KV_STAGES = 4;
+  static constexpr int KV_STAGES = R >= 256 ? 2 : 4;   // 64 KB or 32 KB per C tile
   static constexpr uint32_t Q_BYTES = 128 * R * 2;
   static constexpr uint32_t KV_BYTES = KEYS * R * 2;
   static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
@@ -70,7 +73,7 @@ struct AttnCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(OBUF * R + 2 * KEYS <= 512, "TMEM budget");
-  static_assert(KP == 32 || KP == 64, "softmax chunk");
+  static_assert(KP == 64, "softmax chunk");
 };
 
 // TMEM column (relative to the S buffer) of the packed bf16 P for keys
@@ -540,7 +543,7 @@ cudaError_t launch_r(const CUtensorMap& q, const CUtensorMap& c, const AttnTcPar
 
 }  // namespace
 
-int attn_tc_keys(int r) { return r >= 256 ? 64 : 128; }
+int attn_tc_keys(int) { return 128; }
 
 bool attn_tc_supported(int r) { return r == 64 || r == 128 || r == 256; }
 
