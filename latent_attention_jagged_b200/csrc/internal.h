@@ -58,7 +58,7 @@ struct LayerDev {
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
-struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair; };
+struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair; };
 
 }  // namespace llatte
 
@@ -98,6 +98,7 @@ struct llatte_handle {
   int bn_kv, bn_q, bn_o, bn_f1, bn_f2;
   int attn_keys;                  // keys per attention tile (tensor-core path)
   int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
+  int pair_norm;                  // output / FFN-down projections on SM pairs (d = 512)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
 
   // the per-user context term runs on a side stream, beside the plan and

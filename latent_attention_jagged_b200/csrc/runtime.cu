@@ -198,6 +198,7 @@ bool build_tc_maps(llatte_handle* h) {
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
   h->attn_keys = attn_tc_keys(r);
   h->ffn_fused = ffn_tc_supported(d, f) ? 1 : 0;
+  h->pair_norm = tc_gemm_pair_supported(TC_NORM, d, hr) && tc_gemm_pair_supported(TC_NORM, d, f);
   ok = ok && make_tmap_bf16(&h->tm_Qt, h->Qt, rq * D.heads, r, 128);
   ok = ok && make_tmap_bf16(&h->tm_C, h->C, rh, r, (uint32_t)h->attn_keys);
   auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
@@ -212,6 +213,11 @@ bool build_tc_maps(llatte_handle* h) {
     if (h->ffn_fused) {
       // the SM-pair FFN: each CTA loads half of a weight chunk
       ok = ok && make_tmap_bf16(&M.w1_pair, W.W1, f, d, 64);
+      ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
+    }
+    if (h->pair_norm) {
+      // the SM-pair residual + RMSNorm GEMMs at d = 512: 128-row weight boxes
+      ok = ok && make_tmap_bf16(&M.ov_pair, W.W_ov, d, hr, 128);
       ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
     }
   }
@@ -527,7 +533,8 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, hr);
         q.norm = o_norm;
-        CK(launch_tc_gemm(h->bn_o, TC_NORM, h->tm_Ot, LM.ov, q, h->num_sms, s));
+        if (h->pair_norm) CK(launch_tc_gemm_pair(TC_NORM, h->tm_Ot, LM.ov_pair, q, h->num_sms, s));
+        else CK(launch_tc_gemm(h->bn_o, TC_NORM, h->tm_Ot, LM.ov, q, h->num_sms, s));
         t.done(1);
       } else {
         GemmArgs g = {};
@@ -567,7 +574,8 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, f);
         q.norm = f_norm;
-        CK(launch_tc_gemm(h->bn_f2, TC_NORM, h->tm_Hd, LM.w2, q, h->num_sms, s));
+        if (h->pair_norm) CK(launch_tc_gemm_pair(TC_NORM, h->tm_Hd, LM.w2_pair, q, h->num_sms, s));
+        else CK(launch_tc_gemm(h->bn_f2, TC_NORM, h->tm_Hd, LM.w2, q, h->num_sms, s));
         t.done(1);
       } else {
         GemmArgs g = {};

@@ -28,5 +28,10 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool tc_gemm_supported(int BN, int epi, int N, int K);
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
                            const TcGemmParams& p, int num_sms, cudaStream_t s);
+// Residual + RMSNorm GEMM with N = 512 on pairs of SMs (256-row tiles); b_half:
+// the weight with 128-row boxes (each CTA loads half of a k-block).
+bool tc_gemm_pair_supported(int epi, int N, int K);
+cudaError_t launch_tc_gemm_pair(int epi, const CUtensorMap& a, const CUtensorMap& b_half,
+                                const TcGemmParams& p, int num_sms, cudaStream_t s);
 
 }  // namespace llatte
