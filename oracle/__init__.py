@@ -17,7 +17,9 @@ A.3 "Multi-head Latent Attention"; daiwk.github.io reproduction notes,
 Readings of points the pages leave open (scale 1/sqrt(d_h); candidates see all
 history keys but no query token; keep counts count history rows only; RMSNorm
 on the KV latent; FFN = W2 SiLU(W1 z) without biases; eps = 1e-6; mean-pool +
-linear readout for the upstream workload) are stated where they are used.
+linear readout for the upstream workload; a sequence summary is a SiLU MLP with
+a rank-r bottleneck over the row-major flattened final query tokens) are
+stated where they are used.
 
 Parity status: every function here is pinned by tests against invariants,
 special cases and library routines (see tests/test_oracle.py). The numeric
@@ -25,8 +27,8 @@ forward values themselves are not printed on the pages; parity against the
 pages' own numbers is unpinned for that reason.
 """
 from .plan import plan_layers, LayerPlan
-from .model import forward, layer_forward, absorb, rmsnorm, silu
+from .model import forward, layer_forward, absorb, rmsnorm, silu, summaries
 from .brute import forward_brute
 
 __all__ = ["plan_layers", "LayerPlan", "forward", "layer_forward", "absorb",
-           "rmsnorm", "silu", "forward_brute"]
+           "rmsnorm", "silu", "summaries", "forward_brute"]

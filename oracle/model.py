@@ -15,7 +15,8 @@ display's sqrt(d_c) is read as garbled: only the same scale keeps the two forms
 equal); history query at position p sees keys t <= p; a candidate sees every
 history key of the current layer and no query token; with no visible key the
 attention output is zero; RMSNorm(v) = v / sqrt(mean(v^2) + eps) * g;
-FFN(z) = W2 SiLU(W1 z), SiLU(x) = x / (1 + exp(-x)), no biases.
+FFN(z) = W2 SiLU(W1 z), SiLU(x) = x / (1 + exp(-x)), no biases; a sequence
+summary is W_up SiLU(W_down Flatten(Z_raw)) (see `summaries`).
 
 Absorbed matrices per head j (rows j*d_h:(j+1)*d_h of the per-head blocks):
   W_QK_j = W_uk_j^T W_q_j / sqrt(d_h)      (r x (d + d_ctx))
@@ -100,12 +101,32 @@ def layer_forward(H: np.ndarray, Y: np.ndarray, c: np.ndarray, w: dict, ab: dict
     return X[:n], X[n:]
 
 
+def summaries(z_raw: np.ndarray, sum_w: Sequence[dict]) -> np.ndarray:
+    """Sequence summaries of one user from the final query-token rows.
+
+    LLaTTE notes (huaxiaozhuan.com), appendix A.2 item 4 "Sequence Summaries":
+    the final layer's rows at the query-token positions, Z_raw [n_q, d], are
+    flattened and each of k low-rank adapted MLPs maps the flat vector to a
+    fixed-size summary Z_seq^(k) of width d_seq.
+
+    Reading (the pages name the block but give no formula): Flatten is
+    row-major, token 0's d values first; LoRAMLP_k(v) = W_up,k SiLU(W_down,k v)
+    with W_down,k [sum_rank, n_q*d] the low-rank bottleneck and W_up,k
+    [d_seq, sum_rank], no biases (the layers have none either), SiLU as in
+    the FFN.  Returns [k, d_seq].
+    """
+    v = _f64(z_raw).reshape(-1)
+    return np.stack([_f64(w["W_up"]) @ silu(_f64(w["W_down"]) @ v) for w in sum_w])
+
+
 def forward(inputs, users: Optional[Sequence[int]] = None, return_probs: bool = False,
             return_layers: bool = False):
     """fp64 forward of the whole sequence module for the chosen users.
 
-    Returns out: [U, n_q, d] (final query-token rows) when d_out == 0, otherwise
-    [U, d_out] = W_e @ mean of the final layer's rows (zero if there are none).
+    Returns out: [U, n_q, d] (final query-token rows) when d_out == 0 and
+    n_sum == 0; [U, d_out] = W_e @ mean of the final layer's rows (zero if
+    there are none) when d_out > 0; [U, n_sum, d_seq] sequence summaries of the
+    final query-token rows when n_sum > 0.
     With return_probs, also a list (per user) of lists (per layer) of per-head
     probability matrices. With return_layers, also per user the list of
     (H, Y) after every layer.
@@ -130,6 +151,8 @@ def forward(inputs, users: Optional[Sequence[int]] = None, return_probs: bool = 
             rows = np.concatenate([H, Y], axis=0)
             m = rows.mean(axis=0) if rows.shape[0] > 0 else np.zeros(dims.d)
             outs.append(_f64(inputs.W_e) @ m)
+        elif getattr(dims, "n_sum", 0) > 0:
+            outs.append(summaries(Y, inputs.summaries))
         else:
             outs.append(Y)
         all_probs.append(probs_u)

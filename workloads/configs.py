@@ -11,7 +11,7 @@ L in {1,2,4,8} grid of huaxiaozhuan.com sec. 1.5.2.
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass, field, replace
 from typing import Tuple
 
 
@@ -32,6 +32,9 @@ class Dims:
     eps      RMSNorm epsilon
     kv_norm  1 = RMSNorm on the KV latent, 0 = plain down-projection
     dtype    storage type of activations and weights: "bf16" or "fp32"
+    n_sum    sequence summaries read out of the final query tokens (0 = none)
+    sum_rank hidden (low-rank) width of each summary MLP
+    d_seq    width of each summary
     """
 
     d: int
@@ -46,6 +49,9 @@ class Dims:
     eps: float = 1e-6
     kv_norm: int = 1
     dtype: str = "bf16"
+    n_sum: int = 0
+    sum_rank: int = 0
+    d_seq: int = 0
 
     @property
     def n_layers(self) -> int:
@@ -119,6 +125,20 @@ WORKLOADS = {
         description="skewed jagged batch: B=512, T~lognormal(5.5,0.8) clipped to "
                     "[8,1600], d=256, 4 heads, r=128, 6 layers keep 512>>l, 256 candidates"),
 }
+
+# Sequence summaries (the pages' LoRAMLP readout of the final query tokens):
+# the same batches with k low-rank MLP summaries read out of the flattened
+# final query tokens.  The pages fix neither k, the rank nor d_seq; two
+# summaries of width 1024 make the 2048-wide transfer vector the upstream
+# pipeline hands to downstream models.
+WORKLOADS["tiny_sum"] = Workload(
+    name="tiny_sum", dims=replace(WORKLOADS["tiny"].dims, n_sum=3, sum_rank=8, d_seq=12),
+    batch=4, lengths=("uniform", 16, 64), seed=0,
+    description="tiny fp32 case with 3 summaries (rank 8, width 12)")
+WORKLOADS["online_sum"] = Workload(
+    name="online_sum", dims=replace(WORKLOADS["online"].dims, n_sum=2, sum_rank=128, d_seq=1024),
+    batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
+    description="online ranker + 2 sequence summaries: flatten(64 x 256) -> rank 128 -> 1024")
 
 
 def workload(name: str) -> Workload:

@@ -11,6 +11,9 @@ Draw order, fixed so that every consumer sees the same numbers for a seed:
      (matrices N(0, 1/fan_in); gains are 1 unless random gains are asked for,
      then N(1, 0.1^2))
   7. W_e (readout) when d_out > 0.
+  8. sequence-summary weights when n_sum > 0, summary by summary:
+     W_down [sum_rank, n_q*d] N(0, 1/(n_q*d)), then W_up [d_seq, sum_rank]
+     N(0, 1/sum_rank).
 
 All arrays are returned as float32 already rounded to the storage type
 (round-to-nearest-even to bfloat16 for "bf16" workloads), so that the oracle
@@ -47,6 +50,7 @@ class Inputs:
     ctx: np.ndarray            # float32 [B, d_ctx]   non-sequence context
     layers: List[Dict[str, np.ndarray]]
     W_e: Optional[np.ndarray]  # float32 [d_out, d] or None
+    summaries: Optional[List[Dict[str, np.ndarray]]] = None  # per summary W_down, W_up
 
     @property
     def batch(self) -> int:
@@ -100,6 +104,18 @@ def draw_weights(dims: Dims, rng: np.random.Generator, random_gains: bool = Fals
     return layers, W_e
 
 
+def draw_summaries(dims: Dims, rng: np.random.Generator):
+    """Weights of the n_sum summary MLPs (None when there are none)."""
+    if dims.n_sum <= 0:
+        return None
+    kin = dims.n_q * dims.d
+    out = []
+    for _ in range(dims.n_sum):
+        out.append({"W_down": _normal(rng, (dims.sum_rank, kin), 1.0 / np.sqrt(kin)),
+                    "W_up": _normal(rng, (dims.d_seq, dims.sum_rank), 1.0 / np.sqrt(dims.sum_rank))})
+    return out
+
+
 def make_inputs(wl: Workload, batch: Optional[int] = None,
                 lengths: Optional[np.ndarray] = None, seed: Optional[int] = None,
                 random_gains: bool = False, dims: Optional[Dims] = None) -> Inputs:
@@ -129,12 +145,15 @@ def make_inputs(wl: Workload, batch: Optional[int] = None,
     cand = tokens(B * dims.n_q).reshape(B, dims.n_q, d)
     ctx = _normal(rng, (B, dims.d_ctx))
     layers, W_e = draw_weights(dims, rng, random_gains=random_gains)
+    sums = draw_summaries(dims, rng)
 
     if dims.dtype == "bf16":
         values, cand, ctx = round_to_bf16(values), round_to_bf16(cand), round_to_bf16(ctx)
         layers = [{k: round_to_bf16(v) for k, v in w.items()} for w in layers]
         W_e = round_to_bf16(W_e) if W_e is not None else None
+        if sums is not None:
+            sums = [{k: round_to_bf16(v) for k, v in w.items()} for w in sums]
     elif dims.dtype != "fp32":
         raise ValueError(f"unknown storage dtype {dims.dtype!r}")
     return Inputs(dims=dims, lengths=lens, offsets=offsets, values=values, cand=cand,
-                  ctx=ctx, layers=layers, W_e=W_e)
+                  ctx=ctx, layers=layers, W_e=W_e, summaries=sums)
