@@ -227,14 +227,14 @@ def main():
         shard = shard_batch(offsets, wl.dims, world)[rank]
         inp = make_inputs(wl, lengths=lengths[shard.users], seed=wl.seed + 1000 + rank)
         shared = make_inputs(wl, lengths=np.zeros(1, dtype=np.int64), seed=wl.seed)
-        inp.layers, inp.W_e = shared.layers, shared.W_e
+        inp.layers, inp.W_e, inp.summaries = shared.layers, shared.W_e, shared.summaries
         return inp
 
     def measure(wl, steps, warmup, sample_clocks):
         inp = rank_inputs(wl)
         dt = torch.bfloat16 if inp.dims.dtype == "bf16" else torch.float32
         h = Llatte(inp.dims, inp.layers, inp.W_e, max_batch=inp.batch,
-                   max_len=int(inp.lengths.max()))
+                   max_len=int(inp.lengths.max()), summaries=inp.summaries)
         values = torch.from_numpy(inp.values).cuda().to(dt)
         offsets = torch.from_numpy(inp.offsets).cuda()
         ctx = torch.from_numpy(inp.ctx).cuda().to(dt) if inp.dims.d_ctx else None
@@ -342,6 +342,19 @@ def main():
                 "peak_source": f"{peaks['source']} sustained bf16 (cuBLAS loop)",
                 "traffic": TRAFFIC.get((dom, wl.name)),
                 "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms}
+        # the sequence-summary step (bottleneck GEMM + up-projection), when the
+        # workload has one, against HBM: the final rows and both projections
+        # read once, the summaries written once
+        summary = None
+        if prof.get("summary", {}).get("calls"):
+            s_ms = prof["summary"]["ms"] / prof["summary"]["calls"]
+            s_bytes = cost.summary_bytes(inp.batch, inp.dims)
+            summary = {"bound": "hbm", "achieved": s_bytes / (s_ms / 1e3) / 1e9,
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": s_bytes / (s_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                       "bytes": s_bytes, "ms": s_ms, "launches": prof["summary"]["launches"]
+                       / prof["summary"]["calls"],
+                       "flops": cost.summary_flops(inp.batch, inp.dims)}
         total_flops = cost.total_flops(inp.lengths, inp.dims)
         step_ms = ms / steps
         whole = {"achieved_tflops": total_flops / (step_ms / 1e3) / 1e12,
@@ -350,7 +363,7 @@ def main():
         steps_ms = {k: round(v["ms"] / prof_steps, 4) for k, v in prof.items() if v["calls"]}
         res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
                    clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
-                   dtype=inp.dims.dtype, users_all=users_all)
+                   dtype=inp.dims.dtype, users_all=users_all, summary=summary)
         del graph
         h.close()
         return res
@@ -388,6 +401,7 @@ def main():
             "gpu_launches": int(round(main_res["launches"] * args.steps)),
             "clocks": main_res["clocks"],
             "steps_ms": main_res["steps_ms"],
+            "summary": main_res["summary"],
             "second": second,
         }
         print(json.dumps(line), flush=True)

@@ -20,8 +20,13 @@
  *     history <- X[:n], query tokens <- X[n:], T <- n
  *   Visibility: a history query at position p sees keys t <= p; a query token
  *   sees every current history key and no query token; no key -> zero output.
- *   Output: the final query-token rows, or, with d_out > 0, W_e times the mean
- *   of the final layer's rows.
+ *   Output: the final query-token rows; or, with d_out > 0, W_e times the mean
+ *   of the final layer's rows; or, with n_sum > 0, the sequence summaries
+ *   Z_seq^(k) = W_up,k SiLU(W_down,k Flatten(Z_raw)), k = 1..n_sum, of the
+ *   final query-token rows Z_raw [n_q, d] flattened row-major (token 0 first)
+ *   (appendix A.2 item 4 "Sequence Summaries"; the pages call each map a
+ *   low-rank adapted MLP and give no formula: a SiLU MLP whose hidden layer
+ *   is the rank sum_rank bottleneck, without biases, is the reading taken).
  *
  * Conventions
  *   - All matrices are row-major [out, in] as on the pages.
@@ -83,6 +88,9 @@ enum {
  *   max_batch             largest B a forward may pass
  *   max_len               longest history a user may have
  *   max_total             largest sum of lengths in one batch (0 = max_batch*max_len)
+ *   n_sum                 sequence summaries (0 = none; needs n_q > 0 and d_out == 0;
+ *                         at most LLATTE_MAX_SUMMARIES)
+ *   sum_rank, d_seq       bottleneck width (1 .. 1024) and width (even) of each summary
  */
 typedef struct {
   int32_t d, heads, d_head, rank, d_ctx, n_q, n_layers;
@@ -92,7 +100,10 @@ typedef struct {
   int32_t max_batch;
   int64_t max_len;
   int64_t max_total;
+  int32_t n_sum, sum_rank, d_seq;
 } llatte_dims;
+
+#define LLATTE_MAX_SUMMARIES 16
 
 /*
  * Weights of one layer, non-absorbed, in `dtype` (row-major [out, in]):
@@ -106,6 +117,15 @@ typedef struct {
   const void *W_dkv, *g_kv, *W_q, *W_uk, *W_uv, *W_o, *g1, *W1, *W2, *g2;
 } llatte_layer_w;
 
+/*
+ * Weights of one sequence summary k, in `dtype` (row-major [out, in]):
+ *   W_down [sum_rank, n_q*d]   bottleneck projection of the flattened rows
+ *   W_up   [d_seq, sum_rank]   output projection
+ */
+typedef struct {
+  const void *W_down, *W_up;
+} llatte_summary_w;
+
 typedef struct llatte_handle llatte_handle;
 
 /*
@@ -113,12 +133,14 @@ typedef struct llatte_handle llatte_handle;
  * weights_on_device == 0, device memory otherwise) are copied; the caller may
  * free them afterwards.  The absorbed matrices W_uk^T W_q / sqrt(d_h) and
  * W_o W_uv are formed on the device in fp32 and stored in `dtype`.  W_e is
- * [d_out, d] (ignored when d_out == 0).  The handle owns a workspace sized
- * from max_batch / max_total; llatte_workspace_bytes reports its size.
- * Synchronous.
+ * [d_out, d] (ignored when d_out == 0); summaries points to n_sum
+ * llatte_summary_w (ignored, and may be NULL, when n_sum == 0).  The handle
+ * owns a workspace sized from max_batch / max_total; llatte_workspace_bytes
+ * reports its size.  Synchronous.
  */
 int llatte_create(llatte_handle** handle, const llatte_dims* dims,
-                  const llatte_layer_w* layers, const void* W_e, int weights_on_device);
+                  const llatte_layer_w* layers, const void* W_e,
+                  const llatte_summary_w* summaries, int weights_on_device);
 
 /*
  * One forward pass, asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -131,7 +153,8 @@ int llatte_create(llatte_handle** handle, const llatte_dims* dims,
  *   B       number of users, 0 <= B <= max_batch (B = 0 launches nothing)
  *   context device [B, d_ctx] in dtype (may be NULL when d_ctx == 0)
  *   cand    device [B, n_q, d] in dtype (may be NULL when n_q == 0)
- *   out     device fp32 [B, n_q, d] (d_out == 0) or [B, d_out]
+ *   out     device fp32 [B, n_q, d] (d_out == 0, n_sum == 0), [B, d_out]
+ *           (d_out > 0) or [B, n_sum, d_seq] (n_sum > 0)
  * Inputs are only read; `out` is the only caller memory written.  Calls on
  * one handle must not overlap in time (they share its workspace).
  */
@@ -163,9 +186,9 @@ const char* llatte_error_string(int code);
 /*
  * Per-step device timing, a profiling aid.  With profiling enabled every
  * forward records a CUDA event pair on its stream around each step (plan,
- * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout, and ffn when the FFN
- * runs as one fused kernel); llatte_profile_step synchronises on the recorded
- * events and returns, for step index `step` (0 .. 10), its name, the
+ * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout, ffn when the FFN
+ * runs as one fused kernel, and summary); llatte_profile_step synchronises on
+ * the recorded events and returns, for step index `step` (0 .. 11), its name, the
  * accumulated milliseconds, the number of kernels the
  * step launched and the number of times it ran since the last reset.
  * Returns LLATTE_ERR_ARG for a step index out of range.

@@ -14,7 +14,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libllatte.so")
 MAX_LAYERS = 16
-STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout", "ffn")
+STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout", "ffn",
+         "summary")
 
 LLATTE_OK, LLATTE_ERR_ARG, LLATTE_ERR_UNSUPPORTED, LLATTE_ERR_CUDA, LLATTE_ERR_OOM, \
     LLATTE_ERR_DEVICE = 0, -1, -2, -3, -4, -5
@@ -35,7 +36,8 @@ class llatte_dims(ctypes.Structure):
                 ("d_out", ctypes.c_int32), ("ffn_mult", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("kv_norm", ctypes.c_int32), ("eps", ctypes.c_float),
                 ("max_batch", ctypes.c_int32), ("max_len", ctypes.c_int64),
-                ("max_total", ctypes.c_int64)]
+                ("max_total", ctypes.c_int64), ("n_sum", ctypes.c_int32),
+                ("sum_rank", ctypes.c_int32), ("d_seq", ctypes.c_int32)]
 
 
 LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2")
@@ -43,6 +45,13 @@ LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "
 
 class llatte_layer_w(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in LAYER_KEYS]
+
+
+SUMMARY_KEYS = ("W_down", "W_up")
+
+
+class llatte_summary_w(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in SUMMARY_KEYS]
 
 
 EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
@@ -65,7 +74,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
                            "`python -m latent_attention_jagged_b200.build`")
     lib = ctypes.CDLL(p)
     P, I32, I64, VP = ctypes.POINTER, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
-    lib.llatte_create.argtypes = [P(VP), P(llatte_dims), P(llatte_layer_w), VP, ctypes.c_int]
+    lib.llatte_create.argtypes = [P(VP), P(llatte_dims), P(llatte_layer_w), VP,
+                                  P(llatte_summary_w), ctypes.c_int]
     lib.llatte_create.restype = ctypes.c_int
     lib.llatte_forward.argtypes = [VP, VP, VP, I32, VP, VP, VP, VP]
     lib.llatte_forward.restype = ctypes.c_int
@@ -115,6 +125,9 @@ def make_dims(dims, max_batch: int, max_len: int, max_total: int = 0) -> llatte_
     c.dtype = {"bf16": LLATTE_BF16, "fp32": LLATTE_FP32}[dims.dtype]
     c.kv_norm, c.eps = dims.kv_norm, float(dims.eps)
     c.max_batch, c.max_len, c.max_total = int(max_batch), int(max_len), int(max_total)
+    c.n_sum = int(getattr(dims, "n_sum", 0))
+    c.sum_rank = int(getattr(dims, "sum_rank", 0))
+    c.d_seq = int(getattr(dims, "d_seq", 0))
     return c
 
 
@@ -142,7 +155,8 @@ class Llatte:
     absorbed at construction; `forward` runs the whole sequence module."""
 
     def __init__(self, dims, layers: Sequence[dict], W_e=None, max_batch: int = 1,
-                 max_len: int = 0, max_total: int = 0, lib_path: Optional[str] = None):
+                 max_len: int = 0, max_total: int = 0, lib_path: Optional[str] = None,
+                 summaries: Optional[Sequence[dict]] = None):
         self.lib = load_library(lib_path)
         self.dims = dims
         self.cdims = make_dims(dims, max_batch, max_len, max_total)
@@ -160,9 +174,20 @@ class Llatte:
         if dims.d_out:
             we = _host(W_e, self.dt)
             keep_alive.append(we)
+        n_sum = int(getattr(dims, "n_sum", 0))
+        sarr = None
+        if n_sum:
+            if summaries is None or len(summaries) != n_sum:
+                raise ValueError(f"{n_sum} summary weight dicts are required")
+            sarr = (llatte_summary_w * n_sum)()
+            for i, w in enumerate(summaries):
+                for k in SUMMARY_KEYS:
+                    t = _host(w[k], self.dt)
+                    keep_alive.append(t)
+                    setattr(sarr[i], k, t.data_ptr())
         h = ctypes.c_void_p()
         rc = self.lib.llatte_create(ctypes.byref(h), ctypes.byref(self.cdims), arr,
-                                    _ptr(we), 0)
+                                    _ptr(we), sarr, 0)
         if rc != LLATTE_OK:
             raise LlatteError(rc, "llatte_create")
         self.h = h
@@ -173,6 +198,8 @@ class Llatte:
 
     def out_shape(self, B: int):
         d = self.dims
+        if getattr(d, "n_sum", 0):
+            return (B, d.n_sum, d.d_seq)
         return (B, d.d_out) if d.d_out else (B, d.n_q, d.d)
 
     def forward(self, values: torch.Tensor, offsets: torch.Tensor, context=None, cand=None,

@@ -13,6 +13,9 @@ Per user and layer, with T history rows in, n = min(T, keep) kept, q = n + n_q:
   o       2 q h r d
   ffn1    2 q d (m d)      ffn2  2 q (m d) d        (m = FFN multiplier)
   readout 2 d d_out per user (final layer)
+  summary 2 k R (n_q d + d_seq) per user: k sequence summaries, each a
+          bottleneck of width R over the flattened n_q x d final query rows
+          then the projection to d_seq (appendix A.2 item 4)
 Masked pairs and padding are not counted.
 """
 from __future__ import annotations
@@ -65,7 +68,26 @@ def total_flops(lengths: Sequence[int], dims) -> float:
     tot = sum(sum(w.flops.values()) for w in work)
     if dims.d_out:
         tot += 2.0 * len(lengths) * dims.d * dims.d_out
+    tot += summary_flops(len(lengths), dims)
     return float(tot)
+
+
+def summary_flops(B: int, dims) -> float:
+    k = getattr(dims, "n_sum", 0)
+    if not k:
+        return 0.0
+    return 2.0 * B * k * dims.sum_rank * (dims.n_q * dims.d + dims.d_seq)
+
+
+def summary_bytes(B: int, dims, elem: int = 2) -> float:
+    """Bytes the summary step must move at least: the final query rows and
+    both projections read once (storage type), the summaries written (fp32)."""
+    k = getattr(dims, "n_sum", 0)
+    if not k:
+        return 0.0
+    rows = B * dims.n_q * dims.d * elem
+    w = k * dims.sum_rank * (dims.n_q * dims.d + dims.d_seq) * elem
+    return float(rows + w + B * k * dims.d_seq * 4)
 
 
 def flops_by_step(lengths: Sequence[int], dims) -> Dict[str, float]:
@@ -76,6 +98,8 @@ def flops_by_step(lengths: Sequence[int], dims) -> Dict[str, float]:
     if dims.d_out:
         acc["readout"] = 2.0 * len(lengths) * dims.d * dims.d_out
     acc["ffn"] = acc["ffn1"] + acc["ffn2"]      # the FFN as one fused step
+    if getattr(dims, "n_sum", 0):
+        acc["summary"] = summary_flops(len(lengths), dims)
     return acc
 
 
@@ -88,5 +112,10 @@ def io_bytes(lengths: Sequence[int], dims, elem: int = 2) -> float:
     inp = (lengths.sum() + B * dims.n_q) * d * elem + B * dc * elem + (B + 1) * 8
     per_layer_w = (r * d + r + hd * (d + dc) + 2 * hd * r + d * hd + 2 * d + 2 * f * d) * elem
     w = dims.n_layers * per_layer_w + dims.d_out * d * elem
-    out = B * (dims.d_out if dims.d_out else dims.n_q * d) * 4
+    k = getattr(dims, "n_sum", 0)
+    if k:
+        w += k * dims.sum_rank * (dims.n_q * d + dims.d_seq) * elem
+        out = B * k * dims.d_seq * 4
+    else:
+        out = B * (dims.d_out if dims.d_out else dims.n_q * d) * 4
     return float(inp + w + out)

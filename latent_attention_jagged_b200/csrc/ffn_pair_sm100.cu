@@ -355,8 +355,13 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
           const int64_t jr = row - a.qoff_l[u];
           const int32_t nl = a.n_l[u];
           if (a.last) {
-            if (a.final_rows) f_dst = row;
-            else if (jr >= nl) f_dst = (int64_t)u * a.n_q + (jr - nl);
+            if (a.zraw) {
+              if (jr >= nl) h_dst = (int64_t)u * a.n_q + (jr - nl);   // summary input row
+            } else if (a.final_rows) {
+              f_dst = row;
+            } else if (jr >= nl) {
+              f_dst = (int64_t)u * a.n_q + (jr - nl);
+            }
           } else {
             const int32_t nn = a.n_n[u];
             if (jr < nl) {
@@ -369,6 +374,7 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
         }
       }
       float* const f_base = a.final_rows ? a.final_rows : a.out;
+      __nv_bfloat16* const h_base = (__nv_bfloat16*)(a.last ? a.zraw : a.Xh_n);
       bool w = mbar_wait(v_full, ti & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) break;
 #pragma unroll 1
@@ -413,8 +419,7 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
           for (int k = 0; k < 8; ++k) x[k] *= inv * g8[k];
           const uint4 wb = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
                                       pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          if (hd >= 0)
-            *reinterpret_cast<uint4*>((__nv_bfloat16*)a.Xh_n + hd * D + 8 * lane) = wb;
+          if (hd >= 0) *reinterpret_cast<uint4*>(h_base + hd * D + 8 * lane) = wb;
           if (qd >= 0) {
             *reinterpret_cast<uint4*>((__nv_bfloat16*)a.Xq_n + qd * D + 8 * lane) = wb;
             if (a.Xq_res_n)

@@ -11,17 +11,22 @@
 //               STORE     bf16 store
 //               USERBIAS  + per-user context term (absorbed query projection)
 //               SILU      SiLU (FFN up-projection)
+//               PARTIAL   fp32 partial sums of one k-slice (split-K)
 //               NORM      + residual (read once: the sum is staged back in
 //                         TMEM), RMSNorm over the full row (BN == N; the two
 //                         halves' sums of squares meet in shared memory),
 //                         store bf16 (+ fp16 residual copy) or scatter into the
 //                         next layer's history / query rows (pyramid trimming)
 // The accumulator is double-buffered in TMEM when 2 * BN <= 512 columns, so
-// the epilogue of tile i overlaps the MMAs of tile i + 1.
+// the epilogue of tile i overlaps the MMAs of tile i + 1.  With split-K a tile
+// is (row block, column block, k-slice); the slices of one output tile are
+// consecutive tile indices.
 //
 // Equations (LLaTTE notes, huaxiaozhuan.com, appendix A.2 display and A.3):
 // KV latent RMSNorm(X W_down^KV); absorbed query X (W_uk^T W_q)^T + context
 // term; Z = RMSNorm(R + o~ (W_o W_uv)^T); FFN W2 SiLU(W1 Z) + Z, RMSNorm.
+// Split-K: the bottleneck projection of the sequence summaries (appendix A.2
+// item 4), whose K = n_q * d is long and whose output is small.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -66,8 +71,8 @@ struct GemmCfg {
 // through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
 __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0, int half, float* red, int rrow,
-                                         uint64_t* xbar, uint32_t& xphase,
+                                         bool valid, int n0, int ks, int half, float* red,
+                                         int rrow, uint64_t* xbar, uint32_t& xphase,
                                          volatile int* abort_flag, uint32_t stg,
                                          NormPre<BN, 4>& pre, const __nv_bfloat16* sg) {
   constexpr int HB = BN / 2;                 // columns per thread
@@ -75,6 +80,25 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
                              abort_flag, p.status, stg, pre, sg);
+  } else if constexpr (EPI == TC_PARTIAL) {
+    float* prow = valid ? p.Dp + ks * p.slice_stride + row * p.N + n0 : nullptr;
+#pragma unroll 1
+    for (int c = c0; c < c0 + HB; c += 32) {
+      float v[32];
+      tmem_ld32(taddr + c, v);
+      // 32 fp32 = two 64-byte staged row pieces
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint4 x[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x[j] = make_uint4(__float_as_uint(v[16 * h + 4 * j]), __float_as_uint(v[16 * h + 4 * j + 1]),
+                            __float_as_uint(v[16 * h + 4 * j + 2]),
+                            __float_as_uint(v[16 * h + 4 * j + 3]));
+        stage_store(stg, x, prow ? prow + c + 16 * h : nullptr);
+      }
+    }
+    return true;
   } else {
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = p.row_user[row];
@@ -141,6 +165,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n_tiles = p.N / BN;
   const int KB = p.K / BK;
   const int kb0 = blockIdx.x % KB;
+  const int S = (EPI == TC_PARTIAL && p.k_split > 1) ? p.k_split : 1;   // k-slices (<= KB)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -164,7 +189,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   // everything below reads what earlier kernels wrote
   pdl_wait();
   const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
-  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles * S;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -172,13 +197,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t phase = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
-        for (int kb = 0; kb < KB; ++kb) {
+        const int64_t tt = t / S;
+        const int ks = (int)(t % S);
+        const int mt = (int)(tt / n_tiles), nt = (int)(tt % n_tiles);
+        const int kb_lo = (int)((int64_t)ks * KB / S);
+        const int nkb = (int)((int64_t)(ks + 1) * KB / S) - kb_lo;
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           // k-blocks in a per-CTA rotated order: the SMs do not all read the
           // same weight lines from L2 at the same moment
-          const int kx = ((kb + kb0) % KB) * BK;
+          const int kx = (kb_lo + (kb + kb0) % nkb) * BK;
           tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kx, mt * BM);
 #pragma unroll
           for (int s2 = 0; s2 < NSUB; ++s2)
@@ -199,7 +228,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_base = tmem + acc * BN;
-        for (int kb = 0; kb < KB; ++kb) {
+        const int ks = (int)(t % S);
+        const int nkb = (int)((int64_t)(ks + 1) * KB / S) - (int)((int64_t)ks * KB / S);
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
@@ -233,7 +264,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0, it = 0;
     uint32_t acc_phase = 0, xphase = 0;
     for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
+      const int64_t tt = t / S;
+      const int ks = (int)(t % S);
+      const int mt = (int)(tt / n_tiles), nt = (int)(tt % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
       NormPre<BN, 4> pre;
@@ -241,7 +274,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, half,
+      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, half,
                              red + (it & 1) * 256, rr, xbar, xphase, abort_flag,
                              smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
         break;
@@ -285,7 +318,7 @@ cudaError_t launch_epi(int BN, const CUtensorMap& a, const CUtensorMap& b, const
     case 256: return launch_cfg<256, EPI>(a, b, p, grid, s);
     case 512:
       if constexpr (EPI == TC_NORM) return launch_cfg<512, EPI>(a, b, p, grid, s);
-      return cudaErrorInvalidValue;
+      else return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -297,20 +330,28 @@ bool tc_gemm_supported(int BN, int epi, int N, int K) {
   if (BN != 64 && BN != 128 && BN != 256 && BN != 512) return false;
   if (BN == 512 && epi != TC_NORM) return false;
   if (epi == TC_NORM && N != BN) return false;
+  if (epi == TC_PARTIAL && BN > 128) return false;
   return N % BN == 0;
 }
 
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
                            const TcGemmParams& p, int num_sms, cudaStream_t s) {
   if (!tc_gemm_supported(BN, epi, p.N, p.K)) return cudaErrorInvalidValue;
+  if (epi == TC_PARTIAL && (p.k_split < 1 || p.k_split > p.K / BK || !p.Dp))
+    return cudaErrorInvalidValue;
   // grid: one CTA per SM, never more CTAs than the largest possible tile count
-  const int64_t max_tiles = ((p.M_cap + BM - 1) / BM) * (p.N / BN);
+  const int64_t max_tiles =
+      ((p.M_cap + BM - 1) / BM) * (p.N / BN) * (epi == TC_PARTIAL ? p.k_split : 1);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, max_tiles));
   switch (epi) {
     case TC_STORE: return launch_epi<TC_STORE>(BN, a, b, p, grid, s);
     case TC_USERBIAS: return launch_epi<TC_USERBIAS>(BN, a, b, p, grid, s);
     case TC_SILU: return launch_epi<TC_SILU>(BN, a, b, p, grid, s);
     case TC_NORM: return launch_epi<TC_NORM>(BN, a, b, p, grid, s);
+    case TC_PARTIAL:
+      if (BN == 64) return launch_cfg<64, TC_PARTIAL>(a, b, p, grid, s);
+      if (BN == 128) return launch_cfg<128, TC_PARTIAL>(a, b, p, grid, s);
+      return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }

@@ -13,7 +13,7 @@ namespace llatte {
 
 // Step kinds, for the optional per-step timing.
 enum Step { ST_PLAN = 0, ST_GATHER, ST_CTX, ST_KV, ST_Q, ST_ATTN, ST_O, ST_FFN1, ST_FFN2,
-            ST_READOUT, ST_FFN, ST_COUNT };
+            ST_READOUT, ST_FFN, ST_SUMMARY, ST_COUNT };
 extern const char* const kStepNames[ST_COUNT];
 
 // Device-side pyramid plan.  Layer index l runs over 0..L where l = L is the
@@ -70,6 +70,14 @@ struct llatte_handle {
   int num_sms;
   llatte::LayerDev layers[LLATTE_MAX_LAYERS];
   void* W_e;                      // [d_out, d]
+  // sequence summaries: the stacked bottleneck projections, the output
+  // projections transposed, the final query-token rows and the split-K partials
+  void* W_sdown;                  // [n_sum * sum_rank, n_q * d]
+  void* W_supT;                   // [n_sum][sum_rank][d_seq]
+  void* zraw;                     // [max_batch, n_q * d] storage type
+  float* sum_part;                // [k slices][rows][n_sum * sum_rank] fp32
+  int sum_tc;                     // bottleneck GEMM on the tensor cores
+  int sum_bn;                     // its tile width
   std::vector<void*> allocs;
 
   // workspace
@@ -100,6 +108,7 @@ struct llatte_handle {
   int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
   int pair_norm;                  // output / FFN-down projections on SM pairs (d = 512)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
+  CUtensorMap tm_zraw, tm_sdown;  // summary bottleneck GEMM operands
 
   // the per-user context term runs on a side stream, beside the plan and
   // the gather (forked from and joined back into the caller's stream)
@@ -154,6 +163,9 @@ struct NormArgs {
   // NORM_SCATTER (FFN2 output of layer l -> inputs of layer l+1 / outputs)
   const int64_t *qoff_l, *hoff_n, *qoff_n; const int32_t *n_l, *n_n; int B; int n_q;
   void* Xh_n; void* Xq_n; void* Xq_res_n; int last; float* out; float* final_rows;
+  // last layer with sequence summaries: the query-token rows go, in the
+  // storage type, to zraw[u * n_q + j] instead of the fp32 output
+  void* zraw;
   const int32_t* row_user;           // user of each query row of layer l (tensor-core path)
 };
 enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
@@ -173,6 +185,19 @@ cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
 struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [d_ctx, h*r] per layer
 cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
                             int dc, float* out, cudaStream_t s);
+
+// Sequence summaries after the bottleneck GEMM: h = SiLU(sum of the S split-K
+// partial rows), out[b, k, :] = h[b, k-block] W_up,k^T.
+struct SummaryArgs {
+  const float* P; int S; int64_t slice_stride;   // P[s * slice_stride + b * N + j]
+  int B, N, rank, d_seq, n_sum;                  // N = n_sum * rank
+  const void* Wt;                                // [n_sum][rank][d_seq] storage type
+  float* out;                                    // [B, n_sum, d_seq]
+};
+cudaError_t launch_summary_up(int elem, const SummaryArgs& a, int num_sms, cudaStream_t s);
+// dst[c, r] = src[r, c] for a [rows, cols] matrix of the storage type.
+cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
+                             cudaStream_t s);
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
                              cudaStream_t s);

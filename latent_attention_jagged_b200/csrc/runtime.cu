@@ -15,19 +15,31 @@ using namespace llatte;
 
 namespace llatte {
 const char* const kStepNames[ST_COUNT] = {"plan", "gather", "ctx_bias", "kv",      "q",  "attn",
-                                          "o",    "ffn1",   "ffn2",     "readout", "ffn"};
+                                          "o",    "ffn1",   "ffn2",     "readout", "ffn",
+                                          "summary"};
 }
 
 namespace {
 
 size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
+// Split-K of the summary bottleneck GEMM: about this many CTAs in all (the
+// SM count of a B200); the workspace bound below follows from it.
+constexpr int kSplitCtas = 148;
+constexpr int kSumMaxBN = 128;
+
+int summary_slices(int64_t B, int N, int BN, int K) {
+  const int64_t tiles = ((B + 127) / 128) * (N / BN);
+  const int64_t KB = K / 64;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(KB, kSplitCtas / std::max<int64_t>(tiles, 1)));
+}
+
 struct Layout {
   int64_t rows_h, rows_q;
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
       off_work_count, off_work_next, off_item_off, off_row_user;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
-      off_final, off_mean, off_Zres, off_Xqres[2];
+      off_final, off_mean, off_Zres, off_Xqres[2], off_zraw, off_sum_part;
   size_t total;
   int32_t max_work;
 };
@@ -41,6 +53,11 @@ int check_dims(const llatte_dims* d) {
   if (!(d->eps > 0.f)) return LLATTE_ERR_ARG;
   if (d->max_batch <= 0 || d->max_len < 0 || d->max_total < 0) return LLATTE_ERR_ARG;
   if (d->kv_norm != 0 && d->kv_norm != 1) return LLATTE_ERR_ARG;
+  if (d->n_sum < 0 || d->n_sum > LLATTE_MAX_SUMMARIES) return LLATTE_ERR_ARG;
+  if (d->n_sum > 0) {
+    if (d->n_q <= 0 || d->d_out > 0 || d->sum_rank <= 0 || d->d_seq <= 0) return LLATTE_ERR_ARG;
+    if (d->sum_rank > 1024 || d->d_seq % 2 != 0) return LLATTE_ERR_UNSUPPORTED;
+  }
   for (int l = 0; l < d->n_layers; ++l) {
     if (d->keep[l] < 0) return LLATTE_ERR_ARG;
     if (l && d->keep[l] > d->keep[l - 1]) return LLATTE_ERR_ARG;  // T_{l+1} <= T_l
@@ -92,6 +109,12 @@ Layout layout_of(const llatte_dims* d) {
   L.off_ctxbias = take(sizeof(float) * nl * B * hr);
   L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
   L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
+  // sequence summaries: the final query-token rows and the split-K partials
+  // (S * B <= kSplitCtas * 128 / column tiles, or S = 1)
+  const int64_t sN = (int64_t)d->n_sum * d->sum_rank;
+  L.off_zraw = take(d->n_sum ? (size_t)B * d->n_q * d->d * elem : 0);
+  L.off_sum_part = take(d->n_sum ? sizeof(float) * std::max<int64_t>(
+                                       (int64_t)kSplitCtas * 128 * kSumMaxBN, B * sN) : 0);
   L.total = o;
   return L;
 }
@@ -258,7 +281,7 @@ void llatte_destroy(llatte_handle* h) {
 }
 
 int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_layer_w* layers,
-                  const void* W_e, int weights_on_device) {
+                  const void* W_e, const llatte_summary_w* summaries, int weights_on_device) {
   if (!out) return LLATTE_ERR_ARG;
   *out = nullptr;
   int rc = check_dims(dims);
@@ -272,6 +295,11 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
       return LLATTE_ERR_ARG;
   }
   if (D.d_out > 0 && !W_e) return LLATTE_ERR_ARG;
+  if (D.n_sum > 0) {
+    if (!summaries) return LLATTE_ERR_ARG;
+    for (int k = 0; k < D.n_sum; ++k)
+      if (!summaries[k].W_down || !summaries[k].W_up) return LLATTE_ERR_ARG;
+  }
 
   llatte_handle* h = new (std::nothrow) llatte_handle();
   if (!h) return LLATTE_ERR_OOM;
@@ -334,6 +362,29 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     h->W_e = upload(h, W_e, e * (size_t)D.d_out * d, weights_on_device);
     if (!h->W_e) return fail(LLATTE_ERR_OOM);
   }
+  h->W_sdown = h->W_supT = nullptr;
+  if (D.n_sum > 0) {
+    // bottleneck projections stacked into one [n_sum * sum_rank, n_q * d]
+    // matrix; output projections transposed to [sum_rank][d_seq] each
+    const size_t rs = D.sum_rank, K = (size_t)D.n_q * d, ds = D.d_seq;
+    h->W_sdown = dev_alloc(h, e * D.n_sum * rs * K);
+    h->W_supT = dev_alloc(h, e * D.n_sum * rs * ds);
+    if (!h->W_sdown || !h->W_supT) return fail(LLATTE_ERR_OOM);
+    void* tmp = nullptr;
+    if (cudaMalloc(&tmp, e * rs * ds) != cudaSuccess) return fail(LLATTE_ERR_OOM);
+    const cudaMemcpyKind k = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    bool ok = true;
+    for (int j = 0; j < D.n_sum && ok; ++j) {
+      ok = cudaMemcpy((char*)h->W_sdown + e * j * rs * K, summaries[j].W_down, e * rs * K, k) ==
+               cudaSuccess &&
+           cudaMemcpy(tmp, summaries[j].W_up, e * rs * ds, k) == cudaSuccess &&
+           launch_transpose(h->elem, tmp, (int64_t)ds, (int64_t)rs,
+                            (char*)h->W_supT + e * j * rs * ds, 0) == cudaSuccess &&
+           cudaDeviceSynchronize() == cudaSuccess;
+    }
+    cudaFree(tmp);
+    if (!ok) return fail(LLATTE_ERR_CUDA);
+  }
 
   Layout Lo = layout_of(&D);
   char* ws = (char*)dev_alloc(h, Lo.total);
@@ -369,9 +420,23 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->ctxbias = (float*)(ws + Lo.off_ctxbias);
   h->final_rows = D.d_out ? (float*)(ws + Lo.off_final) : nullptr;
   h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
+  h->zraw = D.n_sum ? (void*)(ws + Lo.off_zraw) : nullptr;
+  h->sum_part = D.n_sum ? (float*)(ws + Lo.off_sum_part) : nullptr;
+  h->sum_tc = 0;
+  h->sum_bn = 0;
   if (want_tc) {
     if (!build_tc_maps(h)) return fail(LLATTE_ERR_CUDA);
     h->use_tc = 1;
+    if (D.n_sum > 0) {
+      const int N = D.n_sum * D.sum_rank, K = D.n_q * d;
+      h->sum_bn = N % 128 == 0 ? 128 : 64;
+      if (tc_gemm_supported(h->sum_bn, TC_PARTIAL, N, K)) {
+        if (!make_tmap_bf16(&h->tm_zraw, h->zraw, D.max_batch, K, 128) ||
+            !make_tmap_bf16(&h->tm_sdown, h->W_sdown, N, K, h->sum_bn))
+          return fail(LLATTE_ERR_CUDA);
+        h->sum_tc = 1;
+      }
+    }
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLATTE_ERR_CUDA);
   *out = h;
@@ -453,6 +518,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     f_norm.Xh_n = Xh_n; f_norm.Xq_n = Xq_n; f_norm.last = last;
     f_norm.Xq_res_n = (res16 && !last) ? h->Xqres[(l + 1) & 1] : nullptr;
     f_norm.out = out; f_norm.final_rows = D.d_out ? h->final_rows : nullptr;
+    f_norm.zraw = (last && D.n_sum > 0) ? h->zraw : nullptr;
     f_norm.row_user = p.ruser(l);
     const LayerMaps& LM = h->lmaps[l];
     auto tcp = [&](const int64_t* Mdev, int64_t cap, int N, int K) {
@@ -595,6 +661,28 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     g.A = h->mean_rows; g.lda = d; g.W = h->W_e; g.D = out; g.ldd = D.d_out;
     g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = D.d_out; g.K = d; g.epi = EPI_F32;
     CK(launch_gemm_simt(4, e, 4, g, s));
+    t.done(2);
+  }
+  if (D.n_sum > 0) {  // sequence summaries of the final query-token rows
+    StepTimer t(h, s, ST_SUMMARY);
+    const int N = D.n_sum * D.sum_rank, K = D.n_q * d;
+    int S = 1;
+    if (h->sum_tc) {
+      S = summary_slices(B, N, h->sum_bn, K);
+      TcGemmParams q = {};
+      q.M_host = B; q.M_dev = nullptr; q.M_cap = B; q.N = N; q.K = K; q.status = p.status;
+      q.Dp = h->sum_part; q.slice_stride = (int64_t)B * N; q.k_split = S;
+      CK(launch_tc_gemm(h->sum_bn, TC_PARTIAL, h->tm_zraw, h->tm_sdown, q, h->num_sms, s));
+    } else {
+      GemmArgs g = {};
+      g.A = h->zraw; g.lda = K; g.W = h->W_sdown; g.D = h->sum_part; g.ldd = N;
+      g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = N; g.K = K; g.epi = EPI_F32;
+      CK(launch_gemm_simt(e, e, 4, g, s));
+    }
+    SummaryArgs sa = {};
+    sa.P = h->sum_part; sa.S = S; sa.slice_stride = (int64_t)B * N; sa.B = B; sa.N = N;
+    sa.rank = D.sum_rank; sa.d_seq = D.d_seq; sa.n_sum = D.n_sum; sa.Wt = h->W_supT; sa.out = out;
+    CK(launch_summary_up(e, sa, h->num_sms, s));
     t.done(2);
   }
   return LLATTE_OK;

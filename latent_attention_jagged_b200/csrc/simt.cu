@@ -10,6 +10,8 @@
 //   FFN   X'   = RMSNorm_{g2}(Z + W2 SiLU(W1 Z))
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -135,8 +137,13 @@ rownorm_kernel(NormArgs a) {
     const int64_t j = m - a.qoff_l[u];
     const int32_t nl = a.n_l[u];
     if (a.last) {
-      if (a.final_rows) f1 = a.final_rows + m * N;
-      else if (j >= nl) f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+      if (a.zraw) {
+        if (j >= nl) d1 = (T*)a.zraw + ((int64_t)u * a.n_q + (j - nl)) * N;
+      } else if (a.final_rows) {
+        f1 = a.final_rows + m * N;
+      } else if (j >= nl) {
+        f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+      }
     } else {
       const int32_t nn = a.n_n[u];
       int64_t q = -1;
@@ -311,6 +318,116 @@ cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int 
                              cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   mean_rows_kernel<<<B, 256, 0, s>>>(rows, qoff, d, mean);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- summaries
+// Sequence summaries (LLaTTE notes, appendix A.2 item 4), the step after the
+// bottleneck GEMM, which has left S partial sums per (user, bottleneck unit).
+// A block takes SUM_UB users and one summary k: h = SiLU(sum of the partials,
+// in slice order, so the result does not depend on timing), then
+// out[b, k, i] = sum_t W_up,k[i, t] h[b, t].  The output projection is stored
+// transposed ([t][i]): a warp reads 64 consecutive outputs' weights of one t
+// in one line, and every thread keeps SUM_UB x 2 accumulators.
+constexpr int SUM_UB = 8;
+
+__device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) summary_up_kernel(SummaryArgs a) {
+  extern __shared__ float4 sh4[];                  // [SUM_UB][r4] fp32, zero padded
+  float* sh = reinterpret_cast<float*>(sh4);
+  const int b0 = blockIdx.x * SUM_UB, k = blockIdx.y;
+  const int r = a.rank, r4 = (r + 3) & ~3;
+  for (int idx = threadIdx.x; idx < SUM_UB * r4; idx += blockDim.x) {
+    const int u = idx / r4, t = idx - u * r4;
+    const int b = b0 + u;
+    float v = 0.f;
+    if (b < a.B && t < r) {
+      const float* p = a.P + (int64_t)b * a.N + (int64_t)k * r + t;
+      for (int s = 0; s < a.S; ++s) v += p[s * a.slice_stride];
+      v = silu_f(v);
+    }
+    sh[idx] = v;
+  }
+  __syncthreads();
+  const int half_d = a.d_seq / 2;
+  const T* W = (const T*)a.Wt + (int64_t)k * r * a.d_seq;
+  const int rq = r & ~3;
+  for (int pi = blockIdx.z * blockDim.x + threadIdx.x; pi < half_d;
+       pi += gridDim.z * blockDim.x) {
+    float acc[SUM_UB][2];
+#pragma unroll
+    for (int u = 0; u < SUM_UB; ++u) acc[u][0] = acc[u][1] = 0.f;
+    const T* w = W + 2 * pi;
+#pragma unroll 1
+    for (int t = 0; t < rq; t += 4) {
+      float2 wf[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wf[i] = load2(w + (int64_t)(t + i) * a.d_seq);
+#pragma unroll
+      for (int u = 0; u < SUM_UB; ++u) {
+        const float4 hv = sh4[(u * r4 + t) >> 2];
+        acc[u][0] = fmaf(wf[0].x, hv.x, acc[u][0]); acc[u][1] = fmaf(wf[0].y, hv.x, acc[u][1]);
+        acc[u][0] = fmaf(wf[1].x, hv.y, acc[u][0]); acc[u][1] = fmaf(wf[1].y, hv.y, acc[u][1]);
+        acc[u][0] = fmaf(wf[2].x, hv.z, acc[u][0]); acc[u][1] = fmaf(wf[2].y, hv.z, acc[u][1]);
+        acc[u][0] = fmaf(wf[3].x, hv.w, acc[u][0]); acc[u][1] = fmaf(wf[3].y, hv.w, acc[u][1]);
+      }
+    }
+    for (int t = rq; t < r; ++t) {
+      const float2 wf = load2(w + (int64_t)t * a.d_seq);
+#pragma unroll
+      for (int u = 0; u < SUM_UB; ++u) {
+        const float hv = sh[u * r4 + t];
+        acc[u][0] = fmaf(wf.x, hv, acc[u][0]);
+        acc[u][1] = fmaf(wf.y, hv, acc[u][1]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SUM_UB; ++u) {
+      const int b = b0 + u;
+      if (b < a.B)
+        *reinterpret_cast<float2*>(a.out + ((int64_t)b * a.n_sum + k) * a.d_seq + 2 * pi) =
+            make_float2(acc[u][0], acc[u][1]);
+    }
+  }
+}
+
+cudaError_t launch_summary_up(int elem, const SummaryArgs& a, int num_sms, cudaStream_t s) {
+  if (a.B <= 0) return cudaSuccess;
+  if (a.d_seq <= 0 || (a.d_seq & 1) || a.rank <= 0 || a.rank > 1024 || a.n_sum <= 0 || a.S < 1)
+    return cudaErrorInvalidValue;
+  const int bx = (a.B + SUM_UB - 1) / SUM_UB;
+  // split the outputs of a (user block, summary) over z until the grid fills the SMs
+  const int pairs_blocks = (a.d_seq / 2 + 255) / 256;
+  const int z = std::max(1, std::min(pairs_blocks, num_sms / std::max(1, bx * a.n_sum)));
+  const dim3 grid(bx, a.n_sum, z);
+  const size_t smem = sizeof(float) * SUM_UB * ((a.rank + 3) & ~3);
+  if (elem == 4) summary_up_kernel<float><<<grid, 256, smem, s>>>(a);
+  else summary_up_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ src, int64_t rows, int64_t cols,
+                                 T* __restrict__ dst) {
+  const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (i >= rows * cols) return;
+  const int64_t r = i / cols, c = i - r * cols;
+  dst[c * rows + r] = src[i];
+}
+
+cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
+                             cudaStream_t s) {
+  const int64_t n = rows * cols;
+  if (n <= 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (elem == 4) transpose_kernel<float><<<blocks, 256, 0, s>>>((const float*)src, rows, cols, (float*)dst);
+  else transpose_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)src, rows, cols,
+                                                                (__nv_bfloat16*)dst);
   return cudaGetLastError();
 }
 

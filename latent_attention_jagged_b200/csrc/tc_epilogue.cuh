@@ -182,8 +182,13 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
       const int64_t j = row - a.qoff_l[u];
       const int32_t nl = a.n_l[u];
       if (a.last) {
-        if (a.final_rows) f1 = a.final_rows + row * N;
-        else if (j >= nl) f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+        if (a.zraw) {
+          if (j >= nl) d1 = (__nv_bfloat16*)a.zraw + ((int64_t)u * a.n_q + (j - nl)) * N;
+        } else if (a.final_rows) {
+          f1 = a.final_rows + row * N;
+        } else if (j >= nl) {
+          f1 = a.out + ((int64_t)u * a.n_q + (j - nl)) * N;
+        }
       } else {
         const int32_t nn = a.n_n[u];
         int64_t q = -1;

@@ -9,7 +9,7 @@
 
 namespace llatte {
 
-enum { TC_STORE = 0, TC_USERBIAS = 1, TC_SILU = 2, TC_NORM = 3 };
+enum { TC_STORE = 0, TC_USERBIAS = 1, TC_SILU = 2, TC_NORM = 3, TC_PARTIAL = 4 };
 
 struct TcGemmParams {
   int64_t M_host;               // rows, unless M_dev != NULL
@@ -20,6 +20,9 @@ struct TcGemmParams {
   const float* bias; const int64_t* seg_off; int B;   // USERBIAS: bias[user(row), n]
   const int32_t* row_user;                             // user of each row
   NormArgs norm;                                       // NORM (acc unused)
+  // PARTIAL: split-K over k_split slices of the k-blocks; slice s writes its
+  // fp32 partial sums to Dp[s * slice_stride + row * N + n]
+  float* Dp; int64_t slice_stride; int k_split;
   int32_t* status;
 };
 

@@ -26,7 +26,7 @@ def make_handle(inp, max_batch=None, max_len=None, max_total=0):
     B = inp.batch
     ml = int(inp.lengths.max()) if max_len is None and B else (max_len or 1)
     return Llatte(inp.dims, inp.layers, inp.W_e, max_batch=max_batch or max(B, 1),
-                  max_len=ml, max_total=max_total)
+                  max_len=ml, max_total=max_total, summaries=inp.summaries)
 
 
 def run(inp, handle=None, **kw):

@@ -45,9 +45,12 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_struct_layout_matches_header(lib):
-    # int32 x 7, keep[16], 4 x int32, float, int32, (pad 4), int64, int64
-    assert ctypes.sizeof(binding.llatte_dims) == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16
+    # int32 x 7, keep[16], 4 x int32, float, int32, (pad 4), int64, int64,
+    # int32 x 3, (pad 4)
+    assert ctypes.sizeof(binding.llatte_dims) == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16 + 16
+    assert binding.llatte_dims.n_sum.offset == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16
     assert ctypes.sizeof(binding.llatte_layer_w) == 10 * ctypes.sizeof(ctypes.c_void_p)
+    assert ctypes.sizeof(binding.llatte_summary_w) == 2 * ctypes.sizeof(ctypes.c_void_p)
 
 
 def _cdims(**kw):
@@ -76,13 +79,25 @@ def test_create_rejects_bad_arguments_on_host(lib):
     layers = (binding.llatte_layer_w * 4)()
     # increasing schedule: rejected before any device call
     bad = _cdims(keep=(10, 20, 30, 40))
-    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, 0) == \
+    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, None, 0) == \
         binding.LLATTE_ERR_ARG
     # null weight pointers
     good = _cdims()
-    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(good), layers, None, 0) == \
+    assert lib.llatte_create(ctypes.byref(h), ctypes.byref(good), layers, None, None, 0) == \
         binding.LLATTE_ERR_ARG
-    assert lib.llatte_create(None, ctypes.byref(good), layers, None, 0) == binding.LLATTE_ERR_ARG
+    assert lib.llatte_create(None, ctypes.byref(good), layers, None, None, 0) == binding.LLATTE_ERR_ARG
+    # summaries: need candidates, no d_out, weights; sizes within the kernels' range
+    for kw, code in ((dict(n_sum=2, sum_rank=8, d_seq=16, n_q=0), binding.LLATTE_ERR_ARG),
+                     (dict(n_sum=2, sum_rank=8, d_seq=16, d_out=32), binding.LLATTE_ERR_ARG),
+                     (dict(n_sum=2, sum_rank=0, d_seq=16), binding.LLATTE_ERR_ARG),
+                     (dict(n_sum=17, sum_rank=8, d_seq=16), binding.LLATTE_ERR_ARG),
+                     (dict(n_sum=2, sum_rank=8, d_seq=15), binding.LLATTE_ERR_UNSUPPORTED),
+                     (dict(n_sum=2, sum_rank=2048, d_seq=16), binding.LLATTE_ERR_UNSUPPORTED)):
+        bad = _cdims(**kw)
+        assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, None, 0) == code
+        assert lib.llatte_workspace_bytes(ctypes.byref(bad)) == 0
+    ok = _cdims(n_sum=2, sum_rank=8, d_seq=16)
+    assert lib.llatte_workspace_bytes(ctypes.byref(ok)) > lib.llatte_workspace_bytes(ctypes.byref(good))
 
 
 def test_forward_and_status_reject_null_handle(lib):
