@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace llatte {
 
@@ -322,14 +323,48 @@ cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int 
 }
 
 // ---------------------------------------------------------------- summaries
-// Sequence summaries (LLaTTE notes, appendix A.2 item 4), the step after the
+// Sequence summaries (LLaTTE notes, appendix A.2 item 4), the steps after the
 // bottleneck GEMM, which has left S partial sums per (user, bottleneck unit).
-// A block takes SUM_UB users and one summary k: h = SiLU(sum of the partials,
-// in slice order, so the result does not depend on timing), then
-// out[b, k, i] = sum_t W_up,k[i, t] h[b, t].  The output projection is stored
-// transposed ([t][i]): a warp reads 64 consecutive outputs' weights of one t
-// in one line, and every thread keeps SUM_UB x 2 accumulators.
+//   reduce  H[b, j] = SiLU(sum of the S partials of (b, j)), summed in slice
+//           order so that the result does not depend on timing; one thread
+//           per (b, j), eight partial loads in flight.  Written in fp32
+//           [B, N], or in bf16 as the A operand of the batched tensor-core
+//           output projection: [k][b_pad][rank]
+//   up      out[b, k, i] = sum_t W_up,k[i, t] H[b, k * R + t]; a block takes
+//           SUM_UB users, one summary and 256 outputs, with H of its users in
+//           shared memory and the output projection stored transposed
+//           ([t][i]: a warp reads 64 consecutive outputs' weights of one t in
+//           one line); the weights of the next eight t are loaded while the
+//           current eight are used
 constexpr int SUM_UB = 8;
+
+__global__ void __launch_bounds__(256) summary_reduce_kernel(SummaryArgs a) {
+  // launched as a dependent of the bottleneck GEMM: the next kernel may start
+  // its set-up at once; the partials are read only after the GEMM is complete
+  tc::pdl_trigger();
+  tc::pdl_wait();
+  const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (i >= (int64_t)a.B * a.N) return;
+  const float* p = a.P + i;
+  float v = 0.f;
+  int s = 0;
+  for (; s + 8 <= a.S; s += 8) {
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = __ldcg(p + (int64_t)(s + q) * a.slice_stride);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v += x[q];
+  }
+  for (; s < a.S; ++s) v += __ldcg(p + (int64_t)s * a.slice_stride);
+  v = silu_f(v);
+  if (a.H) {
+    a.H[i] = v;
+  } else {
+    const int64_t b = i / a.N;
+    const int j = (int)(i - b * a.N), k = j / a.rank, t = j - k * a.rank;
+    a.H16[((int64_t)k * a.b_pad + b) * a.rank + t] = __float2bfloat16_rn(v);
+  }
+}
 
 __device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
 __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
@@ -337,77 +372,75 @@ __device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) summary_up_kernel(SummaryArgs a) {
-  extern __shared__ float4 sh4[];                  // [SUM_UB][r4] fp32, zero padded
+__global__ void __launch_bounds__(128) summary_up_kernel(SummaryArgs a) {
+  extern __shared__ float4 sh4[];                  // [SUM_UB][r8] fp32, zero padded
   float* sh = reinterpret_cast<float*>(sh4);
   const int b0 = blockIdx.x * SUM_UB, k = blockIdx.y;
-  const int r = a.rank, r4 = (r + 3) & ~3;
-  for (int idx = threadIdx.x; idx < SUM_UB * r4; idx += blockDim.x) {
-    const int u = idx / r4, t = idx - u * r4;
+  const int r = a.rank, r8 = (r + 7) & ~7;
+  for (int idx = threadIdx.x; idx < SUM_UB * r8; idx += blockDim.x) {
+    const int u = idx / r8, t = idx - u * r8;
     const int b = b0 + u;
-    float v = 0.f;
-    if (b < a.B && t < r) {
-      const float* p = a.P + (int64_t)b * a.N + (int64_t)k * r + t;
-      for (int s = 0; s < a.S; ++s) v += p[s * a.slice_stride];
-      v = silu_f(v);
-    }
-    sh[idx] = v;
+    sh[idx] = (b < a.B && t < r) ? a.H[(int64_t)b * a.N + (int64_t)k * r + t] : 0.f;
   }
   __syncthreads();
-  const int half_d = a.d_seq / 2;
-  const T* W = (const T*)a.Wt + (int64_t)k * r * a.d_seq;
-  const int rq = r & ~3;
-  for (int pi = blockIdx.z * blockDim.x + threadIdx.x; pi < half_d;
-       pi += gridDim.z * blockDim.x) {
-    float acc[SUM_UB][2];
+  const int pi = blockIdx.z * blockDim.x + threadIdx.x;      // output pair
+  if (pi >= a.d_seq / 2) return;
+  const T* w = (const T*)a.Wt + (int64_t)k * r * a.d_seq + 2 * pi;
+  float acc[SUM_UB][2];
 #pragma unroll
-    for (int u = 0; u < SUM_UB; ++u) acc[u][0] = acc[u][1] = 0.f;
-    const T* w = W + 2 * pi;
+  for (int u = 0; u < SUM_UB; ++u) acc[u][0] = acc[u][1] = 0.f;
+  // t in groups of eight; rows t >= r read as zero weights
+  auto fetch = [&](int t0, float2 (&wf)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      wf[i] = t0 + i < r ? load2(w + (int64_t)(t0 + i) * a.d_seq) : make_float2(0.f, 0.f);
+  };
+  float2 cur[8], nxt[8];
+  fetch(0, cur);
 #pragma unroll 1
-    for (int t = 0; t < rq; t += 4) {
-      float2 wf[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) wf[i] = load2(w + (int64_t)(t + i) * a.d_seq);
-#pragma unroll
-      for (int u = 0; u < SUM_UB; ++u) {
-        const float4 hv = sh4[(u * r4 + t) >> 2];
-        acc[u][0] = fmaf(wf[0].x, hv.x, acc[u][0]); acc[u][1] = fmaf(wf[0].y, hv.x, acc[u][1]);
-        acc[u][0] = fmaf(wf[1].x, hv.y, acc[u][0]); acc[u][1] = fmaf(wf[1].y, hv.y, acc[u][1]);
-        acc[u][0] = fmaf(wf[2].x, hv.z, acc[u][0]); acc[u][1] = fmaf(wf[2].y, hv.z, acc[u][1]);
-        acc[u][0] = fmaf(wf[3].x, hv.w, acc[u][0]); acc[u][1] = fmaf(wf[3].y, hv.w, acc[u][1]);
-      }
-    }
-    for (int t = rq; t < r; ++t) {
-      const float2 wf = load2(w + (int64_t)t * a.d_seq);
-#pragma unroll
-      for (int u = 0; u < SUM_UB; ++u) {
-        const float hv = sh[u * r4 + t];
-        acc[u][0] = fmaf(wf.x, hv, acc[u][0]);
-        acc[u][1] = fmaf(wf.y, hv, acc[u][1]);
-      }
-    }
+  for (int t = 0; t < r8; t += 8) {
+    if (t + 8 < r8) fetch(t + 8, nxt);
 #pragma unroll
     for (int u = 0; u < SUM_UB; ++u) {
-      const int b = b0 + u;
-      if (b < a.B)
-        *reinterpret_cast<float2*>(a.out + ((int64_t)b * a.n_sum + k) * a.d_seq + 2 * pi) =
-            make_float2(acc[u][0], acc[u][1]);
+      const float4 h0 = sh4[(u * r8 + t) >> 2];
+      const float4 h1 = sh4[((u * r8 + t) >> 2) + 1];
+      const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[u][0] = fmaf(cur[i].x, hv[i], acc[u][0]);
+        acc[u][1] = fmaf(cur[i].y, hv[i], acc[u][1]);
+      }
     }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+  }
+#pragma unroll
+  for (int u = 0; u < SUM_UB; ++u) {
+    const int b = b0 + u;
+    if (b < a.B)
+      *reinterpret_cast<float2*>(a.out + ((int64_t)b * a.n_sum + k) * a.d_seq + 2 * pi) =
+          make_float2(acc[u][0], acc[u][1]);
   }
 }
 
-cudaError_t launch_summary_up(int elem, const SummaryArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_summary_reduce(const SummaryArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
-  if (a.d_seq <= 0 || (a.d_seq & 1) || a.rank <= 0 || a.rank > 1024 || a.n_sum <= 0 || a.S < 1)
+  if (a.rank <= 0 || a.n_sum <= 0 || a.N != a.n_sum * a.rank || a.S < 1 ||
+      (!a.H && (!a.H16 || a.b_pad < a.B)))
     return cudaErrorInvalidValue;
-  const int bx = (a.B + SUM_UB - 1) / SUM_UB;
-  // split the outputs of a (user block, summary) over z until the grid fills the SMs
-  const int pairs_blocks = (a.d_seq / 2 + 255) / 256;
-  const int z = std::max(1, std::min(pairs_blocks, num_sms / std::max(1, bx * a.n_sum)));
-  const dim3 grid(bx, a.n_sum, z);
-  const size_t smem = sizeof(float) * SUM_UB * ((a.rank + 3) & ~3);
-  if (elem == 4) summary_up_kernel<float><<<grid, 256, smem, s>>>(a);
-  else summary_up_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a);
+  const int64_t vals = (int64_t)a.B * a.N;
+  return tc::launch_dependent(summary_reduce_kernel, dim3((unsigned)((vals + 255) / 256)),
+                              dim3(256), 0, s, 1, a);
+}
+
+cudaError_t launch_summary_up(int elem, const SummaryArgs& a, cudaStream_t s) {
+  if (a.B <= 0) return cudaSuccess;
+  if (a.d_seq <= 0 || (a.d_seq & 1) || a.rank <= 0 || a.rank > 1024 || a.n_sum <= 0 || !a.H)
+    return cudaErrorInvalidValue;
+  const dim3 grid((a.B + SUM_UB - 1) / SUM_UB, a.n_sum, (a.d_seq / 2 + 127) / 128);
+  const size_t smem = sizeof(float) * SUM_UB * ((a.rank + 7) & ~7);
+  if (elem == 4) summary_up_kernel<float><<<grid, 128, smem, s>>>(a);
+  else summary_up_kernel<__nv_bfloat16><<<grid, 128, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,9 @@ Sources (LLaTTE notes, huaxiaozhuan.com):
   * appendix A.3 first display (non-absorbed MLA):
     K, V = split(RMSNorm(X W_down^KV) W_up^KV),
     MLA(X) = softmax(Q K^T / sqrt(d_k)) V W_out;
-  * daiwk.github.io notes, "core formula": q_t = W_Q [x_t ; c].
+  * daiwk.github.io notes, "core formula": q_t = W_Q [x_t ; c];
+  * appendix A.3 first display, low-rank query (q_rank > 0):
+    Q = RMSNorm([x ; c] W_down^Q) W_up^Q.
 
 Every row of the fused sequence is computed (also the rows the slice then
 drops), with an explicit boolean mask over (row, key): a history row at fused
@@ -54,7 +56,10 @@ def layer_brute(Xf: np.ndarray, T: int, c: np.ndarray, w: dict, dims):
     K = C @ f("W_uk").T                                             # [T, h*dh]
     V = C @ f("W_uv").T
     Xc = np.concatenate([Xf, np.tile(c, (N, 1))], axis=1)
-    Q = Xc @ f("W_q").T                                             # [N, h*dh]
+    if getattr(dims, "q_rank", 0):
+        Q = _rms(Xc @ f("W_dq").T, f("g_q"), eps) @ f("W_uq").T        # [N, h*dh]
+    else:
+        Q = Xc @ f("W_q").T                                         # [N, h*dh]
 
     mask = np.zeros((N, T), dtype=bool)
     for i in range(N):

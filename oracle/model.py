@@ -9,6 +9,8 @@ Sources:
     and the pyramid slice of the last T_{l+1} rows.
   * daiwk.github.io notes, "core formula": target-aware query
     q_t = W_Q [x_t ; c], h_t = sum_i softmax_i(q_t.k_i / sqrt(d)) W_V x_i.
+  * appendix A.3 first display, the low-rank query of the MLA
+    parameterisation: Q = RMSNorm(X W_down^Q) W_up^Q (when q_rank > 0).
 
 Readings: the softmax scale is 1/sqrt(d_h) in both forms (the absorbed
 display's sqrt(d_c) is read as garbled: only the same scale keeps the two forms
@@ -18,8 +20,13 @@ attention output is zero; RMSNorm(v) = v / sqrt(mean(v^2) + eps) * g;
 FFN(z) = W2 SiLU(W1 z), SiLU(x) = x / (1 + exp(-x)), no biases; a sequence
 summary is W_up SiLU(W_down Flatten(Z_raw)) (see `summaries`).
 
+Low-rank query reading: the down-projection acts on the target-aware input
+[x ; c] (so the query stays target-aware), with its own RMSNorm gain g_q;
+W_up^Q then absorbs into the key up-projection like W_Q does.
+
 Absorbed matrices per head j (rows j*d_h:(j+1)*d_h of the per-head blocks):
   W_QK_j = W_uk_j^T W_q_j / sqrt(d_h)      (r x (d + d_ctx))
+  W_QK_j = W_uk_j^T W_uq_j / sqrt(d_h)     (r x q_rank, low-rank query)
   W_OV_j = W_o[:, j-block] W_uv_j          (d x r)
 """
 from __future__ import annotations
@@ -47,7 +54,8 @@ def _f64(a):
 def absorb(w: dict, dims) -> dict:
     """Per-head absorbed matrices in fp64 from the non-absorbed weights."""
     h, dh = dims.heads, dims.d_head
-    W_q, W_uk, W_uv, W_o = _f64(w["W_q"]), _f64(w["W_uk"]), _f64(w["W_uv"]), _f64(w["W_o"])
+    W_q = _f64(w["W_uq"] if getattr(dims, "q_rank", 0) else w["W_q"])
+    W_uk, W_uv, W_o = _f64(w["W_uk"]), _f64(w["W_uv"]), _f64(w["W_o"])
     scale = 1.0 / np.sqrt(dh)
     W_QK, W_OV = [], []
     for j in range(h):
@@ -79,9 +87,13 @@ def layer_forward(H: np.ndarray, Y: np.ndarray, c: np.ndarray, w: dict, ab: dict
         else:
             visible[i, :] = True                                 # candidate: all history keys
 
+    if getattr(dims, "q_rank", 0):
+        Qin = rmsnorm(RC @ _f64(w["W_dq"]).T, _f64(w["g_q"]), eps)   # [q, q_rank]
+    else:
+        Qin = RC
     A = np.zeros((q, dims.d))
     for j in range(dims.heads):
-        Qt = RC @ ab["W_QK"][j].T                                # [q, r] latent queries
+        Qt = Qin @ ab["W_QK"][j].T                               # [q, r] latent queries
         S = Qt @ C.T                                             # [q, T]
         S = np.where(visible, S, -np.inf)
         P = np.zeros_like(S)

@@ -54,6 +54,8 @@ def small_dims(**kw):
     dict(kv_norm=0),
     dict(d_out=7, keep=(10, 3)),
     dict(heads=3, d_head=4, rank=20),     # r > h*d_h
+    dict(q_rank=5),                       # low-rank RMSNorm'd query
+    dict(q_rank=21, d_ctx=0, keep=(6, 0)),
 ])
 def test_absorbed_equals_non_absorbed(lengths, dkw):
     dims = small_dims(**dkw)
@@ -66,8 +68,9 @@ def test_absorbed_equals_non_absorbed(lengths, dkw):
         assert np.abs(a - b).max() <= 1e-11 * scale
 
 
-def test_absorbed_equals_non_absorbed_tiny_workload():
-    inp = make_inputs(workload("tiny"))
+@pytest.mark.parametrize("name", ["tiny", "tiny_lq"])
+def test_absorbed_equals_non_absorbed_tiny_workload(name):
+    inp = make_inputs(workload(name))
     a = oracle.forward(inp)
     b = oracle.forward_brute(inp)
     assert np.abs(a - b).max() < 1e-12
@@ -84,7 +87,12 @@ def _textbook_layer(x, c, w, dims, causal_rows, cand):
     cc = t(c)
 
     def q_of(rows):
-        return F.linear(torch.cat([rows, cc.expand(rows.shape[0], -1)], 1), t(w["W_q"]))
+        xc = torch.cat([rows, cc.expand(rows.shape[0], -1)], 1)
+        if dims.q_rank:                           # Q = RMSNorm([x; c] W_down^Q) W_up^Q
+            lat = F.rms_norm(F.linear(xc, t(w["W_dq"])), (dims.q_rank,), weight=t(w["g_q"]),
+                             eps=dims.eps)
+            return F.linear(lat, t(w["W_uq"]))
+        return F.linear(xc, t(w["W_q"]))
 
     k = F.linear(X, t(w["W_uk"]))                 # C = X because W_dkv = I, no norm
     v = F.linear(X, t(w["W_uv"]))
@@ -111,12 +119,13 @@ def _textbook_layer(x, c, w, dims, causal_rows, cand):
     return hist, cnd
 
 
-@pytest.mark.parametrize("n_q,d_ctx,keep", [(0, 0, (11, 6)), (3, 4, (11, 6)), (2, 0, (5, 0)),
-                                             (4, 3, (0,))])
-def test_textbook_reduction(n_q, d_ctx, keep):
+@pytest.mark.parametrize("n_q,d_ctx,keep,q_rank", [
+    (0, 0, (11, 6), 0), (3, 4, (11, 6), 0), (2, 0, (5, 0), 0), (4, 3, (0,), 0),
+    (3, 4, (11, 6), 5), (2, 0, (7, 0), 9)])
+def test_textbook_reduction(n_q, d_ctx, keep, q_rank):
     d = 12
     dims = Dims(d=d, heads=3, d_head=4, rank=d, d_ctx=d_ctx, n_q=n_q, keep=keep,
-                kv_norm=0, dtype="fp32")
+                kv_norm=0, dtype="fp32", q_rank=q_rank)
     inp = make_inputs(_wl(dims, batch=2), lengths=[11, 7], random_gains=True)
     for w in inp.layers:
         w["W_dkv"] = np.eye(d, dtype=np.float32)
@@ -132,6 +141,23 @@ def test_textbook_reduction(n_q, d_ctx, keep):
             Ho, Yo = layers[u][l]
             np.testing.assert_allclose(Ho, H, rtol=0, atol=1e-12)
             np.testing.assert_allclose(Yo, Y, rtol=0, atol=1e-12)
+
+
+def test_low_rank_query_is_scale_invariant_in_its_down_projection():
+    """RMSNorm on the query latent: scaling W_down^Q by any positive factor
+    leaves the layer unchanged (with eps -> 0); a full-rank or un-normed query
+    would change."""
+    dims = small_dims(q_rank=6, eps=1e-30)
+    inp = make_inputs(_wl(dims), lengths=[9, 4, 1], random_gains=True)
+    a = oracle.forward(inp)
+    for w in inp.layers:
+        w["W_dq"] = w["W_dq"] * np.float32(8.0)
+    b = oracle.forward(inp)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    for w in inp.layers:
+        w["W_uq"] = w["W_uq"] * np.float32(2.0)        # the up-projection is not normed
+    c = oracle.forward(inp)
+    assert np.abs(c - a).max() > 1e-3
 
 
 # ---------------------------------------------------------------- special cases

@@ -35,6 +35,8 @@ class Dims:
     n_sum    sequence summaries read out of the final query tokens (0 = none)
     sum_rank hidden (low-rank) width of each summary MLP
     d_seq    width of each summary
+    q_rank   rank of the low-rank query: Q = RMSNorm([x; c] W_down^Q) W_up^Q
+             (0 = the full-rank query W_Q [x; c])
     """
 
     d: int
@@ -52,6 +54,7 @@ class Dims:
     n_sum: int = 0
     sum_rank: int = 0
     d_seq: int = 0
+    q_rank: int = 0
 
     @property
     def n_layers(self) -> int:
@@ -135,6 +138,21 @@ WORKLOADS["tiny_sum"] = Workload(
     name="tiny_sum", dims=replace(WORKLOADS["tiny"].dims, n_sum=3, sum_rank=8, d_seq=12),
     batch=4, lengths=("uniform", 16, 64), seed=0,
     description="tiny fp32 case with 3 summaries (rank 8, width 12)")
+# The low-rank RMSNorm'd query of the MLA parameterisation (appendix A.3,
+# first display) in place of the full-rank target-aware query; the pages give
+# no query rank: half the token width is taken.
+WORKLOADS["tiny_lq"] = Workload(
+    name="tiny_lq", dims=replace(WORKLOADS["tiny"].dims, q_rank=24),
+    batch=4, lengths=("uniform", 16, 64), seed=0,
+    description="tiny fp32 case with a rank-24 RMSNorm'd query")
+WORKLOADS["online_lq"] = Workload(
+    name="online_lq", dims=replace(WORKLOADS["online"].dims, q_rank=128),
+    batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
+    description="online ranker with a rank-128 RMSNorm'd query")
+WORKLOADS["upstream_lq"] = Workload(
+    name="upstream_lq", dims=replace(WORKLOADS["upstream"].dims, q_rank=256),
+    batch=64, lengths=("fixed", 1600), seed=2,
+    description="upstream user model with a rank-256 RMSNorm'd query")
 WORKLOADS["online_sum"] = Workload(
     name="online_sum", dims=replace(WORKLOADS["online"].dims, n_sum=2, sum_rank=128, d_seq=1024),
     batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,

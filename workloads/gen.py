@@ -9,7 +9,9 @@ Draw order, fixed so that every consumer sees the same numbers for a seed:
   6. weights, layer by layer, in the order
      W_dkv, g_kv, W_q, W_uk, W_uv, W_o, g1, W1, W2, g2
      (matrices N(0, 1/fan_in); gains are 1 unless random gains are asked for,
-     then N(1, 0.1^2))
+     then N(1, 0.1^2)); with a low-rank query, W_q is replaced by
+     W_dq [q_rank, d + d_ctx], g_q [q_rank], W_uq [h*d_h, q_rank] drawn in
+     that order at its place
   7. W_e (readout) when d_out > 0.
   8. sequence-summary weights when n_sum > 0, summary by summary:
      W_down [sum_rank, n_q*d] N(0, 1/(n_q*d)), then W_up [d_seq, sum_rank]
@@ -91,7 +93,13 @@ def draw_weights(dims: Dims, rng: np.random.Generator, random_gains: bool = Fals
         w = {}
         w["W_dkv"] = _normal(rng, (r, d), 1.0 / np.sqrt(d))
         w["g_kv"] = gain(r)
-        w["W_q"] = _normal(rng, (hd, d + dc), 1.0 / np.sqrt(d + dc))
+        if dims.q_rank > 0:
+            rq = dims.q_rank
+            w["W_dq"] = _normal(rng, (rq, d + dc), 1.0 / np.sqrt(d + dc))
+            w["g_q"] = gain(rq)
+            w["W_uq"] = _normal(rng, (hd, rq), 1.0 / np.sqrt(rq))
+        else:
+            w["W_q"] = _normal(rng, (hd, d + dc), 1.0 / np.sqrt(d + dc))
         w["W_uk"] = _normal(rng, (hd, r), 1.0 / np.sqrt(r))
         w["W_uv"] = _normal(rng, (hd, r), 1.0 / np.sqrt(r))
         w["W_o"] = _normal(rng, (d, hd), 1.0 / np.sqrt(hd))
