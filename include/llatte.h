@@ -18,6 +18,9 @@
  *     Z      = RMSNorm_{g1}(R + A)
  *     X      = RMSNorm_{g2}(Z + W2 SiLU(W1 Z))
  *     history <- X[:n], query tokens <- X[n:], T <- n
+ *   With q_rank > 0 the query is low-rank and normalised (appendix A.3, first
+ *   display): q~ = (W_uk,j^T W_up,j^Q) RMSNorm_{g_q}(W_down^Q [R_i ; c]) / sqrt(d_h),
+ *   the down-projection taking the target-aware input [x ; c].
  *   Visibility: a history query at position p sees keys t <= p; a query token
  *   sees every current history key and no query token; no key -> zero output.
  *   Output: the final query-token rows; or, with d_out > 0, W_e times the mean
@@ -91,6 +94,8 @@ enum {
  *   n_sum                 sequence summaries (0 = none; needs n_q > 0 and d_out == 0;
  *                         at most LLATTE_MAX_SUMMARIES)
  *   sum_rank, d_seq       bottleneck width (1 .. 1024) and width (even) of each summary
+ *   q_rank                rank of the low-rank RMSNorm'd query (0 = full-rank W_q;
+ *                         at most 1024)
  */
 typedef struct {
   int32_t d, heads, d_head, rank, d_ctx, n_q, n_layers;
@@ -101,6 +106,7 @@ typedef struct {
   int64_t max_len;
   int64_t max_total;
   int32_t n_sum, sum_rank, d_seq;
+  int32_t q_rank;
 } llatte_dims;
 
 #define LLATTE_MAX_SUMMARIES 16
@@ -112,9 +118,14 @@ typedef struct {
  *   W_uk  [h*d_h, r]    K up-projection            W_uv [h*d_h, r] V up-projection
  *   W_o   [d, h*d_h]    output projection          g1 [d]     post-attention gain
  *   W1    [ffn_mult*d, d]   W2 [d, ffn_mult*d]     g2 [d]     post-FFN gain
+ * With q_rank > 0, W_q is not read (may be NULL) and the query comes from
+ *   W_dq  [q_rank, d+d_ctx] query down-projection  g_q [q_rank] its RMSNorm gain
+ *   W_uq  [h*d_h, q_rank]   query up-projection
+ * (all three ignored, and may be NULL, when q_rank == 0).
  */
 typedef struct {
   const void *W_dkv, *g_kv, *W_q, *W_uk, *W_uv, *W_o, *g1, *W1, *W2, *g2;
+  const void *W_dq, *g_q, *W_uq;
 } llatte_layer_w;
 
 /*
@@ -154,7 +165,7 @@ int llatte_create(llatte_handle** handle, const llatte_dims* dims,
  *   context device [B, d_ctx] in dtype (may be NULL when d_ctx == 0)
  *   cand    device [B, n_q, d] in dtype (may be NULL when n_q == 0)
  *   out     device fp32 [B, n_q, d] (d_out == 0, n_sum == 0), [B, d_out]
- *           (d_out > 0) or [B, n_sum, d_seq] (n_sum > 0)
+ *           (d_out > 0) or [B, n_sum, d_seq] (n_sum > 0, 16-byte aligned)
  * Inputs are only read; `out` is the only caller memory written.  Calls on
  * one handle must not overlap in time (they share its workspace).
  */

@@ -37,10 +37,12 @@ class llatte_dims(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("kv_norm", ctypes.c_int32), ("eps", ctypes.c_float),
                 ("max_batch", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("max_total", ctypes.c_int64), ("n_sum", ctypes.c_int32),
-                ("sum_rank", ctypes.c_int32), ("d_seq", ctypes.c_int32)]
+                ("sum_rank", ctypes.c_int32), ("d_seq", ctypes.c_int32),
+                ("q_rank", ctypes.c_int32)]
 
 
-LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2")
+LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2",
+              "W_dq", "g_q", "W_uq")
 
 
 class llatte_layer_w(ctypes.Structure):
@@ -128,6 +130,7 @@ def make_dims(dims, max_batch: int, max_len: int, max_total: int = 0) -> llatte_
     c.n_sum = int(getattr(dims, "n_sum", 0))
     c.sum_rank = int(getattr(dims, "sum_rank", 0))
     c.d_seq = int(getattr(dims, "d_seq", 0))
+    c.q_rank = int(getattr(dims, "q_rank", 0))
     return c
 
 
@@ -167,6 +170,8 @@ class Llatte:
         arr = (llatte_layer_w * len(layers))()
         for i, w in enumerate(layers):
             for k in LAYER_KEYS:
+                if w.get(k) is None:         # W_q or the low-rank query's matrices
+                    continue
                 t = _host(w[k], self.dt)
                 keep_alive.append(t)
                 setattr(arr[i], k, t.data_ptr())

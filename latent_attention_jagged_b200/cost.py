@@ -9,6 +9,7 @@ visible (query, key) pairs only) with the constants of the absorbed MLA form
 Per user and layer, with T history rows in, n = min(T, keep) kept, q = n + n_q:
   kv      2 T d r
   q       2 q d h r + 2 d_ctx h r          (context term once per user)
+          low-rank query (rank R_q): 2 q d R_q + 2 d_ctx R_q + 2 q R_q h r
   attn    4 h r P,  P = n_q T + n T - n (n - 1) / 2  visible pairs
   o       2 q h r d
   ffn1    2 q d (m d)      ffn2  2 q (m d) d        (m = FFN multiplier)
@@ -44,6 +45,7 @@ def visible_pairs(T: np.ndarray, n: np.ndarray, n_q: int) -> np.ndarray:
 def layer_work(lengths: Sequence[int], dims) -> List[LayerWork]:
     T = np.asarray(lengths, dtype=np.int64)
     d, h, r, dc, m = dims.d, dims.heads, dims.rank, dims.d_ctx, dims.ffn_mult
+    rq = getattr(dims, "q_rank", 0)
     out = []
     for k in dims.keep:
         n = np.minimum(T, k)
@@ -52,7 +54,8 @@ def layer_work(lengths: Sequence[int], dims) -> List[LayerWork]:
         B = T.shape[0]
         f = {
             "kv": 2.0 * T.sum() * d * r,
-            "q": 2.0 * q.sum() * d * h * r + 2.0 * B * dc * h * r,
+            "q": (2.0 * q.sum() * d * h * r + 2.0 * B * dc * h * r) if not rq else
+                 (2.0 * q.sum() * d * rq + 2.0 * B * dc * rq + 2.0 * q.sum() * rq * h * r),
             "attn": 4.0 * h * r * P.sum(),
             "o": 2.0 * q.sum() * h * r * d,
             "ffn1": 2.0 * q.sum() * d * m * d,
@@ -110,7 +113,9 @@ def io_bytes(lengths: Sequence[int], dims, elem: int = 2) -> float:
     B = lengths.shape[0]
     d, hd, r, dc, f = dims.d, dims.heads * dims.d_head, dims.rank, dims.d_ctx, dims.d_ffn
     inp = (lengths.sum() + B * dims.n_q) * d * elem + B * dc * elem + (B + 1) * 8
-    per_layer_w = (r * d + r + hd * (d + dc) + 2 * hd * r + d * hd + 2 * d + 2 * f * d) * elem
+    rq = getattr(dims, "q_rank", 0)
+    qw = rq * (d + dc) + rq + hd * rq if rq else hd * (d + dc)
+    per_layer_w = (r * d + r + qw + 2 * hd * r + d * hd + 2 * d + 2 * f * d) * elem
     w = dims.n_layers * per_layer_w + dims.d_out * d * elem
     k = getattr(dims, "n_sum", 0)
     if k:

@@ -11,22 +11,24 @@
 //               STORE     bf16 store
 //               USERBIAS  + per-user context term (absorbed query projection)
 //               SILU      SiLU (FFN up-projection)
-//               PARTIAL   fp32 partial sums of one k-slice (split-K)
+//               F32       fp32 store (a split-K slice's partial sums, or one
+//                         member of a batch of products)
 //               NORM      + residual (read once: the sum is staged back in
 //                         TMEM), RMSNorm over the full row (BN == N; the two
 //                         halves' sums of squares meet in shared memory),
 //                         store bf16 (+ fp16 residual copy) or scatter into the
 //                         next layer's history / query rows (pyramid trimming)
 // The accumulator is double-buffered in TMEM when 2 * BN <= 512 columns, so
-// the epilogue of tile i overlaps the MMAs of tile i + 1.  With split-K a tile
-// is (row block, column block, k-slice); the slices of one output tile are
-// consecutive tile indices.
+// the epilogue of tile i overlaps the MMAs of tile i + 1.  With F32 a tile is
+// (group, row block, column block, k-slice); the slices of one output tile
+// are consecutive tile indices.
 //
 // Equations (LLaTTE notes, huaxiaozhuan.com, appendix A.2 display and A.3):
 // KV latent RMSNorm(X W_down^KV); absorbed query X (W_uk^T W_q)^T + context
 // term; Z = RMSNorm(R + o~ (W_o W_uv)^T); FFN W2 SiLU(W1 Z) + Z, RMSNorm.
-// Split-K: the bottleneck projection of the sequence summaries (appendix A.2
-// item 4), whose K = n_q * d is long and whose output is small.
+// F32: the sequence summaries (appendix A.2 item 4): the bottleneck
+// projection, whose K = n_q * d is long and whose output is small (split-K),
+// and the per-summary output projections (a batch of products).
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -71,7 +73,7 @@ struct GemmCfg {
 // through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
 __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0, int ks, int half, float* red,
+                                         bool valid, int n0, int ks, int g, int half, float* red,
                                          int rrow, uint64_t* xbar, uint32_t& xphase,
                                          volatile int* abort_flag, uint32_t stg,
                                          NormPre<BN, 4>& pre, const __nv_bfloat16* sg) {
@@ -80,8 +82,9 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
                              abort_flag, p.status, stg, pre, sg);
-  } else if constexpr (EPI == TC_PARTIAL) {
-    float* prow = valid ? p.Dp + ks * p.slice_stride + row * p.N + n0 : nullptr;
+  } else if constexpr (EPI == TC_F32) {
+    float* prow =
+        valid ? p.Dp + ks * p.slice_stride + g * p.d_group_off + row * p.ldp + n0 : nullptr;
 #pragma unroll 1
     for (int c = c0; c < c0 + HB; c += 32) {
       float v[32];
@@ -165,7 +168,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n_tiles = p.N / BN;
   const int KB = p.K / BK;
   const int kb0 = blockIdx.x % KB;
-  const int S = (EPI == TC_PARTIAL && p.k_split > 1) ? p.k_split : 1;   // k-slices (<= KB)
+  const int S = (EPI == TC_F32 && p.k_split > 1) ? p.k_split : 1;   // k-slices (<= KB)
+  const int G = (EPI == TC_F32 && p.groups > 1) ? p.groups : 1;      // batch members
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -189,7 +193,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   // everything below reads what earlier kernels wrote
   pdl_wait();
   const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
-  const int64_t num_tiles = ((M + BM - 1) / BM) * n_tiles * S;
+  const int64_t mn_tiles = ((M + BM - 1) / BM) * n_tiles;
+  const int64_t num_tiles = mn_tiles * G * S;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -199,7 +204,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int64_t tt = t / S;
         const int ks = (int)(t % S);
-        const int mt = (int)(tt / n_tiles), nt = (int)(tt % n_tiles);
+        const int g = (int)(tt / mn_tiles);
+        const int64_t rem = tt % mn_tiles;
+        const int mt = (int)(rem / n_tiles), nt = (int)(rem % n_tiles);
+        const int a_row = (int)(g * p.a_group_rows) + mt * BM;
+        const int w_row = g * p.w_group_rows + nt * BN;
         const int kb_lo = (int)((int64_t)ks * KB / S);
         const int nkb = (int)((int64_t)(ks + 1) * KB / S) - kb_lo;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -208,11 +217,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // k-blocks in a per-CTA rotated order: the SMs do not all read the
           // same weight lines from L2 at the same moment
           const int kx = (kb_lo + (kb + kb0) % nkb) * BK;
-          tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kx, mt * BM);
+          tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kx, a_row);
 #pragma unroll
           for (int s2 = 0; s2 < NSUB; ++s2)
             tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * NI * 128, kx,
-                        nt * BN + s2 * NI);
+                        w_row + s2 * NI);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -266,7 +275,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int64_t tt = t / S;
       const int ks = (int)(t % S);
-      const int mt = (int)(tt / n_tiles), nt = (int)(tt % n_tiles);
+      const int g = (int)(tt / mn_tiles);
+      const int64_t rem = tt % mn_tiles;
+      const int mt = (int)(rem / n_tiles), nt = (int)(rem % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
       NormPre<BN, 4> pre;
@@ -274,7 +285,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, half,
+      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, g, half,
                              red + (it & 1) * 256, rr, xbar, xphase, abort_flag,
                              smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
         break;
@@ -330,27 +341,32 @@ bool tc_gemm_supported(int BN, int epi, int N, int K) {
   if (BN != 64 && BN != 128 && BN != 256 && BN != 512) return false;
   if (BN == 512 && epi != TC_NORM) return false;
   if (epi == TC_NORM && N != BN) return false;
-  if (epi == TC_PARTIAL && BN > 128) return false;
+  if (epi == TC_F32 && BN > 128) return false;
   return N % BN == 0;
 }
 
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
                            const TcGemmParams& p, int num_sms, cudaStream_t s) {
   if (!tc_gemm_supported(BN, epi, p.N, p.K)) return cudaErrorInvalidValue;
-  if (epi == TC_PARTIAL && (p.k_split < 1 || p.k_split > p.K / BK || !p.Dp))
+  if (epi == TC_F32 &&
+      (p.k_split < 1 || p.k_split > p.K / BK || p.groups < 1 || !p.Dp || p.ldp % 4 != 0 ||
+       p.d_group_off % 4 != 0 || p.slice_stride % 4 != 0 ||
+       (p.groups > 1 && ((p.M_cap > p.a_group_rows) ||
+                         (int64_t)p.groups * p.a_group_rows > INT32_MAX ||
+                         (int64_t)p.groups * p.w_group_rows > INT32_MAX))))
     return cudaErrorInvalidValue;
   // grid: one CTA per SM, never more CTAs than the largest possible tile count
-  const int64_t max_tiles =
-      ((p.M_cap + BM - 1) / BM) * (p.N / BN) * (epi == TC_PARTIAL ? p.k_split : 1);
+  const int64_t max_tiles = ((p.M_cap + BM - 1) / BM) * (p.N / BN) *
+                            (epi == TC_F32 ? (int64_t)p.k_split * p.groups : 1);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, max_tiles));
   switch (epi) {
     case TC_STORE: return launch_epi<TC_STORE>(BN, a, b, p, grid, s);
     case TC_USERBIAS: return launch_epi<TC_USERBIAS>(BN, a, b, p, grid, s);
     case TC_SILU: return launch_epi<TC_SILU>(BN, a, b, p, grid, s);
     case TC_NORM: return launch_epi<TC_NORM>(BN, a, b, p, grid, s);
-    case TC_PARTIAL:
-      if (BN == 64) return launch_cfg<64, TC_PARTIAL>(a, b, p, grid, s);
-      if (BN == 128) return launch_cfg<128, TC_PARTIAL>(a, b, p, grid, s);
+    case TC_F32:
+      if (BN == 64) return launch_cfg<64, TC_F32>(a, b, p, grid, s);
+      if (BN == 128) return launch_cfg<128, TC_F32>(a, b, p, grid, s);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,7 +49,12 @@ struct LayerDev {
   void* W_dkv;     // [r, d]
   void* g_kv;      // [r]
   void* W_qk;      // [h*r, d]   absorbed W_uk^T W_q (x columns), scaled 1/sqrt(d_h)
-  float* W_qkc;    // [d_ctx, h*r] fp32 absorbed context columns, transposed (NULL if d_ctx == 0)
+                   //   low-rank query: [h*r, q_rank] absorbed W_uk^T W_uq
+  float* W_qkc;    // [d_ctx, h*r] fp32 absorbed context columns, transposed (NULL if d_ctx == 0
+                   //   or low-rank query)
+  void* W_dqx;     // [q_rank, d] query down-projection, x columns (low-rank query)
+  float* W_dqc;    // [d_ctx, q_rank] fp32 its context columns, transposed (NULL if d_ctx == 0)
+  void* g_q;       // [q_rank] query-latent RMSNorm gain
   void* W_ov;      // [d, h*r]   absorbed W_o W_uv
   void* g1;        // [d]
   void* W1;        // [f, d]
@@ -58,7 +65,7 @@ struct LayerDev {
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
-struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair; };
+struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq; };
 
 }  // namespace llatte
 
@@ -73,11 +80,16 @@ struct llatte_handle {
   // sequence summaries: the stacked bottleneck projections, the output
   // projections transposed, the final query-token rows and the split-K partials
   void* W_sdown;                  // [n_sum * sum_rank, n_q * d]
-  void* W_supT;                   // [n_sum][sum_rank][d_seq]
+  void* W_sup;                    // [n_sum * d_seq, sum_rank] (sum_up_tc), else
+                                  // transposed: [n_sum][sum_rank][d_seq]
   void* zraw;                     // [max_batch, n_q * d] storage type
   float* sum_part;                // [k slices][rows][n_sum * sum_rank] fp32
+  float* sum_h;                   // [max_batch, n_sum * sum_rank] fp32
+  void* sum_h16;                  // [n_sum][sum_bpad][sum_rank] bf16 (sum_up_tc)
+  int64_t sum_bpad;               // max_batch rounded up to 128
   int sum_tc;                     // bottleneck GEMM on the tensor cores
   int sum_bn;                     // its tile width
+  int sum_up_tc;                  // output projections as one batched tensor-core GEMM
   std::vector<void*> allocs;
 
   // workspace
@@ -90,6 +102,7 @@ struct llatte_handle {
   void* Ot;
   void* Z;
   void* Hd;
+  void* Cq;            // [max_rows_q, q_rank] normalised query latent (low-rank query)
   void* Zres;          // fp16 residual copy of Z (bf16 storage only; NULL for fp32)
   void* Xqres[2];      // fp16 residual copy of the query rows (bf16 storage only)
   float* acc32;        // fp32 pre-norm rows (CUDA-core path)
@@ -101,14 +114,15 @@ struct llatte_handle {
 
   // tensor-core path: TMA descriptors of the A operands and the weights,
   // and the tile width (BN) of each GEMM
-  CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd;
+  CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd, tm_Cq;
   llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
-  int bn_kv, bn_q, bn_o, bn_f1, bn_f2;
+  int bn_kv, bn_q, bn_o, bn_f1, bn_f2, bn_dq;
   int attn_keys;                  // keys per attention tile (tensor-core path)
   int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
   int pair_norm;                  // output / FFN-down projections on SM pairs (d = 512)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
   CUtensorMap tm_zraw, tm_sdown;  // summary bottleneck GEMM operands
+  CUtensorMap tm_sh16, tm_sup;    // summary output-projection GEMM operands
 
   // the per-user context term runs on a side stream, beside the plan and
   // the gather (forked from and joined back into the caller's stream)
@@ -145,7 +159,7 @@ struct GemmArgs {
   int epi;                           // EPI_*
   const float* bias; const int64_t* seg_off; int B;  // EPI_USERBIAS
 };
-enum { EPI_STORE = 0, EPI_USERBIAS, EPI_SILU, EPI_F32 };
+enum { EPI_STORE = 0, EPI_USERBIAS, EPI_SILU, EPI_F32, EPI_USERBIAS_F32 };
 cudaError_t launch_gemm_simt(int elem_a, int elem_w, int elem_d, const GemmArgs& g, cudaStream_t s);
 
 // Element type of a residual-stream buffer.
@@ -155,6 +169,8 @@ struct NormArgs {
   const float* acc; int N;           // [M, N] fp32 rows
   const void* resid;                 // [M, N] residual or NULL
   int resid_kind;                    // RES_STORAGE / RES_F32 / RES_F16
+  const int32_t* resid_user;         // non-NULL: the residual is per user, [B, N], row
+                                     //   resid_user[m] for row m (RES_F16 only)
   const void* g; float eps;
   const int64_t* M_dev; int64_t M_max;
   int mode;                          // NORM_PLAIN / NORM_SCATTER
@@ -183,26 +199,36 @@ cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
 
 // Per-user context term of every layer's absorbed query projection.
 struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [d_ctx, h*r] per layer
-cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
-                            int dc, float* out, cudaStream_t s);
+// out[l][b][n] (fp32), or out16 (fp16) when out16 != NULL; N columns.
+cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int N,
+                            int dc, float* out, __half* out16, cudaStream_t s);
+// Split a [rows, d + dc] matrix into its first d columns (storage type, [rows, d])
+// and its last dc columns (fp32, transposed: [dc, rows]).
+cudaError_t launch_split_ctx_cols(int elem, const void* src, int rows, int d, int dc, void* dst_x,
+                                  float* dst_c, cudaStream_t s);
 
-// Sequence summaries after the bottleneck GEMM: h = SiLU(sum of the S split-K
-// partial rows), out[b, k, :] = h[b, k-block] W_up,k^T.
+// Sequence summaries after the bottleneck GEMM: H = SiLU(sum of the S split-K
+// partial rows) (reduce), then out[b, k, :] = H[b, k-block] W_up,k^T (up, on
+// CUDA cores; the tensor-core path runs it as a batched GEMM instead).
 struct SummaryArgs {
   const float* P; int S; int64_t slice_stride;   // P[s * slice_stride + b * N + j]
+  float* H;                                      // [B, N] fp32, or NULL and:
+  __nv_bfloat16* H16; int64_t b_pad;             // [n_sum][b_pad][rank] bf16
   int B, N, rank, d_seq, n_sum;                  // N = n_sum * rank
   const void* Wt;                                // [n_sum][rank][d_seq] storage type
   float* out;                                    // [B, n_sum, d_seq]
 };
-cudaError_t launch_summary_up(int elem, const SummaryArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_summary_reduce(const SummaryArgs& a, cudaStream_t s);
+cudaError_t launch_summary_up(int elem, const SummaryArgs& a, cudaStream_t s);
 // dst[c, r] = src[r, c] for a [rows, cols] matrix of the storage type.
 cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
                              cudaStream_t s);
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
                              cudaStream_t s);
+// W_q has dq + d_ctx columns (dq = d, or q_rank for W_uq of a low-rank query).
 cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
-                          const void* W_o, int d, int d_ctx, int heads, int d_head, int r,
+                          const void* W_o, int d, int dq, int d_ctx, int heads, int d_head, int r,
                           float qscale, void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s);
 
 }  // namespace llatte

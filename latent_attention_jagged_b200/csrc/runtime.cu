@@ -38,8 +38,9 @@ struct Layout {
   int64_t rows_h, rows_q;
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
       off_work_count, off_work_next, off_item_off, off_row_user;
-  size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_acc32, off_ctxbias,
-      off_final, off_mean, off_Zres, off_Xqres[2], off_zraw, off_sum_part;
+  size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_Cq, off_acc32, off_ctxbias,
+      off_final, off_mean, off_Zres, off_Xqres[2], off_zraw, off_sum_part, off_sum_h,
+      off_sum_h16;
   size_t total;
   int32_t max_work;
 };
@@ -54,6 +55,8 @@ int check_dims(const llatte_dims* d) {
   if (d->max_batch <= 0 || d->max_len < 0 || d->max_total < 0) return LLATTE_ERR_ARG;
   if (d->kv_norm != 0 && d->kv_norm != 1) return LLATTE_ERR_ARG;
   if (d->n_sum < 0 || d->n_sum > LLATTE_MAX_SUMMARIES) return LLATTE_ERR_ARG;
+  if (d->q_rank < 0) return LLATTE_ERR_ARG;
+  if (d->q_rank > 1024) return LLATTE_ERR_UNSUPPORTED;
   if (d->n_sum > 0) {
     if (d->n_q <= 0 || d->d_out > 0 || d->sum_rank <= 0 || d->d_seq <= 0) return LLATTE_ERR_ARG;
     if (d->sum_rank > 1024 || d->d_seq % 2 != 0) return LLATTE_ERR_UNSUPPORTED;
@@ -99,14 +102,19 @@ Layout layout_of(const llatte_dims* d) {
   L.off_Ot = take((size_t)L.rows_q * hr * elem);
   L.off_Z = take((size_t)L.rows_q * d->d * elem);
   L.off_Hd = take((size_t)L.rows_q * f * elem);
+  L.off_Cq = take((size_t)L.rows_q * d->q_rank * elem);
   // fp16 copies of the residual stream (bf16 storage keeps bf16 GEMM operands
   // plus these; fp32 storage needs none)
   const size_t res16 = elem == 2 ? 2 * (size_t)L.rows_q * d->d : 0;
   L.off_Zres = take(res16);
   for (int i = 0; i < 2; ++i) L.off_Xqres[i] = take(res16);
-  L.off_acc32 = take(sizeof(float) * std::max<size_t>((size_t)L.rows_h * d->rank,
-                                                      (size_t)L.rows_q * d->d));
-  L.off_ctxbias = take(sizeof(float) * nl * B * hr);
+  L.off_acc32 = take(sizeof(float) * std::max<size_t>(
+                                         std::max<size_t>((size_t)L.rows_h * d->rank,
+                                                          (size_t)L.rows_q * d->d),
+                                         (size_t)L.rows_q * d->q_rank));
+  // per-user context term of every layer's query: h*r columns (full-rank
+  // query), or q_rank columns (low-rank query: it enters before the norm)
+  L.off_ctxbias = take(sizeof(float) * nl * B * std::max<int64_t>(hr, d->q_rank));
   L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
   L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
   // sequence summaries: the final query-token rows and the split-K partials
@@ -115,6 +123,8 @@ Layout layout_of(const llatte_dims* d) {
   L.off_zraw = take(d->n_sum ? (size_t)B * d->n_q * d->d * elem : 0);
   L.off_sum_part = take(d->n_sum ? sizeof(float) * std::max<int64_t>(
                                        (int64_t)kSplitCtas * 128 * kSumMaxBN, B * sN) : 0);
+  L.off_sum_h = take(d->n_sum ? sizeof(float) * B * sN : 0);
+  L.off_sum_h16 = take(d->n_sum ? 2 * (size_t)((B + 127) / 128 * 128) * sN : 0);
   L.total = o;
   return L;
 }
@@ -197,7 +207,10 @@ bool tc_dims_ok(const llatte_dims& D) {
   const int hr = D.heads * D.rank, f = D.ffn_mult * D.d;
   const bool d_ok = D.d == 64 || D.d == 128 || D.d == 256 || D.d == 512;
   const bool r_ok = attn_tc_supported(D.rank);
-  return d_ok && r_ok && hr % 64 == 0 && f % 64 == 0;
+  // low-rank query: its latent is normalised in one 128 x q_rank tile
+  const bool q_ok = D.q_rank == 0 || D.q_rank == 64 || D.q_rank == 128 || D.q_rank == 256 ||
+                    D.q_rank == 512;
+  return d_ok && r_ok && q_ok && hr % 64 == 0 && f % 64 == 0;
 }
 
 int pick_bn(int N) { return N % 256 == 0 ? 256 : N % 128 == 0 ? 128 : 64; }
@@ -210,6 +223,8 @@ bool build_tc_maps(llatte_handle* h) {
   h->bn_o = d;
   h->bn_f1 = pick_bn(f);
   h->bn_f2 = d;
+  h->bn_dq = D.q_rank;
+  const int kq = D.q_rank ? D.q_rank : d;     // input width of the absorbed query GEMM
   const uint64_t rh = std::max<int64_t>(h->max_rows_h, 1), rq = std::max<int64_t>(h->max_rows_q, 1);
   bool ok = true;
   for (int i = 0; i < 2; ++i) {
@@ -219,6 +234,7 @@ bool build_tc_maps(llatte_handle* h) {
   ok = ok && make_tmap_bf16(&h->tm_Ot, h->Ot, rq, hr, 128);
   ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
+  if (D.q_rank) ok = ok && make_tmap_bf16(&h->tm_Cq, h->Cq, rq, D.q_rank, 128);
   h->attn_keys = attn_tc_keys(r);
   h->ffn_fused = ffn_tc_supported(d, f) ? 1 : 0;
   h->pair_norm = tc_gemm_pair_supported(TC_NORM, d, hr) && tc_gemm_pair_supported(TC_NORM, d, f);
@@ -229,7 +245,8 @@ bool build_tc_maps(llatte_handle* h) {
     const LayerDev& W = h->layers[l];
     LayerMaps& M = h->lmaps[l];
     ok = ok && make_tmap_bf16(&M.dkv, W.W_dkv, r, d, box(h->bn_kv));
-    ok = ok && make_tmap_bf16(&M.qk, W.W_qk, hr, d, box(h->bn_q));
+    ok = ok && make_tmap_bf16(&M.qk, W.W_qk, hr, kq, box(h->bn_q));
+    if (D.q_rank) ok = ok && make_tmap_bf16(&M.dq, W.W_dqx, D.q_rank, d, box(h->bn_dq));
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
@@ -290,9 +307,9 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   const llatte_dims& D = *dims;
   for (int l = 0; l < D.n_layers; ++l) {
     const llatte_layer_w& w = layers[l];
-    if (!w.W_dkv || !w.g_kv || !w.W_q || !w.W_uk || !w.W_uv || !w.W_o || !w.g1 || !w.W1 ||
-        !w.W2 || !w.g2)
+    if (!w.W_dkv || !w.g_kv || !w.W_uk || !w.W_uv || !w.W_o || !w.g1 || !w.W1 || !w.W2 || !w.g2)
       return LLATTE_ERR_ARG;
+    if (D.q_rank ? (!w.W_dq || !w.g_q || !w.W_uq) : !w.W_q) return LLATTE_ERR_ARG;
   }
   if (D.d_out > 0 && !W_e) return LLATTE_ERR_ARG;
   if (D.n_sum > 0) {
@@ -320,7 +337,10 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
 
   const size_t e = h->elem;
   const int d = D.d, r = D.rank, hd = D.heads * D.d_head, hr = D.heads * D.rank,
-            f = D.ffn_mult * D.d, dc = D.d_ctx;
+            f = D.ffn_mult * D.d, dc = D.d_ctx, rq = D.q_rank;
+  // columns of the matrix absorbed into the query: W_q [hd, d + dc], or for a
+  // low-rank query W_uq [hd, rq] (the context then enters through W_dq)
+  const int kq = rq ? rq : d, kqc = rq ? 0 : dc;
   // The tensor-core attention takes its scores in log2 units (exp2 in the
   // softmax): fold log2(e) into the absorbed query projection for that path.
   const bool want_tc = h->elem == 2 && tc_dims_ok(D);
@@ -334,24 +354,42 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     L.W1 = upload(h, w.W1, e * (size_t)f * d, weights_on_device);
     L.W2 = upload(h, w.W2, e * (size_t)d * f, weights_on_device);
     L.g2 = upload(h, w.g2, e * d, weights_on_device);
-    L.W_qk = dev_alloc(h, e * (size_t)hr * d);
-    L.W_qkc = dc ? (float*)dev_alloc(h, sizeof(float) * (size_t)hr * dc) : nullptr;
+    L.W_qk = dev_alloc(h, e * (size_t)hr * kq);
+    L.W_qkc = kqc ? (float*)dev_alloc(h, sizeof(float) * (size_t)hr * kqc) : nullptr;
     L.W_ov = dev_alloc(h, e * (size_t)d * hr);
+    L.W_dqx = L.g_q = nullptr;
+    L.W_dqc = nullptr;
+    if (rq) {
+      L.g_q = upload(h, w.g_q, e * rq, weights_on_device);
+      L.W_dqx = dev_alloc(h, e * (size_t)rq * d);
+      L.W_dqc = dc ? (float*)dev_alloc(h, sizeof(float) * (size_t)dc * rq) : nullptr;
+      if (!L.g_q || !L.W_dqx || (dc && !L.W_dqc)) return fail(LLATTE_ERR_OOM);
+      void* tdq = nullptr;
+      bool okq = cudaMalloc(&tdq, e * (size_t)rq * (d + dc)) == cudaSuccess &&
+                 cudaMemcpy(tdq, w.W_dq, e * (size_t)rq * (d + dc),
+                            weights_on_device ? cudaMemcpyDeviceToDevice
+                                              : cudaMemcpyHostToDevice) == cudaSuccess &&
+                 launch_split_ctx_cols(h->elem, tdq, rq, d, dc, L.W_dqx, L.W_dqc, 0) ==
+                     cudaSuccess &&
+                 cudaDeviceSynchronize() == cudaSuccess;
+      cudaFree(tdq);
+      if (!okq) return fail(LLATTE_ERR_CUDA);
+    }
     if (!L.W_dkv || !L.g_kv || !L.g1 || !L.W1 || !L.W2 || !L.g2 || !L.W_qk || !L.W_ov ||
-        (dc && !L.W_qkc))
+        (kqc && !L.W_qkc))
       return fail(LLATTE_ERR_OOM);
     // temporaries for absorption
     void *tq = nullptr, *tuk = nullptr, *tuv = nullptr, *to = nullptr;
-    bool ok = cudaMalloc(&tq, e * (size_t)hd * (d + dc)) == cudaSuccess &&
+    bool ok = cudaMalloc(&tq, e * (size_t)hd * (kq + kqc)) == cudaSuccess &&
               cudaMalloc(&tuk, e * (size_t)hd * r) == cudaSuccess &&
               cudaMalloc(&tuv, e * (size_t)hd * r) == cudaSuccess &&
               cudaMalloc(&to, e * (size_t)d * hd) == cudaSuccess;
     cudaMemcpyKind k = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
-    ok = ok && cudaMemcpy(tq, w.W_q, e * (size_t)hd * (d + dc), k) == cudaSuccess &&
+    ok = ok && cudaMemcpy(tq, rq ? w.W_uq : w.W_q, e * (size_t)hd * (kq + kqc), k) == cudaSuccess &&
          cudaMemcpy(tuk, w.W_uk, e * (size_t)hd * r, k) == cudaSuccess &&
          cudaMemcpy(tuv, w.W_uv, e * (size_t)hd * r, k) == cudaSuccess &&
          cudaMemcpy(to, w.W_o, e * (size_t)d * hd, k) == cudaSuccess;
-    ok = ok && launch_absorb(h->elem, tq, tuk, tuv, to, d, dc, D.heads, D.d_head, r, qscale,
+    ok = ok && launch_absorb(h->elem, tq, tuk, tuv, to, d, kq, kqc, D.heads, D.d_head, r, qscale,
                              L.W_qk, L.W_qkc, L.W_ov, 0) == cudaSuccess;
     ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     cudaFree(tq); cudaFree(tuk); cudaFree(tuv); cudaFree(to);
@@ -362,14 +400,18 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     h->W_e = upload(h, W_e, e * (size_t)D.d_out * d, weights_on_device);
     if (!h->W_e) return fail(LLATTE_ERR_OOM);
   }
-  h->W_sdown = h->W_supT = nullptr;
+  h->W_sdown = h->W_sup = nullptr;
+  // output projections as one batched tensor-core GEMM (bf16, K = sum_rank and
+  // N = d_seq in whole 64-wide blocks); otherwise on CUDA cores
+  h->sum_up_tc = want_tc && D.n_sum > 0 && D.sum_rank % 64 == 0 && D.d_seq % 64 == 0;
   if (D.n_sum > 0) {
     // bottleneck projections stacked into one [n_sum * sum_rank, n_q * d]
-    // matrix; output projections transposed to [sum_rank][d_seq] each
+    // matrix; output projections stacked as given ([n_sum * d_seq, sum_rank],
+    // tensor cores) or each transposed to [sum_rank][d_seq] (CUDA cores)
     const size_t rs = D.sum_rank, K = (size_t)D.n_q * d, ds = D.d_seq;
     h->W_sdown = dev_alloc(h, e * D.n_sum * rs * K);
-    h->W_supT = dev_alloc(h, e * D.n_sum * rs * ds);
-    if (!h->W_sdown || !h->W_supT) return fail(LLATTE_ERR_OOM);
+    h->W_sup = dev_alloc(h, e * D.n_sum * rs * ds);
+    if (!h->W_sdown || !h->W_sup) return fail(LLATTE_ERR_OOM);
     void* tmp = nullptr;
     if (cudaMalloc(&tmp, e * rs * ds) != cudaSuccess) return fail(LLATTE_ERR_OOM);
     const cudaMemcpyKind k = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
@@ -377,10 +419,15 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     for (int j = 0; j < D.n_sum && ok; ++j) {
       ok = cudaMemcpy((char*)h->W_sdown + e * j * rs * K, summaries[j].W_down, e * rs * K, k) ==
                cudaSuccess &&
-           cudaMemcpy(tmp, summaries[j].W_up, e * rs * ds, k) == cudaSuccess &&
-           launch_transpose(h->elem, tmp, (int64_t)ds, (int64_t)rs,
-                            (char*)h->W_supT + e * j * rs * ds, 0) == cudaSuccess &&
-           cudaDeviceSynchronize() == cudaSuccess;
+           cudaMemcpy(tmp, summaries[j].W_up, e * rs * ds, k) == cudaSuccess;
+      if (!ok) break;
+      if (h->sum_up_tc)
+        ok = cudaMemcpy((char*)h->W_sup + e * j * rs * ds, tmp, e * rs * ds,
+                        cudaMemcpyDeviceToDevice) == cudaSuccess;
+      else
+        ok = launch_transpose(h->elem, tmp, (int64_t)ds, (int64_t)rs,
+                              (char*)h->W_sup + e * j * rs * ds, 0) == cudaSuccess;
+      ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     }
     cudaFree(tmp);
     if (!ok) return fail(LLATTE_ERR_CUDA);
@@ -414,6 +461,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->Ot = ws + Lo.off_Ot;
   h->Z = ws + Lo.off_Z;
   h->Hd = ws + Lo.off_Hd;
+  h->Cq = rq ? (void*)(ws + Lo.off_Cq) : nullptr;
   h->Zres = h->elem == 2 ? (void*)(ws + Lo.off_Zres) : nullptr;
   for (int i = 0; i < 2; ++i) h->Xqres[i] = h->elem == 2 ? (void*)(ws + Lo.off_Xqres[i]) : nullptr;
   h->acc32 = (float*)(ws + Lo.off_acc32);
@@ -422,6 +470,9 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
   h->zraw = D.n_sum ? (void*)(ws + Lo.off_zraw) : nullptr;
   h->sum_part = D.n_sum ? (float*)(ws + Lo.off_sum_part) : nullptr;
+  h->sum_h = D.n_sum ? (float*)(ws + Lo.off_sum_h) : nullptr;
+  h->sum_h16 = D.n_sum ? (void*)(ws + Lo.off_sum_h16) : nullptr;
+  h->sum_bpad = ((int64_t)D.max_batch + 127) / 128 * 128;
   h->sum_tc = 0;
   h->sum_bn = 0;
   if (want_tc) {
@@ -430,12 +481,17 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     if (D.n_sum > 0) {
       const int N = D.n_sum * D.sum_rank, K = D.n_q * d;
       h->sum_bn = N % 128 == 0 ? 128 : 64;
-      if (tc_gemm_supported(h->sum_bn, TC_PARTIAL, N, K)) {
+      if (tc_gemm_supported(h->sum_bn, TC_F32, N, K)) {
         if (!make_tmap_bf16(&h->tm_zraw, h->zraw, D.max_batch, K, 128) ||
             !make_tmap_bf16(&h->tm_sdown, h->W_sdown, N, K, h->sum_bn))
           return fail(LLATTE_ERR_CUDA);
         h->sum_tc = 1;
       }
+      if (h->sum_up_tc &&
+          (!make_tmap_bf16(&h->tm_sh16, h->sum_h16, (uint64_t)D.n_sum * h->sum_bpad, D.sum_rank,
+                           128) ||
+           !make_tmap_bf16(&h->tm_sup, h->W_sup, (uint64_t)D.n_sum * D.d_seq, D.sum_rank, 64)))
+        return fail(LLATTE_ERR_CUDA);
     }
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLATTE_ERR_CUDA);
@@ -455,6 +511,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
   const bool has_out = D.d_out > 0 || D.n_q > 0;
   if (has_out && !out) return LLATTE_ERR_ARG;
   if (((uintptr_t)values | (uintptr_t)cand) & 15) return LLATTE_ERR_ARG;  // 16-byte rows
+  if (D.n_sum > 0 && ((uintptr_t)out & 15)) return LLATTE_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   const int L = D.n_layers, e = h->elem;
   const int d = D.d, r = D.rank, hr = D.heads * D.rank, f = D.ffn_mult * D.d;
@@ -464,18 +521,23 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
   // Context term of every layer's query projection, one launch.  It depends
   // on nothing above, so outside profiling it runs on the side stream while
   // the plan and the gather run here; the first query projection waits for it.
+  // With a low-rank query the term belongs to the down-projection (before
+  // its RMSNorm): q_rank columns, fp16 for the tensor-core norm epilogue.
   bool ctx_join = false;
+  const int rq = D.q_rank;
+  const int ctx_n = rq ? rq : hr;
+  __half* ctx16 = (rq && h->use_tc) ? (__half*)h->ctxbias : nullptr;
   if (D.d_ctx > 0) {
     CtxWeights cw = {};
-    for (int l = 0; l < L; ++l) cw.W[l] = h->layers[l].W_qkc;
+    for (int l = 0; l < L; ++l) cw.W[l] = rq ? h->layers[l].W_dqc : h->layers[l].W_qkc;
     if (h->profiling) {
       StepTimer t(h, s, ST_CTX);
-      CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, s));
+      CK(launch_ctx_bias(e, context, cw, L, B, ctx_n, D.d_ctx, h->ctxbias, ctx16, s));
       t.done(1);
     } else {
       CK(cudaEventRecord(h->ev_fork, s));
       CK(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-      CK(launch_ctx_bias(e, context, cw, L, B, hr, D.d_ctx, h->ctxbias, h->side));
+      CK(launch_ctx_bias(e, context, cw, L, B, ctx_n, D.d_ctx, h->ctxbias, ctx16, h->side));
       CK(cudaEventRecord(h->ev_join, h->side));
       ctx_join = true;
     }
@@ -559,7 +621,41 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
         ctx_join = false;
       }
       StepTimer t(h, s, ST_Q);
-      if (tc) {
+      if (rq) {
+        // low-rank query: Cq = RMSNorm_{g_q}(R W_dq,x^T + context term of the
+        // row's user), then the absorbed projection Qt = Cq (W_uk^T W_uq)^T
+        NormArgs qn = {};
+        qn.N = rq; qn.g = W.g_q; qn.eps = D.eps; qn.M_dev = p.query_total(l);
+        qn.M_max = h->max_rows_q; qn.mode = NORM_PLAIN; qn.dst = h->Cq;
+        if (tc) {
+          if (D.d_ctx > 0) {
+            qn.resid = ctx16 + (int64_t)l * B * rq; qn.resid_kind = RES_F16;
+            qn.resid_user = p.ruser(l);
+          }
+          TcGemmParams q1 = tcp(p.query_total(l), h->max_rows_q, rq, d);
+          q1.norm = qn;
+          CK(launch_tc_gemm(h->bn_dq, TC_NORM, h->tm_Xq[l & 1], LM.dq, q1, h->num_sms, s));
+          TcGemmParams q2 = tcp(p.query_total(l), h->max_rows_q, hr, rq);
+          q2.D = (__nv_bfloat16*)h->Qt; q2.ldd = hr;
+          CK(launch_tc_gemm(h->bn_q, TC_STORE, h->tm_Cq, LM.qk, q2, h->num_sms, s));
+          t.done(2);
+        } else {
+          GemmArgs g = {};
+          g.A = Xq_l; g.lda = d; g.W = W.W_dqx; g.D = h->acc32; g.ldd = rq;
+          g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = rq; g.K = d;
+          g.epi = D.d_ctx > 0 ? EPI_USERBIAS_F32 : EPI_F32;
+          g.bias = h->ctxbias + (int64_t)l * B * rq; g.seg_off = p.qoff(l); g.B = B;
+          CK(launch_gemm_simt(e, e, 4, g, s));
+          qn.acc = h->acc32;
+          CK(launch_rownorm(e, qn, s));
+          GemmArgs g2 = {};
+          g2.A = h->Cq; g2.lda = rq; g2.W = W.W_qk; g2.D = h->Qt; g2.ldd = hr;
+          g2.M_dev = p.query_total(l); g2.M_max = h->max_rows_q; g2.N = hr; g2.K = rq;
+          g2.epi = EPI_STORE;
+          CK(launch_gemm_simt(e, e, e, g2, s));
+          t.done(3);
+        }
+      } else if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
         q.bias = h->ctxbias + (int64_t)l * B * hr; q.seg_off = p.qoff(l); q.B = B;
@@ -574,7 +670,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
         g.bias = h->ctxbias + (int64_t)l * B * hr; g.seg_off = p.qoff(l); g.B = B;
         CK(launch_gemm_simt(e, e, e, g, s));
       }
-      t.done(1);
+      if (!rq) t.done(1);
     }
     if (tc) {  // latent attention, tensor cores
       StepTimer t(h, s, ST_ATTN);
@@ -672,7 +768,8 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       TcGemmParams q = {};
       q.M_host = B; q.M_dev = nullptr; q.M_cap = B; q.N = N; q.K = K; q.status = p.status;
       q.Dp = h->sum_part; q.slice_stride = (int64_t)B * N; q.k_split = S;
-      CK(launch_tc_gemm(h->sum_bn, TC_PARTIAL, h->tm_zraw, h->tm_sdown, q, h->num_sms, s));
+      q.groups = 1; q.ldp = N;
+      CK(launch_tc_gemm(h->sum_bn, TC_F32, h->tm_zraw, h->tm_sdown, q, h->num_sms, s));
     } else {
       GemmArgs g = {};
       g.A = h->zraw; g.lda = K; g.W = h->W_sdown; g.D = h->sum_part; g.ldd = N;
@@ -680,10 +777,24 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       CK(launch_gemm_simt(e, e, 4, g, s));
     }
     SummaryArgs sa = {};
-    sa.P = h->sum_part; sa.S = S; sa.slice_stride = (int64_t)B * N; sa.B = B; sa.N = N;
-    sa.rank = D.sum_rank; sa.d_seq = D.d_seq; sa.n_sum = D.n_sum; sa.Wt = h->W_supT; sa.out = out;
-    CK(launch_summary_up(e, sa, h->num_sms, s));
-    t.done(2);
+    sa.P = h->sum_part; sa.S = S; sa.slice_stride = (int64_t)B * N;
+    sa.H = h->sum_up_tc ? nullptr : h->sum_h;
+    sa.H16 = (__nv_bfloat16*)h->sum_h16; sa.b_pad = h->sum_bpad;
+    sa.B = B; sa.N = N;
+    sa.rank = D.sum_rank; sa.d_seq = D.d_seq; sa.n_sum = D.n_sum; sa.Wt = h->W_sup; sa.out = out;
+    CK(launch_summary_reduce(sa, s));
+    if (h->sum_up_tc) {
+      // out[b, k, :] = H16[k, b, :] W_up,k^T for every k, one batched GEMM
+      TcGemmParams q = {};
+      q.M_host = B; q.M_dev = nullptr; q.M_cap = B; q.N = D.d_seq; q.K = D.sum_rank;
+      q.status = p.status; q.Dp = out; q.k_split = 1; q.groups = D.n_sum;
+      q.a_group_rows = h->sum_bpad; q.w_group_rows = D.d_seq; q.d_group_off = D.d_seq;
+      q.ldp = (int64_t)D.n_sum * D.d_seq;
+      CK(launch_tc_gemm(64, TC_F32, h->tm_sh16, h->tm_sup, q, h->num_sms, s));
+    } else {
+      CK(launch_summary_up(e, sa, s));
+    }
+    t.done(3);
   }
   return LLATTE_OK;
 }

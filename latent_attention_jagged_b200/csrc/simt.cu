@@ -64,15 +64,15 @@ gemm_simt_kernel(GemmArgs g) {
     const int64_t m = m0 + ty * 4 + i;
     if (m >= M) continue;
     int u = 0;
-    if (g.epi == EPI_USERBIAS) u = segment_of(g.seg_off, g.B, m);
+    if (g.epi == EPI_USERBIAS || g.epi == EPI_USERBIAS_F32) u = segment_of(g.seg_off, g.B, m);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
       if (n >= g.N) continue;
       float v = acc[i][j];
-      if (g.epi == EPI_USERBIAS) v += g.bias[(int64_t)u * g.N + n];
+      if (g.epi == EPI_USERBIAS || g.epi == EPI_USERBIAS_F32) v += g.bias[(int64_t)u * g.N + n];
       if (g.epi == EPI_SILU) v = silu_f(v);
-      if (g.epi == EPI_F32) ((float*)g.D)[m * g.ldd + n] = v;
+      if (g.epi == EPI_F32 || g.epi == EPI_USERBIAS_F32) ((float*)g.D)[m * g.ldd + n] = v;
       else ((TD*)g.D)[m * g.ldd + n] = from_f<TD>(v);
     }
   }
@@ -111,7 +111,7 @@ rownorm_kernel(NormArgs a) {
   auto val = [&](int c) {
     float v = row[c];
     if (a.resid) {
-      const int64_t i = m * N + c;
+      const int64_t i = (a.resid_user ? (int64_t)a.resid_user[m] : m) * N + c;
       if (a.resid_kind == RES_F32) v += ((const float*)a.resid)[i];
       else if (a.resid_kind == RES_F16) v += __half2float(((const __half*)a.resid)[i]);
       else v += to_f(((const T*)a.resid)[i]);
@@ -265,7 +265,7 @@ constexpr int CTX_COLS = 128;
 template <typename T>
 __global__ void __launch_bounds__(CTX_COLS)
 ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
-                float* __restrict__ out) {
+                float* __restrict__ out, __half* __restrict__ out16) {
   extern __shared__ float cs[];                       // [CTX_USERS][dc]
   const int l = blockIdx.y;
   const int u0 = blockIdx.z * CTX_USERS;
@@ -285,19 +285,23 @@ ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
 #pragma unroll
     for (int uu = 0; uu < CTX_USERS; ++uu) acc[uu] = fmaf(cs[uu * dc + k], wk, acc[uu]);
   }
-  for (int uu = 0; uu < nu; ++uu) out[((int64_t)l * B + u0 + uu) * hr + n] = acc[uu];
+  for (int uu = 0; uu < nu; ++uu) {
+    const int64_t o = ((int64_t)l * B + u0 + uu) * hr + n;
+    if (out16) out16[o] = __float2half_rn(acc[uu]);
+    else out[o] = acc[uu];
+  }
 }
 
 cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
-                            int dc, float* out, cudaStream_t s) {
+                            int dc, float* out, __half* out16, cudaStream_t s) {
   if (B == 0 || dc == 0) return cudaSuccess;
   dim3 grid((hr + CTX_COLS - 1) / CTX_COLS, L, (B + CTX_USERS - 1) / CTX_USERS);
   const size_t sm = sizeof(float) * CTX_USERS * dc;
   if (elem == 4)
-    ctx_bias_kernel<float><<<grid, CTX_COLS, sm, s>>>((const float*)ctx, w, B, hr, dc, out);
+    ctx_bias_kernel<float><<<grid, CTX_COLS, sm, s>>>((const float*)ctx, w, B, hr, dc, out, out16);
   else
     ctx_bias_kernel<__nv_bfloat16><<<grid, CTX_COLS, sm, s>>>((const __nv_bfloat16*)ctx, w, B, hr,
-                                                             dc, out);
+                                                             dc, out, out16);
   return cudaGetLastError();
 }
 
@@ -473,6 +477,7 @@ cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t co
 template <typename T>
 __global__ void absorb_q_kernel(const T* W_q, const T* W_uk, int d, int dc, int heads, int dh,
                                 int r, float qscale, T* W_qk, float* W_qkc) {
+  // d here is the width of the query input (d, or q_rank for a low-rank query)
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int K = d + dc;
   if (idx >= (int64_t)heads * r * K) return;
@@ -503,22 +508,47 @@ __global__ void absorb_o_kernel(const T* W_o, const T* W_uv, int d, int heads, i
 }
 
 cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,
-                          const void* W_o, int d, int dc, int heads, int dh, int r, float qscale,
-                          void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s) {
-  const int64_t nq = (int64_t)heads * r * (d + dc), no = (int64_t)d * heads * r;
+                          const void* W_o, int d, int dq, int dc, int heads, int dh, int r,
+                          float qscale, void* W_qk, float* W_qkc, void* W_ov, cudaStream_t s) {
+  const int64_t nq = (int64_t)heads * r * (dq + dc), no = (int64_t)d * heads * r;
   const unsigned bq = (unsigned)((nq + 255) / 256), bo = (unsigned)((no + 255) / 256);
   if (elem == 4) {
-    absorb_q_kernel<float><<<bq, 256, 0, s>>>((const float*)W_q, (const float*)W_uk, d, dc, heads,
+    absorb_q_kernel<float><<<bq, 256, 0, s>>>((const float*)W_q, (const float*)W_uk, dq, dc, heads,
                                               dh, r, qscale, (float*)W_qk, W_qkc);
     absorb_o_kernel<float><<<bo, 256, 0, s>>>((const float*)W_o, (const float*)W_uv, d, heads, dh,
                                               r, (float*)W_ov);
   } else {
     typedef __nv_bfloat16 bf;
-    absorb_q_kernel<bf><<<bq, 256, 0, s>>>((const bf*)W_q, (const bf*)W_uk, d, dc, heads, dh, r,
+    absorb_q_kernel<bf><<<bq, 256, 0, s>>>((const bf*)W_q, (const bf*)W_uk, dq, dc, heads, dh, r,
                                            qscale, (bf*)W_qk, W_qkc);
     absorb_o_kernel<bf><<<bo, 256, 0, s>>>((const bf*)W_o, (const bf*)W_uv, d, heads, dh, r,
                                            (bf*)W_ov);
   }
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void split_ctx_cols_kernel(const T* __restrict__ src, int rows, int d, int dc,
+                                      T* __restrict__ dst_x, float* __restrict__ dst_c) {
+  const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const int K = d + dc;
+  if (i >= (int64_t)rows * K) return;
+  const int row = (int)(i / K), col = (int)(i % K);
+  if (col < d) dst_x[(int64_t)row * d + col] = src[i];
+  else dst_c[(int64_t)(col - d) * rows + row] = to_f(src[i]);
+}
+
+cudaError_t launch_split_ctx_cols(int elem, const void* src, int rows, int d, int dc, void* dst_x,
+                                  float* dst_c, cudaStream_t s) {
+  const int64_t n = (int64_t)rows * (d + dc);
+  if (n <= 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (elem == 4)
+    split_ctx_cols_kernel<float><<<blocks, 256, 0, s>>>((const float*)src, rows, d, dc,
+                                                         (float*)dst_x, dst_c);
+  else
+    split_ctx_cols_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        (const __nv_bfloat16*)src, rows, d, dc, (__nv_bfloat16*)dst_x, dst_c);
   return cudaGetLastError();
 }
 

@@ -95,7 +95,9 @@ template <int BN, int PDMAX>
 __device__ __forceinline__ void norm_prefetch(const NormArgs& a, int64_t row, bool valid,
                                               int half, NormPre<BN, PDMAX>& pre) {
   if (!a.resid) return;
-  const char* src = valid ? (const char*)a.resid + (row * BN + half * (BN / 2)) * 2 : nullptr;
+  // a per-user residual (context term of a low-rank query) is row user(row)
+  const int64_t res_row = (valid && a.resid_user) ? (int64_t)a.resid_user[row] : row;
+  const char* src = valid ? (const char*)a.resid + (res_row * BN + half * (BN / 2)) * 2 : nullptr;
 #pragma unroll
   for (int i = 0; i < NormPre<BN, PDMAX>::PD; ++i) stage_fetch(src ? src + 64 * i : nullptr, pre.t[i]);
 }
@@ -127,7 +129,8 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   const int c0 = half * HB;
   const int N = BN;
   const bool have = a.resid != nullptr;
-  const char* rsrc = (valid && have) ? (const char*)a.resid + (row * N) * 2 : nullptr;
+  const int64_t res_row = (valid && have && a.resid_user) ? (int64_t)a.resid_user[row] : row;
+  const char* rsrc = (valid && have) ? (const char*)a.resid + (res_row * N) * 2 : nullptr;
   // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
   float ss = 0.f;
   constexpr int PD = NormPre<BN, PDMAX>::PD;

@@ -9,7 +9,7 @@
 
 namespace llatte {
 
-enum { TC_STORE = 0, TC_USERBIAS = 1, TC_SILU = 2, TC_NORM = 3, TC_PARTIAL = 4 };
+enum { TC_STORE = 0, TC_USERBIAS = 1, TC_SILU = 2, TC_NORM = 3, TC_F32 = 4 };
 
 struct TcGemmParams {
   int64_t M_host;               // rows, unless M_dev != NULL
@@ -20,9 +20,13 @@ struct TcGemmParams {
   const float* bias; const int64_t* seg_off; int B;   // USERBIAS: bias[user(row), n]
   const int32_t* row_user;                             // user of each row
   NormArgs norm;                                       // NORM (acc unused)
-  // PARTIAL: split-K over k_split slices of the k-blocks; slice s writes its
-  // fp32 partial sums to Dp[s * slice_stride + row * N + n]
+  // F32: fp32 store, optionally one k-slice of a split-K sum (k_split slices
+  // of the k-blocks) and one member of a batch of `groups` products.  Tile
+  // (group g, rows m, columns n, slice s) reads A rows g * a_group_rows + m
+  // and W rows g * w_group_rows + n, and writes
+  // Dp[s * slice_stride + g * d_group_off + m * ldp + n]  (M, N per group).
   float* Dp; int64_t slice_stride; int k_split;
+  int groups; int64_t a_group_rows; int w_group_rows; int64_t d_group_off; int64_t ldp;
   int32_t* status;
 };
 

@@ -49,7 +49,8 @@ def test_struct_layout_matches_header(lib):
     # int32 x 3, (pad 4)
     assert ctypes.sizeof(binding.llatte_dims) == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16 + 16
     assert binding.llatte_dims.n_sum.offset == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16
-    assert ctypes.sizeof(binding.llatte_layer_w) == 10 * ctypes.sizeof(ctypes.c_void_p)
+    assert binding.llatte_dims.q_rank.offset == binding.llatte_dims.d_seq.offset + 4
+    assert ctypes.sizeof(binding.llatte_layer_w) == 13 * ctypes.sizeof(ctypes.c_void_p)
     assert ctypes.sizeof(binding.llatte_summary_w) == 2 * ctypes.sizeof(ctypes.c_void_p)
 
 
@@ -96,6 +97,10 @@ def test_create_rejects_bad_arguments_on_host(lib):
         bad = _cdims(**kw)
         assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, None, 0) == code
         assert lib.llatte_workspace_bytes(ctypes.byref(bad)) == 0
+    for kw, code in ((dict(q_rank=-1), binding.LLATTE_ERR_ARG),
+                     (dict(q_rank=2048), binding.LLATTE_ERR_UNSUPPORTED)):
+        bad = _cdims(**kw)
+        assert lib.llatte_create(ctypes.byref(h), ctypes.byref(bad), layers, None, None, 0) == code
     ok = _cdims(n_sum=2, sum_rank=8, d_seq=16)
     assert lib.llatte_workspace_bytes(ctypes.byref(ok)) > lib.llatte_workspace_bytes(ctypes.byref(good))
 
