@@ -13,6 +13,9 @@ A.3 "Multi-head Latent Attention"; daiwk.github.io reproduction notes,
   * brute.py  - Form A: the non-absorbed MLA applied to the whole fused
                 sequence with explicit masks, then the pages' tail slice
                 (the brute force that Form B is checked against)
+  * analysis.py - attention-probability statistics of the query tokens
+                (cumulative attention on the most recent / the top-k keys,
+                attention by hours before the request; appendix A.4)
 
 Readings of points the pages leave open (scale 1/sqrt(d_h); candidates see all
 history keys but no query token; keep counts count history rows only; RMSNorm
