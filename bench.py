@@ -29,7 +29,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import draw_lengths, make_inputs, workload  # noqa: E402
+from workloads import draw_lengths, make_event_ages, make_inputs, workload  # noqa: E402
 from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 
 # ncu-measured DRAM traffic per launch (bytes, mean over one forward's layers)
@@ -173,6 +173,8 @@ def main():
                     help="second workload measured in the same run ('' = none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--export-layer", type=int, default=-1,
+                    help="also export the attention statistics of this layer in every step")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every kernel eagerly instead of replaying one CUDA graph")
     args = ap.parse_args()
@@ -241,8 +243,19 @@ def main():
         cand = torch.from_numpy(inp.cand).cuda().to(dt) if inp.dims.n_q else None
         out = torch.empty(h.out_shape(inp.batch), dtype=torch.float32, device="cuda")
         stream = torch.cuda.current_stream()
+        # optional: the attention statistics of one layer's query tokens in every step
+        ages = None
+        if args.export_layer >= 0:
+            ages = torch.from_numpy(make_event_ages(inp.lengths, seed=wl.seed + 77)).cuda()
+
+        def fwd():
+            if args.export_layer >= 0:
+                h.forward_export(values, offsets, ctx, cand, layer=args.export_layer, n_k=11,
+                                 event_age=ages, n_hours=168, out=out)
+            else:
+                h.forward(values, offsets, ctx, cand, out=out)
         for _ in range(warmup):
-            h.forward(values, offsets, ctx, cand, out=out)
+            fwd()
         torch.cuda.synchronize()
         assert h.status() == 0, "device status word set during warm-up"
         # the whole forward as one CUDA graph (no host work between kernels)
@@ -250,7 +263,7 @@ def main():
         if args.graph:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
-                h.forward(values, offsets, ctx, cand, out=out)
+                fwd()
             graph.replay()
             torch.cuda.synchronize()
 
@@ -258,7 +271,7 @@ def main():
             if graph is not None:
                 graph.replay()
             else:
-                h.forward(values, offsets, ctx, cand, out=out)
+                fwd()
 
         # ---- device-resident timing
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -291,7 +304,7 @@ def main():
         prof_steps = max(3, min(steps, 50))
         for _ in range(prof_steps):
             flush.fill_(1)
-            h.forward(values, offsets, ctx, cand, out=out)
+            fwd()
         torch.cuda.synchronize()
         prof = h.profile()
         h.set_profiling(False)
@@ -393,7 +406,8 @@ def main():
                        "seq_len": list(wl.lengths), "d": inp.dims.d, "layers": inp.dims.n_layers,
                        "parallelism": f"users sharded by LPT on FLOPs, dp{world}",
                        "l2": "flushed (256 MiB write) before every timed step",
-                       "launch": "one CUDA graph replay per step" if args.graph else "eager"},
+                       "launch": "one CUDA graph replay per step" if args.graph else "eager",
+                       "attn_export_layer": args.export_layer if args.export_layer >= 0 else None},
             "roofline": main_res["roofline"],
             "whole_step": main_res["whole"],
             "cpu_baseline": cpu,

@@ -198,8 +198,9 @@ const char* llatte_error_string(int code);
  * Per-step device timing, a profiling aid.  With profiling enabled every
  * forward records a CUDA event pair on its stream around each step (plan,
  * gather, ctx_bias, kv, q, attn, o, ffn1, ffn2, readout, ffn when the FFN
- * runs as one fused kernel, and summary); llatte_profile_step synchronises on
- * the recorded events and returns, for step index `step` (0 .. 11), its name, the
+ * runs as one fused kernel, summary, and attn_export); llatte_profile_step
+ * synchronises on the recorded events and returns, for step index `step`
+ * (0 .. 12), its name, the
  * accumulated milliseconds, the number of kernels the
  * step launched and the number of times it ran since the last reset.
  * Returns LLATTE_ERR_ARG for a step index out of range.
@@ -253,6 +254,43 @@ int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t 
  * on `stream`; allocates nothing.
  */
 int llatte_exp2_eval(const float* x, float* y, float* y_hw, int64_t n, void* stream);
+
+/*
+ * Attention-probability statistics (appendix A.4 "Attention Weight
+ * Distribution": how much attention the query tokens give to the most recent
+ * events, to the events with the largest weights, and by hours before the
+ * request).  For layer `layer`, every (user u, query token i, head j) row of
+ * P = softmax over that layer's history keys gives, for k = 2^0 .. 2^(n_k-1):
+ *   recent [B, n_q, h, n_k]  sum of P over the k most recent keys
+ *   topk   [B, n_q, h, n_k]  sum of the k largest entries of P
+ * and, with n_hours > 0 and the age of every input event in hours before the
+ * request (event_age, device float, same jagged layout as values):
+ *   hours  [B, n_q, h, n_hours]  sum of P over keys with floor(age) = b, the
+ *                                last bin also taking every older key
+ * (a user without keys gives zeros).  The keys of layer l are the user's
+ * most recent T_l events.  Reading: the pages plot these curves aggregated
+ * over requests and give no formula; the aggregation is the caller's.
+ * All outputs are device fp32, row-major, written in full.
+ */
+typedef struct {
+  int32_t layer;          /* 0 .. n_layers-1 */
+  int32_t n_k;            /* 1 .. 16 */
+  int32_t n_hours;        /* 0 .. 8192 */
+  const float* event_age; /* required iff n_hours > 0 */
+  float *recent, *topk;   /* required */
+  float* hours;           /* required iff n_hours > 0 */
+} llatte_attn_export;
+
+/*
+ * llatte_forward plus the statistics above, computed right after the
+ * layer's attention from its stored queries and latent keys (scores in fp32).
+ * Needs n_q > 0 and max_len <= LLATTE_EXPORT_MAX_LEN; LLATTE_ERR_ARG for bad
+ * export arguments.  Asynchronous on `stream` like llatte_forward.
+ */
+#define LLATTE_EXPORT_MAX_LEN 4096
+int llatte_forward_export(llatte_handle* handle, const void* values, const int64_t* offsets,
+                          int32_t B, const void* context, const void* cand, float* out,
+                          const llatte_attn_export* ex, void* stream);
 
 /* Free the handle and everything it owns (synchronises its device). */
 void llatte_destroy(llatte_handle* handle);

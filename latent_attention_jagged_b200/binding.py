@@ -15,7 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libllatte.so")
 MAX_LAYERS = 16
 STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "readout", "ffn",
-         "summary")
+         "summary", "attn_export")
 
 LLATTE_OK, LLATTE_ERR_ARG, LLATTE_ERR_UNSUPPORTED, LLATTE_ERR_CUDA, LLATTE_ERR_OOM, \
     LLATTE_ERR_DEVICE = 0, -1, -2, -3, -4, -5
@@ -56,10 +56,16 @@ class llatte_summary_w(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in SUMMARY_KEYS]
 
 
+class llatte_attn_export(ctypes.Structure):
+    _fields_ = [("layer", ctypes.c_int32), ("n_k", ctypes.c_int32), ("n_hours", ctypes.c_int32),
+                ("event_age", ctypes.c_void_p), ("recent", ctypes.c_void_p),
+                ("topk", ctypes.c_void_p), ("hours", ctypes.c_void_p)]
+
+
 EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
            "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
-           "llatte_plan_static", "llatte_exp2_eval")
+           "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export")
 PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
@@ -81,6 +87,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_create.restype = ctypes.c_int
     lib.llatte_forward.argtypes = [VP, VP, VP, I32, VP, VP, VP, VP]
     lib.llatte_forward.restype = ctypes.c_int
+    lib.llatte_forward_export.argtypes = [VP, VP, VP, I32, VP, VP, VP, P(llatte_attn_export), VP]
+    lib.llatte_forward_export.restype = ctypes.c_int
     lib.llatte_plan_export.argtypes = [VP, VP, VP]
     lib.llatte_plan_export.restype = ctypes.c_int
     lib.llatte_get_status.argtypes = [VP, P(I32)]
@@ -236,6 +244,37 @@ class Llatte:
             raise LlatteError(rc, "llatte_forward")
         self.last_B = B
         return out
+
+    def forward_export(self, values: torch.Tensor, offsets: torch.Tensor, context=None,
+                       cand=None, layer: int = 0, n_k: int = 8, event_age=None,
+                       n_hours: int = 0, out: Optional[torch.Tensor] = None, stream=None):
+        """Forward plus the attention statistics of `layer`'s query tokens:
+        returns (out, recent [B, n_q, h, n_k], topk [B, n_q, h, n_k],
+        hours [B, n_q, h, n_hours] or None)."""
+        d = self.dims
+        B = int(offsets.numel()) - 1
+        dev = values.device
+        recent = torch.empty((B, d.n_q, d.heads, n_k), dtype=torch.float32, device=dev)
+        topk = torch.empty_like(recent)
+        hours = None
+        if n_hours:
+            if (event_age is None or not event_age.is_cuda or event_age.dtype != torch.float32
+                    or not event_age.is_contiguous()):
+                raise ValueError("event_age must be a contiguous CUDA float32 tensor")
+            hours = torch.empty((B, d.n_q, d.heads, n_hours), dtype=torch.float32, device=dev)
+        ex = llatte_attn_export(layer=layer, n_k=n_k, n_hours=n_hours,
+                                event_age=event_age.data_ptr() if n_hours else None,
+                                recent=recent.data_ptr(), topk=topk.data_ptr(),
+                                hours=hours.data_ptr() if hours is not None else None)
+        if out is None:
+            out = torch.empty(self.out_shape(B), dtype=torch.float32, device=dev)
+        rc = self.lib.llatte_forward_export(self.h, _ptr(values), _ptr(offsets), B,
+                                            _ptr(context), _ptr(cand), _ptr(out),
+                                            ctypes.byref(ex), _stream_ptr(stream))
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_forward_export")
+        self.last_B = B
+        return out, recent, topk, hours
 
     def plan_export(self, stream=None) -> torch.Tensor:
         L, B = len(self.dims.keep), self.last_B

@@ -15,7 +15,7 @@ namespace llatte {
 
 // Step kinds, for the optional per-step timing.
 enum Step { ST_PLAN = 0, ST_GATHER, ST_CTX, ST_KV, ST_Q, ST_ATTN, ST_O, ST_FFN1, ST_FFN2,
-            ST_READOUT, ST_FFN, ST_SUMMARY, ST_COUNT };
+            ST_READOUT, ST_FFN, ST_SUMMARY, ST_EXPORT, ST_COUNT };
 extern const char* const kStepNames[ST_COUNT];
 
 // Device-side pyramid plan.  Layer index l runs over 0..L where l = L is the
@@ -124,6 +124,9 @@ struct llatte_handle {
   CUtensorMap tm_zraw, tm_sdown;  // summary bottleneck GEMM operands
   CUtensorMap tm_sh16, tm_sup;    // summary output-projection GEMM operands
 
+  // attention-probability export requested for the forward in progress
+  const llatte_attn_export* export_req;
+
   // the per-user context term runs on a side stream, beside the plan and
   // the gather (forked from and joined back into the caller's stream)
   cudaStream_t side;
@@ -223,6 +226,19 @@ cudaError_t launch_summary_up(int elem, const SummaryArgs& a, cudaStream_t s);
 // dst[c, r] = src[r, c] for a [rows, cols] matrix of the storage type.
 cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
                              cudaStream_t s);
+
+// Attention-probability statistics of one layer's query tokens (see the
+// attention-export call of the public header).
+struct ExportArgs {
+  const void* Qt; const void* C;                 // the layer's absorbed queries and latent keys
+  const int64_t *qoff, *hoff, *evoff;            // layer query / history offsets, input offsets
+  const int32_t *T, *n, *T0;                     // layer keys, kept history rows, input lengths
+  int B, n_q, heads, r, n2, n_k, n_hours, log2_scores;
+  const float* event_age;                        // [sum T0] hours, or NULL
+  float *recent, *topk, *hours;                  // [B, n_q, h, n_k] x2, [B, n_q, h, n_hours]
+};
+size_t attn_export_smem(int n2, int r, int n_hours);
+cudaError_t launch_attn_export(int elem, const ExportArgs& a, cudaStream_t s);
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
                              cudaStream_t s);

@@ -16,7 +16,7 @@ using namespace llatte;
 namespace llatte {
 const char* const kStepNames[ST_COUNT] = {"plan", "gather", "ctx_bias", "kv",      "q",  "attn",
                                           "o",    "ffn1",   "ffn2",     "readout", "ffn",
-                                          "summary"};
+                                          "summary", "attn_export"};
 }
 
 namespace {
@@ -325,6 +325,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->use_tc = 0;
   h->profiling = 0;
   h->last_B = 0;
+  h->export_req = nullptr;
   for (int i = 0; i < ST_COUNT; ++i) { h->step_ms[i] = 0; h->step_launches[i] = 0; h->step_calls[i] = 0; }
   auto fail = [&](int code) { llatte_destroy(h); return code; };
   if (cudaGetDevice(&h->device) != cudaSuccess) return fail(LLATTE_ERR_CUDA);
@@ -690,6 +691,21 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
       CK(launch_attn_simt(e, a, s));
       t.done(1);
     }
+    if (h->export_req && h->export_req->layer == l) {  // attention statistics of this layer
+      const llatte_attn_export& ex = *h->export_req;
+      ExportArgs x = {};
+      x.Qt = h->Qt; x.C = h->C; x.qoff = p.qoff(l); x.hoff = p.hoff(l); x.evoff = offsets;
+      x.T = p.Tl(l); x.n = p.nl(l); x.T0 = p.Tl(0);
+      x.B = B; x.n_q = D.n_q; x.heads = D.heads; x.r = r;
+      int n2 = 1;
+      while (n2 < D.max_len) n2 <<= 1;
+      x.n2 = n2; x.n_k = ex.n_k; x.n_hours = ex.n_hours; x.log2_scores = tc ? 1 : 0;
+      x.event_age = ex.n_hours > 0 ? ex.event_age : nullptr;
+      x.recent = ex.recent; x.topk = ex.topk; x.hours = ex.n_hours > 0 ? ex.hours : nullptr;
+      StepTimer t(h, s, ST_EXPORT);
+      CK(launch_attn_export(e, x, s));
+      t.done(1);
+    }
     {  // output projection + residual + RMSNorm
       StepTimer t(h, s, ST_O);
       if (tc) {
@@ -797,6 +813,23 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     t.done(3);
   }
   return LLATTE_OK;
+}
+
+int llatte_forward_export(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
+                          const void* context, const void* cand, float* out,
+                          const llatte_attn_export* ex, void* stream) {
+  if (!h || !ex) return LLATTE_ERR_ARG;
+  const llatte_dims& D = h->dims;
+  if (ex->layer < 0 || ex->layer >= D.n_layers || ex->n_k < 1 || ex->n_k > 16 ||
+      ex->n_hours < 0 || ex->n_hours > 8192 || !ex->recent || !ex->topk ||
+      (ex->n_hours > 0) != (ex->event_age != nullptr) || (ex->n_hours > 0) != (ex->hours != nullptr))
+    return LLATTE_ERR_ARG;
+  if (D.n_q <= 0) return LLATTE_ERR_ARG;
+  if (D.max_len > LLATTE_EXPORT_MAX_LEN) return LLATTE_ERR_UNSUPPORTED;
+  h->export_req = ex;
+  const int rc = llatte_forward(h, values, offsets, B, context, cand, out, stream);
+  h->export_req = nullptr;
+  return rc;
 }
 
 int llatte_plan_export(llatte_handle* h, int64_t* dst, void* stream) {

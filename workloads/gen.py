@@ -124,6 +124,19 @@ def draw_summaries(dims: Dims, rng: np.random.Generator):
     return out
 
 
+def make_event_ages(lengths, seed: int, mean_gap_hours: float = 0.5) -> np.ndarray:
+    """Hours before the request of every history event (jagged like values):
+    exponential gaps between consecutive events (and between the most recent
+    event and the request), so ages fall from the earliest event to the most
+    recent one.  Drawn from a generator of its own (seed), after nothing else."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for T in np.asarray(lengths, dtype=np.int64):
+        gaps = rng.exponential(mean_gap_hours, size=int(T))
+        out.append(np.cumsum(gaps[::-1])[::-1])          # age of event t = sum of gaps t..T-1
+    return np.concatenate(out).astype(np.float32) if out else np.zeros(0, np.float32)
+
+
 def make_inputs(wl: Workload, batch: Optional[int] = None,
                 lengths: Optional[np.ndarray] = None, seed: Optional[int] = None,
                 random_gains: bool = False, dims: Optional[Dims] = None) -> Inputs:
