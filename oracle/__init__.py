@@ -30,8 +30,8 @@ forward values themselves are not printed on the pages; parity against the
 pages' own numbers is unpinned for that reason.
 """
 from .plan import plan_layers, LayerPlan
-from .model import forward, layer_forward, absorb, rmsnorm, silu, summaries
+from .model import forward, layer_forward, absorb, rmsnorm, silu, summaries, time_encoding
 from .brute import forward_brute
 
 __all__ = ["plan_layers", "LayerPlan", "forward", "layer_forward", "absorb",
-           "rmsnorm", "silu", "summaries", "forward_brute"]
+           "rmsnorm", "silu", "summaries", "time_encoding", "forward_brute"]

@@ -24,6 +24,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from .model import history_tokens
+
 
 def _rms(v, g, eps):
     out = np.empty_like(v)
@@ -90,7 +92,7 @@ def forward_brute(inputs, users=None, return_counts: bool = False):
     outs, counts = [], []
     for u in users:
         a, b = int(inputs.offsets[u]), int(inputs.offsets[u + 1])
-        Xf = np.concatenate([np.asarray(inputs.values[a:b], np.float64),
+        Xf = np.concatenate([history_tokens(inputs, u),
                              np.asarray(inputs.cand[u], np.float64)], axis=0)
         T = b - a
         c = np.asarray(inputs.ctx[u], np.float64)

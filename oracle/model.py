@@ -38,6 +38,32 @@ import numpy as np
 from .plan import plan_layers
 
 
+def time_encoding(ages: np.ndarray, d_time: int) -> np.ndarray:
+    """Additive timestamp encoding of history events (LLaTTE notes,
+    huaxiaozhuan.com, appendix A.2 item 1: added on a subset of the hidden
+    dims).  Reading (the pages give no formula): the sinusoidal code of the
+    Transformer applied to the event's age a in hours before the request, on
+    the first d_time dims: pair i = 0 .. d_time/2 - 1 holds
+    (sin(a w_i), cos(a w_i)) with w_i = 10000^(-2i / d_time).  [T, d_time]."""
+    a = np.asarray(ages, dtype=np.float64).reshape(-1, 1)
+    w = 10000.0 ** (-2.0 * np.arange(d_time // 2) / d_time)
+    te = np.empty((a.shape[0], d_time))
+    te[:, 0::2] = np.sin(a * w)
+    te[:, 1::2] = np.cos(a * w)
+    return te
+
+
+def history_tokens(inputs, u: int) -> np.ndarray:
+    """User u's history tokens as the first layer sees them: the input rows,
+    plus the timestamp encoding on the first d_time dims when d_time > 0."""
+    a, b = int(inputs.offsets[u]), int(inputs.offsets[u + 1])
+    H = _f64(inputs.values[a:b]).copy()
+    dt = getattr(inputs.dims, "d_time", 0)
+    if dt:
+        H[:, :dt] += time_encoding(inputs.event_age[a:b], dt)
+    return H
+
+
 def rmsnorm(v: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
     ms = np.mean(v * v, axis=-1, keepdims=True)
     return v / np.sqrt(ms + eps) * g
@@ -149,8 +175,7 @@ def forward(inputs, users: Optional[Sequence[int]] = None, return_probs: bool = 
     abs_w = [absorb(w, dims) for w in inputs.layers]
     outs, all_probs, all_layers = [], [], []
     for u in users:
-        a, b = int(inputs.offsets[u]), int(inputs.offsets[u + 1])
-        H = _f64(inputs.values[a:b])
+        H = history_tokens(inputs, u)
         Y = _f64(inputs.cand[u])
         c = _f64(inputs.ctx[u])
         probs_u, layers_u = [], []

@@ -37,6 +37,8 @@ class Dims:
     d_seq    width of each summary
     q_rank   rank of the low-rank query: Q = RMSNorm([x; c] W_down^Q) W_up^Q
              (0 = the full-rank query W_Q [x; c])
+    d_time   hidden dims carrying the additive timestamp encoding of history
+             tokens (even; 0 = none)
     """
 
     d: int
@@ -55,6 +57,7 @@ class Dims:
     sum_rank: int = 0
     d_seq: int = 0
     q_rank: int = 0
+    d_time: int = 0
 
     @property
     def n_layers(self) -> int:
@@ -153,6 +156,17 @@ WORKLOADS["upstream_lq"] = Workload(
     name="upstream_lq", dims=replace(WORKLOADS["upstream"].dims, q_rank=256),
     batch=64, lengths=("fixed", 1600), seed=2,
     description="upstream user model with a rank-256 RMSNorm'd query")
+# Additive timestamp encoding on a subset of the hidden dims of the history
+# tokens (appendix A.2 item 1); the pages name neither the subset nor the
+# code: a quarter of the width is taken.
+WORKLOADS["tiny_time"] = Workload(
+    name="tiny_time", dims=replace(WORKLOADS["tiny"].dims, d_time=16),
+    batch=4, lengths=("uniform", 16, 64), seed=0,
+    description="tiny fp32 case with the timestamp encoding on 16 of 64 dims")
+WORKLOADS["online_time"] = Workload(
+    name="online_time", dims=replace(WORKLOADS["online"].dims, d_time=64),
+    batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
+    description="online ranker with the timestamp encoding on 64 of 256 dims")
 WORKLOADS["online_sum"] = Workload(
     name="online_sum", dims=replace(WORKLOADS["online"].dims, n_sum=2, sum_rank=128, d_seq=1024),
     batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,

@@ -13,6 +13,9 @@ Draw order, fixed so that every consumer sees the same numbers for a seed:
      W_dq [q_rank, d + d_ctx], g_q [q_rank], W_uq [h*d_h, q_rank] drawn in
      that order at its place
   7. W_e (readout) when d_out > 0.
+  Event ages (hours before the request, for the timestamp encoding when
+  d_time > 0) come from a generator of their own: make_event_ages with seed
+  + 7919.
   8. sequence-summary weights when n_sum > 0, summary by summary:
      W_down [sum_rank, n_q*d] N(0, 1/(n_q*d)), then W_up [d_seq, sum_rank]
      N(0, 1/sum_rank).
@@ -53,6 +56,7 @@ class Inputs:
     layers: List[Dict[str, np.ndarray]]
     W_e: Optional[np.ndarray]  # float32 [d_out, d] or None
     summaries: Optional[List[Dict[str, np.ndarray]]] = None  # per summary W_down, W_up
+    event_age: Optional[np.ndarray] = None  # float32 [sum T] hours before the request
 
     @property
     def batch(self) -> int:
@@ -168,6 +172,10 @@ def make_inputs(wl: Workload, batch: Optional[int] = None,
     layers, W_e = draw_weights(dims, rng, random_gains=random_gains)
     sums = draw_summaries(dims, rng)
 
+    ages = None
+    if dims.d_time > 0:
+        ages = make_event_ages(lens, seed=(wl.seed if seed is None else seed) + 7919)
+
     if dims.dtype == "bf16":
         values, cand, ctx = round_to_bf16(values), round_to_bf16(cand), round_to_bf16(ctx)
         layers = [{k: round_to_bf16(v) for k, v in w.items()} for w in layers]
@@ -177,4 +185,4 @@ def make_inputs(wl: Workload, batch: Optional[int] = None,
     elif dims.dtype != "fp32":
         raise ValueError(f"unknown storage dtype {dims.dtype!r}")
     return Inputs(dims=dims, lengths=lens, offsets=offsets, values=values, cand=cand,
-                  ctx=ctx, layers=layers, W_e=W_e, summaries=sums)
+                  ctx=ctx, layers=layers, W_e=W_e, summaries=sums, event_age=ages)
