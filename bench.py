@@ -243,9 +243,12 @@ def main():
         cand = torch.from_numpy(inp.cand).cuda().to(dt) if inp.dims.n_q else None
         out = torch.empty(h.out_shape(inp.batch), dtype=torch.float32, device="cuda")
         stream = torch.cuda.current_stream()
-        # optional: the attention statistics of one layer's query tokens in every step
+        # event ages: the timestamp code's input (d_time > 0), and the hour bins
+        # of the optional attention statistics of one layer's query tokens
         ages = None
-        if args.export_layer >= 0:
+        if inp.event_age is not None:
+            ages = torch.from_numpy(inp.event_age).cuda()
+        elif args.export_layer >= 0:
             ages = torch.from_numpy(make_event_ages(inp.lengths, seed=wl.seed + 77)).cuda()
 
         def fwd():
@@ -253,7 +256,7 @@ def main():
                 h.forward_export(values, offsets, ctx, cand, layer=args.export_layer, n_k=11,
                                  event_age=ages, n_hours=168, out=out)
             else:
-                h.forward(values, offsets, ctx, cand, out=out)
+                h.forward(values, offsets, ctx, cand, out=out, event_age=ages)
         for _ in range(warmup):
             fwd()
         torch.cuda.synchronize()
@@ -315,6 +318,7 @@ def main():
         ho = torch.from_numpy(inp.offsets).pin_memory()
         hc = torch.from_numpy(inp.ctx).to(dt).pin_memory() if inp.dims.d_ctx else None
         hq = torch.from_numpy(inp.cand).to(dt).pin_memory() if inp.dims.n_q else None
+        ha = torch.from_numpy(inp.event_age).pin_memory() if inp.event_age is not None else None
         hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
         e2e_steps = max(3, min(steps, 50))
         ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -330,6 +334,8 @@ def main():
                 ctx.copy_(hc, non_blocking=True)
             if hq is not None:
                 cand.copy_(hq, non_blocking=True)
+            if ha is not None:
+                ages.copy_(ha, non_blocking=True)
             step()
             hout.copy_(out, non_blocking=True)
             b.record(stream)
@@ -338,7 +344,8 @@ def main():
         ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2))
         h2d = hv.numel() * hv.element_size() + ho.numel() * 8 + \
             (hc.numel() * hc.element_size() if hc is not None else 0) + \
-            (hq.numel() * hq.element_size() if hq is not None else 0)
+            (hq.numel() * hq.element_size() if hq is not None else 0) + \
+            (ha.numel() * 4 if ha is not None else 0)
         e2e = {"value": users_all * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4)}
         assert h.status() == 0

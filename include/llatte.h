@@ -21,6 +21,11 @@
  *   With q_rank > 0 the query is low-rank and normalised (appendix A.3, first
  *   display): q~ = (W_uk,j^T W_up,j^Q) RMSNorm_{g_q}(W_down^Q [R_i ; c]) / sqrt(d_h),
  *   the down-projection taking the target-aware input [x ; c].
+ *   With d_time > 0 every history token first gets an additive timestamp code
+ *   on its first d_time dims (appendix A.2 item 1; the pages give no formula:
+ *   the Transformer's sinusoidal code of the event's age a in hours before
+ *   the request is the reading taken): dims 2i, 2i+1 add sin(a w_i), cos(a w_i),
+ *   w_i = 10000^(-2i/d_time).  Query tokens carry no timestamp.
  *   Visibility: a history query at position p sees keys t <= p; a query token
  *   sees every current history key and no query token; no key -> zero output.
  *   Output: the final query-token rows; or, with d_out > 0, W_e times the mean
@@ -96,6 +101,7 @@ enum {
  *   sum_rank, d_seq       bottleneck width (1 .. 1024) and width (even) of each summary
  *   q_rank                rank of the low-rank RMSNorm'd query (0 = full-rank W_q;
  *                         at most 1024)
+ *   d_time                dims carrying the timestamp code (even, <= d; 0 = none)
  */
 typedef struct {
   int32_t d, heads, d_head, rank, d_ctx, n_q, n_layers;
@@ -107,6 +113,7 @@ typedef struct {
   int64_t max_total;
   int32_t n_sum, sum_rank, d_seq;
   int32_t q_rank;
+  int32_t d_time;
 } llatte_dims;
 
 #define LLATTE_MAX_SUMMARIES 16
@@ -154,6 +161,23 @@ int llatte_create(llatte_handle** handle, const llatte_dims* dims,
                   const llatte_summary_w* summaries, int weights_on_device);
 
 /*
+ * One batch of inputs, for llatte_forward_batch (the fields of llatte_forward
+ * plus the event ages):
+ *   event_age  device float [offsets[B]]: hours before the request of every
+ *              history event, same jagged layout as values; required when
+ *              d_time > 0 (otherwise ignored, may be NULL); the code keeps
+ *              fp32 accuracy for ages below 4e5 hours
+ */
+typedef struct {
+  const void* values;
+  const int64_t* offsets;
+  int32_t B;
+  const void* context;
+  const void* cand;
+  const float* event_age;
+} llatte_batch;
+
+/*
  * One forward pass, asynchronous on `stream` (a cudaStream_t; NULL = legacy
  * default stream), with no host synchronisation.
  *   values  device [offsets[B] rows, d] in dtype: all users' histories, user u
@@ -167,7 +191,9 @@ int llatte_create(llatte_handle** handle, const llatte_dims* dims,
  *   out     device fp32 [B, n_q, d] (d_out == 0, n_sum == 0), [B, d_out]
  *           (d_out > 0) or [B, n_sum, d_seq] (n_sum > 0, 16-byte aligned)
  * Inputs are only read; `out` is the only caller memory written.  Calls on
- * one handle must not overlap in time (they share its workspace).
+ * one handle must not overlap in time (they share its workspace).  With
+ * d_time > 0 it returns LLATTE_ERR_ARG (the ages are needed: use
+ * llatte_forward_batch).
  */
 int llatte_forward(llatte_handle* handle, const void* values, const int64_t* offsets,
                    int32_t B, const void* context, const void* cand, float* out,
@@ -291,6 +317,15 @@ typedef struct {
 int llatte_forward_export(llatte_handle* handle, const void* values, const int64_t* offsets,
                           int32_t B, const void* context, const void* cand, float* out,
                           const llatte_attn_export* ex, void* stream);
+
+/*
+ * The forward pass of one llatte_batch (with the event ages, which the
+ * timestamp code needs when d_time > 0); with ex != NULL it also computes the
+ * attention statistics above (ex->event_age may then be the batch's).
+ * Otherwise as llatte_forward.
+ */
+int llatte_forward_batch(llatte_handle* handle, const llatte_batch* batch, float* out,
+                         const llatte_attn_export* ex, void* stream);
 
 /* Free the handle and everything it owns (synchronises its device). */
 void llatte_destroy(llatte_handle* handle);

@@ -38,7 +38,7 @@ class llatte_dims(ctypes.Structure):
                 ("max_batch", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("max_total", ctypes.c_int64), ("n_sum", ctypes.c_int32),
                 ("sum_rank", ctypes.c_int32), ("d_seq", ctypes.c_int32),
-                ("q_rank", ctypes.c_int32)]
+                ("q_rank", ctypes.c_int32), ("d_time", ctypes.c_int32)]
 
 
 LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2",
@@ -56,6 +56,12 @@ class llatte_summary_w(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in SUMMARY_KEYS]
 
 
+class llatte_batch(ctypes.Structure):
+    _fields_ = [("values", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("B", ctypes.c_int32),
+                ("context", ctypes.c_void_p), ("cand", ctypes.c_void_p),
+                ("event_age", ctypes.c_void_p)]
+
+
 class llatte_attn_export(ctypes.Structure):
     _fields_ = [("layer", ctypes.c_int32), ("n_k", ctypes.c_int32), ("n_hours", ctypes.c_int32),
                 ("event_age", ctypes.c_void_p), ("recent", ctypes.c_void_p),
@@ -65,7 +71,8 @@ class llatte_attn_export(ctypes.Structure):
 EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_status",
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
            "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
-           "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export")
+           "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export",
+           "llatte_forward_batch")
 PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
@@ -89,6 +96,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_forward.restype = ctypes.c_int
     lib.llatte_forward_export.argtypes = [VP, VP, VP, I32, VP, VP, VP, P(llatte_attn_export), VP]
     lib.llatte_forward_export.restype = ctypes.c_int
+    lib.llatte_forward_batch.argtypes = [VP, P(llatte_batch), VP, P(llatte_attn_export), VP]
+    lib.llatte_forward_batch.restype = ctypes.c_int
     lib.llatte_plan_export.argtypes = [VP, VP, VP]
     lib.llatte_plan_export.restype = ctypes.c_int
     lib.llatte_get_status.argtypes = [VP, P(I32)]
@@ -139,6 +148,7 @@ def make_dims(dims, max_batch: int, max_len: int, max_total: int = 0) -> llatte_
     c.sum_rank = int(getattr(dims, "sum_rank", 0))
     c.d_seq = int(getattr(dims, "d_seq", 0))
     c.q_rank = int(getattr(dims, "q_rank", 0))
+    c.d_time = int(getattr(dims, "d_time", 0))
     return c
 
 
@@ -215,14 +225,14 @@ class Llatte:
             return (B, d.n_sum, d.d_seq)
         return (B, d.d_out) if d.d_out else (B, d.n_q, d.d)
 
-    def forward(self, values: torch.Tensor, offsets: torch.Tensor, context=None, cand=None,
-                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    def _check_inputs(self, values, offsets, context, cand, event_age):
         d = self.dims
         B = int(offsets.numel()) - 1
         if B < 0:
             raise ValueError("offsets needs B+1 entries")
         for name, t, dt in (("values", values, self.dt), ("offsets", offsets, torch.int64),
-                            ("context", context, self.dt), ("cand", cand, self.dt)):
+                            ("context", context, self.dt), ("cand", cand, self.dt),
+                            ("event_age", event_age, torch.float32)):
             if t is None:
                 continue
             if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
@@ -233,16 +243,46 @@ class Llatte:
             raise ValueError(f"context must be [{B}, {d.d_ctx}]")
         if d.n_q and (cand is None or tuple(cand.shape) != (B, d.n_q, d.d)):
             raise ValueError(f"cand must be [{B}, {d.n_q}, {d.d}]")
+        if getattr(d, "d_time", 0) and (event_age is None or event_age.dim() != 1 or
+                                        event_age.shape[0] < values.shape[0]):
+            raise ValueError("event_age [rows] (hours before the request) is required")
+        return B
+
+    def _out(self, out, B, device):
         if out is None:
-            out = torch.empty(self.out_shape(B), dtype=torch.float32, device=values.device)
-        elif (tuple(out.shape) != self.out_shape(B) or out.dtype != torch.float32
-              or not out.is_contiguous()):
+            return torch.empty(self.out_shape(B), dtype=torch.float32, device=device)
+        if (tuple(out.shape) != self.out_shape(B) or out.dtype != torch.float32
+                or not out.is_contiguous()):
             raise ValueError(f"out must be a contiguous float32 {self.out_shape(B)} tensor")
-        rc = self.lib.llatte_forward(self.h, _ptr(values), _ptr(offsets), B, _ptr(context),
-                                     _ptr(cand), _ptr(out), _stream_ptr(stream))
+        return out
+
+    def _run(self, values, offsets, context, cand, event_age, out, ex, stream, B):
+        if ex is None and event_age is None:
+            rc = self.lib.llatte_forward(self.h, _ptr(values), _ptr(offsets), B, _ptr(context),
+                                         _ptr(cand), _ptr(out), _stream_ptr(stream))
+            what = "llatte_forward"
+        else:
+            b = llatte_batch(values=values.data_ptr(), offsets=offsets.data_ptr(), B=B,
+                             context=context.data_ptr() if context is not None else None,
+                             cand=cand.data_ptr() if cand is not None else None,
+                             event_age=event_age.data_ptr() if event_age is not None else None)
+            rc = self.lib.llatte_forward_batch(self.h, ctypes.byref(b), _ptr(out),
+                                               ctypes.byref(ex) if ex is not None else None,
+                                               _stream_ptr(stream))
+            what = "llatte_forward_batch"
         if rc != LLATTE_OK:
-            raise LlatteError(rc, "llatte_forward")
+            raise LlatteError(rc, what)
         self.last_B = B
+
+    def forward(self, values: torch.Tensor, offsets: torch.Tensor, context=None, cand=None,
+                out: Optional[torch.Tensor] = None, stream=None, event_age=None) -> torch.Tensor:
+        """One forward pass.  event_age (float32 [rows], hours before the
+        request of every history event) is required when dims.d_time > 0."""
+        B = self._check_inputs(values, offsets, context, cand, event_age)
+        out = self._out(out, B, values.device)
+        if not getattr(self.dims, "d_time", 0):
+            event_age = None
+        self._run(values, offsets, context, cand, event_age, out, None, stream, B)
         return out
 
     def forward_export(self, values: torch.Tensor, offsets: torch.Tensor, context=None,
@@ -250,30 +290,25 @@ class Llatte:
                        n_hours: int = 0, out: Optional[torch.Tensor] = None, stream=None):
         """Forward plus the attention statistics of `layer`'s query tokens:
         returns (out, recent [B, n_q, h, n_k], topk [B, n_q, h, n_k],
-        hours [B, n_q, h, n_hours] or None)."""
+        hours [B, n_q, h, n_hours] or None).  event_age serves both the hour
+        bins and, when dims.d_time > 0, the timestamp code."""
         d = self.dims
-        B = int(offsets.numel()) - 1
+        B = self._check_inputs(values, offsets, context, cand, event_age)
         dev = values.device
         recent = torch.empty((B, d.n_q, d.heads, n_k), dtype=torch.float32, device=dev)
         topk = torch.empty_like(recent)
         hours = None
         if n_hours:
-            if (event_age is None or not event_age.is_cuda or event_age.dtype != torch.float32
-                    or not event_age.is_contiguous()):
-                raise ValueError("event_age must be a contiguous CUDA float32 tensor")
+            if event_age is None:
+                raise ValueError("event_age is required for hour bins")
             hours = torch.empty((B, d.n_q, d.heads, n_hours), dtype=torch.float32, device=dev)
         ex = llatte_attn_export(layer=layer, n_k=n_k, n_hours=n_hours,
                                 event_age=event_age.data_ptr() if n_hours else None,
                                 recent=recent.data_ptr(), topk=topk.data_ptr(),
                                 hours=hours.data_ptr() if hours is not None else None)
-        if out is None:
-            out = torch.empty(self.out_shape(B), dtype=torch.float32, device=dev)
-        rc = self.lib.llatte_forward_export(self.h, _ptr(values), _ptr(offsets), B,
-                                            _ptr(context), _ptr(cand), _ptr(out),
-                                            ctypes.byref(ex), _stream_ptr(stream))
-        if rc != LLATTE_OK:
-            raise LlatteError(rc, "llatte_forward_export")
-        self.last_B = B
+        out = self._out(out, B, dev)
+        self._run(values, offsets, context, cand,
+                  event_age if getattr(d, "d_time", 0) else None, out, ex, stream, B)
         return out, recent, topk, hours
 
     def plan_export(self, stream=None) -> torch.Tensor:

@@ -148,8 +148,10 @@ cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, c
 // The plan kernel on caller-described storage (no work lists).
 cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_total,
                            const int64_t* offsets, int B, cudaStream_t s);
+// Layer-0 rows from the inputs; with ages != NULL (d_time > 0) the rows taken
+// from `values` get the timestamp code on their first d_time dims.
 cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
-                          const void* cand, int B, cudaStream_t s);
+                          const void* cand, const float* ages, int B, cudaStream_t s);
 
 // CUDA-core path
 struct GemmArgs {

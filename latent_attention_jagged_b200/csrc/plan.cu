@@ -217,13 +217,63 @@ cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_t
 
 // ---------------------------------------------------------------- gather
 
+// sin and cos of x: x is reduced to [-pi, pi] by subtracting the nearest
+// multiple of 2 pi in two parts (Cody and Waite's method; 2 pi = 6.28125 +
+// a remainder, the first part short enough that k * 6.28125 is exact for
+// |k| < 2^16, i.e. |x| < 4e5), then the hardware approximation, whose absolute
+// error is below 1e-6 on that interval.
+__device__ __forceinline__ void sincos_reduced(float x, float* s, float* c) {
+  constexpr float kInv2Pi = 0.15915494309189535f;
+  constexpr float kHi = 6.28125f, kLo = 1.9353071795864769e-3f;
+  const float k = rintf(x * kInv2Pi);
+  float r = fmaf(-k, kHi, x);
+  r = fmaf(-k, kLo, r);
+  __sincosf(r, s, c);
+}
+
+// Additive timestamp code (LLaTTE notes, appendix A.2 item 1, read as the
+// Transformer's sinusoidal code of the event's age in hours): the 16-byte
+// vector x holds dims e0 .. e0 + 16/elem - 1 of a history row; dims 2i and
+// 2i + 1 below d_time add sin(age w_i) and cos(age w_i), w_i = 10000^(-2i/d_time).
+__device__ __forceinline__ void add_time_code(uint4& x, int e0, float age, int d_time, int elem) {
+  constexpr float kLog2Base = 13.287712379549449f;       // log2(10000)
+  if (elem == 2) {
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int e = e0 + 2 * k;                            // even: one (sin, cos) pair
+      if (e >= d_time) break;
+      float sn, cs;
+      sincos_reduced(age * exp2f(-(float)e / (float)d_time * kLog2Base), &sn, &cs);
+      float2 f = __bfloat1622float2(h2[k]);
+      f.x += sn;
+      f.y += cs;
+      h2[k] = __floats2bfloat162_rn(f.x, f.y);
+    }
+  } else {
+    float* f = reinterpret_cast<float*>(&x);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = e0 + 2 * k;
+      if (e >= d_time) break;
+      float sn, cs;
+      sincos_reduced(age * exp2f(-(float)e / (float)d_time * kLog2Base), &sn, &cs);
+      f[2 * k] += sn;
+      f[2 * k + 1] += cs;
+    }
+  }
+}
+
 // Block (u, s): slice s of user u's rows.  Rows 0..T-1 are the user's
-// history (copied to the history buffer), rows T..T+q-1 its query rows (the
-// last n history rows, then the query tokens).  One warp per row.
+// history events, each read once and stored to the history buffer and, for
+// the last n, also to the query rows; rows T..T+n_q-1 are the query tokens
+// (query rows n..).  One warp per row.  With ages, every history event gets
+// the timestamp code.
 __global__ void __launch_bounds__(256)
 gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offsets,
               const uint4* __restrict__ cand, PlanDev p, uint4* __restrict__ Xh,
-              uint4* __restrict__ Xq, int row_vecs, int n_q, int n_layers) {
+              uint4* __restrict__ Xq, int row_vecs, int n_q, int n_layers,
+              const float* __restrict__ ages, int d_time, int elem) {
   // a batch the plan rejected has zero rows everywhere: copy nothing
   if (*p.hist_total(0) == 0 && *p.query_total(0) == 0) return;
   const int u = blockIdx.x;
@@ -232,7 +282,7 @@ gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offs
   const int w0 = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t T = p.Tl(0)[u], n = p.nl(0)[u];
   const int64_t hoff = p.hoff(0)[u], qoff = p.qoff(0)[u], src0 = offsets[u];
-  const int64_t rows = T + n + n_q;
+  const int64_t rows = T + n_q;
   // user of every query row of every layer (the epilogues' row -> user map)
   for (int l = 0; l < n_layers; ++l) {
     const int64_t q = (int64_t)p.nl(l)[u] + n_q;
@@ -246,43 +296,58 @@ gather_kernel(const uint4* __restrict__ values, const int64_t* __restrict__ offs
   for (int64_t r0 = w0; r0 < rows; r0 += (int64_t)warps * RG) {
     const uint4* src[RG];
     uint4* dst[RG];
+    uint4* dst2[RG];                     // kept history rows: also a query row
+    float age[RG];                       // -1: no timestamp code (query token / none)
 #pragma unroll
     for (int k = 0; k < RG; ++k) {
       const int64_t r = r0 + (int64_t)k * warps;
       src[k] = nullptr;
       dst[k] = nullptr;
+      dst2[k] = nullptr;
+      age[k] = -1.f;
       if (r >= rows) continue;
       if (r < T) {
         src[k] = values + (src0 + r) * row_vecs;
         dst[k] = Xh + (hoff + r) * row_vecs;
+        if (r >= T - n) dst2[k] = Xq + (qoff + r - (T - n)) * row_vecs;
+        if (ages) age[k] = __ldg(ages + src0 + r);
       } else {
         const int64_t j = r - T;
-        src[k] = j < n ? values + (src0 + T - n + j) * row_vecs
-                       : cand + ((int64_t)u * n_q + (j - n)) * row_vecs;
-        dst[k] = Xq + (qoff + j) * row_vecs;
+        src[k] = cand + ((int64_t)u * n_q + j) * row_vecs;
+        dst[k] = Xq + (qoff + n + j) * row_vecs;
       }
     }
+    const int epv = 16 / elem;           // elements per 16-byte vector
     for (int v = lane; v < row_vecs; v += 32) {
       uint4 x[RG];
 #pragma unroll
       for (int k = 0; k < RG; ++k)
         if (src[k]) x[k] = __ldg(src[k] + v);
+      if (ages && v * epv < d_time) {
 #pragma unroll
-      for (int k = 0; k < RG; ++k)
+        for (int k = 0; k < RG; ++k)
+          if (src[k] && age[k] >= 0.f) add_time_code(x[k], v * epv, age[k], d_time, elem);
+      }
+#pragma unroll
+      for (int k = 0; k < RG; ++k) {
         if (dst[k]) dst[k][v] = x[k];
+        if (dst2[k]) dst2[k][v] = x[k];
+      }
     }
   }
 }
 
 cudaError_t launch_gather(const llatte_handle* h, const void* values, const int64_t* offsets,
-                          const void* cand, int B, cudaStream_t s) {
+                          const void* cand, const float* ages, int B, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   const int row_vecs = h->dims.d * h->elem / 16;
   // enough blocks to cover every SM several times even for small batches
   const int slices = std::max(1, std::min(64, (h->num_sms * 8 + B - 1) / B));
   gather_kernel<<<dim3(B, slices), 256, 0, s>>>((const uint4*)values, offsets, (const uint4*)cand,
                                                 h->plan, (uint4*)h->Xh[0], (uint4*)h->Xq[0],
-                                                row_vecs, h->dims.n_q, h->dims.n_layers);
+                                                row_vecs, h->dims.n_q, h->dims.n_layers,
+                                                h->dims.d_time > 0 ? ages : nullptr,
+                                                h->dims.d_time, h->elem);
   return cudaGetLastError();
 }
 

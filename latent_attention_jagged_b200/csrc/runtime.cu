@@ -56,6 +56,7 @@ int check_dims(const llatte_dims* d) {
   if (d->kv_norm != 0 && d->kv_norm != 1) return LLATTE_ERR_ARG;
   if (d->n_sum < 0 || d->n_sum > LLATTE_MAX_SUMMARIES) return LLATTE_ERR_ARG;
   if (d->q_rank < 0) return LLATTE_ERR_ARG;
+  if (d->d_time < 0 || d->d_time % 2 != 0 || d->d_time > d->d) return LLATTE_ERR_ARG;
   if (d->q_rank > 1024) return LLATTE_ERR_UNSUPPORTED;
   if (d->n_sum > 0) {
     if (d->n_q <= 0 || d->d_out > 0 || d->sum_rank <= 0 || d->d_seq <= 0) return LLATTE_ERR_ARG;
@@ -500,9 +501,25 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   return LLATTE_OK;
 }
 
-int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
-                   const void* context, const void* cand, float* out, void* stream) {
-  if (!h) return LLATTE_ERR_ARG;
+}  // extern "C"
+
+namespace {
+
+// The export arguments, checked on the host.
+int check_export(const llatte_handle* h, const llatte_attn_export* ex) {
+  const llatte_dims& D = h->dims;
+  if (ex->layer < 0 || ex->layer >= D.n_layers || ex->n_k < 1 || ex->n_k > 16 ||
+      ex->n_hours < 0 || ex->n_hours > 8192 || !ex->recent || !ex->topk ||
+      (ex->n_hours > 0) != (ex->event_age != nullptr) || (ex->n_hours > 0) != (ex->hours != nullptr))
+    return LLATTE_ERR_ARG;
+  if (D.n_q <= 0) return LLATTE_ERR_ARG;
+  if (D.max_len > LLATTE_EXPORT_MAX_LEN) return LLATTE_ERR_UNSUPPORTED;
+  return LLATTE_OK;
+}
+
+int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
+                 const void* context, const void* cand, const float* ages, float* out,
+                 void* stream) {
   const llatte_dims& D = h->dims;
   if (B < 0 || B > D.max_batch) return LLATTE_ERR_ARG;
   if (B == 0) { h->last_B = 0; return LLATTE_OK; }
@@ -544,7 +561,7 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
     }
   }
   { StepTimer t(h, s, ST_PLAN); CK(launch_plan(h, offsets, B, s)); t.done(1); }
-  { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, B, s)); t.done(1); }
+  { StepTimer t(h, s, ST_GATHER); CK(launch_gather(h, values, offsets, cand, ages, B, s)); t.done(1); }
 
   for (int l = 0; l < L; ++l) {
     const LayerDev& W = h->layers[l];
@@ -815,19 +832,39 @@ int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets,
   return LLATTE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int llatte_forward(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
+                   const void* context, const void* cand, float* out, void* stream) {
+  if (!h || h->dims.d_time > 0) return LLATTE_ERR_ARG;     // the timestamp code needs ages
+  return forward_impl(h, values, offsets, B, context, cand, nullptr, out, stream);
+}
+
 int llatte_forward_export(llatte_handle* h, const void* values, const int64_t* offsets, int32_t B,
                           const void* context, const void* cand, float* out,
                           const llatte_attn_export* ex, void* stream) {
-  if (!h || !ex) return LLATTE_ERR_ARG;
-  const llatte_dims& D = h->dims;
-  if (ex->layer < 0 || ex->layer >= D.n_layers || ex->n_k < 1 || ex->n_k > 16 ||
-      ex->n_hours < 0 || ex->n_hours > 8192 || !ex->recent || !ex->topk ||
-      (ex->n_hours > 0) != (ex->event_age != nullptr) || (ex->n_hours > 0) != (ex->hours != nullptr))
-    return LLATTE_ERR_ARG;
-  if (D.n_q <= 0) return LLATTE_ERR_ARG;
-  if (D.max_len > LLATTE_EXPORT_MAX_LEN) return LLATTE_ERR_UNSUPPORTED;
+  if (!h || !ex || h->dims.d_time > 0) return LLATTE_ERR_ARG;
+  const int rc0 = check_export(h, ex);
+  if (rc0 != LLATTE_OK) return rc0;
   h->export_req = ex;
-  const int rc = llatte_forward(h, values, offsets, B, context, cand, out, stream);
+  const int rc = forward_impl(h, values, offsets, B, context, cand, nullptr, out, stream);
+  h->export_req = nullptr;
+  return rc;
+}
+
+int llatte_forward_batch(llatte_handle* h, const llatte_batch* b, float* out,
+                         const llatte_attn_export* ex, void* stream) {
+  if (!h || !b) return LLATTE_ERR_ARG;
+  if (h->dims.d_time > 0 && b->B > 0 && !b->event_age) return LLATTE_ERR_ARG;
+  if (ex) {
+    const int rc0 = check_export(h, ex);
+    if (rc0 != LLATTE_OK) return rc0;
+  }
+  h->export_req = ex;
+  const int rc = forward_impl(h, b->values, b->offsets, b->B, b->context, b->cand,
+                              h->dims.d_time > 0 ? b->event_age : nullptr, out, stream);
   h->export_req = nullptr;
   return rc;
 }

@@ -29,10 +29,15 @@ def make_handle(inp, max_batch=None, max_len=None, max_total=0):
                   max_len=ml, max_total=max_total, summaries=inp.summaries)
 
 
+def ages_on_device(inp):
+    a = getattr(inp, "event_age", None)
+    return torch.from_numpy(a).cuda() if a is not None else None
+
+
 def run(inp, handle=None, **kw):
     h = handle or make_handle(inp, **kw)
     values, offsets, ctx, cand = to_device(inp)
-    out = h.forward(values, offsets, ctx, cand)
+    out = h.forward(values, offsets, ctx, cand, event_age=ages_on_device(inp))
     torch.cuda.synchronize()
     return h, out.cpu().numpy().astype(np.float64)
 
