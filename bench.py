@@ -173,6 +173,9 @@ def main():
                     help="second workload measured in the same run ('' = none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn-form", type=int, default=None, choices=[0, 1, 2],
+                    help="MLA form on the GPU: 0 auto, 1 absorbed, 2 per head (default: the "
+                         "workload's)")
     ap.add_argument("--export-layer", type=int, default=-1,
                     help="also export the attention statistics of this layer in every step")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
@@ -185,6 +188,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = workload(args.workload)
+    if args.attn_form is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, dims=dataclasses.replace(wl.dims, attn_form=args.attn_form))
 
     if args.impl == "reference":
         if rank == 0:
@@ -351,7 +357,8 @@ def main():
         assert h.status() == 0
 
         # ---- roofline of the dominant step (largest device time)
-        flops = cost.flops_by_step(inp.lengths, inp.dims)
+        ph = h.per_head_layers()              # layers in MLA's per-head form: their own work
+        flops = cost.flops_by_step(inp.lengths, inp.dims, ph)
         dom = max((k for k in prof if k in flops), key=lambda k: prof[k]["ms"])
         dom_ms = prof[dom]["ms"] / max(1, prof[dom]["calls"])       # per launch of the step
         per_launch_flops = flops[dom] / (prof[dom]["calls"] / prof_steps)
@@ -375,7 +382,7 @@ def main():
                        "bytes": s_bytes, "ms": s_ms, "launches": prof["summary"]["launches"]
                        / prof["summary"]["calls"],
                        "flops": cost.summary_flops(inp.batch, inp.dims)}
-        total_flops = cost.total_flops(inp.lengths, inp.dims)
+        total_flops = cost.total_flops(inp.lengths, inp.dims, ph)
         step_ms = ms / steps
         whole = {"achieved_tflops": total_flops / (step_ms / 1e3) / 1e12,
                  "frac_of_peak": total_flops / (step_ms / 1e3) / 1e12 / peak,
@@ -383,7 +390,8 @@ def main():
         steps_ms = {k: round(v["ms"] / prof_steps, 4) for k, v in prof.items() if v["calls"]}
         res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
                    clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
-                   dtype=inp.dims.dtype, users_all=users_all, summary=summary)
+                   dtype=inp.dims.dtype, users_all=users_all, summary=summary,
+                   per_head_layers=ph)
         del graph
         h.close()
         return res
@@ -396,7 +404,8 @@ def main():
         r2 = measure(wl2, s_steps, args.warmup, sample_clocks=False)
         second = {"workload": wl2.name, "value": r2["value"], "unit": "user-seqs/s",
                   "ms_per_step": r2["ms"], "steps": s_steps, "roofline": r2["roofline"],
-                  "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"]}
+                  "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"],
+                  "mla_per_head_layers": r2["per_head_layers"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -414,7 +423,8 @@ def main():
                        "parallelism": f"users sharded by LPT on FLOPs, dp{world}",
                        "l2": "flushed (256 MiB write) before every timed step",
                        "launch": "one CUDA graph replay per step" if args.graph else "eager",
-                       "attn_export_layer": args.export_layer if args.export_layer >= 0 else None},
+                       "attn_export_layer": args.export_layer if args.export_layer >= 0 else None,
+                       "mla_per_head_layers": main_res["per_head_layers"]},
             "roofline": main_res["roofline"],
             "whole_step": main_res["whole"],
             "cpu_baseline": cpu,

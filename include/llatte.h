@@ -102,6 +102,12 @@ enum {
  *   q_rank                rank of the low-rank RMSNorm'd query (0 = full-rank W_q;
  *                         at most 1024)
  *   d_time                dims carrying the timestamp code (even, <= d; 0 = none)
+ *   attn_form             which form of MLA each layer runs (the same function):
+ *                         LLATTE_ATTN_AUTO (per layer, the cheaper one),
+ *                         LLATTE_ATTN_ABSORBED (latent-space multi-query attention)
+ *                         or LLATTE_ATTN_PER_HEAD (K, V = split(c_kv W_up^KV), scores
+ *                         over d_h; needs bf16, d_h = 64, q_rank = 0 and the
+ *                         tensor-core dims, else LLATTE_ERR_UNSUPPORTED)
  */
 typedef struct {
   int32_t d, heads, d_head, rank, d_ctx, n_q, n_layers;
@@ -114,7 +120,10 @@ typedef struct {
   int32_t n_sum, sum_rank, d_seq;
   int32_t q_rank;
   int32_t d_time;
+  int32_t attn_form;
 } llatte_dims;
+
+enum { LLATTE_ATTN_AUTO = 0, LLATTE_ATTN_ABSORBED = 1, LLATTE_ATTN_PER_HEAD = 2 };
 
 #define LLATTE_MAX_SUMMARIES 16
 
@@ -213,6 +222,13 @@ int llatte_plan_export(llatte_handle* handle, int64_t* dst, void* stream);
  * fault) and clear it.  Returns LLATTE_ERR_DEVICE when it was non-zero.
  */
 int llatte_get_status(llatte_handle* handle, int32_t* device_status);
+
+/*
+ * The form of MLA each layer runs on this handle (bit l set: the per-head
+ * form, K, V = split(c_kv W_up^KV) with scores over d_h; clear: the absorbed
+ * latent-space form).  For cost accounting; the result does not depend on it.
+ */
+int llatte_attn_form_mask(const llatte_handle* handle, uint32_t* per_head_layers);
 
 /* Bytes of device workspace a handle with these dims allocates (0 on bad dims). */
 size_t llatte_workspace_bytes(const llatte_dims* dims);

@@ -38,7 +38,8 @@ class llatte_dims(ctypes.Structure):
                 ("max_batch", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("max_total", ctypes.c_int64), ("n_sum", ctypes.c_int32),
                 ("sum_rank", ctypes.c_int32), ("d_seq", ctypes.c_int32),
-                ("q_rank", ctypes.c_int32), ("d_time", ctypes.c_int32)]
+                ("q_rank", ctypes.c_int32), ("d_time", ctypes.c_int32),
+                ("attn_form", ctypes.c_int32)]
 
 
 LAYER_KEYS = ("W_dkv", "g_kv", "W_q", "W_uk", "W_uv", "W_o", "g1", "W1", "W2", "g2",
@@ -72,7 +73,7 @@ EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
            "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
            "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export",
-           "llatte_forward_batch")
+           "llatte_forward_batch", "llatte_attn_form_mask")
 PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
@@ -149,6 +150,7 @@ def make_dims(dims, max_batch: int, max_len: int, max_total: int = 0) -> llatte_
     c.d_seq = int(getattr(dims, "d_seq", 0))
     c.q_rank = int(getattr(dims, "q_rank", 0))
     c.d_time = int(getattr(dims, "d_time", 0))
+    c.attn_form = int(getattr(dims, "attn_form", 0))
     return c
 
 
@@ -215,6 +217,14 @@ class Llatte:
             raise LlatteError(rc, "llatte_create")
         self.h = h
         self.last_B = 0
+
+    def per_head_layers(self) -> int:
+        """Bit l set: layer l runs MLA in its per-head form on this handle."""
+        m = ctypes.c_uint32(0)
+        rc = self.lib.llatte_attn_form_mask(self.h, ctypes.byref(m))
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_attn_form_mask")
+        return int(m.value)
 
     def workspace_bytes(self) -> int:
         return int(self.lib.llatte_workspace_bytes(ctypes.byref(self.cdims)))

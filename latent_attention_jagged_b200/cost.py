@@ -14,6 +14,12 @@ Per user and layer, with T history rows in, n = min(T, keep) kept, q = n + n_q:
   o       2 q h r d
   ffn1    2 q d (m d)      ffn2  2 q (m d) d        (m = FFN multiplier)
   readout 2 d d_out per user (final layer)
+Layers that run MLA in its per-head form (K, V = split(c_kv W_up^KV), scores
+over d_h; same function) count what that form computes instead:
+  kv      2 T d r + 2 T r (2 h d_h)        (latent, then every head's K and V)
+  q       2 q d h d_h + 2 d_ctx h d_h
+  attn    4 h d_h P
+  o       2 q h d_h d
   summary 2 k R (n_q d + d_seq) per user: k sequence summaries, each a
           bottleneck of width R over the flattened n_q x d final query rows
           then the projection to d_seq (appendix A.2 item 4)
@@ -42,12 +48,13 @@ def visible_pairs(T: np.ndarray, n: np.ndarray, n_q: int) -> np.ndarray:
     return n_q * T + n * T - n * (n - 1) // 2
 
 
-def layer_work(lengths: Sequence[int], dims) -> List[LayerWork]:
+def layer_work(lengths: Sequence[int], dims, per_head_layers: int = 0) -> List[LayerWork]:
     T = np.asarray(lengths, dtype=np.int64)
     d, h, r, dc, m = dims.d, dims.heads, dims.rank, dims.d_ctx, dims.ffn_mult
     rq = getattr(dims, "q_rank", 0)
+    hd = h * dims.d_head
     out = []
-    for k in dims.keep:
+    for li, k in enumerate(dims.keep):
         n = np.minimum(T, k)
         q = n + dims.n_q
         P = visible_pairs(T, n, dims.n_q)
@@ -61,13 +68,18 @@ def layer_work(lengths: Sequence[int], dims) -> List[LayerWork]:
             "ffn1": 2.0 * q.sum() * d * m * d,
             "ffn2": 2.0 * q.sum() * m * d * d,
         }
+        if (per_head_layers >> li) & 1:
+            f["kv"] = 2.0 * T.sum() * d * r + 2.0 * T.sum() * r * 2 * hd
+            f["q"] = 2.0 * q.sum() * d * hd + 2.0 * B * dc * hd
+            f["attn"] = 4.0 * hd * P.sum()
+            f["o"] = 2.0 * q.sum() * hd * d
         out.append(LayerWork(T=T.copy(), n=n, q=q, pairs=P, flops=f))
         T = n
     return out
 
 
-def total_flops(lengths: Sequence[int], dims) -> float:
-    work = layer_work(lengths, dims)
+def total_flops(lengths: Sequence[int], dims, per_head_layers: int = 0) -> float:
+    work = layer_work(lengths, dims, per_head_layers)
     tot = sum(sum(w.flops.values()) for w in work)
     if dims.d_out:
         tot += 2.0 * len(lengths) * dims.d * dims.d_out
@@ -93,9 +105,9 @@ def summary_bytes(B: int, dims, elem: int = 2) -> float:
     return float(rows + w + B * k * dims.d_seq * 4)
 
 
-def flops_by_step(lengths: Sequence[int], dims) -> Dict[str, float]:
+def flops_by_step(lengths: Sequence[int], dims, per_head_layers: int = 0) -> Dict[str, float]:
     acc: Dict[str, float] = {}
-    for w in layer_work(lengths, dims):
+    for w in layer_work(lengths, dims, per_head_layers):
         for k, v in w.flops.items():
             acc[k] = acc.get(k, 0.0) + float(v)
     if dims.d_out:

@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(32 * kWarps, 4) attn_export_kernel(ExportArgs 
   // warp takes 32 keys at a time: every lane forms its partial dot products
   // with all 32 (each key row one coalesced read), then a transposed
   // reduction (31 shuffles) leaves key t0 + l's score in lane l
-  const E* q = (const E*)a.Qt + (m * a.heads + head) * r;
+  const E* q = (const E*)a.Qt + m * a.q_row + head * a.q_head;
   float qv[RV];
 #pragma unroll
   for (int j = 0; j < RV; ++j) {
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(32 * kWarps, 4) attn_export_kernel(ExportArgs 
     qv[j] = c < r ? to_f(q[c]) : 0.f;
   }
   for (int b = lane; b < a.n_hours; b += 32) sh[b] = 0.f;
-  const E* C = (const E*)a.C + a.hoff[u] * r;
+  const E* C = (const E*)a.C + a.hoff[u] * a.c_row + head * a.c_head;
   float mx = -INFINITY;
   for (int t0 = 0; t0 < T; t0 += 32) {
     float v[32];
@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(32 * kWarps, 4) attn_export_kernel(ExportArgs 
     for (int kk = 0; kk < 32; ++kk) {
       v[kk] = 0.f;
       if (t0 + kk < T) {
-        const E* c = C + (int64_t)(t0 + kk) * r;
+        const E* c = C + (int64_t)(t0 + kk) * a.c_row;
 #pragma unroll
         for (int j = 0; j < RV; ++j) {
           const int cc = lane + 32 * j;

@@ -55,6 +55,11 @@ struct LayerDev {
   void* W_dqx;     // [q_rank, d] query down-projection, x columns (low-rank query)
   float* W_dqc;    // [d_ctx, q_rank] fp32 its context columns, transposed (NULL if d_ctx == 0)
   void* g_q;       // [q_rank] query-latent RMSNorm gain
+  // per-head (non-absorbed) form of the layer, d_h = 64 (NULL otherwise)
+  void* W_qh;      // [h*d_h, d] W_q's x columns, scaled log2(e)/sqrt(d_h)
+  float* W_qhc;    // [d_ctx, h*d_h] fp32 its context columns (same scale), transposed
+  void* W_ukv;     // [2*h*d_h, r] W_uk stacked on W_uv
+  void* W_oh;      // [d, h*d_h] W_o
   void* W_ov;      // [d, h*r]   absorbed W_o W_uv
   void* g1;        // [d]
   void* W1;        // [f, d]
@@ -65,7 +70,10 @@ struct LayerDev {
 struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
-struct LayerMaps { CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq; };
+struct LayerMaps {
+  CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq;
+  CUtensorMap qh, ukv, oh, oh_pair;     // per-head form
+};
 
 }  // namespace llatte
 
@@ -122,6 +130,11 @@ struct llatte_handle {
   int pair_norm;                  // output / FFN-down projections on SM pairs (d = 512)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
   CUtensorMap tm_zraw, tm_sdown;  // summary bottleneck GEMM operands
+  // per-head attention form: bit l = layer l runs it; its K | V rows, and the
+  // query / output rows laid out [rows, h*d_h] (in the Qt / Ot memory)
+  uint32_t heads_mask;
+  void* KV;                       // [max_rows_h, 2*h*d_h]
+  CUtensorMap tm_Qh, tm_KV, tm_Oh;
   CUtensorMap tm_sh16, tm_sup;    // summary output-projection GEMM operands
 
   // attention-probability export requested for the forward in progress
@@ -203,14 +216,21 @@ struct AttnArgs {
 cudaError_t launch_attn_simt(int elem, const AttnArgs& a, cudaStream_t s);
 
 // Per-user context term of every layer's absorbed query projection.
-struct CtxWeights { const float* W[LLATTE_MAX_LAYERS]; };   // [d_ctx, h*r] per layer
-// out[l][b][n] (fp32), or out16 (fp16) when out16 != NULL; N columns.
-cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int N,
-                            int dc, float* out, __half* out16, cudaStream_t s);
-// Split a [rows, d + dc] matrix into its first d columns (storage type, [rows, d])
-// and its last dc columns (fp32, transposed: [dc, rows]).
+// Per layer l: W[l] [d_ctx, N[l]] fp32; the term of user u, column n goes to
+// element off[l] + u * N[l] + n of the output.
+struct CtxWeights {
+  const float* W[LLATTE_MAX_LAYERS];
+  int N[LLATTE_MAX_LAYERS];
+  int64_t off[LLATTE_MAX_LAYERS];
+};
+// out (fp32), or out16 (fp16) when out16 != NULL, laid out as CtxWeights says;
+// N_max = the largest N[l].
+cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B,
+                            int N_max, int dc, float* out, __half* out16, cudaStream_t s);
+// Split scale * (a [rows, d + dc] matrix) into its first d columns (storage
+// type, [rows, d]) and its last dc columns (fp32, transposed: [dc, rows]).
 cudaError_t launch_split_ctx_cols(int elem, const void* src, int rows, int d, int dc, void* dst_x,
-                                  float* dst_c, cudaStream_t s);
+                                  float* dst_c, float scale, cudaStream_t s);
 
 // Sequence summaries after the bottleneck GEMM: H = SiLU(sum of the S split-K
 // partial rows) (reduce), then out[b, k, :] = H[b, k-block] W_up,k^T (up, on
@@ -236,6 +256,10 @@ struct ExportArgs {
   const int64_t *qoff, *hoff, *evoff;            // layer query / history offsets, input offsets
   const int32_t *T, *n, *T0;                     // layer keys, kept history rows, input lengths
   int B, n_q, heads, r, n2, n_k, n_hours, log2_scores;
+  // element strides: query (row m, head j) at Qt + m q_row + j q_head; key
+  // row t of head j at C + t c_row + j c_head (absorbed: h r, r, r, 0;
+  // per-head form: h 64, 64, 2 h 64, 64 with C = the K | V rows)
+  int64_t q_row, q_head, c_row, c_head;
   const float* event_age;                        // [sum T0] hours, or NULL
   float *recent, *topk, *hours;                  // [B, n_q, h, n_k] x2, [B, n_q, h, n_hours]
 };

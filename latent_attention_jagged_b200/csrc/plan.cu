@@ -64,7 +64,7 @@ __device__ void block_exscan2(int64_t a, int64_t b, int64_t* out_a, int64_t* out
 // keep_0, ..., keep_{l-1}), so the layers need not wait for one another.
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep, int L, int n_q,
-            int64_t max_len, int64_t max_total, int heads, int attn_keys) {
+            int64_t max_len, int64_t max_total, int heads, int attn_keys, uint32_t heads_mask) {
   __shared__ int s_err;
   const int tid = threadIdx.x;
   const int l = blockIdx.x;
@@ -135,31 +135,38 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   if (attn_keys <= 0 || l == L) return;
 
   // Attention work list of layer l: one item per (user, block of 128 (query
-  // row, head) pairs), ordered by the number of key tiles the block visits,
-  // largest first (a counting sort over at most kBuckets cost classes), so
-  // that the persistent attention CTAs take the longest items first.
+  // row, head) pairs) -- or, for a layer in the per-head form (bit l of
+  // heads_mask), per (user, 128-row block, head) with b = block * heads + head
+  // -- ordered by the number of key tiles the block visits, largest first (a
+  // counting sort over at most kBuckets cost classes), so that the persistent
+  // attention CTAs take the longest items first.
   constexpr int kBuckets = 64;
   __shared__ int32_t hist[kBuckets], cursor[kBuckets];
   __shared__ int32_t total_items;
   const int32_t* Tl = p.T + l * bstride;
   const int32_t* nl = p.n + l * bstride;
   int32_t* item_off = p.item_off + l * p.stride;
+  const bool per_head = (heads_mask >> l) & 1u;
+  auto items_of = [&](int u) -> int64_t {
+    const int64_t q = (int64_t)nl[u] + n_q;
+    return per_head ? ((q + 127) / 128) * heads : (q * heads + 127) / 128;
+  };
   if (tid < kBuckets) hist[tid] = 0;
   // items per user and their exclusive scan (item_off[u] = first item of u)
   int64_t cnt = 0;
-  for (int u = u0; u < u1; ++u) cnt += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+  for (int u = u0; u < u1; ++u) cnt += items_of(u);
   int64_t base, dummy, total, dummy2;
   block_exscan2(cnt, 0, &base, &dummy, &total, &dummy2);
   for (int u = u0; u < u1; ++u) {
     item_off[u] = (int32_t)base;
-    base += (((int64_t)nl[u] + n_q) * heads + 127) / 128;
+    base += items_of(u);
   }
   if (tid == 0) item_off[B] = (int32_t)total;
   __syncthreads();
   auto cost_of = [&](int u, int b) {
     const int64_t q = (int64_t)nl[u] + n_q;
-    const int64_t last = min((int64_t)b * 128 + 127, q * heads - 1);
-    const int64_t jl = last / heads;
+    const int64_t jl = per_head ? min((int64_t)(b / heads) * 128 + 127, q - 1)
+                                : min((int64_t)b * 128 + 127, q * heads - 1) / heads;
     const int64_t kmax = jl < nl[u] ? (int64_t)Tl[u] - nl[u] + jl + 1 : (int64_t)Tl[u];
     const int64_t tiles = (kmax + attn_keys - 1) / attn_keys;
     return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
@@ -202,7 +209,8 @@ cudaError_t launch_plan(const llatte_handle* h, const int64_t* offsets, int B, c
   const int L = h->dims.n_layers;
   for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < L ? h->dims.keep[i] : 0;
   plan_kernel<<<L + 1, kPlanThreads, 0, s>>>(offsets, B, h->plan, k, L, h->dims.n_q, h->dims.max_len,
-                                          h->max_rows_h, h->dims.heads, h->use_tc ? h->attn_keys : 0);
+                                          h->max_rows_h, h->dims.heads, h->use_tc ? h->attn_keys : 0,
+                                          h->heads_mask);
   return cudaGetLastError();
 }
 
@@ -211,7 +219,7 @@ cudaError_t launch_plan_on(const PlanDev& p, const llatte_dims& d, int64_t max_t
   KeepArr k;
   for (int i = 0; i <= LLATTE_MAX_LAYERS; ++i) k.k[i] = i < d.n_layers ? d.keep[i] : 0;
   plan_kernel<<<d.n_layers + 1, kPlanThreads, 0, s>>>(offsets, B, p, k, d.n_layers, d.n_q, d.max_len,
-                                          max_total, d.heads, 0);
+                                          max_total, d.heads, 0, 0u);
   return cudaGetLastError();
 }
 

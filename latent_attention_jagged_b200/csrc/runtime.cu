@@ -40,10 +40,12 @@ struct Layout {
       off_work_count, off_work_next, off_item_off, off_row_user;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_Cq, off_acc32, off_ctxbias,
       off_final, off_mean, off_Zres, off_Xqres[2], off_zraw, off_sum_part, off_sum_h,
-      off_sum_h16;
+      off_sum_h16, off_KV;
   size_t total;
   int32_t max_work;
 };
+
+uint32_t heads_mask_of(const llatte_dims& D);
 
 int check_dims(const llatte_dims* d) {
   if (!d) return LLATTE_ERR_ARG;
@@ -57,6 +59,7 @@ int check_dims(const llatte_dims* d) {
   if (d->n_sum < 0 || d->n_sum > LLATTE_MAX_SUMMARIES) return LLATTE_ERR_ARG;
   if (d->q_rank < 0) return LLATTE_ERR_ARG;
   if (d->d_time < 0 || d->d_time % 2 != 0 || d->d_time > d->d) return LLATTE_ERR_ARG;
+  if (d->attn_form < LLATTE_ATTN_AUTO || d->attn_form > LLATTE_ATTN_PER_HEAD) return LLATTE_ERR_ARG;
   if (d->q_rank > 1024) return LLATTE_ERR_UNSUPPORTED;
   if (d->n_sum > 0) {
     if (d->n_q <= 0 || d->d_out > 0 || d->sum_rank <= 0 || d->d_seq <= 0) return LLATTE_ERR_ARG;
@@ -69,6 +72,7 @@ int check_dims(const llatte_dims* d) {
   const int elem = d->dtype == LLATTE_BF16 ? 2 : 4;
   if ((d->d * elem) % 16 != 0) return LLATTE_ERR_UNSUPPORTED;     // 16-byte row vectors
   if (d->rank > 256) return LLATTE_ERR_UNSUPPORTED;
+  if (d->attn_form == LLATTE_ATTN_PER_HEAD && heads_mask_of(*d) == 0) return LLATTE_ERR_UNSUPPORTED;
   return LLATTE_OK;
 }
 
@@ -81,7 +85,8 @@ Layout layout_of(const llatte_dims* d) {
   const int64_t hr = (int64_t)d->heads * d->rank, f = (int64_t)d->ffn_mult * d->d;
   const int nl = d->n_layers;
   // attention work items: (user, 128-row block of (query row, head) pairs)
-  const int64_t max_work = (L.rows_q * d->heads + 127) / 128 + B;
+  // (absorbed: blocks of 128 (row, head) pairs; per-head: h blocks per 128 rows)
+  const int64_t max_work = (L.rows_q * d->heads + 127) / 128 + B * d->heads;
   L.max_work = (int32_t)std::min<int64_t>(max_work, 1 << 30);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o += align_up(bytes); return r; };
@@ -104,6 +109,8 @@ Layout layout_of(const llatte_dims* d) {
   L.off_Z = take((size_t)L.rows_q * d->d * elem);
   L.off_Hd = take((size_t)L.rows_q * f * elem);
   L.off_Cq = take((size_t)L.rows_q * d->q_rank * elem);
+  const int64_t hdh = (int64_t)d->heads * d->d_head;
+  L.off_KV = take(heads_mask_of(*d) ? (size_t)L.rows_h * 2 * hdh * elem : 0);
   // fp16 copies of the residual stream (bf16 storage keeps bf16 GEMM operands
   // plus these; fp32 storage needs none)
   const size_t res16 = elem == 2 ? 2 * (size_t)L.rows_q * d->d : 0;
@@ -115,7 +122,8 @@ Layout layout_of(const llatte_dims* d) {
                                          (size_t)L.rows_q * d->q_rank));
   // per-user context term of every layer's query: h*r columns (full-rank
   // query), or q_rank columns (low-rank query: it enters before the norm)
-  L.off_ctxbias = take(sizeof(float) * nl * B * std::max<int64_t>(hr, d->q_rank));
+  L.off_ctxbias = take(sizeof(float) * nl * B *
+                       std::max<int64_t>(std::max<int64_t>(hr, d->q_rank), hdh));
   L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
   L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
   // sequence summaries: the final query-token rows and the split-K partials
@@ -214,6 +222,19 @@ bool tc_dims_ok(const llatte_dims& D) {
   return d_ok && r_ok && q_ok && hr % 64 == 0 && f % 64 == 0;
 }
 
+// Layers that run MLA in its per-head form (K, V = split(c_kv W_up^KV),
+// scores over d_h = 64).  Both forms compute the same function; per layer the
+// per-head one does 4 d_h / (4 r) of the absorbed attention's tensor work and
+// smaller query / output projections, at the price of one up-projection of
+// the keys, so "auto" takes it when r > 2 d_h.
+uint32_t heads_mask_of(const llatte_dims& D) {
+  const bool possible = D.dtype == LLATTE_BF16 && tc_dims_ok(D) && D.d_head == 64 &&
+                        D.q_rank == 0;
+  if (!possible || D.attn_form == LLATTE_ATTN_ABSORBED) return 0;
+  if (D.attn_form == LLATTE_ATTN_AUTO && D.rank <= 2 * D.d_head) return 0;
+  return D.n_layers >= 32 ? 0xffffffffu : ((1u << D.n_layers) - 1);
+}
+
 int pick_bn(int N) { return N % 256 == 0 ? 256 : N % 128 == 0 ? 128 : 64; }
 
 bool build_tc_maps(llatte_handle* h) {
@@ -241,6 +262,13 @@ bool build_tc_maps(llatte_handle* h) {
   h->pair_norm = tc_gemm_pair_supported(TC_NORM, d, hr) && tc_gemm_pair_supported(TC_NORM, d, f);
   ok = ok && make_tmap_bf16(&h->tm_Qt, h->Qt, rq * D.heads, r, 128);
   ok = ok && make_tmap_bf16(&h->tm_C, h->C, rh, r, (uint32_t)h->attn_keys);
+  const int hdh = D.heads * D.d_head;
+  if (h->heads_mask) {
+    ok = ok && make_tmap_bf16(&h->tm_Qh, h->Qt, rq, hdh, 128);
+    ok = ok && make_tmap_bf16(&h->tm_KV, h->KV, rh, 2 * hdh, 128);
+    ok = ok && make_tmap_bf16(&h->tm_Oh, h->Ot, rq, hdh, 128);
+    h->pair_norm = h->pair_norm && tc_gemm_pair_supported(TC_NORM, d, hdh);
+  }
   auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
   for (int l = 0; l < D.n_layers && ok; ++l) {
     const LayerDev& W = h->layers[l];
@@ -248,6 +276,12 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.dkv, W.W_dkv, r, d, box(h->bn_kv));
     ok = ok && make_tmap_bf16(&M.qk, W.W_qk, hr, kq, box(h->bn_q));
     if (D.q_rank) ok = ok && make_tmap_bf16(&M.dq, W.W_dqx, D.q_rank, d, box(h->bn_dq));
+    if ((h->heads_mask >> l) & 1u) {
+      ok = ok && make_tmap_bf16(&M.qh, W.W_qh, hdh, d, box(pick_bn(hdh)));
+      ok = ok && make_tmap_bf16(&M.ukv, W.W_ukv, 2 * hdh, r, box(pick_bn(2 * hdh)));
+      ok = ok && make_tmap_bf16(&M.oh, W.W_oh, d, hdh, box(h->bn_o));
+      if (h->pair_norm) ok = ok && make_tmap_bf16(&M.oh_pair, W.W_oh, d, hdh, 128);
+    }
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
@@ -346,6 +380,8 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   // The tensor-core attention takes its scores in log2 units (exp2 in the
   // softmax): fold log2(e) into the absorbed query projection for that path.
   const bool want_tc = h->elem == 2 && tc_dims_ok(D);
+  const uint32_t heads_mask = want_tc ? heads_mask_of(D) : 0u;
+  h->heads_mask = heads_mask;
   const float qscale = want_tc ? 1.4426950408889634f : 1.0f;
   for (int l = 0; l < D.n_layers; ++l) {
     const llatte_layer_w& w = layers[l];
@@ -371,7 +407,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
                  cudaMemcpy(tdq, w.W_dq, e * (size_t)rq * (d + dc),
                             weights_on_device ? cudaMemcpyDeviceToDevice
                                               : cudaMemcpyHostToDevice) == cudaSuccess &&
-                 launch_split_ctx_cols(h->elem, tdq, rq, d, dc, L.W_dqx, L.W_dqc, 0) ==
+                 launch_split_ctx_cols(h->elem, tdq, rq, d, dc, L.W_dqx, L.W_dqc, 1.f, 0) ==
                      cudaSuccess &&
                  cudaDeviceSynchronize() == cudaSuccess;
       cudaFree(tdq);
@@ -380,6 +416,30 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
     if (!L.W_dkv || !L.g_kv || !L.g1 || !L.W1 || !L.W2 || !L.g2 || !L.W_qk || !L.W_ov ||
         (kqc && !L.W_qkc))
       return fail(LLATTE_ERR_OOM);
+    L.W_qh = L.W_ukv = L.W_oh = nullptr;
+    L.W_qhc = nullptr;
+    if ((heads_mask >> l) & 1u) {
+      // per-head form: W_q scaled by log2(e) / sqrt(d_h) (scores in log2
+      // units), split into x and context columns; [W_uk ; W_uv]; W_o
+      L.W_qh = dev_alloc(h, e * (size_t)hd * d);
+      L.W_qhc = dc ? (float*)dev_alloc(h, sizeof(float) * (size_t)dc * hd) : nullptr;
+      L.W_ukv = dev_alloc(h, e * (size_t)2 * hd * r);
+      L.W_oh = upload(h, w.W_o, e * (size_t)d * hd, weights_on_device);
+      if (!L.W_qh || (dc && !L.W_qhc) || !L.W_ukv || !L.W_oh) return fail(LLATTE_ERR_OOM);
+      void* tw = nullptr;
+      const cudaMemcpyKind kk = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+      bool okh = cudaMalloc(&tw, e * (size_t)hd * (d + dc)) == cudaSuccess &&
+                 cudaMemcpy(tw, w.W_q, e * (size_t)hd * (d + dc), kk) == cudaSuccess &&
+                 launch_split_ctx_cols(h->elem, tw, hd, d, dc, L.W_qh, L.W_qhc,
+                                       1.4426950408889634f / sqrtf((float)D.d_head), 0) ==
+                     cudaSuccess &&
+                 cudaMemcpy(L.W_ukv, w.W_uk, e * (size_t)hd * r, kk) == cudaSuccess &&
+                 cudaMemcpy((char*)L.W_ukv + e * (size_t)hd * r, w.W_uv, e * (size_t)hd * r, kk) ==
+                     cudaSuccess &&
+                 cudaDeviceSynchronize() == cudaSuccess;
+      cudaFree(tw);
+      if (!okh) return fail(LLATTE_ERR_CUDA);
+    }
     // temporaries for absorption
     void *tq = nullptr, *tuk = nullptr, *tuv = nullptr, *to = nullptr;
     bool ok = cudaMalloc(&tq, e * (size_t)hd * (kq + kqc)) == cudaSuccess &&
@@ -464,6 +524,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->Z = ws + Lo.off_Z;
   h->Hd = ws + Lo.off_Hd;
   h->Cq = rq ? (void*)(ws + Lo.off_Cq) : nullptr;
+  h->KV = heads_mask ? (void*)(ws + Lo.off_KV) : nullptr;
   h->Zres = h->elem == 2 ? (void*)(ws + Lo.off_Zres) : nullptr;
   for (int i = 0; i < 2; ++i) h->Xqres[i] = h->elem == 2 ? (void*)(ws + Lo.off_Xqres[i]) : nullptr;
   h->acc32 = (float*)(ws + Lo.off_acc32);
@@ -541,13 +602,25 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
   // the plan and the gather run here; the first query projection waits for it.
   // With a low-rank query the term belongs to the down-projection (before
   // its RMSNorm): q_rank columns, fp16 for the tensor-core norm epilogue.
+  // Per-head layers take the term of their non-absorbed W_q (h*d_h columns).
   bool ctx_join = false;
   const int rq = D.q_rank;
-  const int ctx_n = rq ? rq : hr;
+  const int hdh = D.heads * D.d_head;
   __half* ctx16 = (rq && h->use_tc) ? (__half*)h->ctxbias : nullptr;
+  CtxWeights cw = {};
+  int ctx_n = 0;
+  {
+    int64_t off = 0;
+    for (int l = 0; l < L; ++l) {
+      const bool ph = (h->heads_mask >> l) & 1u;
+      cw.W[l] = rq ? h->layers[l].W_dqc : (ph ? h->layers[l].W_qhc : h->layers[l].W_qkc);
+      cw.N[l] = rq ? rq : (ph ? hdh : hr);
+      cw.off[l] = off;
+      off += (int64_t)B * cw.N[l];
+      ctx_n = std::max(ctx_n, cw.N[l]);
+    }
+  }
   if (D.d_ctx > 0) {
-    CtxWeights cw = {};
-    for (int l = 0; l < L; ++l) cw.W[l] = rq ? h->layers[l].W_dqc : h->layers[l].W_qkc;
     if (h->profiling) {
       StepTimer t(h, s, ST_CTX);
       CK(launch_ctx_bias(e, context, cw, L, B, ctx_n, D.d_ctx, h->ctxbias, ctx16, s));
@@ -570,6 +643,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     void* Xh_n = h->Xh[(l + 1) & 1];
     void* Xq_n = h->Xq[(l + 1) & 1];
     const bool last = l == L - 1;
+    const bool per_head = (h->heads_mask >> l) & 1u;   // MLA in its non-absorbed form
 
     const bool tc = h->use_tc != 0;
     // epilogue arguments shared by both paths
@@ -615,7 +689,15 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.D = (__nv_bfloat16*)h->C; q.ldd = r;
         CK(launch_tc_gemm(h->bn_kv, D.kv_norm ? TC_NORM : TC_STORE, h->tm_Xh[l & 1], LM.dkv, q,
                           h->num_sms, s));
-        t.done(1);
+        if (per_head) {
+          // K | V = c_kv [W_uk ; W_uv]^T, every head's keys and values
+          TcGemmParams k2 = tcp(p.hist_total(l), h->max_rows_h, 2 * hdh, r);
+          k2.D = (__nv_bfloat16*)h->KV; k2.ldd = 2 * hdh;
+          CK(launch_tc_gemm(pick_bn(2 * hdh), TC_STORE, h->tm_C, LM.ukv, k2, h->num_sms, s));
+          t.done(2);
+        } else {
+          t.done(1);
+        }
       } else {
         GemmArgs g = {};
         g.A = Xh_l; g.lda = d; g.W = W.W_dkv; g.M_dev = p.hist_total(l); g.M_max = h->max_rows_h;
@@ -639,7 +721,16 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         ctx_join = false;
       }
       StepTimer t(h, s, ST_Q);
-      if (rq) {
+      if (per_head) {
+        // per-head query rows [rows, h*d_h] = R W_q,x^T + context term
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hdh, d);
+        q.D = (__nv_bfloat16*)h->Qt; q.ldd = hdh;
+        q.bias = h->ctxbias + cw.off[l]; q.seg_off = p.qoff(l); q.B = B;
+        q.row_user = p.ruser(l);
+        CK(launch_tc_gemm(pick_bn(hdh), D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1],
+                          LM.qh, q, h->num_sms, s));
+        t.done(1);
+      } else if (rq) {
         // low-rank query: Cq = RMSNorm_{g_q}(R W_dq,x^T + context term of the
         // row's user), then the absorbed projection Qt = Cq (W_uk^T W_uq)^T
         NormArgs qn = {};
@@ -647,7 +738,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         qn.M_max = h->max_rows_q; qn.mode = NORM_PLAIN; qn.dst = h->Cq;
         if (tc) {
           if (D.d_ctx > 0) {
-            qn.resid = ctx16 + (int64_t)l * B * rq; qn.resid_kind = RES_F16;
+            qn.resid = ctx16 + cw.off[l]; qn.resid_kind = RES_F16;
             qn.resid_user = p.ruser(l);
           }
           TcGemmParams q1 = tcp(p.query_total(l), h->max_rows_q, rq, d);
@@ -662,7 +753,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
           g.A = Xq_l; g.lda = d; g.W = W.W_dqx; g.D = h->acc32; g.ldd = rq;
           g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = rq; g.K = d;
           g.epi = D.d_ctx > 0 ? EPI_USERBIAS_F32 : EPI_F32;
-          g.bias = h->ctxbias + (int64_t)l * B * rq; g.seg_off = p.qoff(l); g.B = B;
+          g.bias = h->ctxbias + cw.off[l]; g.seg_off = p.qoff(l); g.B = B;
           CK(launch_gemm_simt(e, e, 4, g, s));
           qn.acc = h->acc32;
           CK(launch_rownorm(e, qn, s));
@@ -676,7 +767,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
       } else if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, hr, d);
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
-        q.bias = h->ctxbias + (int64_t)l * B * hr; q.seg_off = p.qoff(l); q.B = B;
+        q.bias = h->ctxbias + cw.off[l]; q.seg_off = p.qoff(l); q.B = B;
         q.row_user = p.ruser(l);
         CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1], LM.qk,
                           q, h->num_sms, s));
@@ -685,7 +776,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
         g.M_dev = p.query_total(l); g.M_max = h->max_rows_q; g.N = hr; g.K = d;
         g.epi = D.d_ctx > 0 ? EPI_USERBIAS : EPI_STORE;
-        g.bias = h->ctxbias + (int64_t)l * B * hr; g.seg_off = p.qoff(l); g.B = B;
+        g.bias = h->ctxbias + cw.off[l]; g.seg_off = p.qoff(l); g.B = B;
         CK(launch_gemm_simt(e, e, e, g, s));
       }
       if (!rq) t.done(1);
@@ -697,7 +788,8 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
       a.max_items = p.max_work; a.T = p.Tl(l); a.n = p.nl(l); a.hoff = p.hoff(l);
       a.qoff = p.qoff(l); a.n_q = D.n_q; a.heads = D.heads; a.Ot = (__nv_bfloat16*)h->Ot;
       a.status = p.status;
-      CK(launch_attn_tc(r, h->tm_Qt, h->tm_C, a, h->num_sms, s));
+      if (per_head) CK(launch_attn_tc_heads(h->tm_Qh, h->tm_KV, a, h->num_sms, s));
+      else CK(launch_attn_tc(r, h->tm_Qt, h->tm_C, a, h->num_sms, s));
       t.done(1);
     } else {  // latent attention, CUDA cores
       StepTimer t(h, s, ST_ATTN);
@@ -711,9 +803,11 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     if (h->export_req && h->export_req->layer == l) {  // attention statistics of this layer
       const llatte_attn_export& ex = *h->export_req;
       ExportArgs x = {};
-      x.Qt = h->Qt; x.C = h->C; x.qoff = p.qoff(l); x.hoff = p.hoff(l); x.evoff = offsets;
-      x.T = p.Tl(l); x.n = p.nl(l); x.T0 = p.Tl(0);
-      x.B = B; x.n_q = D.n_q; x.heads = D.heads; x.r = r;
+      x.Qt = h->Qt; x.C = per_head ? h->KV : h->C; x.qoff = p.qoff(l); x.hoff = p.hoff(l);
+      x.evoff = offsets; x.T = p.Tl(l); x.n = p.nl(l); x.T0 = p.Tl(0);
+      x.B = B; x.n_q = D.n_q; x.heads = D.heads; x.r = per_head ? 64 : r;
+      if (per_head) { x.q_row = hdh; x.q_head = 64; x.c_row = 2 * hdh; x.c_head = 64; }
+      else { x.q_row = (int64_t)D.heads * r; x.q_head = r; x.c_row = r; x.c_head = 0; }
       int n2 = 1;
       while (n2 < D.max_len) n2 <<= 1;
       x.n2 = n2; x.n_k = ex.n_k; x.n_hours = ex.n_hours; x.log2_scores = tc ? 1 : 0;
@@ -726,10 +820,13 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     {  // output projection + residual + RMSNorm
       StepTimer t(h, s, ST_O);
       if (tc) {
-        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, hr);
+        TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, d, per_head ? hdh : hr);
         q.norm = o_norm;
-        if (h->pair_norm) CK(launch_tc_gemm_pair(TC_NORM, h->tm_Ot, LM.ov_pair, q, h->num_sms, s));
-        else CK(launch_tc_gemm(h->bn_o, TC_NORM, h->tm_Ot, LM.ov, q, h->num_sms, s));
+        const CUtensorMap& oa = per_head ? h->tm_Oh : h->tm_Ot;
+        if (h->pair_norm)
+          CK(launch_tc_gemm_pair(TC_NORM, oa, per_head ? LM.oh_pair : LM.ov_pair, q, h->num_sms, s));
+        else
+          CK(launch_tc_gemm(h->bn_o, TC_NORM, oa, per_head ? LM.oh : LM.ov, q, h->num_sms, s));
         t.done(1);
       } else {
         GemmArgs g = {};
@@ -890,6 +987,12 @@ int llatte_get_status(llatte_handle* h, int32_t* device_status) {
   CK(cudaMemset(h->plan.status, 0, sizeof(int32_t)));
   *device_status = v;
   return v ? LLATTE_ERR_DEVICE : LLATTE_OK;
+}
+
+int llatte_attn_form_mask(const llatte_handle* h, uint32_t* per_head_layers) {
+  if (!h || !per_head_layers) return LLATTE_ERR_ARG;
+  *per_head_layers = h->heads_mask;
+  return LLATTE_OK;
 }
 
 int llatte_set_profiling(llatte_handle* h, int enable) {

@@ -264,7 +264,7 @@ constexpr int CTX_COLS = 128;
 
 template <typename T>
 __global__ void __launch_bounds__(CTX_COLS)
-ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
+ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int dc,
                 float* __restrict__ out, __half* __restrict__ out16) {
   extern __shared__ float cs[];                       // [CTX_USERS][dc]
   const int l = blockIdx.y;
@@ -276,6 +276,7 @@ ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
   }
   __syncthreads();
   const int n = blockIdx.x * CTX_COLS + threadIdx.x;
+  const int hr = w.N[l];
   if (n >= hr) return;
   const float* W = w.W[l] + n;
   float acc[CTX_USERS] = {};
@@ -286,7 +287,7 @@ ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
     for (int uu = 0; uu < CTX_USERS; ++uu) acc[uu] = fmaf(cs[uu * dc + k], wk, acc[uu]);
   }
   for (int uu = 0; uu < nu; ++uu) {
-    const int64_t o = ((int64_t)l * B + u0 + uu) * hr + n;
+    const int64_t o = w.off[l] + (int64_t)(u0 + uu) * hr + n;
     if (out16) out16[o] = __float2half_rn(acc[uu]);
     else out[o] = acc[uu];
   }
@@ -294,14 +295,15 @@ ctx_bias_kernel(const T* __restrict__ ctx, CtxWeights w, int B, int hr, int dc,
 
 cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int L, int B, int hr,
                             int dc, float* out, __half* out16, cudaStream_t s) {
+  // hr: the widest layer; each layer's block uses its own width w.N[l]
   if (B == 0 || dc == 0) return cudaSuccess;
   dim3 grid((hr + CTX_COLS - 1) / CTX_COLS, L, (B + CTX_USERS - 1) / CTX_USERS);
   const size_t sm = sizeof(float) * CTX_USERS * dc;
   if (elem == 4)
-    ctx_bias_kernel<float><<<grid, CTX_COLS, sm, s>>>((const float*)ctx, w, B, hr, dc, out, out16);
+    ctx_bias_kernel<float><<<grid, CTX_COLS, sm, s>>>((const float*)ctx, w, B, dc, out, out16);
   else
-    ctx_bias_kernel<__nv_bfloat16><<<grid, CTX_COLS, sm, s>>>((const __nv_bfloat16*)ctx, w, B, hr,
-                                                             dc, out, out16);
+    ctx_bias_kernel<__nv_bfloat16><<<grid, CTX_COLS, sm, s>>>((const __nv_bfloat16*)ctx, w, B, dc,
+                                                             out, out16);
   return cudaGetLastError();
 }
 
@@ -529,26 +531,28 @@ cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const voi
 
 template <typename T>
 __global__ void split_ctx_cols_kernel(const T* __restrict__ src, int rows, int d, int dc,
-                                      T* __restrict__ dst_x, float* __restrict__ dst_c) {
+                                      T* __restrict__ dst_x, float* __restrict__ dst_c,
+                                      float scale) {
   const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
   const int K = d + dc;
   if (i >= (int64_t)rows * K) return;
   const int row = (int)(i / K), col = (int)(i % K);
-  if (col < d) dst_x[(int64_t)row * d + col] = src[i];
-  else dst_c[(int64_t)(col - d) * rows + row] = to_f(src[i]);
+  const float v = to_f(src[i]) * scale;          // one rounding into the storage type
+  if (col < d) dst_x[(int64_t)row * d + col] = from_f<T>(v);
+  else dst_c[(int64_t)(col - d) * rows + row] = v;
 }
 
 cudaError_t launch_split_ctx_cols(int elem, const void* src, int rows, int d, int dc, void* dst_x,
-                                  float* dst_c, cudaStream_t s) {
+                                  float* dst_c, float scale, cudaStream_t s) {
   const int64_t n = (int64_t)rows * (d + dc);
   if (n <= 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (elem == 4)
     split_ctx_cols_kernel<float><<<blocks, 256, 0, s>>>((const float*)src, rows, d, dc,
-                                                         (float*)dst_x, dst_c);
+                                                         (float*)dst_x, dst_c, scale);
   else
     split_ctx_cols_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)src, rows, d, dc, (__nv_bfloat16*)dst_x, dst_c);
+        (const __nv_bfloat16*)src, rows, d, dc, (__nv_bfloat16*)dst_x, dst_c, scale);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@ struct AttnTcParams {
   const int32_t *T, *n;       // per user: history rows (keys) and kept rows
   const int64_t *hoff, *qoff; // per user: first key row, first query row
   int n_q, heads;
-  __nv_bfloat16* Ot;          // [sum q * heads, r]
+  __nv_bfloat16* Ot;          // [sum q * heads, r]; per-head form: [sum q, heads * 64]
   int32_t* status;
 };
 
@@ -22,5 +22,10 @@ int attn_tc_keys(int r);
 bool attn_tc_supported(int r);
 cudaError_t launch_attn_tc(int r, const CUtensorMap& q, const CUtensorMap& c,
                            const AttnTcParams& p, int num_sms, cudaStream_t s);
+// Per-head form (d_h = 64): q over [sum q, heads * 64] (128-row boxes), kv over
+// [sum T, 2 * heads * 64] (K then V, 128-row boxes); work items (user,
+// 128-row block * heads + head).
+cudaError_t launch_attn_tc_heads(const CUtensorMap& q, const CUtensorMap& kv,
+                                 const AttnTcParams& p, int num_sms, cudaStream_t s);
 
 }  // namespace llatte

@@ -46,8 +46,9 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_struct_layout_matches_header(lib):
     # int32 x 7, keep[16], 4 x int32, float, int32, (pad 4), int64, int64,
-    # int32 x 5 (n_sum, sum_rank, d_seq, q_rank, d_time), (pad 4)
+    # int32 x 6 (n_sum, sum_rank, d_seq, q_rank, d_time, attn_form)
     assert ctypes.sizeof(binding.llatte_dims) == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16 + 24
+    assert binding.llatte_dims.attn_form.offset == binding.llatte_dims.d_time.offset + 4
     assert binding.llatte_dims.n_sum.offset == 4 * (7 + 16 + 4 + 1 + 1) + 4 + 16
     assert binding.llatte_dims.q_rank.offset == binding.llatte_dims.d_seq.offset + 4
     assert ctypes.sizeof(binding.llatte_layer_w) == 13 * ctypes.sizeof(ctypes.c_void_p)
@@ -99,6 +100,9 @@ def test_create_rejects_bad_arguments_on_host(lib):
         assert lib.llatte_workspace_bytes(ctypes.byref(bad)) == 0
     for kw, code in ((dict(q_rank=-1), binding.LLATTE_ERR_ARG),
                      (dict(d_time=3), binding.LLATTE_ERR_ARG),
+                     (dict(attn_form=3), binding.LLATTE_ERR_ARG),
+                     (dict(attn_form=2, q_rank=64), binding.LLATTE_ERR_UNSUPPORTED),
+                     (dict(attn_form=2, d_head=32, heads=8), binding.LLATTE_ERR_UNSUPPORTED),
                      (dict(d_time=512), binding.LLATTE_ERR_ARG),
                      (dict(q_rank=2048), binding.LLATTE_ERR_UNSUPPORTED)):
         bad = _cdims(**kw)

@@ -39,6 +39,8 @@ class Dims:
              (0 = the full-rank query W_Q [x; c])
     d_time   hidden dims carrying the additive timestamp encoding of history
              tokens (even; 0 = none)
+    attn_form which form of MLA the GPU runs (0 auto, 1 absorbed, 2 per
+             head); both compute the same function, the oracle ignores it
     """
 
     d: int
@@ -58,6 +60,7 @@ class Dims:
     d_seq: int = 0
     q_rank: int = 0
     d_time: int = 0
+    attn_form: int = 0
 
     @property
     def n_layers(self) -> int:
