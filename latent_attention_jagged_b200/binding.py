@@ -120,6 +120,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_plan_static.restype = ctypes.c_int
     lib.llatte_exp2_eval.argtypes = [VP, VP, VP, I64, VP]
     lib.llatte_exp2_eval.restype = ctypes.c_int
+    lib.llatte_attn_form_mask.argtypes = [VP, P(ctypes.c_uint32)]
+    lib.llatte_attn_form_mask.restype = ctypes.c_int
     if path is None:
         _lib = lib
     return lib
