@@ -33,10 +33,10 @@ from workloads import draw_lengths, make_event_ages, make_inputs, workload  # no
 from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 
 # ncu-measured DRAM traffic per launch (bytes, mean over one forward's layers)
-# of the dominant kernel, keyed by (step, workload); taken from the committed
+# of the dominant kernel, keyed by (step, workload, MLA form); taken from the committed
 # profiles/dram_traffic_dominant_kernels.md.  Absent = not captured for the
 # current kernel version.
-TRAFFIC = {("ffn", "online"): 7.2008e7, ("attn", "upstream"): 2.5609e8}
+TRAFFIC = {("ffn", "online", "absorbed"): 7.2008e7, ("attn", "upstream", "absorbed"): 2.5609e8}
 
 
 def load_peaks():
@@ -178,6 +178,12 @@ def main():
                          "workload's)")
     ap.add_argument("--export-layer", type=int, default=-1,
                     help="also export the attention statistics of this layer in every step")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="users per batch instead of the workload's (a smaller case for "
+                         "profiler captures; the JSON line then names that batch)")
+    ap.add_argument("--tokenize", action="store_true",
+                    help="each step also builds the history tokens from action ids with the "
+                         "MLP_act tokenizer (per-field embedding tables) before the forward")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every kernel eagerly instead of replaying one CUDA graph")
     args = ap.parse_args()
@@ -191,6 +197,9 @@ def main():
     if args.attn_form is not None:
         import dataclasses
         wl = dataclasses.replace(wl, dims=dataclasses.replace(wl.dims, attn_form=args.attn_form))
+    if args.batch is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, batch=int(args.batch))
 
     if args.impl == "reference":
         if rank == 0:
@@ -257,7 +266,24 @@ def main():
         elif args.export_layer >= 0:
             ages = torch.from_numpy(make_event_ages(inp.lengths, seed=wl.seed + 77)).cuda()
 
+        # optional action tokenizer: the step starts from per-field ids
+        tok = ids = None
+        if args.tokenize:
+            from latent_attention_jagged_b200 import Tokenizer
+            from workloads.tokens import TOKENIZERS, make_token_inputs
+            tdims = next((t for t in TOKENIZERS.values()
+                          if t.d == inp.dims.d and t.dtype == inp.dims.dtype), None)
+            if tdims is None:
+                raise SystemExit(f"no tokenizer workload of width {inp.dims.d}")
+            ti = make_token_inputs(tdims, int(inp.offsets[-1]), seed=wl.seed + 501)
+            tok_tables = [torch.from_numpy(t).cuda().to(dt).contiguous() for t in ti.tables]
+            tok = Tokenizer(tok_tables, ti.W_a1, ti.W_a2, dtype=tdims.dtype,
+                            max_events=max(1, int(inp.offsets[-1])))
+            ids = torch.from_numpy(ti.ids).cuda()
+
         def fwd():
+            if tok is not None:
+                tok(ids, out=values)
             if args.export_layer >= 0:
                 h.forward_export(values, offsets, ctx, cand, layer=args.export_layer, n_k=11,
                                  event_age=ages, n_hours=168, out=out)
@@ -318,9 +344,35 @@ def main():
         prof = h.profile()
         h.set_profiling(False)
         launches_per_fwd = sum(v["launches"] for v in prof.values()) / prof_steps
+        tok_res = None
+        if tok is not None:
+            # the tokenizer alone, timed the same way (3 kernels per call)
+            evt = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(prof_steps)]
+            for a, b in evt:
+                flush.fill_(1)
+                a.record(stream)
+                tok(ids, out=values)
+                b.record(stream)
+            torch.cuda.synchronize()
+            t_ms = sum(a.elapsed_time(b) for a, b in evt) / prof_steps
+            n_ev = int(inp.offsets[-1])
+            t_flops = n_ev * cost.tokenizer_flops(tdims)
+            t_bytes = n_ev * cost.tokenizer_bytes(tdims)
+            tok_res = {"ms": t_ms, "events": n_ev, "launches": 3,
+                       "tensor_cores": tok.uses_tensor_cores(),
+                       "achieved_tflops": t_flops / (t_ms / 1e3) / 1e12,
+                       "frac_of_tensor_peak": t_flops / (t_ms / 1e3) / 1e12
+                       / peaks["bf16_tflops_sustained"],
+                       "achieved_gbs": t_bytes / (t_ms / 1e3) / 1e9,
+                       "frac_of_hbm": t_bytes / (t_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                       "algorithmic_flops": t_flops, "algorithmic_bytes": t_bytes}
+            launches_per_fwd += 3
 
         # ---- end to end: pinned host inputs -> device -> forward -> host output
-        hv = torch.from_numpy(inp.values).to(dt).pin_memory()
+        # (with the tokenizer the host sends the action ids instead of the tokens)
+        hv = (ids.cpu() if tok is not None else torch.from_numpy(inp.values).to(dt)).pin_memory()
+        dv = ids if tok is not None else values
         ho = torch.from_numpy(inp.offsets).pin_memory()
         hc = torch.from_numpy(inp.ctx).to(dt).pin_memory() if inp.dims.d_ctx else None
         hq = torch.from_numpy(inp.cand).to(dt).pin_memory() if inp.dims.n_q else None
@@ -334,7 +386,7 @@ def main():
         for a, b in ev2:
             flush.fill_(1)
             a.record(stream)
-            values.copy_(hv, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
             offsets.copy_(ho, non_blocking=True)
             if hc is not None:
                 ctx.copy_(hc, non_blocking=True)
@@ -367,7 +419,7 @@ def main():
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peaks['source']} sustained bf16 (cuBLAS loop)",
-                "traffic": TRAFFIC.get((dom, wl.name)),
+                "traffic": TRAFFIC.get((dom, wl.name, "per_head" if ph else "absorbed")),
                 "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms}
         # the sequence-summary step (bottleneck GEMM + up-projection), when the
         # workload has one, against HBM: the final rows and both projections
@@ -391,9 +443,11 @@ def main():
         res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
                    clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
                    dtype=inp.dims.dtype, users_all=users_all, summary=summary,
-                   per_head_layers=ph)
+                   per_head_layers=ph, tokenizer=tok_res)
         del graph
         h.close()
+        if tok is not None:
+            tok.close()
         return res
 
     main_res = measure(wl, args.steps, args.warmup, sample_clocks=(rank == 0))
@@ -433,6 +487,7 @@ def main():
             "clocks": main_res["clocks"],
             "steps_ms": main_res["steps_ms"],
             "summary": main_res["summary"],
+            "tokenizer": main_res["tokenizer"],
             "second": second,
         }
         print(json.dumps(line), flush=True)

@@ -77,7 +77,8 @@ enum {
   LLATTE_DEV_BAD_OFFSETS = 1,   /* offsets decrease or are negative            */
   LLATTE_DEV_TOO_LONG = 2,      /* a history longer than max_len               */
   LLATTE_DEV_TOO_MANY_ROWS = 4, /* sum of lengths above max_total              */
-  LLATTE_DEV_TIMEOUT = 8        /* a bounded device wait gave up               */
+  LLATTE_DEV_TIMEOUT = 8,       /* a bounded device wait gave up               */
+  LLATTE_DEV_BAD_ID = 16        /* tokenizer: an id outside its embedding table */
 };
 
 /*
@@ -342,6 +343,80 @@ int llatte_forward_export(llatte_handle* handle, const void* values, const int64
  */
 int llatte_forward_batch(llatte_handle* handle, const llatte_batch* batch, float* out,
                          const llatte_attn_export* ex, void* stream);
+
+/*
+ * Action tokenizer (appendix A.2 item 1 "Action Embeddings"): every history
+ * event a_t = (tau_t, type_t, item_t, surface_t, meta_t) is embedded field by
+ * field and projected to one token,
+ *     x_t = MLP_act(E_type(type_t), E_item(item_t), E_surface(surface_t),
+ *                   E_time(tau_t), E_meta(meta_t)) in R^d.
+ * The pages name the parts and give no formula; the reading taken: each field
+ * (the timestamp as its time-bucket id) is an integer id into its own table,
+ * the embeddings are concatenated in field order, and
+ *     x_t = W_a2 SiLU(W_a1 [e_1 ; ... ; e_F]),  no biases.
+ * The tokens are the `values` rows of llatte_forward (same jagged layout).
+ *
+ *   n_fields        1 .. LLATTE_TOK_MAX_FIELDS tables
+ *   rows[f]         rows of table f;  width[f] its embedding width, with
+ *                   width[f] * element size a multiple of 16 bytes
+ *                   (sum of widths = D_in, D_in * element size <= 2048 B)
+ *   d_hid, d        hidden and token width (d * element size a multiple of 16)
+ *   dtype           LLATTE_BF16 (tensor cores when D_in, d_hid are multiples
+ *                   of 64 and d_hid, d of 64, else CUDA cores) or LLATTE_FP32
+ *   max_events      most events one call may tokenize (<= 65535 * 64)
+ */
+#define LLATTE_TOK_MAX_FIELDS 8
+typedef struct {
+  int32_t n_fields;
+  int64_t rows[LLATTE_TOK_MAX_FIELDS];
+  int32_t width[LLATTE_TOK_MAX_FIELDS];
+  int32_t d_hid, d, dtype;
+  int64_t max_events;
+} llatte_tok_dims;
+
+/*
+ * Tokenizer parameters, in dtype, row-major:
+ *   tables[f]  device [rows[f], width[f]], 16-byte aligned: NOT copied; the
+ *              caller owns them and keeps them alive and unchanged while the
+ *              tokenizer is used (embedding tables can be far larger than
+ *              the rest of the model)
+ *   W_a1       [d_hid, D_in]   W_a2 [d, d_hid]: copied at create (host memory
+ *              if weights_on_device == 0, else device memory)
+ */
+typedef struct {
+  const void* tables[LLATTE_TOK_MAX_FIELDS];
+  const void *W_a1, *W_a2;
+} llatte_tok_w;
+
+typedef struct llatte_tokenizer llatte_tokenizer;
+
+/* Create a tokenizer on the current device (synchronous); it owns copies of
+ * W_a1, W_a2 and a workspace of max_events rows of D_in + d_hid elements. */
+int llatte_tokenizer_create(llatte_tokenizer** tok, const llatte_tok_dims* dims,
+                            const llatte_tok_w* weights, int weights_on_device);
+
+/*
+ * Tokens of n events, asynchronous on `stream`, no host synchronisation.
+ *   ids     device int32 [n, n_fields], 4-byte aligned: event t's id per field
+ *   n       0 <= n <= max_events (0 launches nothing)
+ *   tokens  device [n, d] in dtype, 16-byte aligned: x_t for every event,
+ *           ready to pass as llatte_forward's `values`
+ * An id outside its table sets LLATTE_DEV_BAD_ID in the tokenizer's status
+ * word and contributes a zero embedding (no out-of-range read).  Calls on
+ * one tokenizer must not overlap in time (they share its workspace).
+ */
+int llatte_tokenize(llatte_tokenizer* tok, const int32_t* ids, int64_t n, void* tokens,
+                    void* stream);
+
+/* Synchronise the device, read the status word and clear it (as
+ * llatte_get_status does for a forward handle). */
+int llatte_tokenizer_get_status(llatte_tokenizer* tok, int32_t* device_status);
+
+/* 1 when the two MLP_act GEMMs run on the tensor cores, 0 on CUDA cores. */
+int llatte_tokenizer_uses_tensor_cores(const llatte_tokenizer* tok);
+
+/* Free the tokenizer (synchronises its device); the tables stay the caller's. */
+void llatte_tokenizer_destroy(llatte_tokenizer* tok);
 
 /* Free the handle and everything it owns (synchronises its device). */
 void llatte_destroy(llatte_handle* handle);

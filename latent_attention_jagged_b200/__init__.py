@@ -7,6 +7,6 @@ opened when a handle is created, and a missing library is an error.
 from . import cost
 
 __all__ = ["cost"]
-from .binding import Llatte, LlatteError, load_library  # noqa: E402  (no library load here)
+from .binding import Llatte, LlatteError, Tokenizer, load_library  # noqa: E402  (no library load here)
 
-__all__ += ["Llatte", "LlatteError", "load_library"]
+__all__ += ["Llatte", "LlatteError", "Tokenizer", "load_library"]

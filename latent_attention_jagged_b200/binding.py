@@ -20,7 +20,7 @@ STEPS = ("plan", "gather", "ctx_bias", "kv", "q", "attn", "o", "ffn1", "ffn2", "
 LLATTE_OK, LLATTE_ERR_ARG, LLATTE_ERR_UNSUPPORTED, LLATTE_ERR_CUDA, LLATTE_ERR_OOM, \
     LLATTE_ERR_DEVICE = 0, -1, -2, -3, -4, -5
 LLATTE_BF16, LLATTE_FP32 = 0, 1
-DEV_BAD_OFFSETS, DEV_TOO_LONG, DEV_TOO_MANY_ROWS, DEV_TIMEOUT = 1, 2, 4, 8
+DEV_BAD_OFFSETS, DEV_TOO_LONG, DEV_TOO_MANY_ROWS, DEV_TIMEOUT, DEV_BAD_ID = 1, 2, 4, 8, 16
 
 
 class LlatteError(RuntimeError):
@@ -63,6 +63,17 @@ class llatte_batch(ctypes.Structure):
                 ("event_age", ctypes.c_void_p)]
 
 
+class llatte_tok_dims(ctypes.Structure):
+    _fields_ = [("n_fields", ctypes.c_int32), ("rows", ctypes.c_int64 * 8),
+                ("width", ctypes.c_int32 * 8), ("d_hid", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("max_events", ctypes.c_int64)]
+
+
+class llatte_tok_w(ctypes.Structure):
+    _fields_ = [("tables", ctypes.c_void_p * 8), ("W_a1", ctypes.c_void_p),
+                ("W_a2", ctypes.c_void_p)]
+
+
 class llatte_attn_export(ctypes.Structure):
     _fields_ = [("layer", ctypes.c_int32), ("n_k", ctypes.c_int32), ("n_hours", ctypes.c_int32),
                 ("event_age", ctypes.c_void_p), ("recent", ctypes.c_void_p),
@@ -73,7 +84,10 @@ EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_
            "llatte_workspace_bytes", "llatte_error_string", "llatte_destroy",
            "llatte_set_profiling", "llatte_profile_reset", "llatte_profile_step",
            "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export",
-           "llatte_forward_batch", "llatte_attn_form_mask")
+           "llatte_forward_batch", "llatte_attn_form_mask", "llatte_tokenizer_create",
+           "llatte_tokenize", "llatte_tokenizer_get_status", "llatte_tokenizer_uses_tensor_cores",
+           "llatte_tokenizer_destroy")
+TOK_MAX_FIELDS = 8
 PLAN_STATIC_MAX_BATCH = 4096
 
 _lib = None
@@ -122,6 +136,17 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_exp2_eval.restype = ctypes.c_int
     lib.llatte_attn_form_mask.argtypes = [VP, P(ctypes.c_uint32)]
     lib.llatte_attn_form_mask.restype = ctypes.c_int
+    lib.llatte_tokenizer_create.argtypes = [P(VP), P(llatte_tok_dims), P(llatte_tok_w),
+                                            ctypes.c_int]
+    lib.llatte_tokenizer_create.restype = ctypes.c_int
+    lib.llatte_tokenize.argtypes = [VP, VP, I64, VP, VP]
+    lib.llatte_tokenize.restype = ctypes.c_int
+    lib.llatte_tokenizer_get_status.argtypes = [VP, P(I32)]
+    lib.llatte_tokenizer_get_status.restype = ctypes.c_int
+    lib.llatte_tokenizer_uses_tensor_cores.argtypes = [VP]
+    lib.llatte_tokenizer_uses_tensor_cores.restype = ctypes.c_int
+    lib.llatte_tokenizer_destroy.argtypes = [VP]
+    lib.llatte_tokenizer_destroy.restype = None
     if path is None:
         _lib = lib
     return lib
@@ -407,3 +432,81 @@ def exp2_eval(x: torch.Tensor, with_hw: bool = True, stream=None):
     if rc != LLATTE_OK:
         raise LlatteError(rc, "llatte_exp2_eval")
     return (y, y_hw) if with_hw else y
+
+
+class Tokenizer:
+    """Action tokenizer MLP_act: x_t = W_a2 SiLU(W_a1 [E_1(id_t1); ...; E_F(id_tF)]).
+
+    `tables` are CUDA tensors [rows_f, width_f] in the storage dtype that the
+    tokenizer references (not copied): they must stay alive and unchanged.
+    W_a1 [d_hid, D_in] and W_a2 [d, d_hid] are copied."""
+
+    def __init__(self, tables, W_a1, W_a2, dtype: str = "bf16", max_events: int = 1 << 20):
+        self.lib = load_library()
+        self.dt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
+        if not 1 <= len(tables) <= TOK_MAX_FIELDS:
+            raise ValueError(f"1 .. {TOK_MAX_FIELDS} tables")
+        self.tables = []
+        for t in tables:
+            if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == self.dt
+                    and t.dim() == 2 and t.is_contiguous()):
+                raise ValueError("tables must be contiguous 2-D CUDA tensors of the storage dtype")
+            self.tables.append(t)
+        w1, w2 = _host(W_a1, self.dt), _host(W_a2, self.dt)
+        c = llatte_tok_dims()
+        c.n_fields = len(tables)
+        for f, t in enumerate(tables):
+            c.rows[f], c.width[f] = int(t.shape[0]), int(t.shape[1])
+        c.d_hid, c.d = int(w1.shape[0]), int(w2.shape[0])
+        if w1.shape[1] != sum(int(t.shape[1]) for t in tables) or w2.shape[1] != c.d_hid:
+            raise ValueError("W_a1 must be [d_hid, sum of widths], W_a2 [d, d_hid]")
+        c.dtype = LLATTE_BF16 if dtype == "bf16" else LLATTE_FP32
+        c.max_events = int(max_events)
+        self.cdims = c
+        self.d = c.d
+        w = llatte_tok_w()
+        for f, t in enumerate(tables):
+            w.tables[f] = t.data_ptr()
+        w.W_a1, w.W_a2 = w1.data_ptr(), w2.data_ptr()
+        h = ctypes.c_void_p()
+        rc = self.lib.llatte_tokenizer_create(ctypes.byref(h), ctypes.byref(c), ctypes.byref(w), 0)
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_tokenizer_create")
+        self.h = h
+
+    def uses_tensor_cores(self) -> bool:
+        return self.lib.llatte_tokenizer_uses_tensor_cores(self.h) == 1
+
+    def __call__(self, ids: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        """Tokens [n, d] of ids (int32 CUDA [n, n_fields])."""
+        if (not ids.is_cuda or ids.dtype != torch.int32 or ids.dim() != 2
+                or ids.shape[1] != self.cdims.n_fields or not ids.is_contiguous()):
+            raise ValueError("ids must be a contiguous CUDA int32 [n, n_fields] tensor")
+        n = int(ids.shape[0])
+        if out is None:
+            out = torch.empty((n, self.d), dtype=self.dt, device=ids.device)
+        elif (tuple(out.shape) != (n, self.d) or out.dtype != self.dt or not out.is_contiguous()):
+            raise ValueError(f"out must be a contiguous {self.dt} [{n}, {self.d}] tensor")
+        rc = self.lib.llatte_tokenize(self.h, _ptr(ids), n, _ptr(out), _stream_ptr(stream))
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_tokenize")
+        return out
+
+    def status(self) -> int:
+        v = ctypes.c_int32(0)
+        rc = self.lib.llatte_tokenizer_get_status(self.h, ctypes.byref(v))
+        if rc not in (LLATTE_OK, LLATTE_ERR_DEVICE):
+            raise LlatteError(rc, "llatte_tokenizer_get_status")
+        return int(v.value)
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.llatte_tokenizer_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -136,3 +136,16 @@ def io_bytes(lengths: Sequence[int], dims, elem: int = 2) -> float:
     else:
         out = B * (dims.d_out if dims.d_out else dims.n_q * d) * 4
     return float(inp + w + out)
+
+
+def tokenizer_flops(tdims) -> float:
+    """Algorithmic FLOPs of the action tokenizer per event: the two MLP_act
+    products, 2 D_in d_hid + 2 d_hid d."""
+    return 2.0 * tdims.d_in * tdims.d_hid + 2.0 * tdims.d_hid * tdims.d
+
+
+def tokenizer_bytes(tdims) -> float:
+    """Algorithmic bytes of the action tokenizer per event: its ids read, its
+    embedding rows read once, its token written once (storage type)."""
+    e = 2 if tdims.dtype == "bf16" else 4
+    return 4.0 * tdims.n_fields + e * tdims.d_in + e * tdims.d

@@ -118,3 +118,40 @@ def test_forward_and_status_reject_null_handle(lib):
     assert lib.llatte_plan_export(None, None, None) == binding.LLATTE_ERR_ARG
     lib.llatte_destroy(None)
     assert lib.llatte_error_string(binding.LLATTE_ERR_DEVICE).startswith(b"device")
+
+
+def test_tokenizer_struct_layout_and_host_checks(lib):
+    # int32 (+4 pad), int64 x 8, int32 x 8, int32 x 3 (+4 pad), int64
+    assert ctypes.sizeof(binding.llatte_tok_dims) == 8 + 64 + 32 + 16 + 8
+    assert binding.llatte_tok_dims.max_events.offset == 120
+    assert ctypes.sizeof(binding.llatte_tok_w) == 10 * ctypes.sizeof(ctypes.c_void_p)
+    t = ctypes.c_void_p()
+    w = binding.llatte_tok_w()
+
+    def dims(**kw):
+        c = binding.llatte_tok_dims()
+        f = dict(n_fields=2, rows=(10, 20), width=(8, 8), d_hid=64, d=64,
+                 dtype=binding.LLATTE_BF16, max_events=100)
+        f.update(kw)
+        c.n_fields = f["n_fields"]
+        for i, (r, wd) in enumerate(zip(f["rows"], f["width"])):
+            c.rows[i], c.width[i] = r, wd
+        c.d_hid, c.d, c.dtype, c.max_events = f["d_hid"], f["d"], f["dtype"], f["max_events"]
+        return c
+
+    for kw, code in ((dict(n_fields=0), binding.LLATTE_ERR_ARG),
+                     (dict(n_fields=9), binding.LLATTE_ERR_ARG),
+                     (dict(rows=(0, 20)), binding.LLATTE_ERR_ARG),
+                     (dict(width=(8, 4)), binding.LLATTE_ERR_UNSUPPORTED),     # 8-byte rows
+                     (dict(width=(1024, 8)), binding.LLATTE_ERR_UNSUPPORTED),  # E row > 2 KB
+                     (dict(d=60), binding.LLATTE_ERR_UNSUPPORTED),
+                     (dict(dtype=7), binding.LLATTE_ERR_ARG),
+                     (dict(max_events=-1), binding.LLATTE_ERR_ARG),
+                     (dict(), binding.LLATTE_ERR_ARG)):                      # null weights
+        c = dims(**kw)
+        assert lib.llatte_tokenizer_create(ctypes.byref(t), ctypes.byref(c), ctypes.byref(w),
+                                           0) == code
+    assert lib.llatte_tokenize(None, None, 1, None, None) == binding.LLATTE_ERR_ARG
+    v = ctypes.c_int32()
+    assert lib.llatte_tokenizer_get_status(None, ctypes.byref(v)) == binding.LLATTE_ERR_ARG
+    lib.llatte_tokenizer_destroy(None)
