@@ -187,11 +187,18 @@ struct StepTimer {
       cudaEventRecord(a, s);
     }
   }
+  // Records the step's end once; the start event then belongs to the record
+  // (a second call would put one event into two records).
   void done(int launches) {
-    if (!h->profiling) return;
+    if (!h->profiling || !a) return;
     cudaEvent_t b = take_event(h);
     cudaEventRecord(b, s);
     h->pending.push_back(ProfRec{step, a, b, launches});
+    a = nullptr;
+  }
+  // A step left early (an error return) hands its start event back.
+  ~StepTimer() {
+    if (a) h->event_pool.push_back(a);
   }
 };
 
@@ -729,7 +736,6 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.row_user = p.ruser(l);
         CK(launch_tc_gemm(pick_bn(hdh), D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1],
                           LM.qh, q, h->num_sms, s));
-        t.done(1);
       } else if (rq) {
         // low-rank query: Cq = RMSNorm_{g_q}(R W_dq,x^T + context term of the
         // row's user), then the absorbed projection Qt = Cq (W_uk^T W_uq)^T

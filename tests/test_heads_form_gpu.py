@@ -77,3 +77,24 @@ def test_export_in_a_per_head_layer():
     assert_close(rec.cpu().numpy().astype(np.float64), R, "bf16", "recent")
     assert_close(top.cpu().numpy().astype(np.float64), K, "bf16", "topk")
     assert_close(hrs.cpu().numpy().astype(np.float64), H, "bf16", "hours")
+
+
+@pytest.mark.parametrize("form", [ABSORBED, PER_HEAD])
+def test_profiled_steps_count_each_layer_once_and_handles_close(form):
+    """Per-step timing records each step once per layer in both forms, and a
+    profiled handle closes cleanly (its events are released exactly once)."""
+    inp = _force(make_inputs(workload("online"), batch=16), form)
+    L = inp.dims.n_layers
+    for _ in range(2):
+        h = make_handle(inp)
+        values, offsets, ctx, cand = to_device(inp)
+        h.set_profiling(True)
+        for _ in range(3):
+            h.forward(values, offsets, ctx, cand)
+        prof = h.profile()
+        assert h.status() == 0
+        for step in ("kv", "q", "attn", "o"):
+            assert prof[step]["calls"] == 3 * L, (step, prof[step])
+        h.profile_reset()
+        h.forward(values, offsets, ctx, cand)
+        h.close()
