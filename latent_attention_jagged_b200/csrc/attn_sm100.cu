@@ -395,9 +395,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
         const uint32_t s_addr = lane_base + Cfg::S_COL + (g & 1) * KEYS + part * KP;
         // keys [0, lim) of this warp's KP are visible to the row; masking is
-        // applied only when some row of the warp stops inside them
+        // applied only when some row of the warp stops inside them.  Rows past
+        // the user's last query row (the padding of its last block) are never
+        // stored, so they take every key and do not force the masked path.
         const int64_t lim64 = vis - (int64_t)kt * KEYS - part * KP;
-        const int lim = lim64 <= 0 ? 0 : (lim64 >= KP ? KP : (int)lim64);
+        const int lim = !valid ? KP : (lim64 <= 0 ? 0 : (lim64 >= KP ? KP : (int)lim64));
         const bool masked = __any_sync(0xffffffffu, lim < KP);
         float v[KP];
         tmem_ld_kp<KP>(s_addr, v);
