@@ -26,7 +26,8 @@
 // bytes of both CTAs are counted on rank 0's barriers), warp 1 TMEM owner
 // (in rank 0 the MMA issuer; in rank 1 it forwards that CTA's SiLU and
 // completions to rank 0 with one remote arrival each), warps 2..9 SiLU and
-// the OUT copy, warps 10..13 the row epilogue.  Completion of the pair MMAs is
+// the OUT copy, warps 10..17 the row epilogue (16 rows each: with four warps
+// the row epilogue set the pace of the whole tile).  Completion of the pair MMAs is
 // signalled to both CTAs at once (multicast commit).
 #include <cuda.h>
 
@@ -47,7 +48,8 @@ namespace {
 constexpr int D = 256;                      // model width handled here
 constexpr int HC = 128;                     // hidden chunk
 constexpr int kSiluWarps = 8;               // two per TMEM lane quadrant
-constexpr int kRowWarps = 4;                // row epilogue
+constexpr int kRowWarps = 8;                // row epilogue
+constexpr int kRowsPerWarp = 128 / kRowWarps;
 constexpr int kRowWarp0 = 2 + kSiluWarps;
 constexpr int kThreads = 32 * (2 + kSiluWarps + kRowWarps);
 constexpr int W_STAGES = 3;
@@ -275,20 +277,20 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
         if (!__all_sync(0xffffffffu, w1)) { ok = false; break; }
         tc_fence_after();
         // this warp's 64 hidden columns: SiLU -> bf16 pairs, written over the
-        // first 32 columns of its half of the buffer
+        // first 32 columns of its half of the buffer, 32 columns at a time
+        // (round 1 reads columns 32..63 and writes packed columns 16..31,
+        // which round 0 has already read)
         const uint32_t hcol = lane_base + H_COL + (gc & 1) * HC + half * 64;
-        float v[2][32];
-        tmem_ld32(hcol, v[0]);
-        tmem_ld32(hcol + 32, v[1]);
-        uint32_t pk[2][16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pk[0][i] = pack_bf16(silu_approx(v[0][2 * i]), silu_approx(v[0][2 * i + 1]));
-          pk[1][i] = pack_bf16(silu_approx(v[1][2 * i]), silu_approx(v[1][2 * i + 1]));
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+          tmem_ld32(hcol + 32 * h, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(silu_approx(v[2 * i]), silu_approx(v[2 * i + 1]));
+          tmem_st16u(hcol + 16 * h, pk);
+          tmem_wait_st();
         }
-        tmem_st16u(hcol, pk[0]);
-        tmem_st16u(hcol + 16, pk[1]);
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&hs_local[gc & 1]);
@@ -325,10 +327,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
     // ------------------------------------------------------------ row epilogue
     // Z + OUT, RMSNorm, gain, scatter into the next layer's rows (LLaTTE
     // notes, huaxiaozhuan.com, appendix A.2 display).  Warp w takes rows
-    // 32 (w - kRowWarp0) .. +32 of the CTA's 128; a row is one warp
-    // instruction wide: lane l owns columns [8 l, 8 l + 8).
+    // kRowsPerWarp (w - kRowWarp0) .. + kRowsPerWarp of the CTA's 128; a row
+    // is one warp instruction wide: lane l owns columns [8 l, 8 l + 8).
     const NormArgs& a = p.norm;
-    const int r0 = (warp - kRowWarp0) * 32;
+    const int r0 = (warp - kRowWarp0) * kRowsPerWarp;
     float g8[8];
     {
       const uint4 gw = reinterpret_cast<const uint4*>(sG)[lane];
@@ -341,16 +343,16 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       }
     }
     uint32_t ti = 0;
-    constexpr int RB = 8;                  // rows whose residual is in flight
+    constexpr int RB = kRowsPerWarp < 8 ? kRowsPerWarp : 8;   // rows whose residual is in flight
     for (int64_t t = pair; t < num_tiles; t += n_pairs, ++ti) {
       const int64_t row_base = t * 256 + 128 * rank;
-      // destinations of the warp's 32 rows, lane l -> row r0 + l, found before
+      // destinations of the warp's rows, lane l -> row r0 + l, found before
       // the data is ready (one round of dependent loads for all rows): the
       // next layer's history row, its query row, the final row (-1: none)
       int64_t h_dst = -1, q_dst = -1, f_dst = -1;
       {
         const int64_t row = row_base + r0 + lane;
-        if (row < M) {
+        if (lane < kRowsPerWarp && row < M) {
           const int u = a.row_user[row];
           const int64_t jr = row - a.qoff_l[u];
           const int32_t nl = a.n_l[u];
@@ -378,7 +380,7 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       bool w = mbar_wait(v_full, ti & 1, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w)) break;
 #pragma unroll 1
-      for (int rb = 0; rb < 32; rb += RB) {
+      for (int rb = 0; rb < kRowsPerWarp; rb += RB) {
         uint4 res[RB];
 #pragma unroll
         for (int i = 0; i < RB; ++i) {
