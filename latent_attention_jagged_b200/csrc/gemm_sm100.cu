@@ -1,21 +1,22 @@
 // Tensor-core GEMM for sm_100a: D[m, n] = sum_k A[m, k] W[n, k] (bf16 in,
 // fp32 accumulation in TMEM) with the layer's epilogues fused.
 //
-// Roles (320 threads, one CTA per SM, persistent over 128 x BN tiles):
+// Roles (576 threads, one CTA per SM, persistent over 128 x BN tiles):
 //   warp 0      TMA producer: A (128 x 64) and W (BN x 64) k-blocks into a
 //               STAGES-deep ring of 128-byte-swizzled shared-memory tiles
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (128 x NI x 16) and
 //               commits stage releases / accumulator-ready events
-//   warps 2..9  epilogue, two warps per TMEM lane quadrant, each taking half
-//               of the tile's columns: TMEM -> registers (tcgen05.ld), then one of
+//   warps 2..17 epilogue, four warps per TMEM lane quadrant, each taking a
+//               quarter of the tile's columns (a half for BN = 64; then two of
+//               the four idle): TMEM -> registers (tcgen05.ld), then one of
 //               STORE     bf16 store
 //               USERBIAS  + per-user context term (absorbed query projection)
 //               SILU      SiLU (FFN up-projection)
 //               F32       fp32 store (a split-K slice's partial sums, or one
 //                         member of a batch of products)
 //               NORM      + residual (read once: the sum is staged back in
-//                         TMEM), RMSNorm over the full row (BN == N; the two
-//                         halves' sums of squares meet in shared memory),
+//                         TMEM), RMSNorm over the full row (BN == N; the
+//                         parts' sums of squares meet in shared memory),
 //                         store bf16 (+ fp16 residual copy) or scatter into the
 //                         next layer's history / query rows (pyramid trimming)
 // The accumulator is double-buffered in TMEM when 2 * BN <= 512 columns, so
@@ -47,8 +48,13 @@ using namespace tc;
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kEpiWarps = 8;                        // two per TMEM lane quadrant
+// Four epilogue warps per TMEM lane quadrant: the epilogue (TMEM reads,
+// residual loads, row stores) is the longer leg of a tile, and with two warps
+// per quadrant it ran about twice as long as the tile's MMAs.
+constexpr int kParts = 4;
+constexpr int kEpiWarps = 4 * kParts;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr size_t kSmemMax = 232448;
 
 template <int BN>
 struct GemmCfg {
@@ -61,26 +67,32 @@ struct GemmCfg {
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN >= 512 ? 2 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
-  static constexpr size_t SMEM =
-      1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * 2 * 128 * 4 + kEpiWarps * kStageBytes +
-      BN * 2;
-  static_assert(SMEM <= 232448, "shared memory budget");
+  // epilogue warps that take part: kParts column parts of 32 or more columns
+  static constexpr int P = BN / 32 < kParts ? BN / 32 : kParts;
+  static constexpr size_t FIXED =
+      1024 + 256 + 2 * kParts * 128 * 4 + kEpiWarps * kStageBytes + BN * 2;
+  // as many stages as fit, at most 8
+  static constexpr int STAGES_FIT = (int)((kSmemMax - FIXED) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+  static constexpr size_t SMEM = FIXED + (size_t)STAGES * STAGE_BYTES;
+  static_assert(STAGES >= 2, "pipeline depth");
+  static_assert(SMEM <= kSmemMax, "shared memory budget");
 };
 
-// Epilogue of one 128 x BN tile.  Two warps share each TMEM lane quadrant;
-// `half` selects which half of the columns this thread handles.  Stores pass
-// through the warp's staging buffer `stg` (row-contiguous global writes).
+// Epilogue of one 128 x BN tile.  GemmCfg<BN>::P warps share each TMEM lane
+// quadrant; `part` selects which BN / P columns this thread handles.  Stores
+// pass through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
 __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0, int ks, int g, int half, float* red,
+                                         bool valid, int n0, int ks, int g, int part, float* red,
                                          int rrow, uint64_t* xbar, uint32_t& xphase,
                                          volatile int* abort_flag, uint32_t stg,
-                                         NormPre<BN, 4>& pre, const __nv_bfloat16* sg) {
-  constexpr int HB = BN / 2;                 // columns per thread
-  const int c0 = half * HB;
+                                         NormPre<BN, 1, GemmCfg<BN>::P>& pre,
+                                         const __nv_bfloat16* sg) {
+  constexpr int HB = BN / GemmCfg<BN>::P;    // columns per thread
+  const int c0 = part * HB;
   if constexpr (EPI == TC_NORM) {
-    return norm_epilogue(p.norm, taddr, row, valid, half, red, rrow, xbar, xphase,
+    return norm_epilogue(p.norm, taddr, row, valid, part, red, rrow, xbar, xphase,
                              abort_flag, p.status, stg, pre, sg);
   } else if constexpr (EPI == TC_F32) {
     float* prow =
@@ -106,8 +118,9 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
     int u = 0;
     if (EPI == TC_USERBIAS && valid) u = p.row_user[row];
     __nv_bfloat16* drow = valid ? p.D + row * p.ldd + n0 : nullptr;
-    constexpr int STEP = HB >= 64 ? 64 : 32;
-    // STEP columns per step; the bias loads are issued before the TMEM read
+    // 32 columns per step (the register budget of 576 threads); the bias
+    // loads are issued before the TMEM read
+    constexpr int STEP = 32;
 #pragma unroll 1
     for (int c = c0; c < c0 + HB; c += STEP) {
       const int n = n0 + c;
@@ -118,8 +131,7 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
         for (int j = 0; j < STEP / 4; ++j) b[j] = __ldg(bp + j);
       }
       float v[STEP];
-      if constexpr (STEP == 64) tmem_ld64(taddr + c, v);
-      else tmem_ld32(taddr + c, v);
+      tmem_ld32(taddr + c, v);
       if (EPI == TC_USERBIAS && valid) {
 #pragma unroll
         for (int j = 0; j < STEP / 4; ++j) {
@@ -159,8 +171,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* xbar = drain + 1;                 // epilogue group barrier (norm exchange)
   uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][2 halves][128]
-  uint8_t* sStage = (uint8_t*)(red + 2 * 2 * 128);                  // [epilogue warp][kStageBytes]
+  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][kParts][128]
+  uint8_t* sStage = (uint8_t*)(red + 2 * kParts * 128);             // [epilogue warp][kStageBytes]
   __nv_bfloat16* sG = (__nv_bfloat16*)(sStage + kEpiWarps * kStageBytes);   // RMSNorm gain [BN]
 
   pdl_trigger();
@@ -175,7 +187,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiWarps); }
     mbar_init(drain, 1);
-    mbar_init(xbar, kEpiWarps);
+    mbar_init(xbar, 4 * Cfg::P);              // the epilogue warps that take part
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -268,7 +280,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncwarp();
   } else {
     const int q = warp & 3;                // TMEM lane quadrant this warp may access
-    const int half = (warp - 2) >> 2;      // which half of the tile's columns
+    const int part = (warp - 2) >> 2;      // which part of the tile's columns
+    const bool active = part < Cfg::P;     // BN = 64: two parts, two warps idle
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     int acc = 0, it = 0;
     uint32_t acc_phase = 0, xphase = 0;
@@ -280,13 +293,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int mt = (int)(rem / n_tiles), nt = (int)(rem % n_tiles);
       const int rr = q * 32 + lane;
       const int64_t row = (int64_t)mt * BM + rr;
-      NormPre<BN, 4> pre;
-      if constexpr (EPI == TC_NORM) norm_prefetch(p.norm, row, row < M, half, pre);
+      NormPre<BN, 1, Cfg::P> pre;
+      if constexpr (EPI == TC_NORM) {
+        if (active) norm_prefetch(p.norm, row, row < M, part, pre);
+      }
       const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      if (!epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, g, half,
-                             red + (it & 1) * 256, rr, xbar, xphase, abort_flag,
+      if (active &&
+          !epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, g, part,
+                             red + (it & 1) * kParts * 128, rr, xbar, xphase, abort_flag,
                              smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
         break;
       tc_fence_before();

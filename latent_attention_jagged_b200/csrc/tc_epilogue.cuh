@@ -81,25 +81,28 @@ __device__ __forceinline__ void pack_bf16x32(const float* v, uint4 (&x)[4]) {
                       pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-// Residual chunks of this thread's half row held in registers: the first
-// PD 32-column chunks are fetched before the accumulator is ready (their
-// latency overlaps the wait); pass 1 refills each slot PD chunks ahead.
-template <int BN, int PDMAX = 4>
+// Residual chunks of this thread's part of the row held in registers (the
+// row's BN columns are split into P parts, one per warp of the lane
+// quadrant): the first PD 32-column chunks are fetched before the accumulator
+// is ready (their latency overlaps the wait); pass 1 refills each slot PD
+// chunks ahead.
+template <int BN, int PDMAX = 4, int P = 2>
 struct NormPre {
-  static constexpr int CH = BN / 64;            // 32-column chunks per half row
+  static constexpr int CH = BN / (32 * P);      // 32-column chunks per part
   static constexpr int PD = CH < PDMAX ? CH : PDMAX;   // chunks in flight
   uint4 t[PD][4];
 };
 
-template <int BN, int PDMAX>
+template <int BN, int PDMAX, int P>
 __device__ __forceinline__ void norm_prefetch(const NormArgs& a, int64_t row, bool valid,
-                                              int half, NormPre<BN, PDMAX>& pre) {
+                                              int part, NormPre<BN, PDMAX, P>& pre) {
   if (!a.resid) return;
   // a per-user residual (context term of a low-rank query) is row user(row)
   const int64_t res_row = (valid && a.resid_user) ? (int64_t)a.resid_user[row] : row;
-  const char* src = valid ? (const char*)a.resid + (res_row * BN + half * (BN / 2)) * 2 : nullptr;
+  const char* src = valid ? (const char*)a.resid + (res_row * BN + part * (BN / P)) * 2 : nullptr;
 #pragma unroll
-  for (int i = 0; i < NormPre<BN, PDMAX>::PD; ++i) stage_fetch(src ? src + 64 * i : nullptr, pre.t[i]);
+  for (int i = 0; i < NormPre<BN, PDMAX, P>::PD; ++i)
+    stage_fetch(src ? src + 64 * i : nullptr, pre.t[i]);
 }
 
 // Copy the RMSNorm gain (N bf16) into shared memory; every thread of the CTA
@@ -110,39 +113,42 @@ __device__ __forceinline__ void load_gain(const NormArgs& a, int N, __nv_bfloat1
 }
 
 // Residual + RMSNorm epilogue of one 128-row tile whose accumulator holds the
-// full row (BN == N columns, starting at taddr).  Two warps share each TMEM
-// lane quadrant and take half of the columns each; their partial sums of
-// squares meet in `red` ([2][128] floats) behind the group barrier `xbar`
+// full row (BN == N columns, starting at taddr).  P warps share each TMEM
+// lane quadrant and take BN / P of the columns each; their partial sums of
+// squares meet in `red` ([P][128] floats, added in part order so that every
+// part gets the same sum) behind the group barrier `xbar`
 // (bounded wait; returns false if the CTA is aborting).  Pass 1 reads the
 // accumulator, adds the residual (read once, from the chunks `pre` holds and
 // refills) and stages the sum back in TMEM; pass 2
 // normalises, applies the gain (`sg`, in shared memory) and stores.  Global
 // reads and writes go through the warp's staging buffer `stg`.
-template <int BN, int PDMAX>
+template <int BN, int PDMAX, int P>
 __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
-                                              bool valid, int half, float* red, int rrow,
+                                              bool valid, int part, float* red, int rrow,
                                               uint64_t* xbar, uint32_t& xphase,
                                               volatile int* abort_flag, int32_t* status,
-                                              uint32_t stg, NormPre<BN, PDMAX>& pre,
+                                              uint32_t stg, NormPre<BN, PDMAX, P>& pre,
                                               const __nv_bfloat16* sg) {
-  constexpr int HB = BN / 2;
-  const int c0 = half * HB;
+  constexpr int HB = BN / P;
+  const int c0 = part * HB;
   const int N = BN;
   const bool have = a.resid != nullptr;
   const int64_t res_row = (valid && have && a.resid_user) ? (int64_t)a.resid_user[row] : row;
   const char* rsrc = (valid && have) ? (const char*)a.resid + (res_row * N) * 2 : nullptr;
   // pass 1: v = acc + residual, partial sum of squares; v goes back to TMEM.
   float ss = 0.f;
-  constexpr int PD = NormPre<BN, PDMAX>::PD;
-#pragma unroll
-  for (int ci = 0; ci < NormPre<BN, PDMAX>::CH; ++ci) {
+  constexpr int PD = NormPre<BN, PDMAX, P>::PD;
+  // with one chunk in flight the loop need not be unrolled (the slot index is
+  // always 0), which keeps register pressure down at four parts per row
+#pragma unroll (PD == 1 ? 1 : NormPre<BN, PDMAX, P>::CH)
+  for (int ci = 0; ci < NormPre<BN, PDMAX, P>::CH; ++ci) {
     const int c = c0 + 32 * ci;
     float v[32];
     tmem_ld32(taddr + c, v);
     if (have) {
       uint4 rr[4];
       stage_deliver(stg, pre.t[ci % PD], rr);
-      if (ci + PD < NormPre<BN, PDMAX>::CH)
+      if (ci + PD < NormPre<BN, PDMAX, P>::CH)
         stage_fetch(rsrc ? rsrc + 2 * (c + 32 * PD) : nullptr, pre.t[ci % PD]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -167,9 +173,11 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
     for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     if (have) tmem_st32(taddr + c, v);
   }
-  red[half * 128 + rrow] = ss;
+  red[part * 128 + rrow] = ss;
   if (!group_sync(xbar, xphase, abort_flag, status)) return false;
-  ss += red[(half ^ 1) * 128 + rrow];
+  ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < P; ++q) ss += red[q * 128 + rrow];
   const float inv = rsqrtf(ss / (float)N + a.eps);
   // destinations of this row (null: none)
   __nv_bfloat16* d1 = nullptr;
@@ -214,8 +222,10 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   // pass 2: normalise, scale by the gain, store
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
-    float g[32];
+    float v[32];
+    tmem_ld32(taddr + c, v);
     {
+      // the gain, 8 columns (one 16-byte shared-memory load) at a time
       const uint32_t ga = smem_u32(sg + c);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -224,15 +234,11 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float2 f = __bfloat1622float2(h2[k]);
-          g[8 * j + 2 * k] = f.x;
-          g[8 * j + 2 * k + 1] = f.y;
+          v[8 * j + 2 * k] *= inv * f.x;
+          v[8 * j + 2 * k + 1] *= inv * f.y;
         }
       }
     }
-    float v[32];
-    tmem_ld32(taddr + c, v);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = v[i] * inv * g[i];
     uint4 x[4];
     if (any_d1 || any_d2) {
       pack_bf16x32(v, x);
