@@ -281,26 +281,38 @@ def main():
                             max_events=max(1, int(inp.offsets[-1])))
             ids = torch.from_numpy(ti.ids).cuda()
 
-        def fwd():
+        # device buffers of one step (a second set serves the end-to-end loop)
+        buf0 = dict(values=values, offsets=offsets, ctx=ctx, cand=cand, ages=ages, ids=ids,
+                    out=out)
+
+        def fwd_on(b):
             if tok is not None:
-                tok(ids, out=values)
+                tok(b["ids"], out=b["values"])
             if args.export_layer >= 0:
-                h.forward_export(values, offsets, ctx, cand, layer=args.export_layer, n_k=11,
-                                 event_age=ages, n_hours=168, out=out)
+                h.forward_export(b["values"], b["offsets"], b["ctx"], b["cand"],
+                                 layer=args.export_layer, n_k=11, event_age=b["ages"],
+                                 n_hours=168, out=b["out"])
             else:
-                h.forward(values, offsets, ctx, cand, out=out, event_age=ages)
+                h.forward(b["values"], b["offsets"], b["ctx"], b["cand"], out=b["out"],
+                          event_age=b["ages"])
+
+        def fwd():
+            fwd_on(buf0)
+
+        def capture(b):
+            # the whole forward as one CUDA graph (no host work between kernels)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fwd_on(b)
+            g.replay()
+            torch.cuda.synchronize()
+            return g
+
         for _ in range(warmup):
             fwd()
         torch.cuda.synchronize()
         assert h.status() == 0, "device status word set during warm-up"
-        # the whole forward as one CUDA graph (no host work between kernels)
-        graph = None
-        if args.graph:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                fwd()
-            graph.replay()
-            torch.cuda.synchronize()
+        graph = capture(buf0) if args.graph else None
 
         def step():
             if graph is not None:
@@ -369,44 +381,74 @@ def main():
                        "algorithmic_flops": t_flops, "algorithmic_bytes": t_bytes}
             launches_per_fwd += 3
 
-        # ---- end to end: pinned host inputs -> device -> forward -> host output
+        # ---- end to end: pinned host inputs -> device -> forward -> host output,
+        # double-buffered: step i's inputs are copied in on a copy stream while
+        # step i - 1 computes, and its result is copied out while step i + 1
+        # computes.  Every step's copies are inside the timed region, which
+        # runs from before the first copy-in to after the last copy-out; the L2
+        # flush before each step's forward is inside it too.
         # (with the tokenizer the host sends the action ids instead of the tokens)
-        hv = (ids.cpu() if tok is not None else torch.from_numpy(inp.values).to(dt)).pin_memory()
-        dv = ids if tok is not None else values
-        ho = torch.from_numpy(inp.offsets).pin_memory()
-        hc = torch.from_numpy(inp.ctx).to(dt).pin_memory() if inp.dims.d_ctx else None
-        hq = torch.from_numpy(inp.cand).to(dt).pin_memory() if inp.dims.n_q else None
-        ha = torch.from_numpy(inp.event_age).pin_memory() if inp.event_age is not None else None
-        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        def clone_set(b):
+            return {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in b.items()}
+
+        bufs = [buf0, clone_set(buf0)]
+        graphs = [graph, capture(bufs[1]) if args.graph else None]
+        src_names = ["ids" if tok is not None else "values", "offsets", "ctx", "cand"]
+        if inp.event_age is not None:
+            src_names.append("ages")
+        host = {"values": torch.from_numpy(inp.values).to(dt),
+                "ids": ids.cpu() if tok is not None else None,
+                "offsets": torch.from_numpy(inp.offsets),
+                "ctx": torch.from_numpy(inp.ctx).to(dt) if inp.dims.d_ctx else None,
+                "cand": torch.from_numpy(inp.cand).to(dt) if inp.dims.n_q else None,
+                "ages": torch.from_numpy(inp.event_age) if inp.event_age is not None else None}
+        host = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+        hout = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+        cs = torch.cuda.Stream()
         e2e_steps = max(3, min(steps, 50))
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(e2e_steps)]
+        EV = lambda: torch.cuda.Event()
+        h2d_done, comp_done, d2h_done = [EV(), EV()], [EV(), EV()], [EV(), EV()]
+        t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
-        for a, b in ev2:
+        t_begin.record(cs)
+        for i in range(e2e_steps):
+            k = i % 2
+            b = bufs[k]
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(comp_done[k])          # step i - 2 has read these inputs
+                for name in src_names:
+                    if host[name] is not None and b[name] is not None:
+                        b[name].copy_(host[name], non_blocking=True)
+                h2d_done[k].record(cs)
+            stream.wait_event(h2d_done[k])
+            if i >= 2:
+                stream.wait_event(d2h_done[k])           # step i - 2's result is out
             flush.fill_(1)
-            a.record(stream)
-            dv.copy_(hv, non_blocking=True)
-            offsets.copy_(ho, non_blocking=True)
-            if hc is not None:
-                ctx.copy_(hc, non_blocking=True)
-            if hq is not None:
-                cand.copy_(hq, non_blocking=True)
-            if ha is not None:
-                ages.copy_(ha, non_blocking=True)
-            step()
-            hout.copy_(out, non_blocking=True)
-            b.record(stream)
+            if graphs[k] is not None:
+                graphs[k].replay()
+            else:
+                fwd_on(b)
+            comp_done[k].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(comp_done[k])
+                hout[k].copy_(b["out"], non_blocking=True)
+                d2h_done[k].record(cs)
+        t_end.record(cs)
         torch.cuda.synchronize()
         barrier()
-        ms_e2e = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2))
-        h2d = hv.numel() * hv.element_size() + ho.numel() * 8 + \
-            (hc.numel() * hc.element_size() if hc is not None else 0) + \
-            (hq.numel() * hq.element_size() if hq is not None else 0) + \
-            (ha.numel() * 4 if ha is not None else 0)
+        ms_e2e = max_over_ranks(t_begin.elapsed_time(t_end))
+        h2d = sum(host[n].numel() * host[n].element_size() for n in src_names
+                  if host[n] is not None)
         e2e = {"value": users_all * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout[0].numel() * 4),
+               "pipeline": "double-buffered: copies of step i overlap compute of step i - 1",
+               "steps": e2e_steps}
         assert h.status() == 0
+        for g in graphs:
+            del g
+        graphs = None
 
         # ---- roofline of the dominant step (largest device time)
         ph = h.per_head_layers()              # layers in MLA's per-head form: their own work
