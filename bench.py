@@ -169,8 +169,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="online")
-    ap.add_argument("--second", default="upstream",
-                    help="second workload measured in the same run ('' = none)")
+    ap.add_argument("--second", default="upstream,upstream_abs",
+                    help="further workloads measured in the same run, comma-separated "
+                         "('' = none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-form", type=int, default=None, choices=[0, 1, 2],
@@ -493,15 +494,15 @@ def main():
         return res
 
     main_res = measure(wl, args.steps, args.warmup, sample_clocks=(rank == 0))
-    second = None
-    if args.second and args.second != args.workload:
-        wl2 = workload(args.second)
+    second = []
+    for name2 in [w for w in args.second.split(",") if w and w != args.workload]:
+        wl2 = workload(name2)
         s_steps = max(5, min(args.steps, 40))
         r2 = measure(wl2, s_steps, args.warmup, sample_clocks=False)
-        second = {"workload": wl2.name, "value": r2["value"], "unit": "user-seqs/s",
-                  "ms_per_step": r2["ms"], "steps": s_steps, "roofline": r2["roofline"],
-                  "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"],
-                  "mla_per_head_layers": r2["per_head_layers"]}
+        second.append({"workload": wl2.name, "value": r2["value"], "unit": "user-seqs/s",
+                       "ms_per_step": r2["ms"], "steps": s_steps, "roofline": r2["roofline"],
+                       "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"],
+                       "mla_per_head_layers": r2["per_head_layers"]})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -530,7 +531,7 @@ def main():
             "steps_ms": main_res["steps_ms"],
             "summary": main_res["summary"],
             "tokenizer": main_res["tokenizer"],
-            "second": second,
+            "second": second or None,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -170,6 +170,13 @@ WORKLOADS["online_time"] = Workload(
     name="online_time", dims=replace(WORKLOADS["online"].dims, d_time=64),
     batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
     description="online ranker with the timestamp encoding on 64 of 256 dims")
+# The upstream batch with MLA forced into its absorbed (latent-space) form, the
+# form whose attention is a dense tensor-core contraction at 4 r FLOP per
+# score; "auto" runs the per-head form there (fewer FLOPs, exponential-bound).
+WORKLOADS["upstream_abs"] = Workload(
+    name="upstream_abs", dims=replace(WORKLOADS["upstream"].dims, attn_form=1),
+    batch=64, lengths=("fixed", 1600), seed=2,
+    description="upstream user model, MLA in its absorbed form")
 WORKLOADS["online_sum"] = Workload(
     name="online_sum", dims=replace(WORKLOADS["online"].dims, n_sum=2, sum_rank=128, d_seq=1024),
     batch=256, lengths=("uniform", 100, 400), seed=1, semantic=True,
