@@ -56,7 +56,7 @@ constexpr int kEpiWarps = 4 * kParts;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr size_t kSmemMax = 232448;
 
-template <int BN>
+template <int BN, int EPI>
 struct GemmCfg {
   static constexpr int NI = BN > 256 ? 256 : BN;     // N of one MMA instruction
   static constexpr int NSUB = BN / NI;
@@ -69,8 +69,9 @@ struct GemmCfg {
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   // epilogue warps that take part: kParts column parts of 32 or more columns
   static constexpr int P = BN / 32 < kParts ? BN / 32 : kParts;
-  static constexpr size_t FIXED =
-      1024 + 256 + 2 * kParts * 128 * 4 + kEpiWarps * kStageBytes + BN * 2;
+  // the norm's partial sums and gain only for the norm epilogue
+  static constexpr size_t FIXED = 1024 + 256 + kEpiWarps * kStageBytes +
+                                  (EPI == TC_NORM ? 2 * kParts * 128 * 4 + BN * 2 : 0);
   // as many stages as fit, at most 8
   static constexpr int STAGES_FIT = (int)((kSmemMax - FIXED) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
@@ -79,7 +80,7 @@ struct GemmCfg {
   static_assert(SMEM <= kSmemMax, "shared memory budget");
 };
 
-// Epilogue of one 128 x BN tile.  GemmCfg<BN>::P warps share each TMEM lane
+// Epilogue of one 128 x BN tile.  GemmCfg<BN, EPI>::P warps share each TMEM lane
 // quadrant; `part` selects which BN / P columns this thread handles.  Stores
 // pass through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
@@ -87,9 +88,9 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
                                          bool valid, int n0, int ks, int g, int part, float* red,
                                          int rrow, uint64_t* xbar, uint32_t& xphase,
                                          volatile int* abort_flag, uint32_t stg,
-                                         NormPre<BN, 1, GemmCfg<BN>::P>& pre,
+                                         NormPre<BN, 1, GemmCfg<BN, EPI>::P>& pre,
                                          const __nv_bfloat16* sg) {
-  constexpr int HB = BN / GemmCfg<BN>::P;    // columns per thread
+  constexpr int HB = BN / GemmCfg<BN, EPI>::P;   // columns per thread
   const int c0 = part * HB;
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue(p.norm, taddr, row, valid, part, red, rrow, xbar, xphase,
@@ -157,7 +158,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcGemmParams p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, EPI>;
   constexpr int STAGES = Cfg::STAGES, NI = Cfg::NI, NSUB = Cfg::NSUB, ACC_BUFS = Cfg::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -171,8 +172,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* xbar = drain + 1;                 // epilogue group barrier (norm exchange)
   uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);   // [2 tiles][kParts][128]
-  uint8_t* sStage = (uint8_t*)(red + 2 * kParts * 128);             // [epilogue warp][kStageBytes]
+  // [2 tiles][kParts][128] partial sums of squares (norm epilogue only)
+  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);
+  uint8_t* sStage = (uint8_t*)(red + (EPI == TC_NORM ? 2 * kParts * 128 : 0));   // [warp][kStageBytes]
   __nv_bfloat16* sG = (__nv_bfloat16*)(sStage + kEpiWarps * kStageBytes);   // RMSNorm gain [BN]
 
   pdl_trigger();
@@ -321,7 +323,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 template <int BN, int EPI>
 cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmParams& p,
                        int grid, cudaStream_t s) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, EPI>;
   static uint64_t attr_devices = 0;   // devices on which the smem limit was raised
   int dev = 0;
   cudaGetDevice(&dev);
