@@ -459,7 +459,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int j = 0; j < KP / 2; ++j) {
           float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
-          if ((j & 7) == 7) {
+          // per-head form (d_h = 64): the tensor pipe has slack and the
+          // special-function unit sets the pace, so one pair in four goes to
+          // the FMA pipe; absorbed form: one in eight
+          if (MHA ? (j & 3) == 3 : (j & 7) == 7) {
             x = exp2_fma2(x);
           } else {
             x.x = ex2_approx(x.x);

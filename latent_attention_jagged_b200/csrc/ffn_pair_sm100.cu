@@ -124,8 +124,9 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
-  for (int i = threadIdx.x; i < D / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(sG)[i] = __ldg(reinterpret_cast<const uint4*>(p.norm.g) + i);
+  if (p.norm.mode != NORM_NONE)
+    for (int i = threadIdx.x; i < D / 8; i += blockDim.x)
+      reinterpret_cast<uint4*>(sG)[i] = __ldg(reinterpret_cast<const uint4*>(p.norm.g) + i);
   tc_fence_before();
   __syncthreads();
   cluster_sync();          // both CTAs' barriers exist before either signals the other
@@ -346,6 +347,31 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
     constexpr int RB = kRowsPerWarp < 8 ? kRowsPerWarp : 8;   // rows whose residual is in flight
     for (int64_t t = pair; t < num_tiles; t += n_pairs, ++ti) {
       const int64_t row_base = t * 256 + 128 * rank;
+      if (a.mode == NORM_NONE) {
+        // the block's output rows as they are (the action tokenizer's MLP):
+        // OUT (fp16 in sV) -> bf16 row of dst, one row per warp instruction
+        bool w = mbar_wait(v_full, ti & 1, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, w)) break;
+#pragma unroll 4
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+          const int r = r0 + i;
+          const int64_t row = row_base + r;
+          if (row >= M) break;                          // warp-uniform
+          const uint4 vw = ld_shared_v4(smem_u32(sV) + r * (D * 2) + ((lane ^ (r & 31)) << 4));
+          const __half2* h2 = reinterpret_cast<const __half2*>(&vw);
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(h2[k]);
+            o[k] = pack_bf16(f.x, f.y);
+          }
+          *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dst + row * D + 8 * lane) =
+              make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(v_free);
+        continue;
+      }
       // destinations of the warp's rows, lane l -> row r0 + l, found before
       // the data is ready (one round of dependent loads for all rows): the
       // next layer's history row, its query row, the final row (-1: none)
@@ -481,8 +507,11 @@ bool ffn_tc_supported(int d, int f) { return d == D && f % HC == 0 && f >= HC; }
 
 cudaError_t launch_ffn_pair(const CUtensorMap& z, const CUtensorMap& w1h, const CUtensorMap& w2h,
                             const FfnTcParams& p, int num_sms, cudaStream_t s) {
-  // the row epilogue implements the scatter into the next layer's rows only
-  if (p.norm.mode != NORM_SCATTER || p.F % HC != 0) return cudaErrorInvalidValue;
+  // the row epilogue implements the scatter into the next layer's rows and the
+  // plain store of the tokenizer's MLP
+  if ((p.norm.mode != NORM_SCATTER && p.norm.mode != NORM_NONE) || p.F % HC != 0 ||
+      (p.norm.mode == NORM_NONE && (!p.norm.dst || ((uintptr_t)p.norm.dst & 15))))
+    return cudaErrorInvalidValue;
   static uint64_t attr_devices = 0;
   int dev = 0;
   cudaGetDevice(&dev);

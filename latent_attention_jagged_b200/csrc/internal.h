@@ -202,7 +202,10 @@ struct NormArgs {
   void* zraw;
   const int32_t* row_user;           // user of each query row of layer l (tensor-core path)
 };
-enum { NORM_PLAIN = 0, NORM_SCATTER = 1 };
+// NORM_NONE (fused FFN kernel only): the block's output rows as they are, no
+// residual and no norm, stored in the storage type to dst (the action
+// tokenizer's MLP_act).
+enum { NORM_PLAIN = 0, NORM_SCATTER = 1, NORM_NONE = 2 };
 cudaError_t launch_rownorm(int elem, const NormArgs& a, cudaStream_t s);
 
 struct AttnArgs {

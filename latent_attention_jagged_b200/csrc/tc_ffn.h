@@ -19,7 +19,9 @@ struct FfnTcParams {
 bool ffn_tc_supported(int d, int f);
 // X = RMSNorm(Z + W2 SiLU(W1 Z)) on pairs of SMs (cta_group::2, 256-row
 // tiles).  w1h: W1 with 64-row boxes; w2h: W2 with 128-row boxes (each CTA
-// loads half a chunk).  norm.mode must be NORM_SCATTER.
+// loads half a chunk).  norm.mode NORM_SCATTER (the layer's FFN), or
+// NORM_NONE: X = W2 SiLU(W1 Z) stored as bf16 rows to norm.dst (16-byte
+// aligned; the output passes through fp16, so |X| must stay below 65504).
 cudaError_t launch_ffn_pair(const CUtensorMap& z, const CUtensorMap& w1h, const CUtensorMap& w2h,
                             const FfnTcParams& p, int num_sms, cudaStream_t s);
 

@@ -4,6 +4,9 @@
 //
 //   embed_gather_kernel   E[t] = concatenated table rows of event t (HBM / L2
 //                         bound: 16-byte vectors, four events per warp in flight)
+//   then, for D_in = d = 256 in bf16, the fused FFN kernel on SM pairs
+//   (W_a1 product, SiLU with the hidden layer kept in TMEM, W_a2 product,
+//   bf16 rows stored into the caller's token rows); otherwise two GEMMs:
 //   GEMM 1 (SiLU)         H = SiLU(E W_a1^T)      tcgen05 (bf16) or CUDA cores
 //   GEMM 2 (store)        X = H W_a2^T            into the caller's token rows
 #include <stdio.h>
@@ -14,6 +17,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ffn.h"
 #include "tc_gemm.h"
 
 using namespace llatte;
@@ -26,13 +30,16 @@ struct llatte_tokenizer {
   int num_sms;
   int d_in;
   int bn1, bn2;
+  int fused;                                   // both products in the fused FFN kernel
   const void* tables[LLATTE_TOK_MAX_FIELDS];   // caller-owned
   void* W_a1;                                  // [d_hid, d_in]
   void* W_a2;                                  // [d, d_hid]
   void* E;                                     // [max_events, d_in]
   void* H;                                     // [max_events, d_hid]
   int32_t* status;
+  int64_t* n_dev;                              // events of the call in progress
   CUtensorMap tm_E, tm_H, tm_W1, tm_W2;
+  CUtensorMap tm_W1h, tm_W2h;                  // fused kernel: 64- / 128-row weight boxes
 };
 
 namespace llatte {
@@ -48,6 +55,7 @@ struct EmbedArgs {
   int n_fields, nvec;
   const int32_t* ids;                        // [n, n_fields]
   int64_t n;
+  int64_t* n_dev;                            // receives n (the fused kernel's row count)
   uint4* E;                                  // [n, nvec] vectors
   int32_t* status;
 };
@@ -67,6 +75,7 @@ __global__ void __launch_bounds__(256) embed_gather_kernel(EmbedArgs a) {
     col[k] = v - a.vec_off[f];
     wvec[k] = a.vec_off[f + 1] - a.vec_off[f];
   }
+  if (a.n_dev && blockIdx.x == 0 && threadIdx.x == 0) *a.n_dev = a.n;
   int bad = 0;
   for (int64_t base = warp * kEmbedRows; base < a.n; base += nwarps * kEmbedRows) {
     uint4 buf[kEmbedRows][kEmbedVecs];
@@ -110,6 +119,7 @@ cudaError_t launch_embed(const llatte_tokenizer* t, const int32_t* ids, int64_t 
   a.nvec = a.vec_off[F];
   a.ids = ids;
   a.n = n;
+  a.n_dev = t->n_dev;
   a.E = (uint4*)t->E;
   a.status = t->status;
   const int64_t warps = (n + kEmbedRows - 1) / kEmbedRows;
@@ -183,7 +193,9 @@ int llatte_tokenizer_create(llatte_tokenizer** out, const llatte_tok_dims* dims,
   t->E = dev_alloc(e * (size_t)n * t->d_in);
   t->H = dev_alloc(e * (size_t)n * dims->d_hid);
   t->status = (int32_t*)dev_alloc(sizeof(int32_t));
-  if (!t->W_a1 || !t->W_a2 || !t->E || !t->H || !t->status) return fail(LLATTE_ERR_OOM);
+  t->n_dev = (int64_t*)dev_alloc(sizeof(int64_t));
+  if (!t->W_a1 || !t->W_a2 || !t->E || !t->H || !t->status || !t->n_dev)
+    return fail(LLATTE_ERR_OOM);
   const cudaMemcpyKind kind = weights_on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
   if (cudaMemcpy(t->W_a1, w->W_a1, e * (size_t)dims->d_hid * t->d_in, kind) != cudaSuccess ||
       cudaMemcpy(t->W_a2, w->W_a2, e * (size_t)dims->d * dims->d_hid, kind) != cudaSuccess ||
@@ -203,6 +215,11 @@ int llatte_tokenizer_create(llatte_tokenizer** out, const llatte_tok_dims* dims,
               make_tmap_bf16(&t->tm_W2, t->W_a2, dims->d, dims->d_hid, std::min(t->bn2, 256));
     if (!ok) t->use_tc = 0;
   }
+  // the fused FFN kernel takes 256-wide inputs and outputs and a hidden width
+  // that is a multiple of 128
+  t->fused = t->use_tc && t->d_in == 256 && dims->d == 256 && ffn_tc_supported(256, dims->d_hid) &&
+             make_tmap_bf16(&t->tm_W1h, t->W_a1, dims->d_hid, t->d_in, 64) &&
+             make_tmap_bf16(&t->tm_W2h, t->W_a2, dims->d, dims->d_hid, 128);
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(LLATTE_ERR_CUDA);
   *out = t;
   return LLATTE_OK;
@@ -216,7 +233,13 @@ int llatte_tokenize(llatte_tokenizer* t, const int32_t* ids, int64_t n, void* to
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_embed(t, ids, n, s) != cudaSuccess) return LLATTE_ERR_CUDA;
   const llatte_tok_dims& D = t->dims;
-  if (t->use_tc) {
+  if (t->fused) {
+    FfnTcParams f = {};
+    f.M_dev = t->n_dev; f.M_cap = std::max<int64_t>(D.max_events, 1); f.F = D.d_hid;
+    f.norm.mode = NORM_NONE; f.norm.dst = tokens; f.status = t->status;
+    if (launch_ffn_pair(t->tm_E, t->tm_W1h, t->tm_W2h, f, t->num_sms, s) != cudaSuccess)
+      return LLATTE_ERR_CUDA;
+  } else if (t->use_tc) {
     TcGemmParams g1 = {};
     g1.M_host = n; g1.M_cap = n; g1.N = D.d_hid; g1.K = t->d_in;
     g1.D = (__nv_bfloat16*)t->H; g1.ldd = D.d_hid; g1.status = t->status;
@@ -263,6 +286,7 @@ void llatte_tokenizer_destroy(llatte_tokenizer* t) {
   cudaFree(t->E);
   cudaFree(t->H);
   cudaFree(t->status);
+  cudaFree(t->n_dev);
   delete t;
 }
 
