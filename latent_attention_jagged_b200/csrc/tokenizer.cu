@@ -45,14 +45,18 @@ struct llatte_tokenizer {
 namespace llatte {
 namespace {
 
-constexpr int kEmbedRows = 4;            // events per warp in flight
 constexpr int kEmbedVecs = 4;            // 16-byte vectors per lane and event (row <= 2 KB)
+constexpr int kGatherThreads = 256;
+constexpr int kMaxBlockEvents = 128;     // events per block and round
+constexpr int kGatherSmem = 65536;       // staged table vectors per block
+constexpr int kLoadBatch = 4;            // vectors per thread in flight
 
 struct EmbedArgs {
   const uint4* table[LLATTE_TOK_MAX_FIELDS];
   int64_t rows[LLATTE_TOK_MAX_FIELDS];
   int vec_off[LLATTE_TOK_MAX_FIELDS + 1];   // first vector of each field in an E row
   int n_fields, nvec;
+  int block_events;                          // events per block and round
   const int32_t* ids;                        // [n, n_fields]
   int64_t n;
   int64_t* n_dev;                            // receives n (the fused kernel's row count)
@@ -60,49 +64,85 @@ struct EmbedArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(256) embed_gather_kernel(EmbedArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  // the field and in-field vector of each of this lane's vectors (same for every event)
-  int fld[kEmbedVecs], col[kEmbedVecs], wvec[kEmbedVecs];
-#pragma unroll
-  for (int k = 0; k < kEmbedVecs; ++k) {
-    const int v = lane + 32 * k;
-    int f = 0;
-    while (f + 1 < a.n_fields && a.vec_off[f + 1] <= v) ++f;
-    fld[k] = v < a.nvec ? f : -1;
-    col[k] = v - a.vec_off[f];
-    wvec[k] = a.vec_off[f + 1] - a.vec_off[f];
-  }
-  if (a.n_dev && blockIdx.x == 0 && threadIdx.x == 0) *a.n_dev = a.n;
+__device__ __forceinline__ int field_of(const EmbedArgs& a, int c) {
+  int f = 0;
+  while (f + 1 < a.n_fields && a.vec_off[f + 1] <= c) ++f;
+  return f;
+}
+
+// E rows of a block of events.  Popular ids (Zipf item popularity) make many
+// events read the same table row; read all at once by every SM, such a row's
+// L2 lines serve the reads one after another.  So each block reads every
+// distinct (field, id) of its events once: the first event with that id (its
+// leader) loads the row into shared memory, and every event's E row is
+// written from its leaders' copies.
+__global__ void __launch_bounds__(kGatherThreads) embed_gather_kernel(EmbedArgs a) {
+  extern __shared__ uint4 s_rows[];                     // [block_events][nvec]
+  __shared__ int32_t s_id[kMaxBlockEvents * LLATTE_TOK_MAX_FIELDS];
+  __shared__ int16_t s_lead[kMaxBlockEvents * LLATTE_TOK_MAX_FIELDS];
+  __shared__ int8_t s_field[32 * kEmbedVecs];           // field of each vector of a row
+  const int tid = threadIdx.x;
+  const int F = a.n_fields, NV = a.nvec, EB = a.block_events;
+  for (int c = tid; c < NV; c += kGatherThreads) s_field[c] = (int8_t)field_of(a, c);
+  if (a.n_dev && blockIdx.x == 0 && tid == 0) *a.n_dev = a.n;
   int bad = 0;
-  for (int64_t base = warp * kEmbedRows; base < a.n; base += nwarps * kEmbedRows) {
-    uint4 buf[kEmbedRows][kEmbedVecs];
+  for (int64_t e0 = (int64_t)blockIdx.x * EB; e0 < a.n; e0 += (int64_t)gridDim.x * EB) {
+    const int ne = (int)(a.n - e0 < EB ? a.n - e0 : EB);
+    for (int i = tid; i < ne * F; i += kGatherThreads) s_id[i] = __ldg(a.ids + e0 * F + i);
+    __syncthreads();
+    // leader of (event e, field f): the first event of the block with the same id
+    for (int i = tid; i < ne * F; i += kGatherThreads) {
+      const int e = i / F, f = i - e * F, id = s_id[i];
+      int l = e;
+      for (int e2 = 0; e2 < e; ++e2)
+        if (s_id[e2 * F + f] == id) { l = e2; break; }
+      s_lead[i] = (int16_t)l;
+    }
+    __syncthreads();
+    // leaders load their table vectors into their own slots, kLoadBatch in flight
+    const int total = ne * NV;
+    for (int v0 = tid; v0 < total; v0 += kGatherThreads * kLoadBatch) {
+      uint4 buf[kLoadBatch];
+      int slot[kLoadBatch];
 #pragma unroll
-    for (int j = 0; j < kEmbedRows; ++j) {
-      const int64_t t = base + j;
-#pragma unroll
-      for (int k = 0; k < kEmbedVecs; ++k) {
-        buf[j][k] = make_uint4(0, 0, 0, 0);
-        if (t < a.n && fld[k] >= 0) {
-          const int f = fld[k];
-          const int64_t id = __ldg(a.ids + t * a.n_fields + f);
-          if (id >= 0 && id < a.rows[f]) buf[j][k] = __ldg(a.table[f] + id * wvec[k] + col[k]);
-          else bad = 1;
+      for (int b = 0; b < kLoadBatch; ++b) {
+        const int v = v0 + b * kGatherThreads;
+        slot[b] = -1;
+        buf[b] = make_uint4(0, 0, 0, 0);
+        if (v < total) {
+          const int e = v / NV, c = v - e * NV, f = s_field[c];
+          if (s_lead[e * F + f] == e) {
+            slot[b] = v;
+            const int64_t id = s_id[e * F + f];
+            if (id >= 0 && id < a.rows[f]) {
+              const int w = a.vec_off[f + 1] - a.vec_off[f];
+              buf[b] = __ldg(a.table[f] + id * w + (c - a.vec_off[f]));
+            } else {
+              bad = 1;
+            }
+          }
         }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < kEmbedRows; ++j) {
-      const int64_t t = base + j;
-      if (t >= a.n) break;
-#pragma unroll
-      for (int k = 0; k < kEmbedVecs; ++k)
-        if (fld[k] >= 0) a.E[t * a.nvec + lane + 32 * k] = buf[j][k];
+      for (int b = 0; b < kLoadBatch; ++b)
+        if (slot[b] >= 0) s_rows[slot[b]] = buf[b];
     }
+    __syncthreads();
+    // every event's row from its leaders' copies, coalesced 16-byte stores
+    for (int v = tid; v < total; v += kGatherThreads) {
+      const int e = v / NV, c = v - e * NV, f = s_field[c];
+      const int l = s_lead[e * F + f];
+      a.E[(e0 + e) * NV + c] = s_rows[l * NV + c];
+    }
+    __syncthreads();
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.status, LLATTE_DEV_BAD_ID);
+  if (__syncthreads_or(bad) && tid == 0) atomicOr(a.status, LLATTE_DEV_BAD_ID);
+}
+
+// Events per block and round for rows of nvec 16-byte vectors.
+int gather_block_events(int nvec) {
+  const int fit = kGatherSmem / (nvec * 16);
+  return fit < kMaxBlockEvents ? fit : kMaxBlockEvents;
 }
 
 cudaError_t launch_embed(const llatte_tokenizer* t, const int32_t* ids, int64_t n,
@@ -117,14 +157,25 @@ cudaError_t launch_embed(const llatte_tokenizer* t, const int32_t* ids, int64_t 
     a.vec_off[f + 1] = a.vec_off[f] + t->dims.width[f] * t->elem / 16;
   }
   a.nvec = a.vec_off[F];
+  a.block_events = gather_block_events(a.nvec);
   a.ids = ids;
   a.n = n;
   a.n_dev = t->n_dev;
   a.E = (uint4*)t->E;
   a.status = t->status;
-  const int64_t warps = (n + kEmbedRows - 1) / kEmbedRows;
-  const int64_t blocks = std::min<int64_t>((warps + 7) / 8, (int64_t)t->num_sms * 16);
-  embed_gather_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), 256, 0, s>>>(a);
+  const size_t smem = (size_t)a.block_events * a.nvec * 16;
+  static uint64_t attr_devices = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_devices >> (dev & 63) & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(embed_gather_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherSmem);
+    if (e != cudaSuccess) return e;
+    attr_devices |= 1ull << (dev & 63);
+  }
+  const int64_t groups = (n + a.block_events - 1) / a.block_events;
+  const int64_t blocks = std::min<int64_t>(groups, (int64_t)t->num_sms * 3);
+  embed_gather_kernel<<<(unsigned)std::max<int64_t>(blocks, 1), kGatherThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
