@@ -185,7 +185,9 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (rank 0)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t IDESC1 = idesc_bf16(256, HC, false, false);
+      // Z W1^T: both operands fp16 or both bf16 (the caller's choice)
+      const uint32_t IDESC1 = p.z_f16 ? idesc_f16(256, HC, false, false)
+                                      : idesc_bf16(256, HC, false, false);
       constexpr uint32_t IDESC2 = idesc_bf16(256, D, false, false);
       const uint32_t z_addr = smem_u32(sZ);
       uint32_t w = 0, ti = 0, gc = 0;

@@ -410,20 +410,31 @@ EncodeTiledFn encode_fn() {
 }
 }  // namespace
 
-// 2-D bf16 tensor [rows, cols] (row-major, cols contiguous), box of
+namespace {
+// 2-D 16-bit tensor [rows, cols] (row-major, cols contiguous), box of
 // box_rows x 64 columns (128 bytes), 128-byte swizzle, zero fill outside.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows) {
+bool make_tmap_16(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t rows,
+                  uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || cols % 64 != 0 || ((uintptr_t)base & 15) || box_rows > 256) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  return make_tmap_16(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rows, cols, box_rows);
+}
+bool make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  return make_tmap_16(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rows, cols, box_rows);
 }
 
 }  // namespace llatte

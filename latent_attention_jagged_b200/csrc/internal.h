@@ -63,6 +63,7 @@ struct LayerDev {
   void* W_ov;      // [d, h*r]   absorbed W_o W_uv
   void* g1;        // [d]
   void* W1;        // [f, d]
+  void* W1h;       // [f, d] fp16 copy of W1 (the fused FFN's first product takes fp16 Z)
   void* W2;        // [d, f]
   void* g2;        // [d]
 };
@@ -72,6 +73,7 @@ struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 // TMA descriptors of one layer's weights (B operands of the tensor-core GEMMs).
 struct LayerMaps {
   CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq;
+  CUtensorMap w1h_pair;                 // fp16 W1, 64-row boxes (fused FFN)
   CUtensorMap qh, ukv, oh, oh_pair;     // per-head form
 };
 
@@ -123,6 +125,7 @@ struct llatte_handle {
   // tensor-core path: TMA descriptors of the A operands and the weights,
   // and the tile width (BN) of each GEMM
   CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd, tm_Cq;
+  CUtensorMap tm_Zres;            // fp16 Z (the fused FFN's first operand and its residual)
   llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
   int bn_kv, bn_q, bn_o, bn_f1, bn_f2, bn_dq;
   int attn_keys;                  // keys per attention tile (tensor-core path)
@@ -248,6 +251,8 @@ struct SummaryArgs {
 };
 cudaError_t launch_summary_reduce(const SummaryArgs& a, cudaStream_t s);
 cudaError_t launch_summary_up(int elem, const SummaryArgs& a, cudaStream_t s);
+// fp16 copy of n bf16 values.
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s);
 // dst[c, r] = src[r, c] for a [rows, cols] matrix of the storage type.
 cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
                              cudaStream_t s);

@@ -262,6 +262,7 @@ bool build_tc_maps(llatte_handle* h) {
   }
   ok = ok && make_tmap_bf16(&h->tm_Ot, h->Ot, rq, hr, 128);
   ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
+  if (h->Zres) ok = ok && make_tmap_f16(&h->tm_Zres, h->Zres, rq, d, 128);
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
   if (D.q_rank) ok = ok && make_tmap_bf16(&h->tm_Cq, h->Cq, rq, D.q_rank, 128);
   h->attn_keys = attn_tc_keys(r);
@@ -293,9 +294,16 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
     if (h->ffn_fused) {
-      // the SM-pair FFN: each CTA loads half of a weight chunk
+      // the SM-pair FFN: each CTA loads half of a weight chunk; its first
+      // product takes Z in fp16 (the residual copy), so W1 gets an fp16 copy
       ok = ok && make_tmap_bf16(&M.w1_pair, W.W1, f, d, 64);
       ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
+      LayerDev& Wm = h->layers[l];
+      if (ok && !Wm.W1h) {
+        Wm.W1h = dev_alloc(h, 2 * (size_t)f * d);
+        ok = Wm.W1h && launch_bf16_to_f16(W.W1, Wm.W1h, (int64_t)f * d, 0) == cudaSuccess;
+      }
+      ok = ok && make_tmap_f16(&M.w1h_pair, Wm.W1h, f, d, 64);
     }
     if (h->pair_norm) {
       // the SM-pair residual + RMSNorm GEMMs at d = 512: 128-row weight boxes
@@ -668,7 +676,10 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     o_norm.resid = (l == 0 || !res16) ? Xq_l : h->Xqres[l & 1];
     o_norm.resid_kind = (l == 0 || !res16) ? RES_STORAGE : RES_F16;
     o_norm.M_dev = p.query_total(l); o_norm.M_max = h->max_rows_q; o_norm.mode = NORM_PLAIN;
-    o_norm.dst = h->Z; o_norm.dst_res = res16 ? h->Zres : nullptr;
+    // the fused FFN reads Z only as fp16 (its first operand and its residual),
+    // so then the bf16 copy is not written
+    const bool z16_only = tc && h->ffn_fused && res16;
+    o_norm.dst = z16_only ? nullptr : h->Z; o_norm.dst_res = res16 ? h->Zres : nullptr;
     NormArgs f_norm = {};
     f_norm.N = d; f_norm.resid = res16 ? h->Zres : h->Z;
     f_norm.resid_kind = res16 ? RES_F16 : RES_STORAGE; f_norm.res_kind = RES_F16;
@@ -849,7 +860,9 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
       FfnTcParams q = {};
       q.M_dev = p.query_total(l); q.M_cap = h->max_rows_q; q.F = f; q.norm = f_norm;
       q.status = p.status;
-      CK(launch_ffn_pair(h->tm_Z, LM.w1_pair, LM.w2_pair, q, h->num_sms, s));
+      q.z_f16 = z16_only ? 1 : 0;
+      CK(launch_ffn_pair(z16_only ? h->tm_Zres : h->tm_Z, z16_only ? LM.w1h_pair : LM.w1_pair,
+                         LM.w2_pair, q, h->num_sms, s));
       t.done(1);
       continue;
     }

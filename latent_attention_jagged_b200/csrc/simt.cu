@@ -459,6 +459,22 @@ __global__ void transpose_kernel(const T* __restrict__ src, int64_t rows, int64_
   dst[c * rows + r] = src[i];
 }
 
+// dst[i] = fp16(src[i]) for n bf16 values (exact in fp16's normal range: a
+// bf16 mantissa fits in fp16's).
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                   int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
+  bf16_to_f16_kernel<<<(unsigned)blocks, 256, 0, s>>>((const __nv_bfloat16*)src, (__half*)dst, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_transpose(int elem, const void* src, int64_t rows, int64_t cols, void* dst,
                              cudaStream_t s) {
   const int64_t n = rows * cols;

@@ -268,6 +268,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16: fp16 A and B (both operands of one MMA
+// must have the same type), fp32 D, dense.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Generic-proxy shared-memory writes made visible to the async proxy (TMA,
 // tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -186,7 +186,7 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   __half* r1 = nullptr;
   if (valid) {
     if (a.mode == NORM_PLAIN) {
-      d1 = (__nv_bfloat16*)a.dst + row * N;
+      if (a.dst) d1 = (__nv_bfloat16*)a.dst + row * N;
       if (a.dst_res) r1 = (__half*)a.dst_res + row * N;
     } else {
       const int u = a.row_user[row];

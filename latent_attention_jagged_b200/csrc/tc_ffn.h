@@ -12,6 +12,7 @@ struct FfnTcParams {
   const int64_t* M_dev;   // rows (device)
   int64_t M_cap;          // largest M (sizes the grid)
   int F;                  // hidden width (multiple of 128)
+  int z_f16;              // Z and W1 in fp16 (both operands of the first product), else bf16
   NormArgs norm;          // residual + RMSNorm + scatter of the output rows
   int32_t* status;
 };

@@ -32,6 +32,9 @@ struct TcGemmParams {
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+// The same for an fp16 tensor.
+bool make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows);
 bool tc_gemm_supported(int BN, int epi, int N, int K);
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
                            const TcGemmParams& p, int num_sms, cudaStream_t s);
