@@ -362,7 +362,10 @@ int llatte_forward_batch(llatte_handle* handle, const llatte_batch* batch, float
  *                   (sum of widths = D_in, D_in * element size <= 2048 B)
  *   d_hid, d        hidden and token width (d * element size a multiple of 16)
  *   dtype           LLATTE_BF16 (tensor cores when D_in, d_hid are multiples
- *                   of 64 and d_hid, d of 64, else CUDA cores) or LLATTE_FP32
+ *                   of 64 and d_hid, d of 64, else CUDA cores; for D_in = d =
+ *                   256 and d_hid a multiple of 128 both products run in one
+ *                   kernel whose output passes through fp16, so tokens must
+ *                   stay below 65504 in magnitude) or LLATTE_FP32
  *   max_events      most events one call may tokenize (<= 65535 * 64)
  */
 #define LLATTE_TOK_MAX_FIELDS 8
