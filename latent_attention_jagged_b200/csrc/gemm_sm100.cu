@@ -243,7 +243,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16(128, NI, false, false);
+      // A and the weight: both fp16 or both bf16 (the caller's choice)
+      const uint32_t IDESC = p.ab_f16 ? idesc_f16(128, NI, false, false)
+                                      : idesc_bf16(128, NI, false, false);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;

@@ -63,7 +63,7 @@ struct LayerDev {
   void* W_ov;      // [d, h*r]   absorbed W_o W_uv
   void* g1;        // [d]
   void* W1;        // [f, d]
-  void* W1h;       // [f, d] fp16 copy of W1 (the fused FFN's first product takes fp16 Z)
+  void* W1h;       // [f, d] fp16 copy of W1 (the FFN's first product takes fp16 Z)
   void* W2;        // [d, f]
   void* g2;        // [d]
 };
@@ -74,6 +74,7 @@ struct ProfRec { int step; cudaEvent_t a, b; int launches; };
 struct LayerMaps {
   CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq;
   CUtensorMap w1h_pair;                 // fp16 W1, 64-row boxes (fused FFN)
+  CUtensorMap w1h;                      // fp16 W1, bn_f1-row boxes (FFN-up GEMM)
   CUtensorMap qh, ukv, oh, oh_pair;     // per-head form
 };
 

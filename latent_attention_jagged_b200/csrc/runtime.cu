@@ -293,17 +293,21 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
-    if (h->ffn_fused) {
-      // the SM-pair FFN: each CTA loads half of a weight chunk; its first
-      // product takes Z in fp16 (the residual copy), so W1 gets an fp16 copy
-      ok = ok && make_tmap_bf16(&M.w1_pair, W.W1, f, d, 64);
-      ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
+    // the FFN's first product takes Z in fp16 (the residual copy, so Z crosses
+    // HBM once), so W1 gets an fp16 copy (both operands of an MMA share a type)
+    {
       LayerDev& Wm = h->layers[l];
       if (ok && !Wm.W1h) {
         Wm.W1h = dev_alloc(h, 2 * (size_t)f * d);
         ok = Wm.W1h && launch_bf16_to_f16(W.W1, Wm.W1h, (int64_t)f * d, 0) == cudaSuccess;
       }
-      ok = ok && make_tmap_f16(&M.w1h_pair, Wm.W1h, f, d, 64);
+      ok = ok && make_tmap_f16(&M.w1h, Wm.W1h, f, d, box(h->bn_f1));
+      if (h->ffn_fused) {
+        // the SM-pair FFN: each CTA loads half of a weight chunk
+        ok = ok && make_tmap_bf16(&M.w1_pair, W.W1, f, d, 64);
+        ok = ok && make_tmap_bf16(&M.w2_pair, W.W2, d, f, 128);
+        ok = ok && make_tmap_f16(&M.w1h_pair, Wm.W1h, f, d, 64);
+      }
     }
     if (h->pair_norm) {
       // the SM-pair residual + RMSNorm GEMMs at d = 512: 128-row weight boxes
@@ -676,9 +680,9 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     o_norm.resid = (l == 0 || !res16) ? Xq_l : h->Xqres[l & 1];
     o_norm.resid_kind = (l == 0 || !res16) ? RES_STORAGE : RES_F16;
     o_norm.M_dev = p.query_total(l); o_norm.M_max = h->max_rows_q; o_norm.mode = NORM_PLAIN;
-    // the fused FFN reads Z only as fp16 (its first operand and its residual),
-    // so then the bf16 copy is not written
-    const bool z16_only = tc && h->ffn_fused && res16;
+    // on the tensor cores the FFN reads Z only as fp16 (its first operand and
+    // its residual), so then the bf16 copy is not written
+    const bool z16_only = tc && res16;
     o_norm.dst = z16_only ? nullptr : h->Z; o_norm.dst_res = res16 ? h->Zres : nullptr;
     NormArgs f_norm = {};
     f_norm.N = d; f_norm.resid = res16 ? h->Zres : h->Z;
@@ -871,7 +875,9 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
       if (tc) {
         TcGemmParams q = tcp(p.query_total(l), h->max_rows_q, f, d);
         q.D = (__nv_bfloat16*)h->Hd; q.ldd = f;
-        CK(launch_tc_gemm(h->bn_f1, TC_SILU, h->tm_Z, LM.w1, q, h->num_sms, s));
+        q.ab_f16 = z16_only ? 1 : 0;
+        CK(launch_tc_gemm(h->bn_f1, TC_SILU, z16_only ? h->tm_Zres : h->tm_Z,
+                          z16_only ? LM.w1h : LM.w1, q, h->num_sms, s));
       } else {
         GemmArgs g = {};
         g.A = h->Z; g.lda = d; g.W = W.W1; g.D = h->Hd; g.ldd = f;

@@ -28,6 +28,7 @@ struct TcGemmParams {
   float* Dp; int64_t slice_stride; int k_split;
   int groups; int64_t a_group_rows; int w_group_rows; int64_t d_group_off; int64_t ldp;
   int32_t* status;
+  int ab_f16;                   // A and the weight in fp16 (both operands of every MMA), else bf16
 };
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
