@@ -451,7 +451,7 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
                                       pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
           if (hd >= 0) *reinterpret_cast<uint4*>(h_base + hd * D + 8 * lane) = wb;
           if (qd >= 0) {
-            *reinterpret_cast<uint4*>((__nv_bfloat16*)a.Xq_n + qd * D + 8 * lane) = wb;
+            if (a.Xq_n) *reinterpret_cast<uint4*>((__nv_bfloat16*)a.Xq_n + qd * D + 8 * lane) = wb;
             if (a.Xq_res_n)
               *reinterpret_cast<uint4*>((__half*)a.Xq_res_n + qd * D + 8 * lane) =
                   make_uint4(pack_f16(x[0], x[1]), pack_f16(x[2], x[3]), pack_f16(x[4], x[5]),

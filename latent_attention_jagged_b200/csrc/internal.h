@@ -64,6 +64,8 @@ struct LayerDev {
   void* g1;        // [d]
   void* W1;        // [f, d]
   void* W1h;       // [f, d] fp16 copy of W1 (the FFN's first product takes fp16 Z)
+  void* W_q16;     // fp16 copy of the layer's query weight (W_qk, or W_qh in the per-head
+                   //   form) for layers >= 1: their query rows are read in fp16
   void* W2;        // [d, f]
   void* g2;        // [d]
 };
@@ -75,6 +77,7 @@ struct LayerMaps {
   CUtensorMap dkv, qk, ov, w1, w2, w1_pair, w2_pair, ov_pair, dq;
   CUtensorMap w1h_pair;                 // fp16 W1, 64-row boxes (fused FFN)
   CUtensorMap w1h;                      // fp16 W1, bn_f1-row boxes (FFN-up GEMM)
+  CUtensorMap qk16, qh16;               // fp16 query weights (layers >= 1, full-rank query)
   CUtensorMap qh, ukv, oh, oh_pair;     // per-head form
 };
 
@@ -127,6 +130,7 @@ struct llatte_handle {
   // and the tile width (BN) of each GEMM
   CUtensorMap tm_Xh[2], tm_Xq[2], tm_Ot, tm_Z, tm_Hd, tm_Cq;
   CUtensorMap tm_Zres;            // fp16 Z (the fused FFN's first operand and its residual)
+  CUtensorMap tm_Xqres[2];        // fp16 query rows (the query projection's operand, layers >= 1)
   llatte::LayerMaps lmaps[LLATTE_MAX_LAYERS];
   int bn_kv, bn_q, bn_o, bn_f1, bn_f2, bn_dq;
   int attn_keys;                  // keys per attention tile (tensor-core path)

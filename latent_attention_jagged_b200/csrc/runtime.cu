@@ -263,6 +263,8 @@ bool build_tc_maps(llatte_handle* h) {
   ok = ok && make_tmap_bf16(&h->tm_Ot, h->Ot, rq, hr, 128);
   ok = ok && make_tmap_bf16(&h->tm_Z, h->Z, rq, d, 128);
   if (h->Zres) ok = ok && make_tmap_f16(&h->tm_Zres, h->Zres, rq, d, 128);
+  for (int i = 0; i < 2 && h->Xqres[i]; ++i)
+    ok = ok && make_tmap_f16(&h->tm_Xqres[i], h->Xqres[i], rq, d, 128);
   ok = ok && make_tmap_bf16(&h->tm_Hd, h->Hd, rq, f, 128);
   if (D.q_rank) ok = ok && make_tmap_bf16(&h->tm_Cq, h->Cq, rq, D.q_rank, 128);
   h->attn_keys = attn_tc_keys(r);
@@ -293,6 +295,20 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&M.ov, W.W_ov, d, hr, box(h->bn_o));
     ok = ok && make_tmap_bf16(&M.w1, W.W1, f, d, box(h->bn_f1));
     ok = ok && make_tmap_bf16(&M.w2, W.W2, d, f, box(h->bn_f2));
+    // layers >= 1 with a full-rank query read their query rows in fp16 (the
+    // residual copy), so their query weight gets an fp16 copy
+    if (l >= 1 && !D.q_rank && h->Xqres[0]) {
+      LayerDev& Wm = h->layers[l];
+      const bool ph = (h->heads_mask >> l) & 1u;
+      const int rows = ph ? hdh : hr;
+      if (ok && !Wm.W_q16) {
+        Wm.W_q16 = dev_alloc(h, 2 * (size_t)rows * d);
+        ok = Wm.W_q16 && launch_bf16_to_f16(ph ? W.W_qh : W.W_qk, Wm.W_q16, (int64_t)rows * d, 0) ==
+                             cudaSuccess;
+      }
+      if (ph) ok = ok && make_tmap_f16(&M.qh16, Wm.W_q16, hdh, d, box(pick_bn(hdh)));
+      else ok = ok && make_tmap_f16(&M.qk16, Wm.W_q16, hr, d, box(h->bn_q));
+    }
     // the FFN's first product takes Z in fp16 (the residual copy, so Z crosses
     // HBM once), so W1 gets an fp16 copy (both operands of an MMA share a type)
     {
@@ -683,6 +699,9 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     // on the tensor cores the FFN reads Z only as fp16 (its first operand and
     // its residual), so then the bf16 copy is not written
     const bool z16_only = tc && res16;
+    // layers >= 1 (full-rank query, tensor cores): the query rows are read in
+    // fp16, from the residual copy the previous layer's FFN wrote
+    const bool q16 = tc && res16 && l >= 1 && !rq;
     o_norm.dst = z16_only ? nullptr : h->Z; o_norm.dst_res = res16 ? h->Zres : nullptr;
     NormArgs f_norm = {};
     f_norm.N = d; f_norm.resid = res16 ? h->Zres : h->Z;
@@ -691,7 +710,10 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
     f_norm.M_dev = p.query_total(l); f_norm.M_max = h->max_rows_q; f_norm.mode = NORM_SCATTER;
     f_norm.qoff_l = p.qoff(l); f_norm.n_l = p.nl(l); f_norm.hoff_n = p.hoff(l + 1);
     f_norm.qoff_n = p.qoff(l + 1); f_norm.n_n = p.nl(l + 1); f_norm.B = B; f_norm.n_q = D.n_q;
-    f_norm.Xh_n = Xh_n; f_norm.Xq_n = Xq_n; f_norm.last = last;
+    // the next layer reads its query rows in fp16 on the tensor cores (full-rank
+    // query), so then the bf16 copy is not written
+    const bool next_q16 = tc && res16 && !rq && !last;
+    f_norm.Xh_n = Xh_n; f_norm.Xq_n = next_q16 ? nullptr : Xq_n; f_norm.last = last;
     f_norm.Xq_res_n = (res16 && !last) ? h->Xqres[(l + 1) & 1] : nullptr;
     f_norm.out = out; f_norm.final_rows = D.d_out ? h->final_rows : nullptr;
     f_norm.zraw = (last && D.n_sum > 0) ? h->zraw : nullptr;
@@ -749,8 +771,10 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hdh;
         q.bias = h->ctxbias + cw.off[l]; q.seg_off = p.qoff(l); q.B = B;
         q.row_user = p.ruser(l);
-        CK(launch_tc_gemm(pick_bn(hdh), D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1],
-                          LM.qh, q, h->num_sms, s));
+        q.ab_f16 = q16 ? 1 : 0;
+        CK(launch_tc_gemm(pick_bn(hdh), D.d_ctx > 0 ? TC_USERBIAS : TC_STORE,
+                          q16 ? h->tm_Xqres[l & 1] : h->tm_Xq[l & 1], q16 ? LM.qh16 : LM.qh, q,
+                          h->num_sms, s));
       } else if (rq) {
         // low-rank query: Cq = RMSNorm_{g_q}(R W_dq,x^T + context term of the
         // row's user), then the absorbed projection Qt = Cq (W_uk^T W_uq)^T
@@ -790,7 +814,9 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.D = (__nv_bfloat16*)h->Qt; q.ldd = hr;
         q.bias = h->ctxbias + cw.off[l]; q.seg_off = p.qoff(l); q.B = B;
         q.row_user = p.ruser(l);
-        CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE, h->tm_Xq[l & 1], LM.qk,
+        q.ab_f16 = q16 ? 1 : 0;
+        CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE,
+                          q16 ? h->tm_Xqres[l & 1] : h->tm_Xq[l & 1], q16 ? LM.qk16 : LM.qk,
                           q, h->num_sms, s));
       } else {
         GemmArgs g = {};

@@ -210,7 +210,7 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
           q = a.qoff_n[u] + nn + (j - nl);
         }
         if (q >= 0) {
-          d2 = (__nv_bfloat16*)a.Xq_n + q * N;
+          if (a.Xq_n) d2 = (__nv_bfloat16*)a.Xq_n + q * N;
           if (a.Xq_res_n) r1 = (__half*)a.Xq_res_n + q * N;
         }
       }
