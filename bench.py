@@ -36,7 +36,7 @@ from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 # of the dominant kernel, keyed by (step, workload, MLA form); taken from the committed
 # profiles/dram_traffic_dominant_kernels.md.  Absent = not captured for the
 # current kernel version.
-TRAFFIC = {("ffn", "online", "absorbed"): 4.1997e7}
+TRAFFIC = {("ffn", "online", "absorbed"): 3.2992e7}
 
 
 def load_peaks():
