@@ -309,22 +309,48 @@ cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int 
 
 // ---------------------------------------------------------------- readout mean
 // mean[u] = (1 / rows_u) sum of the user's final rows (zero for no rows).
-__global__ void mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qoff,
-                                 int d, float* __restrict__ mean) {
+// mean[u, :] = mean of user u's rows.  A block takes 128 columns (32 float4)
+// of one user; its eight warps take every eighth row (the sums of many rows
+// in flight at once instead of one long dependent chain per column), then
+// the eight partial sums are added in warp order (deterministic).
+constexpr int kMeanWarps = 8;
+
+__global__ void __launch_bounds__(32 * kMeanWarps)
+mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qoff, int d,
+                 float* __restrict__ mean) {
+  __shared__ float4 part[kMeanWarps][32];
   const int u = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c4 = blockIdx.y * 32 + lane;                 // float4 column of this lane
+  const int d4 = d / 4;
   const int64_t a = qoff[u], b = qoff[u + 1];
-  const float inv = b > a ? 1.f / (float)(b - a) : 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float s = 0.f;
-    for (int64_t i = a; i < b; ++i) s += rows[i * d + c];
-    mean[(int64_t)u * d + c] = s * inv;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (c4 < d4) {
+    const float4* r4 = reinterpret_cast<const float4*>(rows);
+    for (int64_t i = a + warp; i < b; i += kMeanWarps) {
+      const float4 v = __ldg(r4 + i * d4 + c4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+  }
+  part[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && c4 < d4) {
+    float4 t = part[0][lane];
+    for (int w = 1; w < kMeanWarps; ++w) {
+      const float4 p = part[w][lane];
+      t.x += p.x; t.y += p.y; t.z += p.z; t.w += p.w;
+    }
+    const float inv = b > a ? 1.f / (float)(b - a) : 0.f;
+    reinterpret_cast<float4*>(mean)[(int64_t)u * d4 + c4] =
+        make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
   }
 }
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
                              cudaStream_t s) {
   if (B == 0) return cudaSuccess;
-  mean_rows_kernel<<<B, 256, 0, s>>>(rows, qoff, d, mean);
+  if (d % 4 != 0) return cudaErrorInvalidValue;
+  mean_rows_kernel<<<dim3(B, (d / 4 + 31) / 32), 32 * kMeanWarps, 0, s>>>(rows, qoff, d, mean);
   return cudaGetLastError();
 }
 
