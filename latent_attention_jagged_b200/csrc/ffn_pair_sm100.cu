@@ -281,8 +281,8 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
         tc_fence_after();
         // this warp's 64 hidden columns: SiLU -> bf16 pairs, written over the
         // first 32 columns of its half of the buffer, 32 columns at a time
-        // (round 1 reads columns 32..63 and writes packed columns 16..31,
-        // which round 0 has already read)
+        // (pass h = 1 reads columns 32..63 and writes packed columns 16..31,
+        // which pass h = 0 has already read)
         const uint32_t hcol = lane_base + H_COL + (gc & 1) * HC + half * 64;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

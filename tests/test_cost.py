@@ -3,8 +3,8 @@
 The per-form counts follow the two MLA displays (absorbed: scores over the
 rank-r latent; per head: scores over d_h after the K | V up-projection), so
 their ratios are fixed by the dimensions; the upstream total is checked
-against the figure worked out independently for the survey of the method
-(3.256 TFLOP per batch in the absorbed form), and the tokenizer's counts
+against an independent hand count of the upstream workload (3.256 TFLOP per
+batch in the absorbed form), and the tokenizer's counts
 against their closed forms."""
 import numpy as np
 
