@@ -33,10 +33,34 @@ from workloads import draw_lengths, make_event_ages, make_inputs, workload  # no
 from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 
 # ncu-measured DRAM traffic per launch (bytes, mean over one forward's layers)
-# of the dominant kernel, keyed by (step, workload, MLA form); taken from the committed
-# profiles/dram_traffic_dominant_kernels.md.  Absent = not captured for the
-# current kernel version.
-TRAFFIC = {("ffn", "online", "absorbed"): 3.2992e7}
+# of a dominant kernel, keyed by (step, workload, MLA form), each with the
+# kernel sources it was taken on and their hash: the bench reports the figure
+# only while those sources are unchanged (null otherwise).  The captures are
+# summarised under profiles/.
+TRAFFIC = {}
+KERNEL_SOURCES = {
+    "ffn": ["ffn_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "attn": ["attn_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "o": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "ffn2": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "kv": ["gemm_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+}
+
+
+def sources_hash(step: str) -> str:
+    import hashlib
+    hsh = hashlib.sha256()
+    for name in KERNEL_SOURCES.get(step, []):
+        with open(os.path.join(ROOT, "latent_attention_jagged_b200", "csrc", name), "rb") as f:
+            hsh.update(f.read())
+    return hsh.hexdigest()[:16]
+
+
+def traffic_of(step: str, workload_name: str, form: str):
+    t = TRAFFIC.get((step, workload_name, form))
+    if t is None or t["sha16"] != sources_hash(step):
+        return None
+    return t["bytes"]
 
 
 def load_peaks():
@@ -47,6 +71,7 @@ def load_peaks():
         return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
                 "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
                 "source": "measured"}
+    # the profiling recipe's figures for this pool (burst; sustained under the power cap)
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
 
@@ -169,7 +194,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="online")
-    ap.add_argument("--second", default="upstream,upstream_abs",
+    ap.add_argument("--second", default="upstream,upstream_abs,sweep400,sweep1600,skewed",
                     help="further workloads measured in the same run, comma-separated "
                          "('' = none)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -381,7 +406,7 @@ def main():
                        "tensor_cores": tok.uses_tensor_cores(),
                        "achieved_tflops": t_flops / (t_ms / 1e3) / 1e12,
                        "frac_of_tensor_peak": t_flops / (t_ms / 1e3) / 1e12
-                       / peaks["bf16_tflops_sustained"],
+                       / peaks["bf16_tflops"],
                        "achieved_gbs": t_bytes / (t_ms / 1e3) / 1e9,
                        "frac_of_hbm": t_bytes / (t_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                        "algorithmic_flops": t_flops, "algorithmic_bytes": t_bytes}
@@ -447,28 +472,80 @@ def main():
         ms_e2e = max_over_ranks(t_begin.elapsed_time(t_end))
         h2d = sum(host[n].numel() * host[n].element_size() for n in src_names
                   if host[n] is not None)
+        # the host link alone: one step's host-to-device copies (the same pinned
+        # buffers, nothing else on the GPU), and one 256 MiB pinned copy
+        def copy_ms(fn, reps=5):
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fn()
+            torch.cuda.synchronize()
+            ea.record(cs)
+            for _ in range(reps):
+                fn()
+            eb.record(cs)
+            torch.cuda.synchronize()
+            return ea.elapsed_time(eb) / reps
+
+        def step_copies():
+            with torch.cuda.stream(cs):
+                for name in src_names:
+                    if host[name] is not None and bufs[0][name] is not None:
+                        bufs[0][name].copy_(host[name], non_blocking=True)
+
+        big_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+        big_d = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def big_copy():
+            with torch.cuda.stream(cs):
+                big_d.copy_(big_h, non_blocking=True)
+
+        ms_h2d = copy_ms(step_copies)
+        ms_big = copy_ms(big_copy, reps=3)
+        del big_h, big_d
         e2e = {"value": users_all * e2e_steps / (ms_e2e / 1e3), "unit": "user-seqs/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout[0].numel() * 4),
                "pipeline": "double-buffered: copies of step i overlap compute of step i - 1",
-               "steps": e2e_steps}
+               "steps": e2e_steps,
+               "h2d_ms_per_step": ms_h2d, "h2d_gbs": h2d / (ms_h2d / 1e3) / 1e9,
+               "link_peak_gbs": (256 << 20) / (ms_big / 1e3) / 1e9,
+               "link_note": "h2d_gbs: one step's input copies alone from pinned host memory; "
+                            "link_peak_gbs: one 256 MiB pinned host-to-device copy"}
         assert h.status() == 0
         for g in graphs:
             del g
         graphs = None
 
-        # ---- roofline of the dominant step (largest device time)
+        # ---- roofline of every step, and of the dominant one (largest device
+        # time): the slower of its algorithmic FLOPs at the burst bf16 tensor
+        # peak (the kernels run at full clock inside a step of milliseconds)
+        # and its algorithmic bytes at the HBM bandwidth
         ph = h.per_head_layers()              # layers in MLA's per-head form: their own work
         flops = cost.flops_by_step(inp.lengths, inp.dims, ph)
-        dom = max((k for k in prof if k in flops), key=lambda k: prof[k]["ms"])
+        nbytes = cost.bytes_by_step(inp.lengths, inp.dims, ph)
+        peak = peaks["bf16_tflops"]
+        steps_roof = {}
+        for k, v in prof.items():
+            if not v["calls"]:
+                continue
+            ms_k = v["ms"] / prof_steps
+            r = cost.step_roofline(flops.get(k, 0.0), nbytes.get(k, 0.0), ms_k, peak,
+                                   peaks["hbm_gbs"])
+            r["launches"] = v["launches"] / prof_steps
+            steps_roof[k] = {kk: (round(vv, 5) if isinstance(vv, float) else vv)
+                             for kk, vv in r.items()}
+        dom = max((k for k in prof if k in flops and prof[k]["calls"]),
+                  key=lambda k: prof[k]["ms"])
         dom_ms = prof[dom]["ms"] / max(1, prof[dom]["calls"])       # per launch of the step
         per_launch_flops = flops[dom] / (prof[dom]["calls"] / prof_steps)
         achieved = per_launch_flops / (dom_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        form = "per_head" if ph else "absorbed"
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peaks['source']} sustained bf16 (cuBLAS loop)",
-                "traffic": TRAFFIC.get((dom, wl.name, "per_head" if ph else "absorbed")),
-                "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms}
+                "peak_source": f"{peaks['source']} burst bf16 (cuBLAS, best of 10)",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": traffic_of(dom, wl.name, form),
+                "traffic_sources_sha16": sources_hash(dom),
+                "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms,
+                "bytes_per_launch": nbytes.get(dom, 0.0) / (prof[dom]["calls"] / prof_steps)}
         # the sequence-summary step (bottleneck GEMM + up-projection), when the
         # workload has one, against HBM: the final rows and both projections
         # read once, the summaries written once
@@ -486,10 +563,11 @@ def main():
         step_ms = ms / steps
         whole = {"achieved_tflops": total_flops / (step_ms / 1e3) / 1e12,
                  "frac_of_peak": total_flops / (step_ms / 1e3) / 1e12 / peak,
-                 "flops_per_step": total_flops}
+                 "peak": peak, "flops_per_step": total_flops}
         steps_ms = {k: round(v["ms"] / prof_steps, 4) for k, v in prof.items() if v["calls"]}
         res = dict(value=value, ms=step_ms, e2e=e2e, roofline=roof, whole=whole,
                    clocks=clocks, launches=launches_per_fwd, steps_ms=steps_ms, inp=inp,
+                   steps_roof=steps_roof,
                    dtype=inp.dims.dtype, users_all=users_all, summary=summary,
                    per_head_layers=ph, tokenizer=tok_res)
         del graph
@@ -503,10 +581,11 @@ def main():
     for name2 in [w for w in args.second.split(",") if w and w != args.workload]:
         wl2 = workload(name2)
         s_steps = max(5, min(args.steps, 40))
-        r2 = measure(wl2, s_steps, args.warmup, sample_clocks=False)
+        r2 = measure(wl2, s_steps, args.warmup, sample_clocks=(rank == 0))
         second.append({"workload": wl2.name, "value": r2["value"], "unit": "user-seqs/s",
                        "ms_per_step": r2["ms"], "steps": s_steps, "roofline": r2["roofline"],
                        "whole_step": r2["whole"], "e2e": r2["e2e"], "steps_ms": r2["steps_ms"],
+                       "step_roofline": r2["steps_roof"], "clocks": r2["clocks"],
                        "mla_per_head_layers": r2["per_head_layers"]})
 
     cpu = None
@@ -534,6 +613,7 @@ def main():
             "gpu_launches": int(round(main_res["launches"] * args.steps)),
             "clocks": main_res["clocks"],
             "steps_ms": main_res["steps_ms"],
+            "step_roofline": main_res["steps_roof"],
             "summary": main_res["summary"],
             "tokenizer": main_res["tokenizer"],
             "second": second or None,

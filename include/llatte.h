@@ -273,7 +273,9 @@ int llatte_profile_step(llatte_handle* handle, int step, const char** name, doub
  * larger than LLATTE_PLAN_STATIC_MAX_BATCH users returns
  * LLATTE_ERR_UNSUPPORTED without launching anything.  The first call on a
  * device looks up that array's device address (with the device current);
- * make the first call before any stream capture.  Every call on a device
+ * make the first call before any stream capture.  That address is kept for
+ * the life of the process: do not call this across a reset of the device or
+ * of its primary context (the array then moves).  Every call on a device
  * shares the array: calls that can run at the same time on the GPU race, so
  * order them (one stream, or synchronise in between).  Asynchronous on
  * `stream`; it calls no cudaMalloc or cudaFree.

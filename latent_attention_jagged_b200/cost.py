@@ -149,3 +149,87 @@ def tokenizer_bytes(tdims) -> float:
     embedding rows read once, its token written once (storage type)."""
     e = 2 if tdims.dtype == "bf16" else 4
     return 4.0 * tdims.n_fields + e * tdims.d_in + e * tdims.d
+
+
+def bytes_by_step(lengths: Sequence[int], dims, per_head_layers: int = 0,
+                  tensor_cores: bool = True) -> Dict[str, float]:
+    """HBM bytes each step must move at least in this library's data flow:
+    the step's inputs read once, its weights read once, its outputs written
+    once (the rows that pass between steps live in HBM by design).
+
+    Per layer, with T history rows in, n kept, q = n + n_q query rows, storage
+    element e (2 for bf16), and the fp16 residual copies of the bf16 path:
+      gather   read  sum T d e + B n_q d e          (history events, query tokens)
+               write sum T d e + sum q_0 d e        (key rows, query rows)
+                     + 4 sum_l sum q_l              (row -> user maps)
+      kv       read  sum T d e + r d e              write sum T r e
+               per-head form: + read sum T r e + 2 h d_h r e, write sum T 2 h d_h e
+      q        read  sum q d e + w_q e + 4 B w      write sum q w e   (w = h r, or h d_h)
+      attn     read  sum q w e + sum T r e          write sum q w e   (latent keys once per user;
+               per-head form: the K | V rows, sum T 2 h d_h e)
+      o        read  sum q w e + sum q d 2 + d w e  write sum q d 2   (fp16 Z)
+      ffn      read  sum q d 2 + 2 f d e            write the next layer's rows
+               (sum n d e history + sum q' d 2 query rows), or the fp32 output
+               rows of the last layer (sum n_q d 4, or sum q d 4 for the readout)
+      ffn1     read  sum q d 2 + f d e              write sum q f e
+      ffn2     read  sum q f e + sum q d 2 + f d e  write as ffn
+      readout  read  sum q_L d 4 + d_out d e        write B d_out 4
+    """
+    T = np.asarray(lengths, dtype=np.int64)
+    B = T.shape[0]
+    e = 2 if dims.dtype == "bf16" else 4
+    res = 2 if e == 2 else 4                     # residual-stream copies
+    d, h, r, dh, nq = dims.d, dims.heads, dims.rank, dims.d_head, dims.n_q
+    f = dims.ffn_mult * d
+    acc: Dict[str, float] = {}
+
+    def add(k, v):
+        acc[k] = acc.get(k, 0.0) + float(v)
+
+    L = dims.n_layers
+    Ts, ns = [], []
+    t = T.copy()
+    for k in dims.keep:
+        n = np.minimum(t, k)
+        Ts.append(t)
+        ns.append(n)
+        t = n
+    qs = [n + nq for n in ns]
+    add("gather", T.sum() * d * e + B * nq * d * e + T.sum() * d * e + qs[0].sum() * d * e
+        + 4 * sum(q.sum() for q in qs))
+    for l in range(L):
+        Tl, nl, ql = Ts[l].sum(), ns[l].sum(), qs[l].sum()
+        ph = (per_head_layers >> l) & 1
+        w = h * dh if ph else h * r
+        add("kv", Tl * d * e + r * d * e + Tl * r * e)
+        if ph:
+            add("kv", Tl * r * e + 2 * h * dh * r * e + Tl * 2 * h * dh * e)
+        add("q", ql * d * e + w * (d + dims.d_ctx) * e + 4 * B * w + ql * w * e)
+        add("attn", ql * w * e + (Tl * 2 * h * dh * e if ph else Tl * r * e) + ql * w * e)
+        add("o", ql * w * e + ql * d * res + d * w * e + ql * d * res)
+        if l == L - 1:
+            out = (ql * d * 4) if dims.d_out else (B * nq * d * 4)
+        else:
+            out = ns[l].sum() * d * e + qs[l + 1].sum() * d * res
+        add("ffn", ql * d * res + 2 * f * d * e + out)
+        add("ffn1", ql * d * res + f * d * e + ql * f * e)
+        add("ffn2", ql * f * e + ql * d * res + f * d * e + out)
+    if dims.d_out:
+        add("readout", qs[-1].sum() * d * 4 + dims.d_out * d * e + B * dims.d_out * 4)
+    return acc
+
+
+def step_roofline(flops: float, nbytes: float, ms: float, peak_tflops: float,
+                  peak_gbs: float) -> Dict[str, float]:
+    """Roofline of one step: the slower of its FLOPs at the tensor peak and its
+    bytes at the HBM bandwidth, against the measured time."""
+    s = ms / 1e3
+    t_f = flops / (peak_tflops * 1e12) if flops else 0.0
+    t_b = nbytes / (peak_gbs * 1e9) if nbytes else 0.0
+    return {"ms": ms, "flops": flops, "bytes": nbytes,
+            "tflops": flops / s / 1e12 if s > 0 else 0.0,
+            "gbs": nbytes / s / 1e9 if s > 0 else 0.0,
+            "frac_tensor": t_f / s if s > 0 else 0.0,
+            "frac_hbm": t_b / s if s > 0 else 0.0,
+            "bound": "tensor" if t_f >= t_b else "hbm",
+            "frac": max(t_f, t_b) / s if s > 0 else 0.0}

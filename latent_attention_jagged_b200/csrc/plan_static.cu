@@ -12,7 +12,9 @@
 // The array lives on every GPU that loads the library until the process
 // exits.  Its address is looked up once per device (cudaGetSymbolAddress) on
 // the first call made with that device current; make that first call before
-// any stream capture.  All calls on a device share the array, so calls whose
+// any stream capture.  The address stays cached for the life of the process,
+// so the call must not be used across a device reset (cudaDeviceReset or a
+// primary-context reset), after which the array lives at a new address.  All calls on a device share the array, so calls whose
 // executions overlap on the GPU (different streams, no ordering) race; order
 // them on one stream or synchronise between them.
 #include <mutex>
@@ -83,7 +85,8 @@ extern "C" int llatte_plan_static(const llatte_dims* dims, const int64_t* offset
   if (!base) return LLATTE_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(status_out, 0, sizeof(int32_t), s) != cudaSuccess) return LLATTE_ERR_CUDA;
-  if (B == 0) return LLATTE_OK;
+  // B = 0 runs too: the plan of an empty batch is all zeros, and plan_out
+  // gets them like any other batch's plan
 
   llatte::PlanDev p = {};
   p.stride = kMaxBatch + 1;

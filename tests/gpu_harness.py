@@ -5,6 +5,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+import parity_log
 from latent_attention_jagged_b200 import Llatte
 
 # Tolerances fixed by the target: bf16 max-abs <= 3e-2 and relative L2 <= 1e-2;
@@ -50,11 +51,15 @@ def errors(gpu: np.ndarray, ref: np.ndarray):
     return max_abs, rel
 
 
-def assert_close(gpu, ref, dtype, what=""):
+def assert_close(gpu, ref, dtype, what="", tol=None):
+    """Max-abs and relative-L2 error of gpu against ref within the tolerance of
+    the storage type (or `tol`); the errors are returned and recorded for the
+    session's parity summary."""
     assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
     ma, rl = errors(gpu, ref)
-    tol = TOL[dtype]
+    tol = tol or TOL[dtype]
+    parity_log.record(what, ma, rl, tol, dtype)
     assert ma <= tol["max_abs"] and rl <= tol["rel_l2"], \
         f"{what}: max_abs={ma:.3e} (tol {tol['max_abs']}) rel_l2={rl:.3e} (tol {tol['rel_l2']})"
     return ma, rl

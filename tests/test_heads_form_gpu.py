@@ -24,8 +24,8 @@ def _force(inp, form):
     return dataclasses.replace(inp, dims=dataclasses.replace(inp.dims, attn_form=form))
 
 
-@pytest.mark.parametrize("name,n", [("online", 6), ("upstream", 2), ("skewed", 5),
-                                    ("sweep1600", 2), ("sweep200", 4)])
+@pytest.mark.parametrize("name,n", [("online", 8), ("upstream", 8), ("skewed", 8),
+                                    ("sweep1600", 8), ("sweep200", 8)])
 def test_full_size_per_head_sampled_users(name, n):
     inp = _force(make_inputs(workload(name)), PER_HEAD)
     h, out = run(inp)

@@ -16,8 +16,9 @@ pytestmark = pytest.mark.gpu
 
 FULL = ["online", "upstream", "sweep200", "sweep400", "sweep800", "sweep1600", "skewed"]
 # users the oracle recomputes one by one at full size (the GPU runs the whole batch)
-SAMPLE = {"online": 8, "upstream": 2, "sweep200": 4, "sweep400": 4, "sweep800": 3,
-          "sweep1600": 2, "skewed": 6}
+# (the first ones, plus the longest and the shortest user of the batch)
+SAMPLE = {"online": 8, "upstream": 8, "sweep200": 8, "sweep400": 8, "sweep800": 8,
+          "sweep1600": 8, "skewed": 8}
 
 
 def check_plan(h, inp):

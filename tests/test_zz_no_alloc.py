@@ -74,3 +74,40 @@ def test_plan_static_rejects_oversized_batch_and_reports_bad_offsets():
     torch.cuda.synchronize()
     assert int(st2.item()) == 0 and torch.equal(out2.cpu(), ref)
     h.close()
+
+
+def test_plan_static_reports_long_users_and_row_totals():
+    """The other rejections of the same plan kernel, through the dims this
+    entry point builds: a user longer than max_len, and more rows than
+    max_total.  A rejected batch leaves zeros; the next valid batch is exact."""
+    inp = make_inputs(workload("online"), batch=8)
+    offs = torch.from_numpy(inp.offsets).cuda()
+    h, ref = _reference_plan(inp)
+    longest = int(inp.lengths.max())
+    out, st = binding.plan_static(inp.dims, offs, max_batch=8, max_len=longest - 1)
+    torch.cuda.synchronize()
+    assert int(st.item()) & binding.DEV_TOO_LONG
+    assert int(out.abs().sum().item()) == 0
+    total = int(inp.offsets[-1])
+    out, st = binding.plan_static(inp.dims, offs, max_batch=8, max_len=longest,
+                                  max_total=total - 1)
+    torch.cuda.synchronize()
+    assert int(st.item()) & binding.DEV_TOO_MANY_ROWS
+    assert int(out.abs().sum().item()) == 0
+    out, st = binding.plan_static(inp.dims, offs, max_batch=8, max_len=longest, max_total=total)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and torch.equal(out.cpu(), ref)
+    h.close()
+
+
+def test_plan_static_empty_batch_writes_zeros():
+    """B = 0: every layer's offsets are the single entry 0, written over
+    whatever the caller's buffer held."""
+    inp = make_inputs(workload("online"), batch=8)
+    offs = torch.from_numpy(inp.offsets[:1]).cuda()
+    out = torch.full((len(inp.dims.keep), 2, 1), 77, dtype=torch.int64, device="cuda")
+    st = torch.full((1,), 5, dtype=torch.int32, device="cuda")
+    binding.plan_static(inp.dims, offs, max_batch=8, max_len=400, out=out, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert int(out.abs().sum().item()) == 0
