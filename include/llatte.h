@@ -231,6 +231,25 @@ int llatte_get_status(llatte_handle* handle, int32_t* device_status);
  */
 int llatte_attn_form_mask(const llatte_handle* handle, uint32_t* per_head_layers);
 
+/*
+ * Failure-detection aid; the paper has no counterpart.  Every wait inside the
+ * tensor-core kernels is bounded: a wait that exceeds its limit records
+ * LLATTE_DEV_TIMEOUT in the status word, and the kernel winds down (it lets
+ * its own loads and matrix products in flight finish first) instead of
+ * hanging.  With enable = 1 the forward calls that follow on this handle make
+ * such a wait run out on purpose: in the attention of every layer in MLA's
+ * per-head form, each CTA's matrix-product issuer, once its first products
+ * and tiles are in flight, waits 20 us for an event that never happens.
+ * enable = 0 switches that off.
+ *
+ * A forward during which a wait ran out leaves `out` unspecified and the
+ * status bit set; the handle stays usable, and the next forward without the
+ * injection computes the usual result.  Returns LLATTE_ERR_UNSUPPORTED when no
+ * layer of the handle runs in the per-head form on the tensor cores (see
+ * llatte_attn_form_mask), LLATTE_ERR_ARG for another enable value.
+ */
+int llatte_inject_timeout(llatte_handle* handle, int enable);
+
 /* Bytes of device workspace a handle with these dims allocates (0 on bad dims). */
 size_t llatte_workspace_bytes(const llatte_dims* dims);
 
@@ -286,7 +305,8 @@ int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t 
 
 /*
  * Self-check of an arithmetic building block; the paper has no counterpart.
- * The attention softmax computes one probability pair in eight with an
+ * The attention softmax computes some probability pairs (one in four or one
+ * in eight, by MLA form) with an
  * exponential built from fused multiply-adds (range reduction x = j + f,
  * |f| <= 1/2, a fitted cubic for 2^f, j added to the exponent field) instead
  * of the special-function unit.  This evaluates exactly that device function:

@@ -86,7 +86,7 @@ EXPORTS = ("llatte_create", "llatte_forward", "llatte_plan_export", "llatte_get_
            "llatte_plan_static", "llatte_exp2_eval", "llatte_forward_export",
            "llatte_forward_batch", "llatte_attn_form_mask", "llatte_tokenizer_create",
            "llatte_tokenize", "llatte_tokenizer_get_status", "llatte_tokenizer_uses_tensor_cores",
-           "llatte_tokenizer_destroy")
+           "llatte_tokenizer_destroy", "llatte_inject_timeout")
 TOK_MAX_FIELDS = 8
 PLAN_STATIC_MAX_BATCH = 4096
 
@@ -136,6 +136,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.llatte_exp2_eval.restype = ctypes.c_int
     lib.llatte_attn_form_mask.argtypes = [VP, P(ctypes.c_uint32)]
     lib.llatte_attn_form_mask.restype = ctypes.c_int
+    lib.llatte_inject_timeout.argtypes = [VP, ctypes.c_int]
+    lib.llatte_inject_timeout.restype = ctypes.c_int
     lib.llatte_tokenizer_create.argtypes = [P(VP), P(llatte_tok_dims), P(llatte_tok_w),
                                             ctypes.c_int]
     lib.llatte_tokenizer_create.restype = ctypes.c_int
@@ -252,6 +254,14 @@ class Llatte:
         if rc != LLATTE_OK:
             raise LlatteError(rc, "llatte_attn_form_mask")
         return int(m.value)
+
+    def inject_timeout(self, enable: bool = True):
+        """Failure-detection aid: the forward calls that follow make a bounded
+        wait of the per-head attention run out on purpose (status bit
+        DEV_TIMEOUT, output unspecified) until switched off again."""
+        rc = self.lib.llatte_inject_timeout(self.h, 1 if enable else 0)
+        if rc != LLATTE_OK:
+            raise LlatteError(rc, "llatte_inject_timeout")
 
     def workspace_bytes(self) -> int:
         return int(self.lib.llatte_workspace_bytes(ctypes.byref(self.cdims)))

@@ -1,0 +1,526 @@
+// Fused attention for sm_100a, MLA in its per-head form (LLaTTE notes,
+// huaxiaozhuan.com, appendix A.3 first display: K, V = split(c_kv W_up^KV),
+// scores over d_h = 64; target-aware causal / candidate masking of appendix
+// A.2): per query row and head, s_t = q . k_t over the visible keys,
+// softmax, o = sum_t a_t v_t.
+//
+// At d_h = 64 the work per 128 x 128 tile is four S products of N = 128 and
+// eight P V products of N = 64, which the tensor pipe runs one after the
+// other at a fixed cost each, so the kernel is built to keep that pipe fed:
+// two CTAs per SM, each with one 128-row query tile at a time, so that one
+// CTA's products run while the other CTA's softmax works (the SM interleaves
+// the two CTAs' product streams).  Per CTA:
+//   TMEM   O | S | P        (64 + 128 + 64 = 256 columns, half of the SM's)
+// P is kept apart from S, so S(kt + 1) is computed while the softmax still
+// turns the scores of tile kt into probabilities: the softmax signals "S
+// read" once its last TMEM load of the scores is done, and the MMA issuer
+// starts S(kt + 1) then; O += P(kt) V follows once P(kt) is written.
+//
+// Work item: one user, one head and a block of 128 query rows (the attention
+// work list of the layer, longest first).
+// Roles (192 threads):
+//   warp 0       TMA: the item's query tile (double-buffered, so the next
+//                item's arrives during this one), then its key and value tiles
+//                into a 2-stage ring
+//   warp 1       TMEM owner; lane 0 issues, per key tile, S(kt) once the
+//                softmax has read S(kt - 1), then O += P(kt - 1) V once P(kt - 1)
+//                is written
+//   warps 2..5   softmax, one warp per TMEM lane quadrant: all 128 keys of the
+//                tile for the quadrant's 32 rows, one row per thread, in two
+//                passes over the scores (row max; then 2^(s - m) in fp32), 64
+//                keys at a time (a whole row of S in registers would spill);
+//                masking: a history row at position p sees keys t <= p, a
+//                query token every key t < T; lazy rescale of O when the
+//                running max grows by more than 2^8; P written to TMEM as
+//                bf16 once the previous P V product has read it.  The same
+//                warps divide O by the row sums and store it through shared-
+//                memory staging, deferred into the next item's first tile so
+//                that the softmax never waits for the last product of an item.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_attn.h"
+#include "tc_common.cuh"
+#include "tc_epilogue.cuh"
+
+namespace llatte {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kSoftWarps = 4;                      // one per TMEM lane quadrant
+constexpr int kThreads = 32 * (2 + kSoftWarps);
+constexpr int KEYS = 128;                          // keys per tile
+constexpr int DH = 64;                             // head width
+constexpr int QBUF = 2;                            // query tiles in flight
+constexpr int KS = 2;                              // key / value tiles in the ring
+constexpr uint32_t Q_BYTES = 128 * DH * 2;         // 16 KB
+constexpr uint32_t KV_BYTES = 2 * KEYS * DH * 2;   // K tile + V tile, 32 KB
+constexpr uint32_t V_OFF = KEYS * DH * 2;
+constexpr uint32_t O_COL = 0;
+constexpr uint32_t S_COL = DH;
+constexpr uint32_t P_COL = S_COL + KEYS;           // bf16 pairs: keys 2j, 2j + 1 in column j
+constexpr uint32_t TMEM_COLS = 256;
+static_assert(P_COL + KEYS / 2 <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t BAR_BYTES = 256;
+constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)KS * KV_BYTES + BAR_BYTES +
+                        kSoftWarps * kStageBytes;
+// two CTAs per SM
+static_assert(2 * (SMEM + 1024) <= 233472, "shared memory budget");
+
+struct Item {
+  int u, b;
+  int32_t T, n, q;
+  int nk;            // key tiles (0: no key at all)
+  int64_t hoff, qoff;
+};
+
+// Work entries (user, 128-row block * heads + head) arrive through a
+// two-stage prefetch, so no role waits on a dependent pair of global loads
+// at an item boundary.
+struct ItemStream {
+  int idx;
+  int2 ub;
+  int u, b;
+  int32_t T, n;
+  int64_t hoff, qoff;
+
+  __device__ __forceinline__ static int2 entry(const AttnTcParams& p, int i, int n_items) {
+    return i < n_items ? reinterpret_cast<const int2*>(p.work)[i] : make_int2(-1, 0);
+  }
+  __device__ __forceinline__ void fetch(const AttnTcParams& p, int2 e) {
+    u = e.x;
+    b = e.y;
+    if (u >= 0) {
+      T = p.T[u]; n = p.n[u]; hoff = p.hoff[u]; qoff = p.qoff[u];
+    } else {
+      T = n = 0; hoff = qoff = 0;
+    }
+  }
+  __device__ __forceinline__ void start(const AttnTcParams& p, int first, int n_items, int step) {
+    idx = first;
+    fetch(p, entry(p, first, n_items));
+    ub = entry(p, first + step, n_items);
+  }
+  __device__ __forceinline__ Item next(const AttnTcParams& p, int n_items, int step) {
+    Item it;
+    it.u = u; it.b = b; it.T = T; it.n = n; it.hoff = hoff; it.qoff = qoff;
+    it.q = n + p.n_q;
+    it.nk = 0;
+    if (u >= 0) {
+      // keys visible to the block's last row
+      const int64_t jl = min((int64_t)(b / p.heads) * 128 + 127, (int64_t)it.q - 1);
+      const int64_t kmax = jl < n ? (int64_t)T - n + jl + 1 : T;
+      it.nk = (int)((kmax + KEYS - 1) / KEYS);
+    }
+    fetch(p, ub);
+    idx += step;
+    ub = entry(p, idx + step, n_items);
+    return it;
+  }
+};
+
+// Wait for a phase without giving up on the CTA's abort flag (drains only):
+// still bounded by the default wait limit.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  int never = 0;
+  mbar_wait(bar, parity, &never, status);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+                  const AttnTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;                             // [QBUF][Q_BYTES]
+  uint8_t* sKV = sQ + QBUF * Q_BYTES;             // [KS][KV_BYTES]
+  uint8_t* sStage = sKV + KS * KV_BYTES;          // [kSoftWarps][kStageBytes]
+  uint64_t* bars = (uint64_t*)(sStage + kSoftWarps * kStageBytes);
+  uint64_t* q_full = bars;                        // [QBUF]
+  uint64_t* q_empty = q_full + QBUF;              // [QBUF]
+  uint64_t* kv_full = q_empty + QBUF;             // [KS]
+  uint64_t* kv_empty = kv_full + KS;              // [KS]
+  uint64_t* s_full = kv_empty + KS;               // S(kt) in TMEM
+  uint64_t* s_free = s_full + 1;                  // the softmax has read S(kt)
+  uint64_t* p_full = s_free + 1;                  // P(kt) written
+  uint64_t* pv_done = p_full + 1;                 // O += P(kt) V done (P free)
+  uint64_t* o_free = pv_done + 1;                 // the previous item's O has been read
+  uint64_t* drain = o_free + 1;
+  uint64_t* never = drain + 1;                    // nothing arrives (injected timeout)
+  uint32_t* tmem_slot = (uint32_t*)(never + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  static_assert((2 * QBUF + 2 * KS + 7) * 8 + 8 <= BAR_BYTES, "barrier area");
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int step = gridDim.x;
+  const uint64_t lim = kWaitTimeoutNs;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < QBUF; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+    for (int s = 0; s < KS; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftWarps);
+    mbar_init(p_full, kSoftWarps);
+    mbar_init(pv_done, 1);
+    mbar_init(o_free, kSoftWarps);
+    mbar_init(drain, 1);
+    mbar_init(never, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmKV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  const int n_items = *p.work_count;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t qi = 0, g = 0;          // query tiles, key tiles loaded
+      bool ok = true;
+      ItemStream items;
+      items.start(p, blockIdx.x, n_items, step);
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+        const Item it = items.next(p, n_items, step);
+        if (it.nk == 0) continue;
+        const int head = it.b % p.heads;
+        const int qb = (int)(qi % QBUF);
+        if (!mbar_wait(&q_empty[qb], ((qi / QBUF) & 1) ^ 1, abort_flag, p.status, lim)) break;
+        mbar_arrive_expect_tx(&q_full[qb], Q_BYTES);
+        tma_load_2d(&tmQ, &q_full[qb], sQ + qb * Q_BYTES, head * DH,
+                    (int32_t)(it.qoff + (int64_t)(it.b / p.heads) * 128));
+        ++qi;
+        for (int kt = 0; kt < it.nk; ++kt, ++g) {
+          const int st = g % KS;
+          if (!mbar_wait(&kv_empty[st], ((g / KS) & 1) ^ 1, abort_flag, p.status, lim)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[st], KV_BYTES);
+          const int32_t krow = (int32_t)(it.hoff + (int64_t)kt * KEYS);
+          uint8_t* dst = sKV + st * KV_BYTES;
+          // K then V of this head: columns 64 j and h * 64 + 64 j
+          tma_load_2d(&tmKV, &kv_full[st], dst, head * DH, krow);
+          tma_load_2d(&tmKV, &kv_full[st], dst + V_OFF, (p.heads + head) * DH, krow);
+        }
+      }
+      // no load may still be landing in shared memory when the CTA exits:
+      // wait for the last key tiles and query tiles issued (they complete on
+      // their own; the waits are bounded all the same)
+      for (uint32_t k = 0; k < (uint32_t)KS && k < g; ++k) {
+        const uint32_t gg = g - 1 - k;
+        drain_wait(&kv_full[gg % KS], (gg / KS) & 1, p.status);
+      }
+      for (uint32_t k = 0; k < (uint32_t)QBUF && k < qi; ++k) {
+        const uint32_t qq = qi - 1 - k;
+        drain_wait(&q_full[qq % QBUF], (qq / QBUF) & 1, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(128, KEYS, false, false);
+      constexpr uint32_t IDESC_O = idesc_bf16(128, DH, false, true);
+      uint32_t qi = 0, g = 0;          // query tiles, key tiles consumed (= S products)
+      uint32_t pc = 0, oi = 0;         // P V products issued, items with keys started
+      bool inject = p.inject_timeout != 0;
+      bool ok = true;
+      // the P V product still to be issued
+      struct Pending { int st; bool first, valid; };
+      Pending pend = {0, false, false};
+      auto flush = [&]() -> bool {
+        if (!pend.valid) return true;
+        if (inject) {
+          // failure-detection test: with an S product and key tiles in
+          // flight, wait on a barrier that nothing arrives on, with a short
+          // limit; the wait runs out, records the timeout and winds the CTA
+          // down
+          inject = false;
+          if (!mbar_wait(never, 0, abort_flag, p.status, 20000)) return false;
+        }
+        if (!mbar_wait(p_full, pc & 1, abort_flag, p.status, lim)) return false;
+        // the first product of an item overwrites O: the softmax must have
+        // read the previous item's O
+        if (pend.first && !mbar_wait(o_free, (oi & 1) ^ 1, abort_flag, p.status, lim)) return false;
+        if (pend.first) ++oi;
+        ++pc;
+        tc_fence_after();
+        const uint64_t bd0 =
+            sdesc_sw128(smem_u32(sKV + pend.st * KV_BYTES) + V_OFF, KEYS * 128, 1024);
+#pragma unroll
+        for (int k = 0; k < KEYS / 16; ++k)
+          // 16 keys per MMA step = 2048 bytes of V (MN-major), 8 packed P columns
+          umma_bf16_ts(tmem + O_COL, tmem + P_COL + 8 * k, bd0 + (uint64_t)(128 * k), IDESC_O,
+                       (!pend.first || k > 0) ? 1u : 0u);
+        umma_commit(pv_done);
+        umma_commit(&kv_empty[pend.st]);
+        pend.valid = false;
+        return true;
+      };
+      ItemStream items;
+      items.start(p, blockIdx.x, n_items, step);
+      for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+        const Item it = items.next(p, n_items, step);
+        if (it.nk == 0) continue;
+        const int qb = (int)(qi % QBUF);
+        for (int kt = 0; kt < it.nk; ++kt, ++g) {
+          const int st = g % KS;
+          // S(g) once the softmax has read S(g - 1), the key tile is in and
+          // (first tile of the item) the query tile
+          if (g > 0 && !mbar_wait(s_free, (g - 1) & 1, abort_flag, p.status, lim)) { ok = false; break; }
+          if (!mbar_wait(&kv_full[st], (g / KS) & 1, abort_flag, p.status, lim)) { ok = false; break; }
+          if (kt == 0) {
+            if (!mbar_wait(&q_full[qb], (qi / QBUF) & 1, abort_flag, p.status, lim)) { ok = false; break; }
+            ++qi;
+          }
+          tc_fence_after();
+          const uint64_t ad0 = sdesc_sw128(smem_u32(sQ + qb * Q_BYTES), 16, 1024);
+          const uint64_t bd0 = sdesc_sw128(smem_u32(sKV + st * KV_BYTES), 16, 1024);
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k)   // 16 head dims = 32 bytes per step
+            umma_bf16(tmem + S_COL, ad0 + (uint64_t)(2 * k), bd0 + (uint64_t)(2 * k), IDESC_S,
+                      k > 0 ? 1u : 0u);
+          umma_commit(s_full);
+          if (kt == it.nk - 1) umma_commit(&q_empty[qb]);
+          // then the P V product of the previous key tile
+          if (!flush()) { ok = false; break; }
+          pend = {st, kt == 0, true};
+        }
+      }
+      if (ok) flush();
+      // every MMA of this CTA must be complete before TMEM is released
+      umma_commit(drain);
+      drain_wait(drain, 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int sw = warp - 2;
+    const int quad = warp & 3;                       // TMEM lane quadrant
+    const int row = quad * 32 + lane;                // row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_base = lane_base + S_COL;
+    const uint32_t p_base = lane_base + P_COL;
+    const uint32_t o_base = lane_base + O_COL;
+    const uint32_t stg = smem_u32(sStage + sw * kStageBytes);
+    uint32_t sc = 0;
+    bool ok = true;
+    // The epilogue of an item is deferred into the next item's first tile:
+    // its O is read once the P V product before that tile's P is done (the
+    // wait that tile makes anyway) and that P is handed over (the first
+    // product of the new item also waits for o_free), so the softmax never
+    // stalls for the last product of an item.  The rows and 1 / l of that item:
+    __nv_bfloat16* prev_orow = nullptr;
+    float prev_inv = 0.f;
+    bool prev_pending = false;
+    // O / l of the pending item -> bf16 rows (O holds its last product)
+    auto finish_prev = [&]() {
+      uint4 x[2][4];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float o[32];
+        tmem_ld32(o_base + 32 * c, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= prev_inv;
+        pack_bf16x32(o, x[c]);
+      }
+      // O may take the next item's first product
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) stage_store(stg, x[c], prev_orow ? prev_orow + 32 * c : nullptr);
+      prev_pending = false;
+    };
+    ItemStream items;
+    items.start(p, blockIdx.x, n_items, step);
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
+      const Item it = items.next(p, n_items, step);
+      // this lane's query row jl within the user, and where its 64 output
+      // columns go (null: padding past the user's last row)
+      const int64_t jl = (int64_t)(it.b / p.heads) * 128 + row;
+      const bool valid = it.u >= 0 && jl < (int64_t)it.q;
+      __nv_bfloat16* orow =
+          valid ? p.Ot + (it.qoff + jl) * (int64_t)(p.heads * DH) + (it.b % p.heads) * DH : nullptr;
+      if (it.nk == 0) {                 // no key at all: the attention output is zero
+        const uint4 z[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                            make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        for (int c = 0; c < DH; c += 32) stage_store(stg, z, orow ? orow + c : nullptr);
+        continue;
+      }
+      const int64_t vis = !valid ? 0 : (jl < it.n ? (int64_t)it.T - it.n + jl + 1 : it.T);
+      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
+      for (int kt = 0; kt < it.nk; ++kt) {
+        bool w = mbar_wait(s_full, sc & 1, abort_flag, p.status, lim);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        // keys [0, lim_k) of the tile are visible to the row; masking only
+        // when some row of the warp stops inside the tile.  Padding rows take
+        // every key (they are never stored).
+        const int64_t lim64 = vis - (int64_t)kt * KEYS;
+        const int lim_k = !valid ? KEYS : (lim64 <= 0 ? 0 : (lim64 >= KEYS ? KEYS : (int)lim64));
+        const bool masked = __any_sync(0xffffffffu, lim_k < KEYS);
+        // pass 1: the row max, 64 keys at a time
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float v[64];
+          tmem_ld64(s_base + 64 * h, v);
+          if (masked) {
+            const int lh = lim_k - 64 * h;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = i < lh ? v[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int i = 0; i < 64; i += 16) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
+          }
+        }
+        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        // lazy rescale (only when the max grows by > 8 in log2): l now, O
+        // once the previous P V product is in it (below)
+        float scale = 1.f;
+        bool resc = false;
+        if (kt == 0) {
+          m_run = mt;
+        } else if (mt > m_run + 8.f) {
+          scale = ex2_approx(m_run - mt);
+          m_run = mt;
+          resc = true;
+        }
+        l_run *= scale;
+        // pass 2: probabilities 2^(s - m) as bf16 pairs (keys 2j, 2j + 1 in
+        // packed column j); one pair in four takes the FMA-pipe exponential,
+        // the rest the special-function unit; both give exactly 0 for a masked
+        // score (-inf).  A row that sees no key keeps m = -inf and subtracts
+        // 0 instead.
+        const float m_use = m_run > -INFINITY ? m_run : 0.f;
+        const float2 nm2 = make_float2(-m_use, -m_use);
+        float2 l4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) l4[i] = make_float2(0.f, 0.f);
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[64];
+          tmem_ld64(s_base + 64 * h, v);
+          if (h == 1) {
+            // the scores are in registers: S may take the next tile
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+          }
+          if (masked) {
+            const int lh = lim_k - 64 * h;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = i < lh ? v[i] : -INFINITY;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
+            if ((j & 3) == 3) {
+              x = exp2_fma2(x);
+            } else {
+              x.x = ex2_approx(x.x);
+              x.y = ex2_approx(x.y);
+            }
+            l4[j & 3] = add_f2(l4[j & 3], x);
+            pk[h][j] = pack_bf16(x.x, x.y);
+          }
+        }
+        l_run += ((l4[0].x + l4[0].y) + (l4[1].x + l4[1].y)) +
+                 ((l4[2].x + l4[2].y) + (l4[3].x + l4[3].y));
+        // P and O are free once the previous P V product is done
+        if (sc > 0) {
+          w = mbar_wait(pv_done, (sc - 1) & 1, abort_flag, p.status, lim);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tc_fence_after();
+        }
+        ++sc;
+        if (__any_sync(0xffffffffu, resc)) {
+          float o[32];
+#pragma unroll 1
+          for (int c = 0; c < DH; c += 32) {
+            tmem_ld32(o_base + c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= scale;
+            tmem_st32(o_base + c, o);
+          }
+        }
+        {
+          float f[32];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(pk[h][j]);
+            tmem_st32(p_base + 32 * h, f);          // waits for the store
+          }
+        }
+        // P(kt) written: the MMA may read it once the four warps are in
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        // first tile of an item: the previous item's O is complete (the
+        // product waited for above); this item's first product waits for o_free
+        if (prev_pending) finish_prev();
+      }
+      if (!ok) break;
+      // this item's epilogue waits for the next item's first tile (or the end)
+      prev_orow = orow;
+      prev_inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      prev_pending = true;
+    }
+    if (ok && prev_pending) {
+      // the last item: its final P V product, then its rows
+      bool w = mbar_wait(pv_done, (sc - 1) & 1, abort_flag, p.status, lim);
+      if (__all_sync(0xffffffffu, w)) {
+        tc_fence_after();
+        finish_prev();
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_heads(const CUtensorMap& q, const CUtensorMap& kv, const AttnTcParams& p,
+                              int num_sms, cudaStream_t s) {
+  static uint64_t attr_devices = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_devices >> (dev & 63) & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(attn_heads_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+    if (e != cudaSuccess) return e;
+    attr_devices |= 1ull << (dev & 63);
+  }
+  // two CTAs per SM
+  const int grid = std::max(1, std::min(2 * num_sms, p.max_items));
+  return launch_dependent(attn_heads_kernel, dim3(grid), dim3(kThreads), SMEM, s, 1, q, kv, p);
+}
+
+}  // namespace llatte

@@ -84,17 +84,21 @@ struct GemmCfg {
 // quadrant; `part` selects which BN / P columns this thread handles.  Stores
 // pass through the warp's staging buffer `stg` (row-contiguous global writes).
 template <int BN, int EPI>
-__device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, int64_t row,
-                                         bool valid, int n0, int ks, int g, int part, float* red,
-                                         int rrow, uint64_t* xbar, uint32_t& xphase,
-                                         volatile int* abort_flag, uint32_t stg,
+__device__ __forceinline__ bool epilogue(const TcGemmParams& p, const CUtensorMap* tmD,
+                                         uint32_t taddr, int64_t row, bool valid, int n0, int ks,
+                                         int g, int part, float* red, int rrow, uint64_t* xbar,
+                                         uint32_t& xphase, volatile int* abort_flag, uint32_t stg,
                                          NormPre<BN, 1, GemmCfg<BN, EPI>::P>& pre,
                                          const __nv_bfloat16* sg) {
   constexpr int HB = BN / GemmCfg<BN, EPI>::P;   // columns per thread
   const int c0 = part * HB;
+  // the warp's 32 rows start here; with a store map its rows go out as TMA
+  // boxes of 32 rows x 32 columns (the first row in use decides)
+  const int64_t row0 = row - (threadIdx.x & 31);
+  const bool box_live = __any_sync(0xffffffffu, valid);
   if constexpr (EPI == TC_NORM) {
     return norm_epilogue(p.norm, taddr, row, valid, part, red, rrow, xbar, xphase,
-                             abort_flag, p.status, stg, pre, sg);
+                         abort_flag, p.status, stg, pre, sg, p.d_tma ? tmD : nullptr, row0);
   } else if constexpr (EPI == TC_F32) {
     float* prow =
         valid ? p.Dp + ks * p.slice_stride + g * p.d_group_off + row * p.ldp + n0 : nullptr;
@@ -147,7 +151,10 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
           for (int i = 0; i < 32; ++i) v[32 * h + i] = silu_approx(v[32 * h + i]);
         }
         pack_bf16x32(&v[32 * h], x);
-        stage_store(stg, x, drow ? drow + c + 32 * h : nullptr);
+        if (p.d_tma)
+          stage_store_tma(stg, x, tmD, n0 + c + 32 * h, (int32_t)row0, box_live);
+        else
+          stage_store(stg, x, drow ? drow + c + 32 * h : nullptr);
       }
     }
     return true;
@@ -157,14 +164,17 @@ __device__ __forceinline__ bool epilogue(const TcGemmParams& p, uint32_t taddr, 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const TcGemmParams p) {
+               const __grid_constant__ CUtensorMap tmD, const TcGemmParams p) {
   using Cfg = GemmCfg<BN, EPI>;
   constexpr int STAGES = Cfg::STAGES, NI = Cfg::NI, NSUB = Cfg::NSUB, ACC_BUFS = Cfg::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint64_t* full = (uint64_t*)(sB + STAGES * Cfg::B_BYTES);
+  // per-warp staging buffers right after the ring (1024-byte aligned: they
+  // double as TMA store boxes with the 64-byte swizzle)
+  uint8_t* sStage = sB + STAGES * Cfg::B_BYTES;                          // [warp][kStageBytes]
+  uint64_t* full = (uint64_t*)(sStage + kEpiWarps * kStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + ACC_BUFS;
@@ -173,9 +183,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   // [2 tiles][kParts][128] partial sums of squares (norm epilogue only)
-  float* red = (float*)(smem + STAGES * Cfg::STAGE_BYTES + 256);
-  uint8_t* sStage = (uint8_t*)(red + (EPI == TC_NORM ? 2 * kParts * 128 : 0));   // [warp][kStageBytes]
-  __nv_bfloat16* sG = (__nv_bfloat16*)(sStage + kEpiWarps * kStageBytes);   // RMSNorm gain [BN]
+  float* red = (float*)((uint8_t*)full + 256);
+  __nv_bfloat16* sG = (__nv_bfloat16*)(red + (EPI == TC_NORM ? 2 * kParts * 128 : 0));   // gain [BN]
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -305,7 +314,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       if (active &&
-          !epilogue<BN, EPI>(p, lane_base + acc * BN, row, row < M, nt * BN, ks, g, part,
+          !epilogue<BN, EPI>(p, &tmD, lane_base + acc * BN, row, row < M, nt * BN, ks, g, part,
                              red + (it & 1) * kParts * 128, rr, xbar, xphase, abort_flag,
                              smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
         break;
@@ -314,6 +323,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (lane == 0) mbar_arrive(&tempty[acc]);
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1; }
     }
+    // the bulk stores must be complete before the CTA ends
+    if (p.d_tma) stage_tma_drain();
   }
   __syncthreads();
   if (warp == 1) {
@@ -323,8 +334,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 }
 
 template <int BN, int EPI>
-cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmParams& p,
-                       int grid, cudaStream_t s) {
+cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
+                       const TcGemmParams& p, int grid, cudaStream_t s) {
   using Cfg = GemmCfg<BN, EPI>;
   static uint64_t attr_devices = 0;   // devices on which the smem limit was raised
   int dev = 0;
@@ -337,18 +348,18 @@ cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const TcGemmP
     attr_devices |= 1ull << (dev & 63);
   }
   return launch_dependent(tc_gemm_kernel<BN, EPI>, dim3(grid), dim3(kThreads), Cfg::SMEM, s, 1,
-                          a, b, p);
+                          a, b, d, p);
 }
 
 template <int EPI>
-cudaError_t launch_epi(int BN, const CUtensorMap& a, const CUtensorMap& b, const TcGemmParams& p,
-                       int grid, cudaStream_t s) {
+cudaError_t launch_epi(int BN, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
+                       const TcGemmParams& p, int grid, cudaStream_t s) {
   switch (BN) {
-    case 64: return launch_cfg<64, EPI>(a, b, p, grid, s);
-    case 128: return launch_cfg<128, EPI>(a, b, p, grid, s);
-    case 256: return launch_cfg<256, EPI>(a, b, p, grid, s);
+    case 64: return launch_cfg<64, EPI>(a, b, d, p, grid, s);
+    case 128: return launch_cfg<128, EPI>(a, b, d, p, grid, s);
+    case 256: return launch_cfg<256, EPI>(a, b, d, p, grid, s);
     case 512:
-      if constexpr (EPI == TC_NORM) return launch_cfg<512, EPI>(a, b, p, grid, s);
+      if constexpr (EPI == TC_NORM) return launch_cfg<512, EPI>(a, b, d, p, grid, s);
       else return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
@@ -366,8 +377,18 @@ bool tc_gemm_supported(int BN, int epi, int N, int K) {
 }
 
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
-                           const TcGemmParams& p, int num_sms, cudaStream_t s) {
-  if (!tc_gemm_supported(BN, epi, p.N, p.K)) return cudaErrorInvalidValue;
+                           const TcGemmParams& p_in, int num_sms, cudaStream_t s,
+                           const CUtensorMap* d) {
+  if (!tc_gemm_supported(BN, epi, p_in.N, p_in.K)) return cudaErrorInvalidValue;
+  TcGemmParams p = p_in;
+  // bulk tensor stores: the plain-store epilogues, and the norm epilogue with
+  // one plain output (bf16 dst, or its fp16 residual copy alone)
+  p.d_tma = 0;
+  if (d && (epi == TC_STORE || epi == TC_USERBIAS || epi == TC_SILU ||
+            (epi == TC_NORM && p.norm.mode == NORM_PLAIN && ((p.norm.dst != nullptr) !=
+                                                              (p.norm.dst_res != nullptr)))))
+    p.d_tma = 1;
+  const CUtensorMap& dm = p.d_tma ? *d : a;     // (unused without bulk stores)
   if (epi == TC_F32 &&
       (p.k_split < 1 || p.k_split > p.K / BK || p.groups < 1 || !p.Dp || p.ldp % 4 != 0 ||
        p.d_group_off % 4 != 0 || p.slice_stride % 4 != 0 ||
@@ -380,13 +401,13 @@ cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensor
                             (epi == TC_F32 ? (int64_t)p.k_split * p.groups : 1);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms, max_tiles));
   switch (epi) {
-    case TC_STORE: return launch_epi<TC_STORE>(BN, a, b, p, grid, s);
-    case TC_USERBIAS: return launch_epi<TC_USERBIAS>(BN, a, b, p, grid, s);
-    case TC_SILU: return launch_epi<TC_SILU>(BN, a, b, p, grid, s);
-    case TC_NORM: return launch_epi<TC_NORM>(BN, a, b, p, grid, s);
+    case TC_STORE: return launch_epi<TC_STORE>(BN, a, b, dm, p, grid, s);
+    case TC_USERBIAS: return launch_epi<TC_USERBIAS>(BN, a, b, dm, p, grid, s);
+    case TC_SILU: return launch_epi<TC_SILU>(BN, a, b, dm, p, grid, s);
+    case TC_NORM: return launch_epi<TC_NORM>(BN, a, b, dm, p, grid, s);
     case TC_F32:
-      if (BN == 64) return launch_cfg<64, TC_F32>(a, b, p, grid, s);
-      if (BN == 128) return launch_cfg<128, TC_F32>(a, b, p, grid, s);
+      if (BN == 64) return launch_cfg<64, TC_F32>(a, b, dm, p, grid, s);
+      if (BN == 128) return launch_cfg<128, TC_F32>(a, b, dm, p, grid, s);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
@@ -429,6 +450,20 @@ bool make_tmap_16(CUtensorMap* map, CUtensorMapDataType type, const void* base, 
   return r == CUDA_SUCCESS;
 }
 }  // namespace
+
+bool make_tmap_store16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, bool f16) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols % 32 != 0 || ((uintptr_t)base & 15)) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows) {

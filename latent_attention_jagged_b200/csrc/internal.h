@@ -137,10 +137,16 @@ struct llatte_handle {
   int ffn_fused;                  // FFN up + SiLU + down in one kernel (d = 256)
   int pair_norm;                  // output / FFN-down projections on SM pairs (d = 512)
   CUtensorMap tm_Qt, tm_C;        // attention operands: [sum q * h, r] and [sum T, r]
+  // store maps of the GEMM outputs (boxes of 32 rows x 32 columns): latent C,
+  // the per-head K | V rows, the query rows ([rows, h r] and per-head
+  // [rows, h d_h]), the low-rank query latent, fp16 Z, the FFN hidden rows
+  CUtensorMap tms_C, tms_KV, tms_Qt, tms_Qh, tms_Cq, tms_Zres, tms_Hd;
   CUtensorMap tm_zraw, tm_sdown;  // summary bottleneck GEMM operands
   // per-head attention form: bit l = layer l runs it; its K | V rows, and the
   // query / output rows laid out [rows, h*d_h] (in the Qt / Ot memory)
   uint32_t heads_mask;
+  int inject_timeout;             // failure-detection test: the next forwards' per-head
+                                  //   attention runs a wait out on purpose
   void* KV;                       // [max_rows_h, 2*h*d_h]
   CUtensorMap tm_Qh, tm_KV, tm_Oh;
   CUtensorMap tm_sh16, tm_sup;    // summary output-projection GEMM operands

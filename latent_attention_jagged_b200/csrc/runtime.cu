@@ -279,6 +279,15 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&h->tm_Oh, h->Ot, rq, hdh, 128);
     h->pair_norm = h->pair_norm && tc_gemm_pair_supported(TC_NORM, d, hdh);
   }
+  ok = ok && make_tmap_store16(&h->tms_C, h->C, rh, r, false);
+  ok = ok && make_tmap_store16(&h->tms_Qt, h->Qt, rq, hr, false);
+  ok = ok && make_tmap_store16(&h->tms_Hd, h->Hd, rq, f, false);
+  if (h->Zres) ok = ok && make_tmap_store16(&h->tms_Zres, h->Zres, rq, d, true);
+  if (D.q_rank) ok = ok && make_tmap_store16(&h->tms_Cq, h->Cq, rq, D.q_rank, false);
+  if (h->heads_mask) {
+    ok = ok && make_tmap_store16(&h->tms_KV, h->KV, rh, 2 * hdh, false);
+    ok = ok && make_tmap_store16(&h->tms_Qh, h->Qt, rq, hdh, false);
+  }
   auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
   for (int l = 0; l < D.n_layers && ok; ++l) {
     const LayerDev& W = h->layers[l];
@@ -393,6 +402,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->dims = D;
   h->elem = D.dtype == LLATTE_BF16 ? 2 : 4;
   h->use_tc = 0;
+  h->inject_timeout = 0;
   h->profiling = 0;
   h->last_B = 0;
   h->export_req = nullptr;
@@ -732,12 +742,13 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.norm = kv_norm;
         q.D = (__nv_bfloat16*)h->C; q.ldd = r;
         CK(launch_tc_gemm(h->bn_kv, D.kv_norm ? TC_NORM : TC_STORE, h->tm_Xh[l & 1], LM.dkv, q,
-                          h->num_sms, s));
+                          h->num_sms, s, &h->tms_C));
         if (per_head) {
           // K | V = c_kv [W_uk ; W_uv]^T, every head's keys and values
           TcGemmParams k2 = tcp(p.hist_total(l), h->max_rows_h, 2 * hdh, r);
           k2.D = (__nv_bfloat16*)h->KV; k2.ldd = 2 * hdh;
-          CK(launch_tc_gemm(pick_bn(2 * hdh), TC_STORE, h->tm_C, LM.ukv, k2, h->num_sms, s));
+          CK(launch_tc_gemm(pick_bn(2 * hdh), TC_STORE, h->tm_C, LM.ukv, k2, h->num_sms, s,
+                            &h->tms_KV));
           t.done(2);
         } else {
           t.done(1);
@@ -774,7 +785,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.ab_f16 = q16 ? 1 : 0;
         CK(launch_tc_gemm(pick_bn(hdh), D.d_ctx > 0 ? TC_USERBIAS : TC_STORE,
                           q16 ? h->tm_Xqres[l & 1] : h->tm_Xq[l & 1], q16 ? LM.qh16 : LM.qh, q,
-                          h->num_sms, s));
+                          h->num_sms, s, &h->tms_Qh));
       } else if (rq) {
         // low-rank query: Cq = RMSNorm_{g_q}(R W_dq,x^T + context term of the
         // row's user), then the absorbed projection Qt = Cq (W_uk^T W_uq)^T
@@ -788,10 +799,11 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
           }
           TcGemmParams q1 = tcp(p.query_total(l), h->max_rows_q, rq, d);
           q1.norm = qn;
-          CK(launch_tc_gemm(h->bn_dq, TC_NORM, h->tm_Xq[l & 1], LM.dq, q1, h->num_sms, s));
+          CK(launch_tc_gemm(h->bn_dq, TC_NORM, h->tm_Xq[l & 1], LM.dq, q1, h->num_sms, s,
+                            &h->tms_Cq));
           TcGemmParams q2 = tcp(p.query_total(l), h->max_rows_q, hr, rq);
           q2.D = (__nv_bfloat16*)h->Qt; q2.ldd = hr;
-          CK(launch_tc_gemm(h->bn_q, TC_STORE, h->tm_Cq, LM.qk, q2, h->num_sms, s));
+          CK(launch_tc_gemm(h->bn_q, TC_STORE, h->tm_Cq, LM.qk, q2, h->num_sms, s, &h->tms_Qt));
           t.done(2);
         } else {
           GemmArgs g = {};
@@ -817,7 +829,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.ab_f16 = q16 ? 1 : 0;
         CK(launch_tc_gemm(h->bn_q, D.d_ctx > 0 ? TC_USERBIAS : TC_STORE,
                           q16 ? h->tm_Xqres[l & 1] : h->tm_Xq[l & 1], q16 ? LM.qk16 : LM.qk,
-                          q, h->num_sms, s));
+                          q, h->num_sms, s, &h->tms_Qt));
       } else {
         GemmArgs g = {};
         g.A = Xq_l; g.lda = d; g.W = W.W_qk; g.D = h->Qt; g.ldd = hr;
@@ -834,8 +846,8 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
       a.work = p.work + (int64_t)l * 2 * p.max_work; a.work_count = p.work_count + l;
       a.max_items = p.max_work; a.T = p.Tl(l); a.n = p.nl(l); a.hoff = p.hoff(l);
       a.qoff = p.qoff(l); a.n_q = D.n_q; a.heads = D.heads; a.Ot = (__nv_bfloat16*)h->Ot;
-      a.status = p.status;
-      if (per_head) CK(launch_attn_tc_heads(h->tm_Qh, h->tm_KV, a, h->num_sms, s));
+      a.status = p.status; a.inject_timeout = h->inject_timeout;
+      if (per_head) CK(launch_attn_heads(h->tm_Qh, h->tm_KV, a, h->num_sms, s));
       else CK(launch_attn_tc(r, h->tm_Qt, h->tm_C, a, h->num_sms, s));
       t.done(1);
     } else {  // latent attention, CUDA cores
@@ -873,7 +885,8 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         if (h->pair_norm)
           CK(launch_tc_gemm_pair(TC_NORM, oa, per_head ? LM.oh_pair : LM.ov_pair, q, h->num_sms, s));
         else
-          CK(launch_tc_gemm(h->bn_o, TC_NORM, oa, per_head ? LM.oh : LM.ov, q, h->num_sms, s));
+          CK(launch_tc_gemm(h->bn_o, TC_NORM, oa, per_head ? LM.oh : LM.ov, q, h->num_sms, s,
+                            &h->tms_Zres));
         t.done(1);
       } else {
         GemmArgs g = {};
@@ -903,7 +916,7 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
         q.D = (__nv_bfloat16*)h->Hd; q.ldd = f;
         q.ab_f16 = z16_only ? 1 : 0;
         CK(launch_tc_gemm(h->bn_f1, TC_SILU, z16_only ? h->tm_Zres : h->tm_Z,
-                          z16_only ? LM.w1h : LM.w1, q, h->num_sms, s));
+                          z16_only ? LM.w1h : LM.w1, q, h->num_sms, s, &h->tms_Hd));
       } else {
         GemmArgs g = {};
         g.A = h->Z; g.lda = d; g.W = W.W1; g.D = h->Hd; g.ldd = f;
@@ -1043,6 +1056,13 @@ int llatte_get_status(llatte_handle* h, int32_t* device_status) {
 int llatte_attn_form_mask(const llatte_handle* h, uint32_t* per_head_layers) {
   if (!h || !per_head_layers) return LLATTE_ERR_ARG;
   *per_head_layers = h->heads_mask;
+  return LLATTE_OK;
+}
+
+int llatte_inject_timeout(llatte_handle* h, int enable) {
+  if (!h || (enable != 0 && enable != 1)) return LLATTE_ERR_ARG;
+  if (!h->use_tc || h->heads_mask == 0) return LLATTE_ERR_UNSUPPORTED;
+  h->inject_timeout = enable;
   return LLATTE_OK;
 }
 

@@ -16,6 +16,8 @@ struct AttnTcParams {
   int n_q, heads;
   __nv_bfloat16* Ot;          // [sum q * heads, r]; per-head form: [sum q, heads * 64]
   int32_t* status;
+  int inject_timeout;         // per-head kernel: every CTA's MMA issuer waits once on a barrier
+                              //   that nothing arrives on (failure-detection test)
 };
 
 int attn_tc_keys(int r);
@@ -24,7 +26,11 @@ cudaError_t launch_attn_tc(int r, const CUtensorMap& q, const CUtensorMap& c,
                            const AttnTcParams& p, int num_sms, cudaStream_t s);
 // Per-head form (d_h = 64): q over [sum q, heads * 64] (128-row boxes), kv over
 // [sum T, 2 * heads * 64] (K then V, 128-row boxes); work items (user,
-// 128-row block * heads + head).
+// 128-row block * heads + head); two CTAs per SM.
+cudaError_t launch_attn_heads(const CUtensorMap& q, const CUtensorMap& kv, const AttnTcParams& p,
+                              int num_sms, cudaStream_t s);
+// The same with one query tile per CTA over eight softmax warps (the layout of
+// the absorbed kernel); kept for comparison.
 cudaError_t launch_attn_tc_heads(const CUtensorMap& q, const CUtensorMap& kv,
                                  const AttnTcParams& p, int num_sms, cudaStream_t s);
 

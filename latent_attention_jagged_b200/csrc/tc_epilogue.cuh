@@ -52,6 +52,35 @@ __device__ __forceinline__ void stage_store(uint32_t stg, const uint4 (&x)[4], v
   __syncwarp();
 }
 
+// The same 32 x 64-byte staging, stored by one bulk tensor copy instead of
+// per-lane global stores: the staging layout (16-byte chunk k of row r at
+// chunk k ^ ((r >> 1) & 3), buffer 512-byte aligned) is the 64-byte swizzle
+// of a TMA box of 32 rows x 32 16-bit columns, so lane l's row goes to row
+// y + l, columns x .. x + 31 of the map's tensor (rows past the tensor's end
+// are dropped by the copy).  `store` false stages nothing to global memory
+// (a box that lies wholly past the rows in use).  The buffer is reused only
+// after the previous copy out of it has read it; call stage_tma_drain once
+// after the last box.
+__device__ __forceinline__ void stage_store_tma(uint32_t stg, const uint4 (&x)[4],
+                                                const CUtensorMap* map, int32_t cx, int32_t cy,
+                                                bool store) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) tma_store_wait_read();
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_shared_v4(stage_slot(stg, lane, j), x[j]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && store) {
+    tma_store_2d(map, stg, cx, cy);
+    tma_store_commit();
+  }
+}
+__device__ __forceinline__ void stage_tma_drain() {
+  if ((threadIdx.x & 31) == 0) tma_store_wait_all();
+  __syncwarp();
+}
+
 // Global loads of the 64 bytes at lane r's `src` (zeros for a null pointer),
 // 8 rows per instruction; stage_deliver then hands each lane its own row.
 __device__ __forceinline__ void stage_fetch(const void* src, uint4 (&t)[4]) {
@@ -121,14 +150,18 @@ __device__ __forceinline__ void load_gain(const NormArgs& a, int N, __nv_bfloat1
 // accumulator, adds the residual (read once, from the chunks `pre` holds and
 // refills) and stages the sum back in TMEM; pass 2
 // normalises, applies the gain (`sg`, in shared memory) and stores.  Global
-// reads and writes go through the warp's staging buffer `stg`.
+// reads and writes go through the warp's staging buffer `stg`.  With `tmap`
+// (NORM_PLAIN with a single output, dst or dst_res, of the map's type) the
+// rows leave as TMA boxes of 32 rows (from row0) x 32 columns.
 template <int BN, int PDMAX, int P>
 __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr, int64_t row,
                                               bool valid, int part, float* red, int rrow,
                                               uint64_t* xbar, uint32_t& xphase,
                                               volatile int* abort_flag, int32_t* status,
                                               uint32_t stg, NormPre<BN, PDMAX, P>& pre,
-                                              const __nv_bfloat16* sg) {
+                                              const __nv_bfloat16* sg,
+                                              const CUtensorMap* tmap = nullptr,
+                                              int64_t row0 = 0) {
   constexpr int HB = BN / P;
   const int c0 = part * HB;
   const int N = BN;
@@ -219,6 +252,7 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
   const unsigned full = 0xffffffffu;
   const bool any_d1 = __any_sync(full, d1 != nullptr), any_d2 = __any_sync(full, d2 != nullptr);
   const bool any_f1 = __any_sync(full, f1 != nullptr), any_r1 = __any_sync(full, r1 != nullptr);
+  const bool box_live = __any_sync(full, valid);
   // pass 2: normalise, scale by the gain, store
 #pragma unroll 1
   for (int c = c0; c < c0 + HB; c += 32) {
@@ -240,6 +274,19 @@ __device__ __forceinline__ bool norm_epilogue(const NormArgs& a, uint32_t taddr,
       }
     }
     uint4 x[4];
+    if (tmap) {
+      // one plain output: bf16 dst or the fp16 residual copy, by TMA
+      if (a.dst) {
+        pack_bf16x32(v, x);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x[j] = make_uint4(pack_f16(v[8 * j], v[8 * j + 1]), pack_f16(v[8 * j + 2], v[8 * j + 3]),
+                            pack_f16(v[8 * j + 4], v[8 * j + 5]), pack_f16(v[8 * j + 6], v[8 * j + 7]));
+      }
+      stage_store_tma(stg, x, tmap, c, (int32_t)row0, box_live);
+      continue;
+    }
     if (any_d1 || any_d2) {
       pack_bf16x32(v, x);
       if (any_d1) stage_store(stg, x, d1 ? d1 + c : nullptr);

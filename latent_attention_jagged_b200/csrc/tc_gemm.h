@@ -29,6 +29,7 @@ struct TcGemmParams {
   int groups; int64_t a_group_rows; int w_group_rows; int64_t d_group_off; int64_t ldp;
   int32_t* status;
   int ab_f16;                   // A and the weight in fp16 (both operands of every MMA), else bf16
+  int d_tma;                    // (set by the launcher) output stored by TMA boxes
 };
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
@@ -37,8 +38,15 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                    uint32_t box_rows);
 bool tc_gemm_supported(int BN, int epi, int N, int K);
+// d: a store map of the output (make_tmap_store16), or NULL: STORE / USERBIAS /
+// SILU and a NORM_PLAIN epilogue with one output then write their rows as TMA
+// boxes of 32 x 32 (rows past M up to the map's row count may be written).
 cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensorMap& b,
-                           const TcGemmParams& p, int num_sms, cudaStream_t s);
+                           const TcGemmParams& p, int num_sms, cudaStream_t s,
+                           const CUtensorMap* d = nullptr);
+// Store map of a 16-bit [rows, cols] tensor for the epilogues: boxes of 32 rows x
+// 32 columns with the 64-byte swizzle (the staging layout).  fp16 when f16.
+bool make_tmap_store16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, bool f16);
 // Residual + RMSNorm GEMM with N = 512 on pairs of SMs (256-row tiles); b_half:
 // the weight with 128-row boxes (each CTA loads half of a k-block).
 bool tc_gemm_pair_supported(int epi, int N, int K);
