@@ -139,7 +139,13 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   // heads_mask), per (user, 128-row block, head) with b = block * heads + head
   // -- ordered by the number of key tiles the block visits, largest first (a
   // counting sort over at most kBuckets cost classes), so that the persistent
-  // attention CTAs take the longest items first.
+  // attention CTAs take the longest items first.  A per-head layer orders its
+  // items by user instead (users with the most key tiles first; within a
+  // user head by head, the longest block first), so that the blocks of one
+  // (user, head), which read the same key and value tiles, run at the same
+  // time on neighbouring CTAs and share those tiles through L2 (ordered by
+  // cost, all users' blocks of one cost class ran together and their key /
+  // value tiles did not fit in L2).
   constexpr int kBuckets = 64;
   __shared__ int32_t hist[kBuckets], cursor[kBuckets];
   __shared__ int32_t total_items;
@@ -179,6 +185,40 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     }
     return lo;
   };
+  int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
+  if (per_head) {
+    // users by the key tiles of their last row (bucketed, descending); each
+    // user claims one consecutive range of the list for its items
+    auto ucost = [&](int u) {
+      const int64_t tiles = ((int64_t)Tl[u] + attn_keys - 1) / attn_keys;
+      return (int)(tiles < kBuckets - 1 ? tiles : kBuckets - 1);
+    };
+    for (int u = u0; u < u1; ++u) atomicAdd(&hist[ucost(u)], (int32_t)items_of(u));
+    __syncthreads();
+    if (tid == 0) {
+      int32_t acc = 0;
+      for (int k = kBuckets - 1; k >= 0; --k) { cursor[k] = acc; acc += hist[k]; }
+      total_items = acc;
+    }
+    __syncthreads();
+    for (int u = u0; u < u1; ++u) {
+      const int32_t n_items_u = (int32_t)items_of(u);
+      if (n_items_u == 0) continue;
+      const int32_t nblk = n_items_u / heads;
+      const int32_t ubase = atomicAdd(&cursor[ucost(u)], n_items_u);
+      for (int32_t b = 0; b < n_items_u; ++b) {
+        const int32_t blk = b / heads, head = b % heads;
+        const int32_t pos = ubase + head * nblk + (nblk - 1 - blk);
+        W[2 * pos] = u;
+        W[2 * pos + 1] = b;
+      }
+    }
+    if (tid == 0) {
+      p.work_count[l] = total_items;
+      p.work_next[l] = 0;
+    }
+    return;
+  }
   for (int i = tid; i < (int)total; i += kPlanThreads) {
     const int u = user_of(i);
     atomicAdd(&hist[cost_of(u, i - item_off[u])], 1);
@@ -190,7 +230,6 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     total_items = acc;
   }
   __syncthreads();
-  int32_t* W = p.work + (int64_t)l * 2 * p.max_work;
   for (int i = tid; i < (int)total; i += kPlanThreads) {
     const int u = user_of(i);
     const int b = i - item_off[u];
