@@ -60,6 +60,7 @@ template <int BN, int EPI>
 struct GemmCfg {
   static constexpr int NI = BN > 256 ? 256 : BN;     // N of one MMA instruction
   static constexpr int NSUB = BN / NI;
+  static constexpr int WB = BN < 128 ? BN : 128;     // weight rows per TMA box
   static constexpr int ACC_BUFS = 2 * BN <= 512 ? 2 : 1;
   static constexpr uint32_t TMEM_COLS =
       ACC_BUFS * BN <= 32 ? 32 : ACC_BUFS * BN <= 64 ? 64 : ACC_BUFS * BN <= 128 ? 128
@@ -241,10 +242,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // same weight lines from L2 at the same moment
           const int kx = (kb_lo + (kb + kb0) % nkb) * BK;
           tma_load_2d(&tmA, &full[stage], sA + stage * Cfg::A_BYTES, kx, a_row);
+          // the weight k-block in boxes of at most 128 rows (stacked, they
+          // form the same 128-byte-swizzled tile as one box of BN rows)
 #pragma unroll
-          for (int s2 = 0; s2 < NSUB; ++s2)
-            tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * NI * 128, kx,
-                        w_row + s2 * NI);
+          for (int s2 = 0; s2 < BN / Cfg::WB; ++s2)
+            tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * Cfg::WB * 128, kx,
+                        w_row + s2 * Cfg::WB);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -351,6 +354,248 @@ cudaError_t launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
                           a, b, d, p);
 }
 
+// ---------------------------------------------------------------- SM pairs
+// The same GEMM on pairs of SMs for BN = 256: a cluster of two CTAs takes
+// 256-row tiles, rank 0 issues cta_group::2 MMAs (M = 256, N = 256), each CTA
+// loads its own 128 rows of A and 128 of the 256 weight rows of every k-block
+// (the pair's tensor cores read both halves), so that per FLOP a CTA moves
+// two thirds of the bytes the one-SM tile moves through L2 and shared
+// memory (the one-SM 128 x 256 tile is bound by that traffic).  Each CTA's
+// TMEM holds its 128 rows of the accumulator, double-buffered (2 x 256
+// columns), and its 16 epilogue warps run the usual epilogues on them.
+// Completion of the pair MMAs reaches both CTAs by multicast commit; rank 1's
+// "accumulator free" is forwarded to rank 0 by one thread, one remote arrival
+// per tile.
+template <int EPI>
+struct Pair2Cfg {
+  static constexpr int BN = 256;
+  static constexpr uint32_t A_BYTES = 128 * BK * 2;   // this CTA's 128 rows
+  static constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's half of the weight rows
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr size_t FIXED = 1024 + 256 + kEpiWarps * kStageBytes +
+                                  (EPI == TC_NORM ? 2 * kParts * 128 * 4 + BN * 2 : 0);
+  static constexpr int STAGES_FIT = (int)((kSmemMax - FIXED) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT < 8 ? STAGES_FIT : 8;
+  static constexpr size_t SMEM = FIXED + (size_t)STAGES * STAGE_BYTES;
+  static_assert(STAGES >= 3, "pipeline depth");
+  static_assert(SMEM <= kSmemMax, "shared memory budget");
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmD, const TcGemmParams p) {
+  using Cfg = Pair2Cfg<EPI>;
+  constexpr int BN = 256, STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* sStage = sB + STAGES * Cfg::B_BYTES;                          // [warp][kStageBytes]
+  uint64_t* full = (uint64_t*)(sStage + kEpiWarps * kStageBytes);         // [STAGES] rank 0: both CTAs' bytes
+  uint64_t* empty = full + STAGES;                                        // [STAGES] both
+  uint64_t* tfull = empty + STAGES;                                       // [2] both
+  uint64_t* tempty = tfull + 2;                                           // [2] this CTA's epilogue done
+  uint64_t* tempty_peer = tempty + 2;                                     // [2] rank 0: rank 1's done
+  uint64_t* drain = tempty_peer + 2;
+  uint64_t* xbar = drain + 1;                 // epilogue group barrier (norm exchange)
+  uint32_t* tmem_slot = (uint32_t*)(xbar + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* red = (float*)((uint8_t*)full + 256);
+  __nv_bfloat16* sG = (__nv_bfloat16*)(red + (EPI == TC_NORM ? 2 * kParts * 128 : 0));
+  static_assert((2 * STAGES + 8) * 8 + 8 <= 256, "barrier area");
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_tiles = p.N / BN;
+  const int KB = p.K / BK;
+  const int kb0 = pair % KB;
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < STAGES; ++s2) { mbar_init(&full[s2], 1); mbar_init(&empty[s2], 1); }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty_peer[a], 1);
+    }
+    mbar_init(drain, 1);
+    mbar_init(xbar, 4 * kParts);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  if constexpr (EPI == TC_NORM) load_gain(p.norm, BN, sG);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();          // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // everything below reads what earlier kernels wrote
+  pdl_wait();
+  const int64_t M = p.M_dev ? *p.M_dev : p.M_host;
+  const int64_t num_tiles = ((M + 2 * BM - 1) / (2 * BM)) * n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t t = pair; t < num_tiles && ok; t += n_pairs) {
+        const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
+        const int32_t a_row = mt * 2 * BM + BM * (int)rank;
+        const int32_t w_row = nt * BN + 128 * (int)rank;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+          const uint32_t full_c = cluster_addr(&full[stage], 0);
+          // k-blocks in a per-pair rotated order: the SMs do not all read the
+          // same weight lines from L2 at the same moment
+          const int kx = ((kb + kb0) % KB) * BK;
+          tma_load_2d_pair(&tmA, full_c, sA + stage * Cfg::A_BYTES, kx, a_row);
+          tma_load_2d_pair(&tmB, full_c, sB + stage * Cfg::B_BYTES, kx, w_row);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      // A and the weight: both fp16 or both bf16 (the caller's choice)
+      const uint32_t IDESC = p.ab_f16 ? idesc_f16(2 * BM, BN, false, false)
+                                      : idesc_bf16(2 * BM, BN, false, false);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = pair; t < num_tiles && ok; t += n_pairs) {
+        // both CTAs' epilogues have read this accumulator's previous tile
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status) ||
+            !mbar_wait_cluster(&tempty_peer[acc], acc_phase ^ 1, abort_flag, p.status))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad0 = sdesc_sw128(smem_u32(sA + stage * Cfg::A_BYTES), 16, 1024);
+          const uint64_t bd0 = sdesc_sw128(smem_u32(sB + stage * Cfg::B_BYTES), 16, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)   // 16 elements of K = 32 bytes per step
+            umma_bf16_pair(d, ad0 + (uint64_t)(2 * k), bd0 + (uint64_t)(2 * k), IDESC,
+                           (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // every pair MMA must be complete before either CTA releases TMEM
+      umma_commit_pair(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, &dummy, p.status);
+    } else if (lane == 0) {
+      // rank 1: forward this CTA's "accumulator free" to rank 0
+      const uint32_t peer_c[2] = {cluster_addr(&tempty_peer[0], 0), cluster_addr(&tempty_peer[1], 0)};
+      uint32_t ti = 0;
+      for (int64_t t = pair; t < num_tiles; t += n_pairs, ++ti) {
+        if (!mbar_wait(&tempty[ti & 1], (ti >> 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_cluster(peer_c[ti & 1]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                // TMEM lane quadrant this warp may access
+    const int part = (warp - 2) >> 2;      // which quarter of the tile's columns
+    const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    int acc = 0, it = 0;
+    uint32_t acc_phase = 0, xphase = 0;
+    for (int64_t t = pair; t < num_tiles; t += n_pairs, ++it) {
+      const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
+      const int rr = q * 32 + lane;
+      const int64_t row = (int64_t)mt * 2 * BM + BM * (int64_t)rank + rr;
+      NormPre<BN, 1, GemmCfg<BN, EPI>::P> pre;
+      if constexpr (EPI == TC_NORM) norm_prefetch(p.norm, row, row < M, part, pre);
+      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      if (!epilogue<BN, EPI>(p, &tmD, lane_base + acc * BN, row, row < M, nt * BN, 0, 0, part,
+                             red + (it & 1) * kParts * 128, rr, xbar, xphase, abort_flag,
+                             smem_u32(sStage + (warp - 2) * kStageBytes), pre, sG))
+        break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    // the bulk stores must be complete before the CTA ends
+    if (p.d_tma) stage_tma_drain();
+  }
+  __syncthreads();
+  cluster_sync();          // rank 0's MMAs into both TMEMs are complete
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// Pairs of this kernel that can be resident at once.
+template <int EPI>
+int pair2_max(int num_sms) {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev]) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms / 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Pair2Cfg<EPI>::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_pair2_kernel<EPI>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms / 2;
+  }
+  n = std::min(n, num_sms / 2);
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <int EPI>
+cudaError_t launch_pair2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
+                         const TcGemmParams& p, int num_sms, cudaStream_t s) {
+  using Cfg = Pair2Cfg<EPI>;
+  static uint64_t attr_devices = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_devices >> (dev & 63) & 1)) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_pair2_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_devices |= 1ull << (dev & 63);
+  }
+  const int64_t max_tiles = ((p.M_cap + 2 * BM - 1) / (2 * BM)) * (p.N / 256);
+  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(pair2_max<EPI>(num_sms), max_tiles));
+  return launch_dependent(tc_gemm_pair2_kernel<EPI>, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM, s,
+                          2, a, b, d, p);
+}
+
 template <int EPI>
 cudaError_t launch_epi(int BN, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
                        const TcGemmParams& p, int grid, cudaStream_t s) {
@@ -396,6 +641,11 @@ cudaError_t launch_tc_gemm(int BN, int epi, const CUtensorMap& a, const CUtensor
                          (int64_t)p.groups * p.a_group_rows > INT32_MAX ||
                          (int64_t)p.groups * p.w_group_rows > INT32_MAX))))
     return cudaErrorInvalidValue;
+  // The FFN up-projection (SiLU, K >= 512) on SM pairs: its one-SM tiles wait
+  // on operand traffic.  Measured on the other BN = 256 GEMMs (plain store,
+  // per-user bias, norm; K = 256 or N = 256) the pair tiles were no faster or
+  // slower, so they keep the one-SM kernel.
+  if (BN == 256 && epi == TC_SILU && p.K >= 512) return launch_pair2<TC_SILU>(a, b, dm, p, num_sms, s);
   // grid: one CTA per SM, never more CTAs than the largest possible tile count
   const int64_t max_tiles = ((p.M_cap + BM - 1) / BM) * (p.N / BN) *
                             (epi == TC_F32 ? (int64_t)p.k_split * p.groups : 1);

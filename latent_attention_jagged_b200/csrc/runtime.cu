@@ -288,7 +288,9 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_store16(&h->tms_KV, h->KV, rh, 2 * hdh, false);
     ok = ok && make_tmap_store16(&h->tms_Qh, h->Qt, rq, hdh, false);
   }
-  auto box = [](int bn) { return (uint32_t)std::min(bn, 256); };
+  // weight tiles load in boxes of at most 128 rows (an SM pair's CTA loads
+  // one 128-row half of a 256-row tile; the one-SM kernel stacks boxes)
+  auto box = [](int bn) { return (uint32_t)std::min(bn, 128); };
   for (int l = 0; l < D.n_layers && ok; ++l) {
     const LayerDev& W = h->layers[l];
     LayerMaps& M = h->lmaps[l];

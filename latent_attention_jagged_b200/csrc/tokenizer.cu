@@ -262,8 +262,8 @@ int llatte_tokenizer_create(llatte_tokenizer** out, const llatte_tok_dims* dims,
   if (t->use_tc) {
     bool ok = make_tmap_bf16(&t->tm_E, t->E, n, t->d_in, 128) &&
               make_tmap_bf16(&t->tm_H, t->H, n, dims->d_hid, 128) &&
-              make_tmap_bf16(&t->tm_W1, t->W_a1, dims->d_hid, t->d_in, std::min(t->bn1, 256)) &&
-              make_tmap_bf16(&t->tm_W2, t->W_a2, dims->d, dims->d_hid, std::min(t->bn2, 256));
+              make_tmap_bf16(&t->tm_W1, t->W_a1, dims->d_hid, t->d_in, std::min(t->bn1, 128)) &&
+              make_tmap_bf16(&t->tm_W2, t->W_a2, dims->d, dims->d_hid, std::min(t->bn2, 128));
     if (!ok) t->use_tc = 0;
   }
   // the fused FFN kernel takes 256-wide inputs and outputs and a hidden width
