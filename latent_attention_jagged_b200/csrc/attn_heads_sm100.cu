@@ -124,6 +124,46 @@ struct ItemStream {
   }
 };
 
+// Largest growth of the running max (log2 domain) that the one-pass softmax
+// absorbs without rescaling: the probabilities of a tile stay below 2^kGrow.
+constexpr float kGrow = 8.f;
+
+// Keys at or past lim of this 64-key half take -inf.
+__device__ __forceinline__ void mask_keys(float (&v)[64], int lim) {
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = i < lim ? v[i] : -INFINITY;
+}
+// Four running maxima over 64 scores (three-input max).
+__device__ __forceinline__ void max_keys(float (&m4)[4], const float (&v)[64]) {
+#pragma unroll
+  for (int i = 0; i < 64; i += 8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[i + k], v[i + 4 + k]);
+  }
+}
+// 2^(s - m) for 64 scores: bf16 pairs (keys 2j, 2j + 1 in word j) and the
+// fp32 sums of four interleaved partial rows (two packed pairs).
+__device__ __forceinline__ void exp_keys(const float (&v)[64], float m, float2 (&l2)[2],
+                                         uint32_t (&pk)[32]) {
+  const float2 nm2 = make_float2(-m, -m);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
+    x.x = ex2_approx(x.x);
+    x.y = ex2_approx(x.y);
+    l2[j & 1] = add_f2(l2[j & 1], x);
+    pk[j] = pack_bf16(x.x, x.y);
+  }
+}
+
+// 32 packed probability words into TMEM (one lane's row), waiting for the store.
+__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t (&pk)[32]) {
+  float f[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(pk[j]);
+  tmem_st32(taddr, f);
+}
+
 // Wait for a phase without giving up on the CTA's abort flag (drains only):
 // still bounded by the default wait limit.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
@@ -375,86 +415,88 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int64_t lim64 = vis - (int64_t)kt * KEYS;
         const int lim_k = !valid ? KEYS : (lim64 <= 0 ? 0 : (lim64 >= KEYS ? KEYS : (int)lim64));
         const bool masked = __any_sync(0xffffffffu, lim_k < KEYS);
-        // pass 1: the row max, 64 keys at a time
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
+        // One pass over the scores, 64 keys at a time: the row max on the
+        // side and, past the item's first tile, the probabilities 2^(s - m)
+        // against the running max m (they may exceed 1 until m catches up, by
+        // at most 2^kGrow).  On the item's first tile (no m yet), or when the
+        // tile's max exceeds m by more than kGrow in some row of the warp, the
+        // warp takes a second pass with the new max instead.  Every
+        // exponential goes to the special-function unit: the softmax is bound
+        // by issue slots, and the FMA-pipe form costs seven times the
+        // instructions.  A masked score (-inf) gives exactly 0; a row that
+        // sees no key keeps m = -inf and subtracts 0 instead.
+        const bool have_m = kt > 0;
+        const float m_use = m_run > -INFINITY ? m_run : 0.f;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // P and O are free once the previous P V product is done
+        bool pv_waited = sc == 0;
+        auto wait_pv = [&]() -> bool {
+          if (pv_waited) return true;
+          pv_waited = true;
+          const bool w2 = mbar_wait(pv_done, (sc - 1) & 1, abort_flag, p.status, lim);
+          if (!__all_sync(0xffffffffu, w2)) return false;
+          tc_fence_after();
+          return true;
+        };
+        {
           float v[64];
-          tmem_ld64(s_base + 64 * h, v);
-          if (masked) {
-            const int lh = lim_k - 64 * h;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = i < lh ? v[i] : -INFINITY;
-          }
-#pragma unroll
-          for (int i = 0; i < 64; i += 16) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], v[i + k], v[i + 8 + k]);
+          tmem_ld64(s_base, v);
+          if (masked) mask_keys(v, lim_k);
+          max_keys(m4, v);
+          if (have_m) {
+            uint32_t pk[32];
+            exp_keys(v, m_use, l2, pk);
+            if (!wait_pv()) { ok = false; break; }
+            store_p(p_base, pk);
           }
         }
-        const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        // lazy rescale (only when the max grows by > 8 in log2): l now, O
-        // once the previous P V product is in it (below)
+        float v[64];
+        tmem_ld64(s_base + 64, v);
+        if (masked) mask_keys(v, lim_k - 64);
+        max_keys(m4, v);
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const bool redo = !have_m || __any_sync(0xffffffffu, mt > m_use + kGrow);
         float scale = 1.f;
         bool resc = false;
-        if (kt == 0) {
-          m_run = mt;
-        } else if (mt > m_run + 8.f) {
-          scale = ex2_approx(m_run - mt);
-          m_run = mt;
-          resc = true;
-        }
-        l_run *= scale;
-        // pass 2: probabilities 2^(s - m) as bf16 pairs (keys 2j, 2j + 1 in
-        // packed column j); one pair in four takes the FMA-pipe exponential,
-        // the rest the special-function unit; both give exactly 0 for a masked
-        // score (-inf).  A row that sees no key keeps m = -inf and subtracts
-        // 0 instead.
-        const float m_use = m_run > -INFINITY ? m_run : 0.f;
-        const float2 nm2 = make_float2(-m_use, -m_use);
-        float2 l4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) l4[i] = make_float2(0.f, 0.f);
-        uint32_t pk[2][32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v[64];
-          tmem_ld64(s_base + 64 * h, v);
-          if (h == 1) {
-            // the scores are in registers: S may take the next tile
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free);
-          }
-          if (masked) {
-            const int lh = lim_k - 64 * h;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = i < lh ? v[i] : -INFINITY;
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
-            if ((j & 3) == 3) {
-              x = exp2_fma2(x);
-            } else {
-              x.x = ex2_approx(x.x);
-              x.y = ex2_approx(x.y);
+        if (!redo) {
+          // the scores are in registers: S may take the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+          uint32_t pk[32];
+          exp_keys(v, m_use, l2, pk);
+          store_p(p_base + 32, pk);
+        } else {
+          // the new max: O and l rescaled (O once the previous P V product
+          // is in it, below)
+          if (mt > m_run) {
+            if (have_m) {
+              scale = ex2_approx(m_run - mt);
+              resc = true;
             }
-            l4[j & 3] = add_f2(l4[j & 3], x);
-            pk[h][j] = pack_bf16(x.x, x.y);
+            m_run = mt;
+          }
+          const float m_new = m_run > -INFINITY ? m_run : 0.f;
+          l2[0] = l2[1] = make_float2(0.f, 0.f);
+          if (!wait_pv()) { ok = false; break; }
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            float u[64];
+            tmem_ld64(s_base + 64 * h, u);
+            if (h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(s_free);
+            }
+            if (masked) mask_keys(u, lim_k - 64 * h);
+            uint32_t pk[32];
+            exp_keys(u, m_new, l2, pk);
+            store_p(p_base + 32 * h, pk);
           }
         }
-        l_run += ((l4[0].x + l4[0].y) + (l4[1].x + l4[1].y)) +
-                 ((l4[2].x + l4[2].y) + (l4[3].x + l4[3].y));
-        // P and O are free once the previous P V product is done
-        if (sc > 0) {
-          w = mbar_wait(pv_done, (sc - 1) & 1, abort_flag, p.status, lim);
-          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-          tc_fence_after();
-        }
+        l_run = l_run * scale + ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y));
+        if (!wait_pv()) { ok = false; break; }
         ++sc;
         if (__any_sync(0xffffffffu, resc)) {
           float o[32];
@@ -464,15 +506,6 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= scale;
             tmem_st32(o_base + c, o);
-          }
-        }
-        {
-          float f[32];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(pk[h][j]);
-            tmem_st32(p_base + 32 * h, f);          // waits for the store
           }
         }
         // P(kt) written: the MMA may read it once the four warps are in
