@@ -123,6 +123,7 @@ struct llatte_handle {
   float* ctxbias;      // [n_layers][B][h*r] (this forward's B)
   float* final_rows;   // [max_rows_q, d] fp32 (readout only)
   float* mean_rows;    // [max_batch, d] fp32
+  void* mean16;        // [max_batch, d] bf16 copy: the tensor-core readout's operand
   size_t ws_bytes;
   int last_B;
 
@@ -150,6 +151,8 @@ struct llatte_handle {
   void* KV;                       // [max_rows_h, 2*h*d_h]
   CUtensorMap tm_Qh, tm_KV, tm_Oh;
   CUtensorMap tm_sh16, tm_sup;    // summary output-projection GEMM operands
+  CUtensorMap tm_mean16, tm_We;   // readout GEMM operands (readout_tc)
+  int readout_tc;                 // the readout projection runs on the tensor cores
 
   // attention-probability export requested for the forward in progress
   const llatte_attn_export* export_req;
@@ -286,6 +289,7 @@ size_t attn_export_smem(int n2, int r, int n_hours);
 cudaError_t launch_attn_export(int elem, const ExportArgs& a, cudaStream_t s);
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
+                             void* mean16,
                              cudaStream_t s);
 // W_q has dq + d_ctx columns (dq = d, or q_rank for W_uq of a low-rank query).
 cudaError_t launch_absorb(int elem, const void* W_q, const void* W_uk, const void* W_uv,

@@ -39,7 +39,7 @@ struct Layout {
   size_t off_hist_off, off_query_off, off_T, off_n, off_totals, off_status, off_work,
       off_work_count, off_work_next, off_item_off, off_row_user;
   size_t off_Xh[2], off_Xq[2], off_C, off_Qt, off_Ot, off_Z, off_Hd, off_Cq, off_acc32, off_ctxbias,
-      off_final, off_mean, off_Zres, off_Xqres[2], off_zraw, off_sum_part, off_sum_h,
+      off_final, off_mean, off_mean16, off_Zres, off_Xqres[2], off_zraw, off_sum_part, off_sum_h,
       off_sum_h16, off_KV;
   size_t total;
   int32_t max_work;
@@ -126,6 +126,7 @@ Layout layout_of(const llatte_dims* d) {
                        std::max<int64_t>(std::max<int64_t>(hr, d->q_rank), hdh));
   L.off_final = take(d->d_out ? sizeof(float) * L.rows_q * d->d : 0);
   L.off_mean = take(d->d_out ? sizeof(float) * B * d->d : 0);
+  L.off_mean16 = take(d->d_out && elem == 2 ? 2 * (size_t)B * d->d : 0);
   // sequence summaries: the final query-token rows and the split-K partials
   // (S * B <= kSplitCtas * 128 / column tiles, or S = 1)
   const int64_t sN = (int64_t)d->n_sum * d->sum_rank;
@@ -278,6 +279,12 @@ bool build_tc_maps(llatte_handle* h) {
     ok = ok && make_tmap_bf16(&h->tm_KV, h->KV, rh, 2 * hdh, 128);
     ok = ok && make_tmap_bf16(&h->tm_Oh, h->Ot, rq, hdh, 128);
     h->pair_norm = h->pair_norm && tc_gemm_pair_supported(TC_NORM, d, hdh);
+  }
+  // readout projection: [max_batch, d] bf16 means times E^T, 64-column tiles
+  h->readout_tc = D.d_out > 0 && h->mean16 && D.d_out % 64 == 0 ? 1 : 0;
+  if (h->readout_tc) {
+    ok = ok && make_tmap_bf16(&h->tm_mean16, h->mean16, std::max(D.max_batch, 1), d, 128);
+    ok = ok && make_tmap_bf16(&h->tm_We, h->W_e, D.d_out, d, 64);
   }
   ok = ok && make_tmap_store16(&h->tms_C, h->C, rh, r, false);
   ok = ok && make_tmap_store16(&h->tms_Qt, h->Qt, rq, hr, false);
@@ -578,6 +585,7 @@ int llatte_create(llatte_handle** out, const llatte_dims* dims, const llatte_lay
   h->ctxbias = (float*)(ws + Lo.off_ctxbias);
   h->final_rows = D.d_out ? (float*)(ws + Lo.off_final) : nullptr;
   h->mean_rows = D.d_out ? (float*)(ws + Lo.off_mean) : nullptr;
+  h->mean16 = D.d_out > 0 && D.dtype == LLATTE_BF16 ? (void*)(ws + Lo.off_mean16) : nullptr;
   h->zraw = D.n_sum ? (void*)(ws + Lo.off_zraw) : nullptr;
   h->sum_part = D.n_sum ? (float*)(ws + Lo.off_sum_part) : nullptr;
   h->sum_h = D.n_sum ? (float*)(ws + Lo.off_sum_h) : nullptr;
@@ -948,11 +956,21 @@ int forward_impl(llatte_handle* h, const void* values, const int64_t* offsets, i
   }
   if (D.d_out > 0) {
     StepTimer t(h, s, ST_READOUT);
-    CK(launch_mean_rows(h->final_rows, p.qoff(L - 1), B, d, h->mean_rows, s));
-    GemmArgs g = {};
-    g.A = h->mean_rows; g.lda = d; g.W = h->W_e; g.D = out; g.ldd = D.d_out;
-    g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = D.d_out; g.K = d; g.epi = EPI_F32;
-    CK(launch_gemm_simt(4, e, 4, g, s));
+    CK(launch_mean_rows(h->final_rows, p.qoff(L - 1), B, d, h->mean_rows,
+                        h->readout_tc ? h->mean16 : nullptr, s));
+    if (h->readout_tc) {
+      // out = mean E^T on the tensor cores: the mean in bf16, fp32 out
+      TcGemmParams q = {};
+      q.M_host = B; q.M_dev = nullptr; q.M_cap = D.max_batch; q.N = D.d_out; q.K = d;
+      q.status = p.status; q.Dp = out; q.slice_stride = 0; q.k_split = 1; q.groups = 1;
+      q.ldp = D.d_out;
+      CK(launch_tc_gemm(64, TC_F32, h->tm_mean16, h->tm_We, q, h->num_sms, s));
+    } else {
+      GemmArgs g = {};
+      g.A = h->mean_rows; g.lda = d; g.W = h->W_e; g.D = out; g.ldd = D.d_out;
+      g.M_host = B; g.M_dev = nullptr; g.M_max = B; g.N = D.d_out; g.K = d; g.epi = EPI_F32;
+      CK(launch_gemm_simt(4, e, 4, g, s));
+    }
     t.done(2);
   }
   if (D.n_sum > 0) {  // sequence summaries of the final query-token rows

@@ -310,14 +310,16 @@ cudaError_t launch_ctx_bias(int elem, const void* ctx, const CtxWeights& w, int 
 // ---------------------------------------------------------------- readout mean
 // mean[u] = (1 / rows_u) sum of the user's final rows (zero for no rows).
 // mean[u, :] = mean of user u's rows.  A block takes 128 columns (32 float4)
-// of one user; its eight warps take every eighth row (the sums of many rows
-// in flight at once instead of one long dependent chain per column), then
-// the eight partial sums are added in warp order (deterministic).
+// of one user; its eight warps take every eighth row, four rows' loads in
+// flight per warp (the sums of many rows in flight at once instead of one
+// long dependent chain per column), then the eight partial sums are added in
+// warp order (deterministic).  With mean16 set the mean is also written in
+// bf16: the A operand of the tensor-core readout projection.
 constexpr int kMeanWarps = 8;
 
 __global__ void __launch_bounds__(32 * kMeanWarps)
 mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qoff, int d,
-                 float* __restrict__ mean) {
+                 float* __restrict__ mean, __nv_bfloat16* __restrict__ mean16) {
   __shared__ float4 part[kMeanWarps][32];
   const int u = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -327,6 +329,7 @@ mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qof
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (c4 < d4) {
     const float4* r4 = reinterpret_cast<const float4*>(rows);
+#pragma unroll 4
     for (int64_t i = a + warp; i < b; i += kMeanWarps) {
       const float4 v = __ldg(r4 + i * d4 + c4);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
@@ -341,16 +344,21 @@ mean_rows_kernel(const float* __restrict__ rows, const int64_t* __restrict__ qof
       t.x += p.x; t.y += p.y; t.z += p.z; t.w += p.w;
     }
     const float inv = b > a ? 1.f / (float)(b - a) : 0.f;
-    reinterpret_cast<float4*>(mean)[(int64_t)u * d4 + c4] =
-        make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+    const float4 m = make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+    reinterpret_cast<float4*>(mean)[(int64_t)u * d4 + c4] = m;
+    if (mean16) {
+      const uint2 w = make_uint2(tc::pack_bf16(m.x, m.y), tc::pack_bf16(m.z, m.w));
+      reinterpret_cast<uint2*>(mean16)[(int64_t)u * d4 + c4] = w;
+    }
   }
 }
 
 cudaError_t launch_mean_rows(const float* rows, const int64_t* qoff, int B, int d, float* mean,
-                             cudaStream_t s) {
+                             void* mean16, cudaStream_t s) {
   if (B == 0) return cudaSuccess;
   if (d % 4 != 0) return cudaErrorInvalidValue;
-  mean_rows_kernel<<<dim3(B, (d / 4 + 31) / 32), 32 * kMeanWarps, 0, s>>>(rows, qoff, d, mean);
+  mean_rows_kernel<<<dim3(B, (d / 4 + 31) / 32), 32 * kMeanWarps, 0, s>>>(
+      rows, qoff, d, mean, (__nv_bfloat16*)mean16);
   return cudaGetLastError();
 }
 
