@@ -13,28 +13,32 @@
 //   TMEM   O | S | P        (64 + 128 + 64 = 256 columns, half of the SM's)
 // P is kept apart from S, so S(kt + 1) is computed while the softmax still
 // turns the scores of tile kt into probabilities: the softmax signals "S
-// read" once its last TMEM load of the scores is done, and the MMA issuer
-// starts S(kt + 1) then; O += P(kt) V follows once P(kt) is written.
+// read" once its TMEM loads of the scores are done and the row max is known,
+// and the MMA issuer starts S(kt + 1) then; O += P(kt) V follows once P(kt)
+// is written.
 //
 // Work item: one user, one head and a block of 128 query rows (the attention
-// work list of the layer, longest first).
-// Roles (192 threads):
+// work list of the layer, ordered by user).
+// Roles (320 threads):
 //   warp 0       TMA: the item's query tile (double-buffered, so the next
 //                item's arrives during this one), then its key and value tiles
 //                into a 2-stage ring
 //   warp 1       TMEM owner; lane 0 issues, per key tile, S(kt) once the
 //                softmax has read S(kt - 1), then O += P(kt - 1) V once P(kt - 1)
 //                is written
-//   warps 2..5   softmax, one warp per TMEM lane quadrant: all 128 keys of the
-//                tile for the quadrant's 32 rows, one row per thread, in two
-//                passes over the scores (row max; then 2^(s - m) in fp32), 64
-//                keys at a time (a whole row of S in registers would spill);
-//                masking: a history row at position p sees keys t <= p, a
-//                query token every key t < T; lazy rescale of O when the
-//                running max grows by more than 2^8; P written to TMEM as
-//                bf16 once the previous P V product has read it.  The same
-//                warps divide O by the row sums and store it through shared-
-//                memory staging, deferred into the next item's first tile so
+//   warps 2..9   softmax, two warps per TMEM lane quadrant, each taking 64 of
+//                the tile's 128 keys for the quadrant's 32 rows (one row per
+//                thread), 32 keys at a time; past an item's first tile in one
+//                pass (probabilities against the running max, the tile max on
+//                the side), the two warps' maxima meeting in shared memory
+//                behind a bounded pair barrier; a second pass only on an
+//                item's first tile or when a row's max grows by more than 2^8
+//                (then O and l are rescaled).  Masking: a history row at
+//                position p sees keys t <= p, a query token every key t < T.
+//                P goes to TMEM as bf16 16 columns at a time once the previous
+//                P V product has read it.  The same warps divide O by the row
+//                sums (each warp 32 of its 64 columns) and store it straight
+//                from registers, deferred into the next item's first tile so
 //                that the softmax never waits for the last product of an item.
 #include <cuda.h>
 
@@ -52,9 +56,11 @@ using namespace tc;
 
 namespace {
 
-constexpr int kSoftWarps = 4;                      // one per TMEM lane quadrant
+constexpr int kSplit = 2;                          // softmax warps per TMEM lane quadrant
+constexpr int kSoftWarps = 4 * kSplit;
 constexpr int kThreads = 32 * (2 + kSoftWarps);
 constexpr int KEYS = 128;                          // keys per tile
+constexpr int KP = KEYS / kSplit;                  // keys per softmax warp
 constexpr int DH = 64;                             // head width
 constexpr int QBUF = 2;                            // query tiles in flight
 constexpr int KS = 2;                              // key / value tiles in the ring
@@ -67,8 +73,10 @@ constexpr uint32_t P_COL = S_COL + KEYS;           // bf16 pairs: keys 2j, 2j + 
 constexpr uint32_t TMEM_COLS = 256;
 static_assert(P_COL + KEYS / 2 <= TMEM_COLS, "TMEM budget");
 constexpr uint32_t BAR_BYTES = 256;
-constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)KS * KV_BYTES + BAR_BYTES +
-                        kSoftWarps * kStageBytes;
+constexpr uint32_t MX_BYTES = 2 * kSplit * 128 * 4;   // partial row maxima, by tile parity
+constexpr uint32_t LX_BYTES = kSplit * 128 * 4;       // partial row sums at an item's end
+constexpr size_t SMEM = 1024 + QBUF * Q_BYTES + (size_t)KS * KV_BYTES + BAR_BYTES + MX_BYTES +
+                        LX_BYTES;
 // two CTAs per SM
 static_assert(2 * (SMEM + 1024) <= 233472, "shared memory budget");
 
@@ -128,26 +136,26 @@ struct ItemStream {
 // absorbs without rescaling: the probabilities of a tile stay below 2^kGrow.
 constexpr float kGrow = 8.f;
 
-// Keys at or past lim of this 64-key half take -inf.
-__device__ __forceinline__ void mask_keys(float (&v)[64], int lim) {
+// Keys at or past lim of these 32 take -inf.
+__device__ __forceinline__ void mask_keys(float (&v)[32], int lim) {
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = i < lim ? v[i] : -INFINITY;
+  for (int i = 0; i < 32; ++i) v[i] = i < lim ? v[i] : -INFINITY;
 }
-// Four running maxima over 64 scores (three-input max).
-__device__ __forceinline__ void max_keys(float (&m4)[4], const float (&v)[64]) {
+// Four running maxima over 32 scores (three-input max).
+__device__ __forceinline__ void max_keys(float (&m4)[4], const float (&v)[32]) {
 #pragma unroll
-  for (int i = 0; i < 64; i += 8) {
+  for (int i = 0; i < 32; i += 8) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[i + k], v[i + 4 + k]);
   }
 }
-// 2^(s - m) for 64 scores: bf16 pairs (keys 2j, 2j + 1 in word j) and the
+// 2^(s - m) for 32 scores: bf16 pairs (keys 2j, 2j + 1 in word j) and the
 // fp32 sums of four interleaved partial rows (two packed pairs).
-__device__ __forceinline__ void exp_keys(const float (&v)[64], float m, float2 (&l2)[2],
-                                         uint32_t (&pk)[32]) {
+__device__ __forceinline__ void exp_keys(const float (&v)[32], float m, float2 (&l2)[2],
+                                         uint32_t (&pk)[16]) {
   const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < 16; ++j) {
     float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
     x.x = ex2_approx(x.x);
     x.y = ex2_approx(x.y);
@@ -156,12 +164,10 @@ __device__ __forceinline__ void exp_keys(const float (&v)[64], float m, float2 (
   }
 }
 
-// 32 packed probability words into TMEM (one lane's row), waiting for the store.
-__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t (&pk)[32]) {
-  float f[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(pk[j]);
-  tmem_st32(taddr, f);
+// 16 packed probability words into TMEM (one lane's row), waiting for the store.
+__device__ __forceinline__ void store_p(uint32_t taddr, const uint32_t (&pk)[16]) {
+  tmem_st16u(taddr, pk);
+  tmem_wait_st();
 }
 
 // Wait for a phase without giving up on the CTA's abort flag (drains only):
@@ -178,8 +184,7 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                             // [QBUF][Q_BYTES]
   uint8_t* sKV = sQ + QBUF * Q_BYTES;             // [KS][KV_BYTES]
-  uint8_t* sStage = sKV + KS * KV_BYTES;          // [kSoftWarps][kStageBytes]
-  uint64_t* bars = (uint64_t*)(sStage + kSoftWarps * kStageBytes);
+  uint64_t* bars = (uint64_t*)(sKV + KS * KV_BYTES);
   uint64_t* q_full = bars;                        // [QBUF]
   uint64_t* q_empty = q_full + QBUF;              // [QBUF]
   uint64_t* kv_full = q_empty + QBUF;             // [KS]
@@ -191,9 +196,12 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   uint64_t* o_free = pv_done + 1;                 // the previous item's O has been read
   uint64_t* drain = o_free + 1;
   uint64_t* never = drain + 1;                    // nothing arrives (injected timeout)
-  uint32_t* tmem_slot = (uint32_t*)(never + 1);
+  uint64_t* pair_bar = never + 1;                 // [4] the two softmax warps of a quadrant
+  uint32_t* tmem_slot = (uint32_t*)(pair_bar + 4);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  static_assert((2 * QBUF + 2 * KS + 7) * 8 + 8 <= BAR_BYTES, "barrier area");
+  static_assert((2 * QBUF + 2 * KS + 11) * 8 + 8 <= BAR_BYTES, "barrier area");
+  float* mx = (float*)((uint8_t*)bars + BAR_BYTES);    // [2][kSplit][128]
+  float* lx = mx + 2 * kSplit * 128;                   // [kSplit][128]
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,6 +218,7 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     mbar_init(o_free, kSoftWarps);
     mbar_init(drain, 1);
     mbar_init(never, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], kSplit);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -352,79 +361,87 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     // ------------------------------------------------------------ softmax + epilogue
     const int sw = warp - 2;
     const int quad = warp & 3;                       // TMEM lane quadrant
+    const int part = sw >> 2;                        // which KP keys of the tile, O columns
     const int row = quad * 32 + lane;                // row within the tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t s_base = lane_base + S_COL;
-    const uint32_t p_base = lane_base + P_COL;
-    const uint32_t o_base = lane_base + O_COL;
-    const uint32_t stg = smem_u32(sStage + sw * kStageBytes);
-    uint32_t sc = 0;
+    const uint32_t s_base = lane_base + S_COL + part * KP;
+    const uint32_t p_base = lane_base + P_COL + part * (KP / 2);
+    const uint32_t o_base = lane_base + O_COL + part * (DH / 2);
+    uint32_t sc = 0, pphase = 0;
     bool ok = true;
     // The epilogue of an item is deferred into the next item's first tile:
     // its O is read once the P V product before that tile's P is done (the
     // wait that tile makes anyway) and that P is handed over (the first
     // product of the new item also waits for o_free), so the softmax never
-    // stalls for the last product of an item.  The rows and 1 / l of that item:
+    // stalls for the last product of an item.  The row (this warp's 32
+    // columns of it) and 1 / l of that item:
     __nv_bfloat16* prev_orow = nullptr;
     float prev_inv = 0.f;
     bool prev_pending = false;
-    // O / l of the pending item -> bf16 rows (O holds its last product)
+    // O / l of the pending item -> 32 bf16 columns of the row (O holds its
+    // last product); 64 bytes per lane, straight from registers
     auto finish_prev = [&]() {
-      uint4 x[2][4];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float o[32];
-        tmem_ld32(o_base + 32 * c, o);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] *= prev_inv;
-        pack_bf16x32(o, x[c]);
-      }
+      float o[32];
+      tmem_ld32(o_base, o);
       // O may take the next item's first product
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_free);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) stage_store(stg, x[c], prev_orow ? prev_orow + 32 * c : nullptr);
+      for (int i = 0; i < 32; ++i) o[i] *= prev_inv;
+      uint4 x[4];
+      pack_bf16x32(o, x);
+      if (prev_orow) {
+        uint4* dst = reinterpret_cast<uint4*>(prev_orow);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[c] = x[c];
+      }
       prev_pending = false;
     };
     ItemStream items;
     items.start(p, blockIdx.x, n_items, step);
     for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
       const Item it = items.next(p, n_items, step);
-      // this lane's query row jl within the user, and where its 64 output
-      // columns go (null: padding past the user's last row)
+      // this lane's query row jl within the user, and where this warp's 32
+      // output columns go (null: padding past the user's last row)
       const int64_t jl = (int64_t)(it.b / p.heads) * 128 + row;
       const bool valid = it.u >= 0 && jl < (int64_t)it.q;
-      __nv_bfloat16* orow =
-          valid ? p.Ot + (it.qoff + jl) * (int64_t)(p.heads * DH) + (it.b % p.heads) * DH : nullptr;
+      __nv_bfloat16* orow = valid ? p.Ot + (it.qoff + jl) * (int64_t)(p.heads * DH) +
+                                        (it.b % p.heads) * DH + part * (DH / 2)
+                                  : nullptr;
       if (it.nk == 0) {                 // no key at all: the attention output is zero
-        const uint4 z[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                            make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        for (int c = 0; c < DH; c += 32) stage_store(stg, z, orow ? orow + c : nullptr);
+        if (orow) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        }
         continue;
       }
       const int64_t vis = !valid ? 0 : (jl < it.n ? (int64_t)it.T - it.n + jl + 1 : it.T);
-      float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and sum
+      // running max (log2 domain; the same in both warps of the quadrant)
+      // and this warp's part of the row sum
+      float m_run = -INFINITY, l_run = 0.f;
       for (int kt = 0; kt < it.nk; ++kt) {
         bool w = mbar_wait(s_full, sc & 1, abort_flag, p.status, lim);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
-        // keys [0, lim_k) of the tile are visible to the row; masking only
-        // when some row of the warp stops inside the tile.  Padding rows take
+        // keys [0, lim_k) of this warp's KP are visible to the row; masking
+        // only when some row of the warp stops inside them.  Padding rows take
         // every key (they are never stored).
-        const int64_t lim64 = vis - (int64_t)kt * KEYS;
-        const int lim_k = !valid ? KEYS : (lim64 <= 0 ? 0 : (lim64 >= KEYS ? KEYS : (int)lim64));
-        const bool masked = __any_sync(0xffffffffu, lim_k < KEYS);
-        // One pass over the scores, 64 keys at a time: the row max on the
+        const int64_t lim64 = vis - (int64_t)kt * KEYS - part * KP;
+        const int lim_k = !valid ? KP : (lim64 <= 0 ? 0 : (lim64 >= KP ? KP : (int)lim64));
+        const bool masked = __any_sync(0xffffffffu, lim_k < KP);
+        // One pass over the scores, 32 keys at a time: the row max on the
         // side and, past the item's first tile, the probabilities 2^(s - m)
         // against the running max m (they may exceed 1 until m catches up, by
-        // at most 2^kGrow).  On the item's first tile (no m yet), or when the
-        // tile's max exceeds m by more than kGrow in some row of the warp, the
-        // warp takes a second pass with the new max instead.  Every
-        // exponential goes to the special-function unit: the softmax is bound
-        // by issue slots, and the FMA-pipe form costs seven times the
-        // instructions.  A masked score (-inf) gives exactly 0; a row that
-        // sees no key keeps m = -inf and subtracts 0 instead.
+        // at most 2^kGrow).  The two warps of the quadrant then agree on the
+        // row max; on the item's first tile (no m yet), or when that max
+        // exceeds m by more than kGrow in some row, both take a second pass
+        // with the new max instead.  Every exponential goes to the special-
+        // function unit: the softmax is bound by issue slots, and the FMA-pipe
+        // form costs seven times the instructions.  A masked score (-inf)
+        // gives exactly 0; a row that sees no key keeps m = -inf and
+        // subtracts 0 instead.
         const bool have_m = kt > 0;
         const float m_use = m_run > -INFINITY ? m_run : 0.f;
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -440,22 +457,27 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           return true;
         };
         {
-          float v[64];
-          tmem_ld64(s_base, v);
+          float v[32];
+          tmem_ld32(s_base, v);
           if (masked) mask_keys(v, lim_k);
           max_keys(m4, v);
           if (have_m) {
-            uint32_t pk[32];
+            uint32_t pk[16];
             exp_keys(v, m_use, l2, pk);
             if (!wait_pv()) { ok = false; break; }
             store_p(p_base, pk);
           }
         }
-        float v[64];
-        tmem_ld64(s_base + 64, v);
-        if (masked) mask_keys(v, lim_k - 64);
+        float v[32];
+        tmem_ld32(s_base + 32, v);
+        if (masked) mask_keys(v, lim_k - 32);
         max_keys(m4, v);
-        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        // the row max over both halves of the tile
+        float* mxs = mx + (sc & 1) * kSplit * 128;
+        mxs[part * 128 + row] = mt;
+        if (!group_sync(&pair_bar[quad], pphase, abort_flag, p.status)) { ok = false; break; }
+        mt = fmaxf(mt, mxs[(part ^ 1) * 128 + row]);
         const bool redo = !have_m || __any_sync(0xffffffffu, mt > m_use + kGrow);
         float scale = 1.f;
         bool resc = false;
@@ -464,9 +486,10 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
-          uint32_t pk[32];
+          uint32_t pk[16];
           exp_keys(v, m_use, l2, pk);
-          store_p(p_base + 32, pk);
+          if (!wait_pv()) { ok = false; break; }
+          store_p(p_base + 16, pk);
         } else {
           // the new max: O and l rescaled (O once the previous P V product
           // is in it, below)
@@ -481,18 +504,18 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           l2[0] = l2[1] = make_float2(0.f, 0.f);
           if (!wait_pv()) { ok = false; break; }
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            float u[64];
-            tmem_ld64(s_base + 64 * h, u);
-            if (h == 1) {
+          for (int c = 0; c < 2; ++c) {
+            float u[32];
+            tmem_ld32(s_base + 32 * c, u);
+            if (c == 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(s_free);
             }
-            if (masked) mask_keys(u, lim_k - 64 * h);
-            uint32_t pk[32];
+            if (masked) mask_keys(u, lim_k - 32 * c);
+            uint32_t pk[16];
             exp_keys(u, m_new, l2, pk);
-            store_p(p_base + 32 * h, pk);
+            store_p(p_base + 16 * c, pk);
           }
         }
         l_run = l_run * scale + ((l2[0].x + l2[0].y) + (l2[1].x + l2[1].y));
@@ -500,15 +523,12 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         ++sc;
         if (__any_sync(0xffffffffu, resc)) {
           float o[32];
-#pragma unroll 1
-          for (int c = 0; c < DH; c += 32) {
-            tmem_ld32(o_base + c, o);
+          tmem_ld32(o_base, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= scale;
-            tmem_st32(o_base + c, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= scale;
+          tmem_st32(o_base, o);
         }
-        // P(kt) written: the MMA may read it once the four warps are in
+        // P(kt) written: the MMA may read it once the eight warps are in
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
@@ -517,9 +537,13 @@ attn_heads_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (prev_pending) finish_prev();
       }
       if (!ok) break;
-      // this item's epilogue waits for the next item's first tile (or the end)
+      // the row sum over both halves; this item's epilogue waits for the next
+      // item's first tile (or the end)
+      lx[part * 128 + row] = l_run;
+      if (!group_sync(&pair_bar[quad], pphase, abort_flag, p.status)) { ok = false; break; }
+      const float l_row = l_run + lx[(part ^ 1) * 128 + row];
       prev_orow = orow;
-      prev_inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      prev_inv = l_row > 0.f ? 1.f / l_row : 0.f;
       prev_pending = true;
     }
     if (ok && prev_pending) {
