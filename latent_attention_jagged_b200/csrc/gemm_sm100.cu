@@ -236,7 +236,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int kb_lo = (int)((int64_t)ks * KB / S);
         const int nkb = (int)((int64_t)(ks + 1) * KB / S) - kb_lo;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait_sleep(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           // k-blocks in a per-CTA rotated order: the SMs do not all read the
           // same weight lines from L2 at the same moment
@@ -262,13 +262,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait_sleep(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_base = tmem + acc * BN;
         const int ks = (int)(t % S);
         const int nkb = (int)((int64_t)(ks + 1) * KB / S) - (int)((int64_t)ks * KB / S);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait_sleep(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * Cfg::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * Cfg::B_BYTES);
@@ -291,7 +291,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // every MMA of this CTA must be complete before TMEM is released
       umma_commit(drain);
       int dummy = 0;
-      mbar_wait(drain, 0, &dummy, p.status);
+      mbar_wait_sleep(drain, 0, &dummy, p.status);
     }
     __syncwarp();
   } else {
@@ -313,7 +313,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if constexpr (EPI == TC_NORM) {
         if (active) norm_prefetch(p.norm, row, row < M, part, pre);
       }
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      const bool ok = mbar_wait_sleep(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       if (active &&
@@ -453,7 +453,7 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int32_t a_row = mt * 2 * BM + BM * (int)rank;
         const int32_t w_row = nt * BN + 128 * (int)rank;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait_sleep(&empty[stage], phase ^ 1, abort_flag, p.status)) { ok = false; break; }
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
           const uint32_t full_c = cluster_addr(&full[stage], 0);
           // k-blocks in a per-pair rotated order: the SMs do not all read the
@@ -477,13 +477,13 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       bool ok = true;
       for (int64_t t = pair; t < num_tiles && ok; t += n_pairs) {
         // both CTAs' epilogues have read this accumulator's previous tile
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status) ||
+        if (!mbar_wait_sleep(&tempty[acc], acc_phase ^ 1, abort_flag, p.status) ||
             !mbar_wait_cluster(&tempty_peer[acc], acc_phase ^ 1, abort_flag, p.status))
           break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait_sleep(&full[stage], phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad0 = sdesc_sw128(smem_u32(sA + stage * Cfg::A_BYTES), 16, 1024);
           const uint64_t bd0 = sdesc_sw128(smem_u32(sB + stage * Cfg::B_BYTES), 16, 1024);
@@ -501,13 +501,13 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       // every pair MMA must be complete before either CTA releases TMEM
       umma_commit_pair(drain);
       int dummy = 0;
-      mbar_wait(drain, 0, &dummy, p.status);
+      mbar_wait_sleep(drain, 0, &dummy, p.status);
     } else if (lane == 0) {
       // rank 1: forward this CTA's "accumulator free" to rank 0
       const uint32_t peer_c[2] = {cluster_addr(&tempty_peer[0], 0), cluster_addr(&tempty_peer[1], 0)};
       uint32_t ti = 0;
       for (int64_t t = pair; t < num_tiles; t += n_pairs, ++ti) {
-        if (!mbar_wait(&tempty[ti & 1], (ti >> 1) & 1, abort_flag, p.status)) break;
+        if (!mbar_wait_sleep(&tempty[ti & 1], (ti >> 1) & 1, abort_flag, p.status)) break;
         mbar_arrive_cluster(peer_c[ti & 1]);
       }
     }
@@ -525,7 +525,7 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const int64_t row = (int64_t)mt * 2 * BM + BM * (int64_t)rank + rr;
       NormPre<BN, 1, GemmCfg<BN, EPI>::P> pre;
       if constexpr (EPI == TC_NORM) norm_prefetch(p.norm, row, row < M, part, pre);
-      const bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      const bool ok = mbar_wait_sleep(&tfull[acc], acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       if (!epilogue<BN, EPI>(p, &tmD, lane_base + acc * BN, row, row < M, nt * BN, 0, 0, part,

@@ -61,6 +61,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with a suspend-time hint: a thread whose phase is not complete
+// sleeps until it completes (or up to kSuspendHintNs) instead of coming back
+// to poll.  Measured: faster for the GEMMs, whose epilogue warps wait a whole
+// tile for their accumulator; slower for the attention softmax, whose waits
+// are short and on its critical path.
+constexpr uint32_t kSuspendHintNs = 100000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Test, without waiting, whether the phase with the given parity has
 // completed (try_wait may suspend the thread for a while before it answers;
 // this returns at once).
@@ -85,6 +103,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicOr(status, LLATTE_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// mbar_wait through mbar_try_wait_sleep: the same contract (the abort flag
+// and the limit are checked every 64 suspensions).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                volatile int* abort_flag, int32_t* status,
+                                                uint64_t limit_ns = kWaitTimeoutNs) {
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
