@@ -11,6 +11,13 @@ from latent_attention_jagged_b200 import Llatte
 # Tolerances fixed by the target: bf16 max-abs <= 3e-2 and relative L2 <= 1e-2;
 # the fp32 configuration max-abs <= 1e-4.
 TOL = {"bf16": dict(max_abs=3e-2, rel_l2=1e-2), "fp32": dict(max_abs=1e-4, rel_l2=1e-5)}
+# Attention-probability statistics (sums of probabilities, each in [0, 1],
+# accumulated in fp32): in a bf16 forward their error comes from the scores
+# the probabilities are made of (bf16 operands), not from the fp32 sums, so
+# they get a bound of their own, a third of the row-output bound; the
+# largest error measured on any tested workload is 2.9e-3 max-abs and 2.4e-3
+# rel-L2.  The fp32 forward keeps the fp32 bound.
+EXPORT_TOL = {"bf16": dict(max_abs=1e-2, rel_l2=5e-3), "fp32": TOL["fp32"]}
 
 
 def to_device(inp):

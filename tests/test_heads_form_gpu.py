@@ -13,7 +13,7 @@ import oracle
 from oracle.analysis import attention_stats
 from workloads import Dims, Workload, make_event_ages, make_inputs, workload
 
-from gpu_harness import assert_close, make_handle, run, sample_users, to_device
+from gpu_harness import EXPORT_TOL, assert_close, make_handle, run, sample_users, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -74,9 +74,10 @@ def test_export_in_a_per_head_layer():
     torch.cuda.synchronize()
     assert h.status() == 0
     R, K, H = attention_stats(inp, 1, 9, ages, 48)
-    assert_close(rec.cpu().numpy().astype(np.float64), R, "bf16", "recent")
-    assert_close(top.cpu().numpy().astype(np.float64), K, "bf16", "topk")
-    assert_close(hrs.cpu().numpy().astype(np.float64), H, "bf16", "hours")
+    tol = EXPORT_TOL["bf16"]
+    assert_close(rec.cpu().numpy().astype(np.float64), R, "bf16", "recent", tol)
+    assert_close(top.cpu().numpy().astype(np.float64), K, "bf16", "topk", tol)
+    assert_close(hrs.cpu().numpy().astype(np.float64), H, "bf16", "hours", tol)
 
 
 @pytest.mark.parametrize("form", [ABSORBED, PER_HEAD])

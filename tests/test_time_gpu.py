@@ -11,7 +11,8 @@ import oracle
 from oracle.analysis import attention_stats
 from workloads import Dims, Workload, make_inputs, workload
 
-from gpu_harness import ages_on_device, assert_close, make_handle, run, sample_users, to_device
+from gpu_harness import (EXPORT_TOL, ages_on_device, assert_close, make_handle, run, sample_users,
+                         to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -75,6 +76,7 @@ def test_forward_without_ages_is_rejected_and_export_uses_them():
     assert h.status() == 0
     assert_close(out.cpu().numpy().astype(np.float64), oracle.forward(inp), "bf16", "out")
     R, K, H = attention_stats(inp, 1, 9, inp.event_age, 72)
-    assert_close(rec.cpu().numpy().astype(np.float64), R, "bf16", "recent")
-    assert_close(top.cpu().numpy().astype(np.float64), K, "bf16", "topk")
-    assert_close(hrs.cpu().numpy().astype(np.float64), H, "bf16", "hours")
+    tol = EXPORT_TOL["bf16"]
+    assert_close(rec.cpu().numpy().astype(np.float64), R, "bf16", "recent", tol)
+    assert_close(top.cpu().numpy().astype(np.float64), K, "bf16", "topk", tol)
+    assert_close(hrs.cpu().numpy().astype(np.float64), H, "bf16", "hours", tol)
