@@ -37,10 +37,18 @@ from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 # kernel sources it was taken on and their hash: the bench reports the figure
 # only while those sources are unchanged (null otherwise).  The captures are
 # summarised under profiles/.
-TRAFFIC = {}
+TRAFFIC = {
+    # fused FFN, online (B = 256): the four layers' launches of one forward,
+    # DRAM read + write 130.4 MB in all
+    ("ffn", "online", "absorbed"): {"bytes": 32.6e6, "sha16": "13ca53a41f9c37eb"},
+    # per-head attention, upstream: captured at B = 16 (222.8 MB over the eight
+    # layers' launches), scaled by the users (x 4: every launch's key and query
+    # tiles grow in proportion)
+    ("attn", "upstream", "per_head"): {"bytes": 111.4e6, "sha16": "c57d4e9cb4cfa754"},
+}
 KERNEL_SOURCES = {
     "ffn": ["ffn_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
-    "attn": ["attn_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "attn": ["attn_sm100.cu", "attn_heads_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "o": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "ffn2": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "kv": ["gemm_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
