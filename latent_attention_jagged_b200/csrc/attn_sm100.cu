@@ -25,12 +25,7 @@
 //                by more than 2^8)
 //   warps 10..13 epilogue: O / l from TMEM to HBM, so the softmax warps move
 //                on to the next item at once
-// Per-head form (MHA = true, the MLA display of appendix A.3 before
-// absorption: K, V = split(c_kv W_up^KV), scores over d_h = 64): an item is
-// one user, one head and a block of 128 query rows; Q, K and V are 64-wide
-// column blocks (head j at columns 64 j) of row-major [rows, h * 64] buffers
-// (K and V side by side in one [rows, 2 h * 64] buffer), the smem stage holds
-// a K tile and a V tile, and O goes to columns 64 j of [rows, h * 64].
+// (MLA in its per-head form runs in its own kernel, attn_heads_sm100.cu.)
 // TMEM: O (double-buffered across items when 2 r + 2 KEYS <= 512 columns),
 // then S double-buffered across key tiles; P(kt) overwrites S(kt) and the
 // P V product reads it from TMEM.  The MMAs of one thread run in issue order,
@@ -57,7 +52,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kEpiWarp0 = 2 + kSoftWarps;
 constexpr int kThreads = 32 * (2 + kSoftWarps + kEpiWarps);
 
-template <int R, bool MHA = false>
+template <int R>
 struct AttnCfg {
   // 128 keys per tile for every rank: the S MMA then has N = 128 (an N = 64
   // MMA takes about 54 cycles instead of 32 on this part)
@@ -68,9 +63,8 @@ struct AttnCfg {
   static constexpr int QBUF = R <= 128 ? 2 : 1;          // query blocks in flight
   static constexpr int KV_STAGES = R >= 256 ? 2 : 4;   // 64 KB or 32 KB per C tile
   static constexpr uint32_t Q_BYTES = 128 * R * 2;
-  static constexpr uint32_t KV_BYTES = KEYS * R * 2 * (MHA ? 2 : 1);   // K (+ V) tile
+  static constexpr uint32_t KV_BYTES = KEYS * R * 2;    // one latent tile (K = V)
   static constexpr uint32_t KV_SUB_BYTES = KEYS * 128;  // one 64-wide sub-tile of a C tile
-  static constexpr uint32_t V_OFF = MHA ? KEYS * R * 2 : 0;   // V tile within a stage
   static constexpr uint32_t S_COL = OBUF * R;           // S buffers after O
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t L_BYTES = 2 * 128 * 4;      // row sums handed to the epilogue
@@ -81,7 +75,6 @@ struct AttnCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(OBUF * R + 2 * KEYS <= 512, "TMEM budget");
   static_assert(KP == 64, "softmax chunk");
-  static_assert(!MHA || R == 64, "per-head form: d_h = 64");
 };
 
 // TMEM column (relative to the S buffer) of the packed bf16 P for keys
@@ -129,9 +122,8 @@ struct ItemStream {
     ub = entry(p, first + step, n_items);
   }
   // The current item, fully derived; then the prefetch moves one item on.
-  // Absorbed form: block b covers (query row, head) pairs 128 b .. 128 b + 127
-  // (heads interleaved).  Per-head form: b = 128-row block * heads + head.
-  template <bool MHA>
+  // Block b covers (query row, head) pairs 128 b .. 128 b + 127 (heads
+  // interleaved).
   __device__ __forceinline__ Item next(const AttnTcParams& p, int n_items, int step, int keys) {
     Item it;
     it.u = u; it.b = b; it.T = T; it.n = n; it.hoff = hoff; it.qoff = qoff;
@@ -139,8 +131,7 @@ struct ItemStream {
     if (u < 0) {
       it.nk = 0;
     } else {
-      const int64_t jl = MHA ? min((int64_t)(b / p.heads) * 128 + 127, (int64_t)it.q - 1)
-                             : min((int64_t)b * 128 + 127, (int64_t)it.q * p.heads - 1) / p.heads;
+      const int64_t jl = min((int64_t)b * 128 + 127, (int64_t)it.q * p.heads - 1) / p.heads;
       const int64_t kmax = jl < n ? (int64_t)T - n + jl + 1 : T;
       it.nk = (int)((kmax + keys - 1) / keys);
     }
@@ -172,11 +163,11 @@ __device__ __forceinline__ void tmem_st_packed(uint32_t taddr, const uint32_t (&
   }
 }
 
-template <int R, bool MHA>
+template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
                const AttnTcParams p) {
-  using Cfg = AttnCfg<R, MHA>;
+  using Cfg = AttnCfg<R>;
   constexpr int KEYS = Cfg::KEYS, KP = Cfg::KP, RSUB = Cfg::RSUB, KS = Cfg::KV_STAGES,
                 OBUF = Cfg::OBUF, QBUF = Cfg::QBUF;
   extern __shared__ uint8_t smem_raw[];
@@ -243,35 +234,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ItemStream items;
       items.start(p, blockIdx.x, n_items, step);
       for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-        const Item it = items.template next<MHA>(p, n_items, step, KEYS);
+        const Item it = items.next(p, n_items, step, KEYS);
         if (it.nk == 0) continue;
         const int qb = itm % QBUF;
         if (!mbar_wait(&q_empty[qb], ((itm / QBUF) & 1) ^ 1, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&q_full[qb], Cfg::Q_BYTES);
         uint8_t* qdst = sQ + qb * Cfg::Q_BYTES;
-        // per-head form: the head's 64 columns of 128 query rows; absorbed:
         // 128 interleaved (row, head) pairs of r columns
-        const int head = MHA ? it.b % p.heads : 0;
-        const int32_t qrow = MHA ? (int32_t)(it.qoff + (int64_t)(it.b / p.heads) * 128)
-                                 : (int32_t)(it.qoff * p.heads + (int64_t)it.b * 128);
+        const int32_t qrow = (int32_t)(it.qoff * p.heads + (int64_t)it.b * 128);
 #pragma unroll
         for (int s = 0; s < RSUB; ++s)
-          tma_load_2d(&tmQ, &q_full[qb], qdst + s * 16384, head * 64 + s * 64, qrow);
+          tma_load_2d(&tmQ, &q_full[qb], qdst + s * 16384, s * 64, qrow);
         for (int kt = 0; kt < it.nk; ++kt, ++g) {
           const int st = g % KS;
           if (!mbar_wait(&kv_empty[st], ((g / KS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&kv_full[st], Cfg::KV_BYTES);
           const int32_t krow = (int32_t)(it.hoff + (int64_t)kt * KEYS);
           uint8_t* dst = sKV + st * Cfg::KV_BYTES;
-          if constexpr (MHA) {
-            // K then V of this head: columns 64 j and h * 64 + 64 j
-            tma_load_2d(&tmC, &kv_full[st], dst, head * 64, krow);
-            tma_load_2d(&tmC, &kv_full[st], dst + Cfg::V_OFF, (p.heads + head) * 64, krow);
-          } else {
 #pragma unroll
-            for (int s = 0; s < RSUB; ++s)
-              tma_load_2d(&tmC, &kv_full[st], dst + s * Cfg::KV_SUB_BYTES, s * 64, krow);
-          }
+          for (int s = 0; s < RSUB; ++s)
+            tma_load_2d(&tmC, &kv_full[st], dst + s * Cfg::KV_SUB_BYTES, s * 64, krow);
         }
         ++itm;
       }
@@ -313,7 +295,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           return false;
         tc_fence_after();
         const int st = gg % KS;
-        const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES) + Cfg::V_OFF;   // V
+        const uint32_t kv_addr = smem_u32(sKV + st * Cfg::KV_BYTES);   // the same tile as V
         const uint32_t p_tmem = tmem + Cfg::S_COL + (gg & 1) * KEYS;
 #pragma unroll
         for (int k = 0; k < KEYS / 16; ++k) {
@@ -344,7 +326,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ItemStream items;
       items.start(p, blockIdx.x, n_items, step);
       for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-        const Item it = items.template next<MHA>(p, n_items, step, KEYS);
+        const Item it = items.next(p, n_items, step, KEYS);
         if (it.nk == 0) continue;
         const int ob = itm % OBUF, qb = itm % QBUF;
         // with one query buffer the next block only arrives after the last S
@@ -377,14 +359,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ItemStream items;
     items.start(p, blockIdx.x, n_items, step);
     for (int idx = blockIdx.x; idx < n_items && ok; idx += step) {
-      const Item it = items.template next<MHA>(p, n_items, step, KEYS);
+      const Item it = items.next(p, n_items, step, KEYS);
       if (it.nk == 0) continue;
       const int ob = itm % OBUF;
       const uint32_t o_col = ob * R + part * (R / 2);   // this warp's half of O
       // this lane's query row jl within the user (absorbed: of its pair)
-      const int64_t pair = MHA ? (int64_t)(it.b / p.heads) * 128 + row : (int64_t)it.b * 128 + row;
-      const bool valid = MHA ? pair < (int64_t)it.q : pair < (int64_t)it.q * p.heads;
-      const int64_t jl = MHA ? pair : pair / p.heads;
+      const int64_t pair = (int64_t)it.b * 128 + row;
+      const bool valid = pair < (int64_t)it.q * p.heads;
+      const int64_t jl = pair / p.heads;
       const int64_t vis = !valid ? 0 : (jl < it.n ? (int64_t)it.T - it.n + jl + 1 : it.T);
       float m_run = -INFINITY, l_run = 0.f;   // running max (log2 domain) and partial sum
       for (int kt = 0; kt < it.nk; ++kt, ++g) {
@@ -459,10 +441,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int j = 0; j < KP / 2; ++j) {
           float2 x = add_f2(make_float2(v[2 * j], v[2 * j + 1]), nm2);
-          // per-head form (d_h = 64): the tensor pipe has slack and the
-          // special-function unit sets the pace, so one pair in four goes to
-          // the FMA pipe; absorbed form: one in eight
-          if (MHA ? (j & 3) == 3 : (j & 7) == 7) {
+          // one pair in eight on the FMA pipe
+          if ((j & 7) == 7) {
             x = exp2_fma2(x);
           } else {
             x.x = ex2_approx(x.x);
@@ -509,17 +489,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     ItemStream items;
     items.start(p, blockIdx.x, n_items, step);
     for (int idx = blockIdx.x; idx < n_items; idx += step) {
-      const Item it = items.template next<MHA>(p, n_items, step, KEYS);
-      __nv_bfloat16* orow;
-      if constexpr (MHA) {
-        const int64_t jl = (int64_t)(it.b / p.heads) * 128 + row;
-        orow = jl < (int64_t)it.q
-                   ? p.Ot + (it.qoff + jl) * (int64_t)(p.heads * 64) + (it.b % p.heads) * 64
-                   : nullptr;
-      } else {
-        const int64_t pair = (int64_t)it.b * 128 + row;
-        orow = pair < (int64_t)it.q * p.heads ? p.Ot + (it.qoff * p.heads + pair) * R : nullptr;
-      }
+      const Item it = items.next(p, n_items, step, KEYS);
+      const int64_t pair = (int64_t)it.b * 128 + row;
+      __nv_bfloat16* orow =
+          pair < (int64_t)it.q * p.heads ? p.Ot + (it.qoff * p.heads + pair) * R : nullptr;
       if (it.nk == 0) {                 // no key: the attention output is zero
         const uint4 z[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
                             make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -559,21 +532,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
 }
 
-template <int R, bool MHA>
+template <int R>
 cudaError_t launch_r(const CUtensorMap& q, const CUtensorMap& c, const AttnTcParams& p, int grid,
                      cudaStream_t s) {
-  using Cfg = AttnCfg<R, MHA>;
+  using Cfg = AttnCfg<R>;
   static uint64_t attr_devices = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_devices >> (dev & 63) & 1)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<R, MHA>,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::SMEM);
     if (e != cudaSuccess) return e;
     attr_devices |= 1ull << (dev & 63);
   }
-  return launch_dependent(attn_tc_kernel<R, MHA>, dim3(grid), dim3(kThreads), Cfg::SMEM, s, 1, q,
+  return launch_dependent(attn_tc_kernel<R>, dim3(grid), dim3(kThreads), Cfg::SMEM, s, 1, q,
                           c, p);
 }
 
@@ -587,17 +560,11 @@ cudaError_t launch_attn_tc(int r, const CUtensorMap& q, const CUtensorMap& c,
                            const AttnTcParams& p, int num_sms, cudaStream_t s) {
   const int grid = std::max(1, std::min(num_sms, p.max_items));
   switch (r) {
-    case 64: return launch_r<64, false>(q, c, p, grid, s);
-    case 128: return launch_r<128, false>(q, c, p, grid, s);
-    case 256: return launch_r<256, false>(q, c, p, grid, s);
+    case 64: return launch_r<64>(q, c, p, grid, s);
+    case 128: return launch_r<128>(q, c, p, grid, s);
+    case 256: return launch_r<256>(q, c, p, grid, s);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_attn_tc_heads(const CUtensorMap& q, const CUtensorMap& kv,
-                                 const AttnTcParams& p, int num_sms, cudaStream_t s) {
-  const int grid = std::max(1, std::min(num_sms, p.max_items));
-  return launch_r<64, true>(q, kv, p, grid, s);
 }
 
 }  // namespace llatte

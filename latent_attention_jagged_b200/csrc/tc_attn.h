@@ -29,9 +29,5 @@ cudaError_t launch_attn_tc(int r, const CUtensorMap& q, const CUtensorMap& c,
 // 128-row block * heads + head); two CTAs per SM.
 cudaError_t launch_attn_heads(const CUtensorMap& q, const CUtensorMap& kv, const AttnTcParams& p,
                               int num_sms, cudaStream_t s);
-// The same with one query tile per CTA over eight softmax warps (the layout of
-// the absorbed kernel); kept for comparison.
-cudaError_t launch_attn_tc_heads(const CUtensorMap& q, const CUtensorMap& kv,
-                                 const AttnTcParams& p, int num_sms, cudaStream_t s);
 
 }  // namespace llatte
