@@ -44,21 +44,23 @@ TRAFFIC = {
     # per-head attention, upstream: captured at B = 16 (222.8 MB over the eight
     # layers' launches), scaled by the users (x 4: every launch's key and query
     # tiles grow in proportion)
-    ("attn", "upstream", "per_head"): {"bytes": 111.4e6, "sha16": "c57d4e9cb4cfa754"},
+    ("attn", "upstream", "per_head"): {"bytes": 111.4e6, "sha16": "f2260204a05194e5"},
 }
 KERNEL_SOURCES = {
     "ffn": ["ffn_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
-    "attn": ["attn_sm100.cu", "attn_heads_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    "attn": ["attn_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
+    # MLA's per-head form runs its own attention kernel
+    ("attn", "per_head"): ["attn_heads_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "o": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "ffn2": ["gemm_sm100.cu", "gemm_pair_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
     "kv": ["gemm_sm100.cu", "tc_common.cuh", "tc_epilogue.cuh"],
 }
 
 
-def sources_hash(step: str) -> str:
+def sources_hash(step: str, form: str = "absorbed") -> str:
     import hashlib
     hsh = hashlib.sha256()
-    for name in KERNEL_SOURCES.get(step, []):
+    for name in KERNEL_SOURCES.get((step, form), KERNEL_SOURCES.get(step, [])):
         with open(os.path.join(ROOT, "latent_attention_jagged_b200", "csrc", name), "rb") as f:
             hsh.update(f.read())
     return hsh.hexdigest()[:16]
@@ -66,7 +68,7 @@ def sources_hash(step: str) -> str:
 
 def traffic_of(step: str, workload_name: str, form: str):
     t = TRAFFIC.get((step, workload_name, form))
-    if t is None or t["sha16"] != sources_hash(step):
+    if t is None or t["sha16"] != sources_hash(step, form):
         return None
     return t["bytes"]
 
@@ -551,7 +553,7 @@ def main():
                 "peak_source": f"{peaks['source']} burst bf16 (cuBLAS, best of 10)",
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": traffic_of(dom, wl.name, form),
-                "traffic_sources_sha16": sources_hash(dom),
+                "traffic_sources_sha16": sources_hash(dom, form),
                 "flops_per_launch": per_launch_flops, "ms_per_launch": dom_ms,
                 "bytes_per_launch": nbytes.get(dom, 0.0) / (prof[dom]["calls"] / prof_steps)}
         # the sequence-summary step (bottleneck GEMM + up-projection), when the
