@@ -149,6 +149,12 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   constexpr int kBuckets = 64;
   __shared__ int32_t hist[kBuckets], cursor[kBuckets];
   __shared__ int32_t total_items;
+  // the users' first items, also in shared memory for batches of at most
+  // kSmemUsers users: every item finds its user by a binary search over them,
+  // which in global memory is a chain of dependent L2 round trips
+  constexpr int kSmemUsers = 4096;
+  __shared__ int32_t s_item_off[kSmemUsers + 1];
+  const bool off_smem = B <= kSmemUsers;
   const int32_t* Tl = p.T + l * bstride;
   const int32_t* nl = p.n + l * bstride;
   int32_t* item_off = p.item_off + l * p.stride;
@@ -165,10 +171,15 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   block_exscan2(cnt, 0, &base, &dummy, &total, &dummy2);
   for (int u = u0; u < u1; ++u) {
     item_off[u] = (int32_t)base;
+    if (off_smem) s_item_off[u] = (int32_t)base;
     base += items_of(u);
   }
-  if (tid == 0) item_off[B] = (int32_t)total;
+  if (tid == 0) {
+    item_off[B] = (int32_t)total;
+    if (off_smem) s_item_off[B] = (int32_t)total;
+  }
   __syncthreads();
+  const int32_t* ioff = off_smem ? s_item_off : item_off;
   auto cost_of = [&](int u, int b) {
     const int64_t q = (int64_t)nl[u] + n_q;
     const int64_t jl = per_head ? min((int64_t)(b / heads) * 128 + 127, q - 1)
@@ -181,7 +192,7 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
     int lo = 0, hi = B - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (item_off[mid] <= i) lo = mid; else hi = mid - 1;
+      if (ioff[mid] <= i) lo = mid; else hi = mid - 1;
     }
     return lo;
   };
@@ -221,7 +232,7 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   }
   for (int i = tid; i < (int)total; i += kPlanThreads) {
     const int u = user_of(i);
-    atomicAdd(&hist[cost_of(u, i - item_off[u])], 1);
+    atomicAdd(&hist[cost_of(u, i - ioff[u])], 1);
   }
   __syncthreads();
   if (tid == 0) {
@@ -232,7 +243,7 @@ plan_kernel(const int64_t* __restrict__ offsets, int B, PlanDev p, KeepArr keep,
   __syncthreads();
   for (int i = tid; i < (int)total; i += kPlanThreads) {
     const int u = user_of(i);
-    const int b = i - item_off[u];
+    const int b = i - ioff[u];
     const int pos = atomicAdd(&cursor[cost_of(u, b)], 1);
     W[2 * pos] = u;
     W[2 * pos + 1] = b;
