@@ -305,8 +305,8 @@ int llatte_plan_static(const llatte_dims* dims, const int64_t* offsets, int32_t 
 
 /*
  * Self-check of an arithmetic building block; the paper has no counterpart.
- * The attention softmax computes some probability pairs (one in four or one
- * in eight, by MLA form) with an
+ * The absorbed-form attention softmax computes one probability pair in eight
+ * with an
  * exponential built from fused multiply-adds (range reduction x = j + f,
  * |f| <= 1/2, a fitted cubic for 2^f, j added to the exponent field) instead
  * of the special-function unit.  This evaluates exactly that device function:
