@@ -22,13 +22,14 @@
 // epilogue on OUT and scatter each row into the next layer's history / query
 // rows.
 // Roles per CTA: warp 0 TMA (Z block, then this CTA's halves of the W1 / W2
-// chunks through a 4-stage ring, in the order the MMAs consume them; the
+// chunks through a 3-stage ring, in the order the MMAs consume them; the
 // bytes of both CTAs are counted on rank 0's barriers), warp 1 TMEM owner
-// (in rank 0 the MMA issuer; in rank 1 it forwards that CTA's SiLU and
-// completions to rank 0 with one remote arrival each), warps 2..9 SiLU and
-// the OUT copy, warps 10..17 the row epilogue (16 rows each: with four warps
-// the row epilogue set the pace of the whole tile).  Completion of the pair MMAs is
-// signalled to both CTAs at once (multicast commit).
+// (in rank 0 also the MMA issuer), warps 2..9 SiLU and the OUT copy, warps
+// 10..17 the row epilogue (16 rows each: with four warps the row epilogue set
+// the pace of the whole tile).  Completion of the pair MMAs is signalled to
+// both CTAs at once (multicast commit); the SiLU and OUT-copy warps of both
+// CTAs arrive directly on rank 0's barriers (rank 1's with remote arrivals),
+// so the issuer waits on one barrier per chunk.
 #include <cuda.h>
 
 #include <algorithm>
@@ -77,12 +78,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
   uint64_t* w_full = bars + 2;                         // [W_STAGES] rank 0: both halves in
   uint64_t* w_empty = w_full + W_STAGES;               // [W_STAGES] both
   uint64_t* h_full = w_empty + W_STAGES;               // [2] both
-  uint64_t* hs_local = h_full + 2;                     // [2] both: this CTA's 8 SiLU warps done
-  uint64_t* hs_peer = hs_local + 2;                    // [2] rank 0: rank 1's SiLU chunk done
-  uint64_t* out_full = hs_peer + 2;                    // both
-  uint64_t* out_local = out_full + 1;                  // both: this CTA's epilogue done
-  uint64_t* out_peer = out_local + 1;                  // rank 0: rank 1's epilogue done
-  uint64_t* v_full = out_peer + 1;                     // both: OUT copied to sV
+  uint64_t* hs_done = h_full + 2;                      // [2] rank 0: both CTAs' SiLU warps done
+  uint64_t* out_full = hs_done + 2;                    // both
+  uint64_t* out_free = out_full + 1;                   // rank 0: both CTAs' OUT copies done
+  uint64_t* v_full = out_free + 1;                     // both: OUT copied to sV
   uint64_t* v_free = v_full + 1;                       // both: row epilogue done with sV
   uint64_t* drain = v_free + 1;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
@@ -105,12 +104,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
     for (int s = 0; s < W_STAGES; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&h_full[b], 1);
-      mbar_init(&hs_local[b], kSiluWarps);
-      mbar_init(&hs_peer[b], 1);
+      mbar_init(&hs_done[b], 2 * kSiluWarps);
     }
     mbar_init(out_full, 1);
-    mbar_init(out_local, kSiluWarps);
-    mbar_init(out_peer, 1);
+    mbar_init(out_free, 2 * kSiluWarps);
     mbar_init(v_full, kSiluWarps);
     mbar_init(v_free, kRowWarps);
     mbar_init(drain, 1);
@@ -189,7 +186,11 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       const uint32_t IDESC1 = p.z_f16 ? idesc_f16(256, HC, false, false)
                                       : idesc_bf16(256, HC, false, false);
       constexpr uint32_t IDESC2 = idesc_bf16(256, D, false, false);
-      const uint32_t z_addr = smem_u32(sZ);
+      // shared-memory descriptors: the start-address field is (address >> 4),
+      // so a k-step or stage offset is a constant added to a base descriptor
+      // (every address here is below 256 KB: no carry out of the field)
+      const uint64_t z_desc = sdesc_sw128(smem_u32(sZ), 16, 1024);
+      const uint64_t w_desc = sdesc_sw128(smem_u32(sW), 16, 1024);
       uint32_t w = 0, ti = 0, gc = 0;
       bool ok = true;
       auto mma1 = [&](int j, uint32_t gcj) -> bool {   // H[gcj&1] = Z W1[chunk(j)]^T
@@ -197,13 +198,11 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
         const int st = w % W_STAGES;
         if (!mbar_wait(&w_full[st], (w / W_STAGES) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t wb = smem_u32(sW + st * W_STAGE_BYTES);
+        const uint64_t wd = w_desc + (uint64_t)(st * (W_STAGE_BYTES >> 4));
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(z_addr + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(wb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024);
-          umma_bf16_pair(d, ad, bd, IDESC1, k != 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < D / 16; ++k)
+          umma_bf16_pair(d, z_desc + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
+                         wd + (uint64_t)((k >> 2) * (8192 >> 4) + (k & 3) * 2), IDESC1, k != 0 ? 1u : 0u);
         umma_commit_pair(&w_empty[st]);
         ++w;
         umma_commit_pair(&h_full[gcj & 1]);
@@ -212,25 +211,21 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       };
       auto mma2 = [&](int j, uint32_t gcj) -> bool {   // OUT += SiLU(H_j) W2[:, chunk(j)]^T
         // SiLU(H_j) of both CTAs in TMEM; for the first chunk of a tile also
-        // both CTAs' epilogues done with OUT
-        if (!mbar_wait(&hs_local[gcj & 1], (gcj >> 1) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait_cluster(&hs_peer[gcj & 1], (gcj >> 1) & 1, abort_flag, p.status)) return false;
-        if (j == 0 && (!mbar_wait(out_local, (ti & 1) ^ 1, abort_flag, p.status) ||
-                       !mbar_wait_cluster(out_peer, (ti & 1) ^ 1, abort_flag, p.status)))
-          return false;
+        // both CTAs' OUT copies done
+        if (!mbar_wait_cluster(&hs_done[gcj & 1], (gcj >> 1) & 1, abort_flag, p.status)) return false;
+        if (j == 0 && !mbar_wait_cluster(out_free, (ti & 1) ^ 1, abort_flag, p.status)) return false;
         const int st = w % W_STAGES;
         if (!mbar_wait(&w_full[st], (w / W_STAGES) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
         // A = SiLU(H_j) as bf16 pairs: hidden columns [64 h, 64 h + 64) were
         // packed into the first 32 columns of that half of the buffer
         const uint32_t ha = tmem + H_COL + (gcj & 1) * HC;
-        const uint32_t wb = smem_u32(sW + st * W_STAGE_BYTES);
+        const uint64_t wd = w_desc + (uint64_t)(st * (W_STAGE_BYTES >> 4));
 #pragma unroll
-        for (int k = 0; k < HC / 16; ++k) {
-          const uint64_t bd = sdesc_sw128(wb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-          umma_bf16_pair_ts(tmem + OUT_COL, ha + (k >> 2) * 64 + (k & 3) * 8, bd, IDESC2,
+        for (int k = 0; k < HC / 16; ++k)
+          umma_bf16_pair_ts(tmem + OUT_COL, ha + (k >> 2) * 64 + (k & 3) * 8,
+                            wd + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2), IDESC2,
                             (j | k) != 0 ? 1u : 0u);
-        }
         umma_commit_pair(&w_empty[st]);
         ++w;
         if (j == NC - 1) umma_commit_pair(out_full);
@@ -248,21 +243,6 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       umma_commit_pair(drain);
       int dummy = 0;
       mbar_wait(drain, 0, &dummy, p.status);
-    } else if (lane == 0) {
-      // rank 1: forward this CTA's SiLU / epilogue completions to rank 0 with
-      // one cluster-scope arrival each, so that the 8 warps only arrive locally
-      const uint32_t hs_peer_c[2] = {cluster_addr(&hs_peer[0], 0), cluster_addr(&hs_peer[1], 0)};
-      const uint32_t out_peer_c = cluster_addr(out_peer, 0);
-      uint32_t gc = 0, ti = 0;
-      bool ok = true;
-      for (int64_t t = pair; t < num_tiles && ok; t += n_pairs, ++ti) {
-        for (int j = 0; j < NC; ++j, ++gc) {
-          if (!mbar_wait(&hs_local[gc & 1], (gc >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_cluster(hs_peer_c[gc & 1]);
-        }
-        if (!ok || !mbar_wait(out_local, ti & 1, abort_flag, p.status)) break;
-        mbar_arrive_cluster(out_peer_c);
-      }
     }
     __syncwarp();
   } else if (warp < kRowWarp0) {
@@ -296,7 +276,10 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&hs_local[gc & 1]);
+        if (lane == 0) {       // on rank 0's barrier (cluster release for rank 1's TMEM writes)
+          if (rank == 0) mbar_arrive(&hs_done[gc & 1]);
+          else mbar_arrive_cluster(cluster_addr(&hs_done[gc & 1], 0));
+        }
       }
       if (!ok) break;
       // OUT (this warp's 128 columns of its row) -> fp16 -> sV, which frees
@@ -322,7 +305,8 @@ ffn_pair_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(out_local);     // OUT may be overwritten
+        if (rank == 0) mbar_arrive(out_free);     // OUT may be overwritten
+        else mbar_arrive_cluster(cluster_addr(out_free, 0));
         mbar_arrive(v_full);        // the row warps may read sV
       }
     }
