@@ -39,8 +39,8 @@ from latent_attention_jagged_b200.sharding import shard_batch  # noqa: E402
 # summarised under profiles/.
 TRAFFIC = {
     # fused FFN, online (B = 256): the four layers' launches of one forward,
-    # DRAM read + write 130.4 MB in all
-    ("ffn", "online", "absorbed"): {"bytes": 32.6e6, "sha16": "13ca53a41f9c37eb"},
+    # DRAM read + write 130.6 MB in all
+    ("ffn", "online", "absorbed"): {"bytes": 32.6e6, "sha16": "33cec15c170da4d5"},
     # per-head attention, upstream: captured at B = 16 (222.8 MB over the eight
     # layers' launches), scaled by the users (x 4: every launch's key and query
     # tiles grow in proportion)
