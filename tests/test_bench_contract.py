@@ -66,3 +66,36 @@ def test_peaks_from_the_measured_file(bench):
         assert peaks["source"] == "fallback"
     # the burst figure is the denominator; the sustained one is never above it
     assert peaks["bf16_tflops_sustained"] <= peaks["bf16_tflops"]
+
+
+def _bench(args, env_extra):
+    import subprocess
+    import sys
+    env = dict(os.environ, LLATTE_REF_STEP_S="0.5", **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, env=env, cwd=ROOT,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return r.stdout
+
+
+def test_reference_arm_prints_one_line_with_the_contract_keys():
+    # the oracle on the host cores, a bounded sample per step, the same metric
+    # and workload as the CUDA arm's main line
+    out = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3"], {})
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["metric"] == "user-seqs/s" and j["unit"] == "user-seqs/s"
+    assert j["value"] > 0 and j["higher_is_better"] is True and j["steps"] == 1 and j["warmup"] == 3
+    assert j["config"]["workload"] == "online"
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
+    e = j["e2e"]
+    assert e["value"] == j["value"] and e["unit"] == j["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    out = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3"],
+                 {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert out.strip() == ""
