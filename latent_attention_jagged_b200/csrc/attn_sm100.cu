@@ -38,6 +38,7 @@
 #include "internal.h"
 #include "tc_attn.h"
 #include "tc_common.cuh"
+#include "tc_drain.cuh"
 #include "tc_epilogue.cuh"
 
 namespace llatte {
@@ -229,7 +230,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t itm = 0, g = 0;
+      uint32_t itm = 0, g = 0, qi = 0;        // items, key tiles, query tiles issued
       bool ok = true;
       ItemStream items;
       items.start(p, blockIdx.x, n_items, step);
@@ -245,6 +246,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int s = 0; s < RSUB; ++s)
           tma_load_2d(&tmQ, &q_full[qb], qdst + s * 16384, s * 64, qrow);
+        ++qi;
         for (int kt = 0; kt < it.nk; ++kt, ++g) {
           const int st = g % KS;
           if (!mbar_wait(&kv_empty[st], ((g / KS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
@@ -256,6 +258,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_2d(&tmC, &kv_full[st], dst + s * Cfg::KV_SUB_BYTES, s * 64, krow);
         }
         ++itm;
+      }
+      // after an abort the MMA thread may have left key / query tiles unread
+      if (*abort_flag) {
+        drain_ring(kv_full, KS, g, p.status);
+        drain_ring(q_full, QBUF, qi, p.status);
       }
     }
     __syncwarp();

@@ -21,6 +21,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tc_drain.cuh"
 #include "tc_epilogue.cuh"
 #include "tc_gemm.h"
 
@@ -100,7 +101,7 @@ gemm_pair_norm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, issued = 0;
       bool ok = true;
       for (int64_t t = pair; t < num_tiles && ok; t += n_pairs) {
         const int32_t arow = (int32_t)(t * 2 * BM + BM * rank);
@@ -116,9 +117,13 @@ gemm_pair_norm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
           for (int s2 = 0; s2 < 2; ++s2)
             tma_load_2d_pair(&tmB, full_c, sB + stage * B_BYTES + s2 * B_SUB, kx,
                              s2 * NI + 128 * (int)rank);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // after an abort: rank 0's full barriers count both CTAs' bytes, and
+      // the cluster barrier at the end holds rank 1 until rank 0 is past here
+      if (rank == 0 && *abort_flag) drain_ring(full, STAGES, issued, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {

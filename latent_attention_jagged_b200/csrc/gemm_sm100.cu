@@ -38,6 +38,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tc_drain.cuh"
 #include "tc_epilogue.cuh"
 #include "tc_gemm.h"
 
@@ -223,7 +224,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, issued = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int64_t tt = t / S;
@@ -248,9 +249,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int s2 = 0; s2 < BN / Cfg::WB; ++s2)
             tma_load_2d(&tmB, &full[stage], sB + stage * Cfg::B_BYTES + s2 * Cfg::WB * 128, kx,
                         w_row + s2 * Cfg::WB);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // after an abort the MMA thread may have left stages unread
+      if (*abort_flag) drain_ring(full, STAGES, issued, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -446,7 +450,7 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, issued = 0;
       bool ok = true;
       for (int64_t t = pair; t < num_tiles && ok; t += n_pairs) {
         const int mt = (int)(t / n_tiles), nt = (int)(t % n_tiles);
@@ -461,9 +465,13 @@ tc_gemm_pair2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           const int kx = ((kb + kb0) % KB) * BK;
           tma_load_2d_pair(&tmA, full_c, sA + stage * Cfg::A_BYTES, kx, a_row);
           tma_load_2d_pair(&tmB, full_c, sB + stage * Cfg::B_BYTES, kx, w_row);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // after an abort: rank 0's full barriers count both CTAs' bytes, and
+      // the cluster barrier at the end holds rank 1 until rank 0 is past here
+      if (rank == 0 && *abort_flag) drain_ring(full, STAGES, issued, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
